@@ -1,0 +1,217 @@
+/*
+ * mk.h -- C ABI of the B200 decode megakernel.
+ *
+ * One call of mk_decode_step() runs one whole greedy decode step of a
+ * Qwen3-style transformer decoder (embedding gather, then per layer RMSNorm ->
+ * QKV projection -> QK-norm + RoPE + KV append -> paged attention -> O
+ * projection + residual -> RMSNorm -> SwiGLU MLP + residual, then final
+ * RMSNorm -> LM head -> argmax) as ONE persistent kernel launch: one CTA per
+ * SM, tasks taken from an in-GPU queue and released by dependency counters,
+ * with no host round trip inside the step.
+ *
+ * Sources: the mega-kernel execution model and the GPU-internal event-driven
+ * task dispatch follow the MPK write-up, "2.1 Mega-Kernel执行模型" (task
+ * descriptors, events with trigger/required counts); the paged shared-memory
+ * allocation and the overlap of the next task's pre-load with the current
+ * task's compute follow its "3.1 分页共享内存管理" and "3.2 任务预取与流水线";
+ * warp roles (loader / consumer / storer) follow the Ada-MK summary,
+ * "Methodik", Phase II ("Warp-Spezialisierung"); the decoder it runs is the
+ * "Transformer-Decoder und LM-Head" of the same summary's Phase I.  None of the
+ * pages defines an interface; this one is the library's own.
+ *
+ * Conventions for every function below:
+ *   - Pointers named d_* (and every pointer inside mk_weights / mk_kv_cache)
+ *     are CUDA device pointers on the plan's device; h_* are host pointers.
+ *   - bf16 = IEEE bfloat16 stored as 2 bytes.  Weight matrices are row-major
+ *     [out, in] (nn.Linear convention): y = W x.
+ *   - Every device pointer must be 16-byte aligned.
+ *   - The caller owns all weights, the KV cache, the block table and all step
+ *     inputs/outputs; the plan only reads/writes them during a step.  The plan
+ *     owns its task array, counters and workspace and frees them in
+ *     mk_plan_destroy().
+ *   - Return values: MK_OK (0) or a negative MK_ERR_* code.  Argument errors
+ *     are detected on the host before any launch and leave the plan
+ *     unchanged; mk_last_error() then describes the problem.
+ *   - A plan serves one stream at a time and is not thread-safe.
+ */
+#ifndef MK_H_
+#define MK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MK_API __attribute__((visibility("default")))
+#else
+#define MK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MK_OK 0
+#define MK_ERR_INVALID_ARG (-1) /* bad pointer / size / alignment (host)      */
+#define MK_ERR_UNSUPPORTED (-2) /* valid but not supported shape (host)       */
+#define MK_ERR_CUDA (-3)        /* a CUDA runtime call failed (host)          */
+#define MK_ERR_RANGE (-4)       /* device: token id >= vocab, position out of
+                                   range, or block-table entry out of range  */
+#define MK_ERR_TIMEOUT (-5)     /* device: a dependency wait exceeded the
+                                   plan's wait limit; the step was abandoned  */
+#define MK_ERR_STATE (-6)       /* the plan holds an unread/uncleared device
+                                   error; call mk_plan_reset()                */
+
+#define MK_MAX_LAYERS 128
+#define MK_MAX_BATCH 16
+
+/* Model shape.  hidden, n_q_heads*head_dim and ffn must be multiples of 8;
+ * head_dim one of 32, 64, 128, 256; n_q_heads a multiple of n_kv_heads with
+ * at most 8 query heads per KV head.  Other shapes: MK_ERR_UNSUPPORTED. */
+typedef struct {
+  int n_layers;     /* 1 .. MK_MAX_LAYERS                                   */
+  int hidden;       /* H                                                    */
+  int n_q_heads;    /* Hq                                                   */
+  int n_kv_heads;   /* Hkv                                                  */
+  int head_dim;     /* d                                                    */
+  int ffn;          /* F (SwiGLU inner width)                               */
+  int vocab;        /* V                                                    */
+  float rms_eps;    /* epsilon of every RMSNorm                             */
+  float rope_theta; /* RoPE base; pair i turns by pos * theta^(-2i/d),
+                       pairing element i with i + d/2                       */
+  int qk_norm;      /* 1: per-head RMSNorm of q and k before RoPE           */
+  int max_seq_len;  /* positions must satisfy 0 <= pos < max_seq_len        */
+} mk_model_config;
+
+/* Per-layer weights, all bf16 device pointers:
+ *   attn_norm [H], wq [Hq*d, H], wk [Hkv*d, H], wv [Hkv*d, H],
+ *   q_norm [d], k_norm [d] (ignored when qk_norm == 0), wo [H, Hq*d],
+ *   mlp_norm [H], w_gate [F, H], w_up [F, H], w_down [H, F]. */
+typedef struct {
+  const void *attn_norm, *wq, *wk, *wv, *q_norm, *k_norm, *wo, *mlp_norm,
+      *w_gate, *w_up, *w_down;
+} mk_layer_weights;
+
+/* embed [V, H], final_norm [H], lm_head [V, H] (bf16 device pointers; embed
+ * and lm_head may be the same pointer).  `layers` is a HOST array of
+ * n_layers entries.  The plan copies the pointers, not the weights: the
+ * weights must stay allocated and unchanged for the plan's lifetime. */
+typedef struct {
+  const void *embed;
+  const mk_layer_weights *layers;
+  const void *final_norm;
+  const void *lm_head;
+} mk_weights;
+
+/* Paged KV cache.  For layer l, k_pages[l] and v_pages[l] point to bf16
+ * arrays [num_pages, n_kv_heads, page_size, head_dim] (head-major inside a
+ * page, so one head's page is contiguous).  k_pages / v_pages are HOST
+ * arrays of n_layers device pointers.  block_table is a device int32 array
+ * [max_batch, max_pages_per_seq]: sequence b's position p lives in physical
+ * page block_table[b*max_pages_per_seq + p/page_size], slot p%page_size.
+ * Every page a step touches must already be mapped. */
+typedef struct {
+  void *const *k_pages;
+  void *const *v_pages;
+  const int32_t *block_table;
+  int num_pages;
+  int max_pages_per_seq;
+} mk_kv_cache;
+
+/* Plan options (pass NULL to mk_plan_create_ex for the defaults). */
+typedef struct {
+  int max_batch;          /* 1 .. MK_MAX_BATCH (default 1)                  */
+  int kv_page_size;       /* tokens per KV page, multiple of 16 (default 16) */
+  int num_ctas;           /* persistent CTAs; 0 = one per SM                 */
+  int64_t wait_limit_ns;  /* bound on every in-kernel wait (default 2 s)    */
+  int rows_per_task[5];   /* override rows per task for QKV, O, gate/up (per
+                             matrix), down, LM head; 0 = automatic          */
+  int debug_unsatisfiable_dep; /* fault-injection for tests: the first QKV
+                             task waits for one completion more than can
+                             ever happen, so the step must end in
+                             MK_ERR_TIMEOUT after wait_limit_ns             */
+} mk_plan_options;
+
+typedef struct mk_plan mk_plan;
+
+/* Build a plan: validate the shape, tile every operator of every layer into
+ * tasks with dependency counters, build the RoPE table (angles in double
+ * precision), allocate and upload the task array, counters and workspace.
+ * No kernel runs.  On success *out receives the plan. */
+MK_API int mk_plan_create(const mk_model_config *cfg, const mk_weights *weights,
+                   int max_batch, int kv_page_size, mk_plan **out);
+MK_API int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *weights,
+                      const mk_plan_options *opts, mk_plan **out);
+
+/* Execution modes of a step. */
+#define MK_MODE_MEGAKERNEL 0 /* one persistent cooperative launch            */
+#define MK_MODE_PER_OP 1     /* the same task code, one launch per operator
+                                (embed, then per layer QKV, attention, O,
+                                gate/up, down, then LM head), ordered by the
+                                stream instead of by in-GPU counters        */
+
+/* Everything one step reads and writes. */
+typedef struct {
+  const int32_t *d_ids;   /* [batch] token fed by each sequence             */
+  const int32_t *d_pos;   /* [batch] its position; K/V are written at pos and
+                             attention covers positions 0..pos              */
+  const mk_kv_cache *kv;  /* host struct, read during the call              */
+  int batch;              /* 1 .. max_batch                                 */
+  int32_t *d_out_ids;     /* [batch] argmax token (lowest index on ties);
+                             may alias d_ids only if not read afterwards     */
+  float *d_out_logits;    /* [batch, V] fp32, or NULL                       */
+  int32_t *d_out_pos;     /* [batch] receives pos+1, or NULL                 */
+  float *d_hidden;        /* [n_layers, batch, H] fp32 residual stream after
+                             each layer (debug/parity), or NULL             */
+  int mode;               /* MK_MODE_*                                      */
+} mk_step_args;
+
+/* Enqueue one decode step on `stream` (a cudaStream_t; NULL = legacy default
+ * stream).  Asynchronous: device-side errors (MK_ERR_RANGE, MK_ERR_TIMEOUT)
+ * are reported by mk_plan_status().  A step enqueued while the plan holds a
+ * device error does nothing on the device. */
+MK_API int mk_decode_step(mk_plan *plan, const int32_t *d_ids, const int32_t *d_pos,
+                   const mk_kv_cache *kv, int batch, int32_t *d_out_ids,
+                   float *d_out_logits, void *stream);
+MK_API int mk_decode_step_ex(mk_plan *plan, const mk_step_args *args, void *stream);
+
+/* The same step from HOST buffers: copies h_ids/h_pos to the device, runs
+ * the step, copies the argmax ids (and logits if h_out_logits != NULL) back
+ * and synchronizes `stream`.  Returns MK_OK or the device error code. */
+MK_API int mk_decode_step_host(mk_plan *plan, const int32_t *h_ids,
+                        const int32_t *h_pos, const mk_kv_cache *kv, int batch,
+                        int32_t *h_out_ids, float *h_out_logits, void *stream);
+
+/* Synchronize the device and return the device-side status of the plan:
+ * MK_OK, MK_ERR_RANGE or MK_ERR_TIMEOUT.  The status is sticky until
+ * mk_plan_reset(). */
+MK_API int mk_plan_status(mk_plan *plan);
+
+/* Details of the first device error: which task, which event, the value
+ * seen.  `info` receives 4 int32. */
+MK_API int mk_plan_error_info(mk_plan *plan, int32_t *info);
+
+/* Synchronize, then clear all counters and the status so the plan can run
+ * again (the caller's KV cache is not touched). */
+MK_API int mk_plan_reset(mk_plan *plan);
+
+/* Plan facts, for tests and benchmarks. */
+typedef struct {
+  int num_ctas, threads_per_cta, smem_bytes, n_pages, page_bytes;
+  int n_tasks, n_events, attn_slots, tokens_per_smem_page;
+  int rows_per_task[5];   /* QKV, O, gate/up, down, LM head                 */
+  int page_cols[4];       /* columns per weight page: K=H, K=Hq*d, K=F, LM  */
+  int64_t weight_bytes;   /* bytes of weights one step streams (excluding the
+                             embedding rows)                                */
+} mk_plan_info_t;
+MK_API int mk_plan_info(const mk_plan *plan, mk_plan_info_t *info);
+
+/* Message of the last error on the calling thread ("" if none). */
+MK_API const char *mk_last_error(void);
+
+/* Free everything the plan owns (synchronizes first).  NULL is a no-op. */
+MK_API void mk_plan_destroy(mk_plan *plan);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MK_H_ */

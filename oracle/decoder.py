@@ -303,13 +303,16 @@ def decode_step(cfg: DecoderConfig, W: Weights, cache: KVCache,
         cache.length[b] = max(cache.length[b], int(pos[b]) + 1)
     x = rms_norm(h, W.final_norm(), cfg.rms_eps)
     logits = x @ W.lm_head().T
+    def stack(xs, shape):
+        return np.stack(xs) if xs else np.zeros((0,) + shape)
+
     return {
         "logits": logits,
         "next_ids": np.argmax(logits, axis=-1),
-        "hidden": np.stack(hidden),
-        "q": np.stack(qs),
-        "k_new": np.stack(ks),
-        "v_new": np.stack(vs),
+        "hidden": stack(hidden, (B, cfg.hidden)),
+        "q": stack(qs, (B, cfg.n_q_heads, d)),
+        "k_new": stack(ks, (B, cfg.n_kv_heads, d)),
+        "v_new": stack(vs, (B, cfg.n_kv_heads, d)),
     }
 
 

@@ -1,0 +1,146 @@
+// Internal layout shared by the host plan builder (mk_api.cu) and the
+// persistent kernel (mk_kernel.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mk.h"
+
+namespace mk {
+
+// ---- CTA shape -------------------------------------------------------------
+constexpr int kComputeWarps = 8;                  // consumers
+constexpr int kLoaderWarp = 0;                    // producer (TMA issue, queue)
+constexpr int kStorerWarp = 1 + kComputeWarps;    // epilogues + signalling
+constexpr int kThreads = 32 * (kComputeWarps + 2);
+constexpr int kComputeThreads = 32 * kComputeWarps;
+constexpr int kTaskSlots = 4;                     // tasks in flight per CTA
+constexpr int kOutSlots = 2;                      // compute -> storer buffers
+constexpr int kMaxPages = 16;                     // ring entries (upper bound)
+constexpr int kMaxMTiles = 8;                     // 16-row tiles per GEMV task
+constexpr int kMaxGroup = 8;                      // query heads per KV head
+constexpr int kMaxSmem = 232448;                  // opt-in smem per CTA (B200)
+
+// ---- task descriptor (32 bytes, two 16-byte loads) ----------------------------
+enum TaskType : uint8_t {
+  T_EMBED = 1,
+  T_QKV = 2,
+  T_ATTN = 3,
+  T_OPROJ = 4,
+  T_GATEUP = 5,
+  T_DOWN = 6,
+  T_LMHEAD = 7,
+  T_END = 255,
+};
+
+struct alignas(16) Task {
+  uint8_t type;
+  uint8_t n_m;        // 16-row tiles (GEMV); gate/up: gate tiles + up tiles
+  uint16_t layer;
+  uint32_t row0;      // first output row within its matrix
+  uint32_t nrows;     // valid output rows (<= 16 * n_m; gate/up: per matrix)
+  uint32_t dep_event; // event this task waits on (kNoEvent = none)
+  uint32_t dep_count; // completions of dep_event per step
+  uint32_t out_event; // event incremented once the task's output is visible
+  uint32_t aux;       // QKV: matrix (0 q, 1 k, 2 v); ATTN: slot index
+  uint32_t aux2;      // QKV: global head index; epilogue count in high 16 bits
+};
+static_assert(sizeof(Task) == 32, "task descriptor must be 32 bytes");
+constexpr uint32_t kNoEvent = 0xffffffffu;
+
+// ---- per-layer weight pointers (device table) ------------------------------
+struct LayerW {
+  const __nv_bfloat16 *attn_norm, *wq, *wk, *wv, *q_norm, *k_norm, *wo,
+      *mlp_norm, *w_gate, *w_up, *w_down;
+};
+
+// ---- counters region (uint32 words) ----------------------------------------
+enum SyncWord : int {
+  S_QUEUE = 0,     // next ticket
+  S_EXIT = 1,      // CTAs that finished the launch
+  S_STATUS = 2,    // first device error (0 = none)
+  S_ABORT = 3,     // nonzero: every CTA leaves as soon as it sees it
+  S_INFO = 4,      // 4 words: task index, event, value seen, code detail
+  S_LMCTR = 8,     // LM-head tasks finished this step (reset by the last)
+  S_EVENTS = 16,   // events start here
+};
+
+// ---- op classes for page geometry --------------------------------------------
+enum OpK : int { K_HID = 0, K_ATT = 1, K_FFN = 2, K_LM = 3 };
+
+// ---- kernel parameters (passed by value, < 4 KB) ----------------------------
+struct Params {
+  // plan (static)
+  const Task *tasks;
+  const LayerW *layers;
+  const __nv_bfloat16 *embed, *final_norm, *lm_head;
+  const float2 *rope_cs;        // [max_seq_len][d/2] (cos, sin)
+  float *h;                     // [maxB][H]      residual stream
+  float *qkv;                   // [maxB][NQKV]   raw projections
+  float *qrot;                  // [maxB][Hq][d]  q after norm + RoPE
+  float *attn_part;             // [slots][G][d+2] chunk partials (acc, m, l)
+  float *o;                     // [maxB][Hq*d]   attention output
+  float *u;                     // [maxB][F]      SwiGLU output
+  unsigned long long *argmax;   // [maxB]         packed (value, ~index)
+  uint32_t *sync;               // counters
+  uint32_t *head_ctr;           // [L][Hq+2Hkv]   QKV tasks done per head
+  uint32_t *comb_ctr;           // [maxB][Hkv]    attention chunks done
+
+  int L, H, Hq, Hkv, d, F, V, G, NQKV;
+  float eps;
+  int qk_norm;
+  int max_batch, page_size, max_pos, num_kv_pages, max_pages_per_seq;
+  int attn_slots, attn_target, tpp;   // slots per layer, chunk target, tokens per smem page
+  int kp[4];                          // page columns per op class
+  int x_cap;                          // bytes of the activation staging area
+  int page_bytes, n_pages;
+  int off_slots, off_red, off_out, out_bytes, off_x, off_pages;  // smem carve-up
+  int n_tasks;
+  int ev_embed, ev_layer0, ev_per_layer;   // event numbering
+  int n_lm_tasks;
+  long long wait_limit_ns;
+
+  // per step
+  uint32_t epoch;
+  int batch;
+  int task_begin, task_end;   // launch covers tickets mapped onto [begin, end)
+  int mode;
+  const int32_t *ids, *pos;
+  int32_t *out_ids, *out_pos;
+  float *out_logits, *hidden_dump;
+  const int32_t *block_table;
+  __nv_bfloat16 *k_pages[MK_MAX_LAYERS];
+  __nv_bfloat16 *v_pages[MK_MAX_LAYERS];
+};
+
+// event numbering helpers (host and device)
+__host__ __device__ inline int ev_attn_ready(const Params &p, int l, int g) {
+  return p.ev_layer0 + l * p.ev_per_layer + g;
+}
+__host__ __device__ inline int ev_o_ready(const Params &p, int l) {
+  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv;
+}
+__host__ __device__ inline int ev_oproj(const Params &p, int l) {
+  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + 1;
+}
+__host__ __device__ inline int ev_gateup(const Params &p, int l) {
+  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + 2;
+}
+__host__ __device__ inline int ev_down(const Params &p, int l) {
+  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + 3;
+}
+
+// smem pitch of one 16-row weight page row / one activation row, in bytes:
+// rounded to 128 and offset by 64 so rows g and g+1 fall in opposite halves
+// of the 32 banks (conflict-free 16-byte fragment loads).
+__host__ __device__ inline int row_pitch_bytes(int cols) {
+  return ((cols * 2 + 127) / 128) * 128 + 64;
+}
+
+cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative,
+                        cudaStream_t stream);
+cudaError_t configure_kernel(int smem);
+
+}  // namespace mk
