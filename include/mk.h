@@ -163,6 +163,12 @@ typedef struct {
   float *d_hidden;        /* [n_layers, batch, H] fp32 residual stream after
                              each layer (debug/parity), or NULL             */
   int mode;               /* MK_MODE_*                                      */
+  uint64_t *d_trace;      /* per-task timeline, or NULL: [n_tasks][8] u64 =
+                             {CTA index, loader: slot written, loader: last
+                             page issued, compute: slot received, compute:
+                             input event satisfied, compute: activation
+                             staged, compute: done, storer: output released},
+                             times in ns of the GPU global timer           */
 } mk_step_args;
 
 /* Enqueue one decode step on `stream` (a cudaStream_t; NULL = legacy default

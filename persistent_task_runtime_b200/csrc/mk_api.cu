@@ -512,6 +512,7 @@ int mk_decode_step_ex(mk_plan *plan, const mk_step_args *a, void *stream) {
   p.out_pos = a->d_out_pos;
   p.out_logits = a->d_out_logits;
   p.hidden_dump = a->d_hidden;
+  p.trace = reinterpret_cast<unsigned long long *>(a->d_trace);
   p.block_table = a->kv->block_table;
   p.num_kv_pages = a->kv->num_pages;
   p.max_pages_per_seq = a->kv->max_pages_per_seq;

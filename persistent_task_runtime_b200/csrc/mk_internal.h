@@ -110,6 +110,7 @@ struct Params {
   const int32_t *ids, *pos;
   int32_t *out_ids, *out_pos;
   float *out_logits, *hidden_dump;
+  unsigned long long *trace;  // optional [n_tasks][8] timeline
   const int32_t *block_table;
   __nv_bfloat16 *k_pages[MK_MAX_LAYERS];
   __nv_bfloat16 *v_pages[MK_MAX_LAYERS];

@@ -169,6 +169,11 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// optional timeline: record k of task `idx`
+__device__ __forceinline__ void trace_mark(const Params &p, int idx, int k) {
+  if (p.trace != nullptr) p.trace[static_cast<size_t>(idx) * 8 + k] = gtimer();
+}
+
 // ============================================================================
 // shared-memory control block
 // ============================================================================
@@ -435,6 +440,12 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     if (lane == 0) {
       S = info;
       mbar_arrive(&ctl->slot_full[ts]);
+      if (p.trace != nullptr) {
+        p.trace[static_cast<size_t>(tix) * 8] =
+            blockIdx.x | (static_cast<unsigned long long>(t.type) << 32) |
+            (static_cast<unsigned long long>(t.layer) << 40);
+        trace_mark(p, tix, 1);
+      }
     }
     if (++ts == kTaskSlots) {
       ts = 0;
@@ -511,6 +522,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
         }
       }
     }
+    if (lane == 0) trace_mark(p, tix, 2);
     if (!ok) break;
   }
 
@@ -674,6 +686,7 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     st.sat_ev = t.dep_event;
     st.sat_cnt = t.dep_count;
   }
+  if (ctid == 0) trace_mark(p, S.idx, 4);
 
   float acc[kMaxMTiles][NN][4];
 #pragma unroll
@@ -689,6 +702,7 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
       stage_x(p, ctl, smem, t, geo, xc0, xend - xc0, B, ctid);
       st.xkey = geo.whole ? key : 0xffffffffu;
     }
+    if (ctid == 0 && xc0 == 0) trace_mark(p, S.idx, 5);
     for (int m = 0; m < t.n_m; ++m) {
       for (int c0 = xc0; c0 < xend; c0 += geo.kp) {
         const int nc = min(geo.kp, xend - c0);
@@ -772,6 +786,7 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     bool okl = true;
     if (ctid == 0) okl = wait_event(p, ctl, ev, static_cast<uint32_t>(G + 2), S.idx);
     if (!st.gs.share(ctl, ctid, okl)) return false;
+    if (ctid == 0) trace_mark(p, S.idx, 4);
   }
   // q (normed, rotated) for the G query heads of KV head g, pre-scaled so
   // that scores are in log2 units: s = q.k / sqrt(d) * log2(e).
@@ -779,6 +794,7 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   for (int i = ctid; i < G * d; i += kComputeThreads)
     qs[i] = __ldcg(p.qrot + (static_cast<size_t>(b) * p.Hq + g * G) * d + i) * qscale;
   compute_bar();
+  if (ctid == 0) trace_mark(p, S.idx, 5);
 
   float qv[kMaxGroup][DL];
   float mrun[kMaxGroup], lrun[kMaxGroup], acc[kMaxGroup][DL];
@@ -948,6 +964,7 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     }
     mbar_try_wait(&ctl->slot_full[ts], ts_par);
     const Slot S = slots[ts];
+    if (ctid == 0 && S.t.type != T_END) trace_mark(p, S.idx, 3);
     if (ctid == 0) okl = wait_mbar(p, ctl, &ctl->out_empty[os], os_par ^ 1u, 0xfff60000u, 2);
     if (!st.gs.share(ctl, ctid, okl)) {
       ok = false;
@@ -978,7 +995,10 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       break;
     }
     compute_bar();
-    if (ctid == 0) mbar_arrive(&ctl->out_full[os]);
+    if (ctid == 0) {
+      if (S.t.type != T_END) trace_mark(p, S.idx, 6);
+      mbar_arrive(&ctl->out_full[os]);
+    }
     if (S.t.type == T_END) break;
     if (++ts == kTaskSlots) {
       ts = 0;
@@ -1234,6 +1254,7 @@ __device__ void storer_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     const float *out = reinterpret_cast<const float *>(smem + p.off_out + os * p.out_bytes);
     storer_epilogue(p, ctl, S, out, lane);
     __syncwarp();
+    if (lane == 0) trace_mark(p, S.idx, 7);
     if (lane == 0) {
       mbar_arrive(&ctl->out_empty[os]);
       mbar_arrive(&ctl->slot_empty[ts]);

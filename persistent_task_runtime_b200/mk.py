@@ -71,7 +71,8 @@ class mk_plan_options(C.Structure):
 class mk_step_args(C.Structure):
     _fields_ = [("d_ids", C.c_void_p), ("d_pos", C.c_void_p), ("kv", C.POINTER(mk_kv_cache)),
                 ("batch", C.c_int), ("d_out_ids", C.c_void_p), ("d_out_logits", C.c_void_p),
-                ("d_out_pos", C.c_void_p), ("d_hidden", C.c_void_p), ("mode", C.c_int)]
+                ("d_out_pos", C.c_void_p), ("d_hidden", C.c_void_p), ("mode", C.c_int),
+                ("d_trace", C.c_void_p)]
 
 
 class mk_plan_info_t(C.Structure):
@@ -196,11 +197,12 @@ class Plan:
     def step(self, ids: torch.Tensor, pos: torch.Tensor, kv: KVCacheView, out_ids: torch.Tensor,
              out_logits: Optional[torch.Tensor] = None, out_pos: Optional[torch.Tensor] = None,
              hidden: Optional[torch.Tensor] = None, mode: int = MODE_MEGAKERNEL,
-             batch: Optional[int] = None, stream=None) -> None:
+             batch: Optional[int] = None, trace: Optional[torch.Tensor] = None,
+             stream=None) -> None:
         """Enqueue one decode step (asynchronous; see status())."""
         b = ids.shape[0] if batch is None else batch
         a = mk_step_args(_ptr(ids), _ptr(pos), C.pointer(kv.struct), b, _ptr(out_ids),
-                         _ptr(out_logits), _ptr(out_pos), _ptr(hidden), mode)
+                         _ptr(out_logits), _ptr(out_pos), _ptr(hidden), mode, _ptr(trace))
         _check(self._lib.mk_decode_step_ex(self._h, C.byref(a), _stream_handle(stream)))
 
     def step_plain(self, ids, pos, kv: KVCacheView, batch, out_ids, out_logits=None,
