@@ -217,6 +217,34 @@ MK_API const char *mk_last_error(void);
 /* Free everything the plan owns (synchronizes first).  NULL is a no-op. */
 MK_API void mk_plan_destroy(mk_plan *plan);
 
+/* ---- Decode step without any device allocation ---------------------------
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot call cudaMalloc (a host that routes every device allocation
+ * through its own pool, a memory-capped sandbox, a callback that must not
+ * allocate).  It runs the same kernel as mk_decode_step() without a plan:
+ * the task array, tables, activations and counters live in one file-scope
+ * __device__ array of MK_NOALLOC_SCRATCH_BYTES, which every GPU that loads
+ * this library holds until the process exits.  No cudaMalloc, cudaFree or
+ * other allocating call is made.
+ *
+ * The caller passes the model, the weights, the KV page size and the step
+ * exactly as for a plan built with max_batch = args->batch; args->mode must
+ * be MK_MODE_MEGAKERNEL.  Each call rebuilds and uploads the tables, zeroes
+ * the counters, launches on `stream`, synchronizes it and returns the device
+ * status (MK_OK, MK_ERR_RANGE, MK_ERR_TIMEOUT) or a host error code.  A shape,
+ * batch or max_seq_len whose scratch would exceed the array is rejected with
+ * MK_ERR_UNSUPPORTED and a message in mk_last_error().
+ *
+ * Every call uses the same array and leaves the previous call's contents
+ * behind: calls that overlap on the GPU (several streams or threads) race
+ * and must not be issued.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) and sets the kernel's
+ * shared-memory limit; make that first call before any stream capture. */
+#define MK_NOALLOC_SCRATCH_BYTES (16u << 20)
+MK_API int mk_decode_step_noalloc(const mk_model_config *cfg,
+                                  const mk_weights *weights, int kv_page_size,
+                                  const mk_step_args *args, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

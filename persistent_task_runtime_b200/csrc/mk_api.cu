@@ -52,6 +52,10 @@ struct Range {
 
 }  // namespace
 
+namespace mk {
+void set_last_error(const char *msg) { g_err = msg; }
+}  // namespace mk
+
 struct mk_plan {
   mk_model_config cfg;
   Params base;  // static part of the kernel parameters

@@ -143,5 +143,6 @@ __host__ __device__ inline int row_pitch_bytes(int cols) {
 cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative,
                         cudaStream_t stream);
 cudaError_t configure_kernel(int smem);
+void set_last_error(const char *msg);  // message returned by mk_last_error()
 
 }  // namespace mk

@@ -36,7 +36,10 @@ ERROR_NAMES = {MK_OK: "MK_OK", MK_ERR_INVALID_ARG: "MK_ERR_INVALID_ARG",
 #: every symbol include/mk.h declares
 EXPORTS = ["mk_plan_create", "mk_plan_create_ex", "mk_decode_step", "mk_decode_step_ex",
            "mk_decode_step_host", "mk_plan_status", "mk_plan_error_info", "mk_plan_reset",
-           "mk_plan_info", "mk_last_error", "mk_plan_destroy"]
+           "mk_plan_info", "mk_last_error", "mk_plan_destroy", "mk_decode_step_noalloc"]
+
+#: bytes of the library's static scratch array used by mk_decode_step_noalloc
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class mk_model_config(C.Structure):
@@ -111,6 +114,9 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
     lib.mk_last_error.argtypes = []
     lib.mk_plan_destroy.argtypes = [P]
     lib.mk_plan_destroy.restype = None
+    lib.mk_decode_step_noalloc.argtypes = [C.POINTER(mk_model_config), C.POINTER(mk_weights),
+                                           C.c_int, C.POINTER(mk_step_args), P]
+    lib.mk_decode_step_noalloc.restype = C.c_int
     for name in ("mk_plan_create", "mk_plan_create_ex", "mk_decode_step", "mk_decode_step_ex",
                  "mk_decode_step_host", "mk_plan_status", "mk_plan_error_info",
                  "mk_plan_reset", "mk_plan_info"):
@@ -244,3 +250,42 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def decode_step_noalloc(plan_like: "Plan", ids: torch.Tensor, pos: torch.Tensor, kv: KVCacheView,
+                        out_ids: torch.Tensor, out_logits: Optional[torch.Tensor] = None,
+                        page_size: int = 16, stream=None) -> int:
+    """mk_decode_step_noalloc: one step with no device allocation by the library.
+
+    ``plan_like`` only supplies the model config and weight pointers (its
+    ctypes structs); the call does not use the plan's device memory.  Returns
+    the device status (raises on host-side errors)."""
+    lib = load_library()
+    a = mk_step_args(_ptr(ids), _ptr(pos), C.pointer(kv.struct), ids.shape[0], _ptr(out_ids),
+                     _ptr(out_logits), None, None, MODE_MEGAKERNEL, None)
+    rc = lib.mk_decode_step_noalloc(C.byref(plan_like._c), C.byref(plan_like._w), page_size,
+                                    C.byref(a), _stream_handle(stream))
+    if rc in (MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_CUDA):
+        _check(rc)
+    return rc
+
+
+class ModelRef:
+    """The config and weight-pointer structs of a model, without a plan (for
+    mk_decode_step_noalloc)."""
+
+    def __init__(self, cfg: Dict, weights: Dict, max_seq_len: int = 4096):
+        self._c = mk_model_config(cfg["n_layers"], cfg["hidden"], cfg["n_q_heads"],
+                                  cfg["n_kv_heads"], cfg["head_dim"], cfg["ffn"], cfg["vocab"],
+                                  cfg.get("rms_eps", 1e-6), cfg.get("rope_theta", 1e6),
+                                  1 if cfg.get("qk_norm", True) else 0, max_seq_len)
+        L = cfg["n_layers"]
+        self._weights = weights
+        lw = (mk_layer_weights * L)()
+        for l, w in enumerate(weights["layers"]):
+            lw[l] = mk_layer_weights(*[_ptr(w[k]) for k in (
+                "attn_norm", "wq", "wk", "wv", "q_norm", "k_norm", "wo", "mlp_norm",
+                "w_gate", "w_up", "w_down")])
+        self._lw = lw
+        self._w = mk_weights(_ptr(weights["embed"]), lw, _ptr(weights["final_norm"]),
+                             _ptr(weights["lm_head"]))
