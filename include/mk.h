@@ -65,7 +65,7 @@ extern "C" {
 #define MK_MAX_BATCH 16
 
 /* Model shape.  hidden, n_q_heads*head_dim and ffn must be multiples of 8;
- * head_dim one of 32, 64, 128, 256; n_q_heads a multiple of n_kv_heads with
+ * head_dim one of 32, 64, 128; n_q_heads a multiple of n_kv_heads with
  * at most 8 query heads per KV head.  Other shapes: MK_ERR_UNSUPPORTED. */
 typedef struct {
   int n_layers;     /* 1 .. MK_MAX_LAYERS                                   */
@@ -129,6 +129,9 @@ typedef struct {
                              task waits for one completion more than can
                              ever happen, so the step must end in
                              MK_ERR_TIMEOUT after wait_limit_ns             */
+  int l2_prefetch_kb;     /* per-CTA budget of upcoming weights requested
+                             into L2 ahead of the shared-memory ring, in
+                             KB; 0 = off (the default)                      */
 } mk_plan_options;
 
 typedef struct mk_plan mk_plan;

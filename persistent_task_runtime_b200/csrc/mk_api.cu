@@ -91,8 +91,8 @@ int validate_cfg(const mk_model_config *c) {
   if (!(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f))
     return fail(MK_ERR_INVALID_ARG, "rms_eps must be >= 0 and rope_theta > 0");
   const int d = c->head_dim;
-  if (d != 32 && d != 64 && d != 128 && d != 256)
-    return fail(MK_ERR_UNSUPPORTED, "head_dim %d: supported 32, 64, 128, 256", d);
+  if (d != 32 && d != 64 && d != 128)
+    return fail(MK_ERR_UNSUPPORTED, "head_dim %d: supported 32, 64, 128", d);
   if (c->n_q_heads % c->n_kv_heads != 0)
     return fail(MK_ERR_INVALID_ARG, "n_q_heads %d not a multiple of n_kv_heads %d",
                 c->n_q_heads, c->n_kv_heads);
@@ -178,7 +178,11 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
 
   // ---- shared-memory carve-up ------------------------------------------------
   const int Kmax = std::max(H, std::max(Hq * d, F));
-  const int att_need = G * d * 4 + mk::kComputeWarps * G * (d + 2) * 4;
+  // attention scratch in the staging area: q [G][d] plus either the warps'
+  // running states [warps][G][d+4] or the combine's per-chunk (m, l) pairs
+  const int max_chunks = (c.max_seq_len + P - 1) / P;
+  const int att_need = G * d * 4 + std::max(mk::kComputeWarps * G * (d + 4),
+                                            2 * max_chunks * G + 2 * G) * 4;
   // activation staging: the whole widest input of one sequence, or a
   // 1024-column chunk of every sequence, whichever is larger (<= 64 KB)
   const int chunk_need = 2 * maxB * mk::row_pitch_bytes(std::min(1024, align_up(Kmax, 32)));
@@ -207,11 +211,12 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   }
   tpp = std::min(tpp, 16 * P);
 
-  const int off_slots = 1024;
+  const int off_look = 1024;   // loader lookahead (8 x 48 B)
+  const int off_slots = off_look + 512;
   const int off_red = align_up(off_slots + mk::kTaskSlots * 64, 128);
   const int red_bytes = mk::kComputeWarps * 16 * (maxB > 8 ? 16 : 8) * 4;
   const int off_out = align_up(off_red + red_bytes, 128);
-  const int out_bytes = align_up(std::max(maxB * 16 * mk::kMaxMTiles * 4, G * (d + 2) * 4), 128);
+  const int out_bytes = align_up(maxB * 16 * mk::kMaxMTiles * 4, 128);
   const int off_x = align_up(off_out + mk::kOutSlots * out_bytes, 128);
   const int off_pages = align_up(off_x + x_cap, 128);
   const int n_pages = std::min(mk::kMaxPages, (smem_max - off_pages) / page_bytes);
@@ -239,6 +244,7 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   p.x_cap = x_cap;
   p.page_bytes = page_bytes;
   p.n_pages = n_pages;
+  p.off_look = off_look;
   p.off_slots = off_slots;
   p.off_red = off_red;
   p.off_out = off_out;
@@ -248,6 +254,7 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   p.attn_target = grid;
   p.attn_slots = grid + maxB * Hkv;
   p.wait_limit_ns = o.wait_limit_ns;
+  p.pf_bytes = o.l2_prefetch_kb > 0 ? 1024u * static_cast<uint32_t>(o.l2_prefetch_kb) : 0u;
   p.ev_embed = 0;
   p.ev_layer0 = 1;
   p.ev_per_layer = Hkv + 4;
@@ -407,7 +414,7 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   const size_t o_h = carve(sizeof(float) * maxB * H);
   const size_t o_qkv = carve(sizeof(float) * maxB * NQKV);
   const size_t o_qrot = carve(sizeof(float) * maxB * Hq * d);
-  const size_t o_part = carve(sizeof(float) * static_cast<size_t>(p.attn_slots) * G * (d + 2));
+  const size_t o_part = carve(sizeof(float) * static_cast<size_t>(p.attn_slots) * G * (d + 4));
   const size_t o_o = carve(sizeof(float) * maxB * Hq * d);
   const size_t o_u = carve(sizeof(float) * maxB * F);
   const size_t o_arg = carve(sizeof(unsigned long long) * maxB);

@@ -11,13 +11,15 @@
 namespace mk {
 
 // ---- CTA shape -------------------------------------------------------------
-constexpr int kComputeWarps = 8;                  // consumers
+// 8 warps per CTA: registers are granted per group of four warps, so 8 warps
+// (not 10) leave 255 registers per thread and the consumers run spill-free.
+constexpr int kComputeWarps = 6;                  // consumers
 constexpr int kLoaderWarp = 0;                    // producer (TMA issue, queue)
 constexpr int kStorerWarp = 1 + kComputeWarps;    // epilogues + signalling
 constexpr int kThreads = 32 * (kComputeWarps + 2);
 constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kTaskSlots = 4;                     // tasks in flight per CTA
-constexpr int kOutSlots = 2;                      // compute -> storer buffers
+constexpr int kOutSlots = 4;                      // compute -> storer buffers
 constexpr int kMaxPages = 16;                     // ring entries (upper bound)
 constexpr int kMaxMTiles = 8;                     // 16-row tiles per GEMV task
 constexpr int kMaxGroup = 8;                      // query heads per KV head
@@ -96,7 +98,8 @@ struct Params {
   int kp[4];                          // page columns per op class
   int x_cap;                          // bytes of the activation staging area
   int page_bytes, n_pages;
-  int off_slots, off_red, off_out, out_bytes, off_x, off_pages;  // smem carve-up
+  int off_look, off_slots, off_red, off_out, out_bytes, off_x, off_pages;  // smem carve-up
+  uint32_t pf_bytes;                  // L2 prefetch budget per CTA (0 = off)
   int n_tasks;
   int ev_embed, ev_layer0, ev_per_layer;   // event numbering
   int n_lm_tasks;

@@ -88,6 +88,16 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
       : "memory");
 }
 
+// 1-D bulk copy without a cache hint.
+__device__ __forceinline__ void bulk_load_plain(void *dst, const void *src, uint32_t bytes,
+                                                uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ uint64_t gtimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -142,7 +152,7 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
 // D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.
 __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(  // pure register op: the compiler may schedule it freely
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
       "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -185,10 +195,12 @@ struct Ctl {
   uint64_t slot_empty[kTaskSlots];
   uint64_t out_full[kOutSlots];
   uint64_t out_empty[kOutSlots];
+  uint64_t xbar;                    // activation bulk copy landed
   volatile int cta_abort;
   int skip;
   int flag[2];
-  float rs[MK_MAX_BATCH];
+  float rs[MK_MAX_BATCH];           // RMSNorm scale per sequence
+  float ss[MK_MAX_BATCH];           // running sum of squares per sequence
   float red8[kComputeWarps][MK_MAX_BATCH];
 };
 static_assert(sizeof(Ctl) <= 1024, "control block exceeds its 1 KB slot");
@@ -231,7 +243,9 @@ __device__ bool wait_mbar(const Params &p, Ctl *ctl, uint64_t *bar, uint32_t par
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 7u) == 7u) {
-      if (aborted(p, ctl)) return false;
+      // the CTA flag is a shared-memory read; the global flag is polled rarely
+      if (ctl->cta_abort != 0) return false;
+      if ((it & 255u) == 255u && ld_relaxed(p.sync + S_ABORT) != 0u) return false;
       const uint64_t now = gtimer();
       if (t0 == 0) {
         t0 = now;
@@ -294,7 +308,10 @@ struct Geo {
   int cls;      // OpK
 };
 
-__device__ __forceinline__ int x_bytes(int B, int cols) { return 2 * B * row_pitch_bytes(cols); }
+// Staged activation: fp32 rows, pitch rounded to 128 B and offset by 16 B so
+// the fragments of consecutive sequences fall on complementary banks.
+__device__ __forceinline__ int x_row_bytes(int cols) { return ((cols * 4 + 127) / 128) * 128 + 16; }
+__device__ __forceinline__ int x_bytes(int B, int cols) { return B * x_row_bytes(cols); }
 
 __device__ Geo gemv_geo(const Params &p, const Task &t, int B) {
   Geo g;
@@ -394,10 +411,53 @@ __device__ __forceinline__ int kv_phys_page(const Params &p, int b, int logical)
 // loader (warp 0)
 // ============================================================================
 
+__device__ __forceinline__ bool is_gemv(uint8_t type) {
+  return type == T_QKV || type == T_OPROJ || type == T_GATEUP || type == T_DOWN ||
+         type == T_LMHEAD;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Ask L2 for (up to `budget` bytes of) a GEMV task's weight rows: each task
+// covers whole rows, so its weights are one contiguous region per matrix.
+// Lanes issue 32 KB pieces.  Returns the bytes requested.
+__device__ uint32_t l2_prefetch_task(const Params &p, const Task &t, uint32_t budget, int lane) {
+  if (!is_gemv(t.type) || budget == 0) return 0;
+  const int K = t.type == T_OPROJ ? p.Hq * p.d : (t.type == T_DOWN ? p.F : p.H);
+  const int regions = t.type == T_GATEUP ? 2 : 1;
+  const uint32_t bytes = t.nrows * static_cast<uint32_t>(K) * 2u;
+  uint32_t want = min(budget, bytes * regions);
+  uint32_t done = 0;
+  for (int r = 0; r < regions && done < want; ++r) {
+    const __nv_bfloat16 *W;
+    int row, rv;
+    gemv_tile(p, t, r == 0 ? 0 : (t.n_m >> 1), W, row, rv);
+    const char *base = reinterpret_cast<const char *>(W + static_cast<size_t>(row) * K);
+    const uint32_t n = min(bytes, want - done);
+    for (uint32_t off = static_cast<uint32_t>(lane) * 32768u; off < n; off += 32u * 32768u)
+      prefetch_l2(base + off, min(32768u, n - off));
+    done += n;
+  }
+  return done;
+}
+
+// Tasks popped from the queue but not yet handed to the compute warps.
+constexpr int kLook = 8;
+struct Look {
+  Task t;
+  int tix;
+  uint32_t pf;   // bytes of its weights already requested into L2
+  int pad[2];
+};
+static_assert(sizeof(Look) == 48, "lookahead entry size");
+
 __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol = l2_evict_first_policy();
   Slot *slots = reinterpret_cast<Slot *>(smem + p.off_slots);
+  Look *la = reinterpret_cast<Look *>(smem + p.off_look);
   uint8_t *pages = smem + p.off_pages;
   const int B = p.batch;
 
@@ -411,32 +471,71 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   const int n_launch = p.task_end - p.task_begin;
   uint32_t next = 0;
   if (lane == 0) next = atomicAdd(p.sync + S_QUEUE, 1u);
+  int la_head = 0, la_count = 0;
+  bool exhausted = false;
+  uint32_t pf_ahead = 0;
+
+  // Pop one task into the lookahead (warp-uniform).  With an L2 budget the
+  // loader keeps up to p.pf_bytes of future weights requested into L2, so
+  // HBM keeps streaming while the compute warps wait at a dependency.
+  auto pop_one = [&]() {
+    const uint32_t ticket = __shfl_sync(0xffffffffu, next, 0);
+    if (static_cast<int>(ticket) >= n_launch) {
+      exhausted = true;
+      return;
+    }
+    if (lane == 0) next = atomicAdd(p.sync + S_QUEUE, 1u);
+    const int tix = p.task_begin + static_cast<int>(ticket);
+    const Task t = p.tasks[tix];
+    const uint32_t room = p.pf_bytes > pf_ahead ? p.pf_bytes - pf_ahead : 0u;
+    const uint32_t pf = l2_prefetch_task(p, t, room, lane);
+    const int e = (la_head + la_count) % kLook;
+    if (lane == 0) {
+      la[e].t = t;
+      la[e].tix = tix;
+      la[e].pf = pf;
+    }
+    ++la_count;
+    pf_ahead += pf;
+  };
+  auto top_up = [&](int max_pops) {
+    for (int k = 0; k < max_pops; ++k) {
+      if (exhausted || la_count == kLook) break;
+      // one task ahead; more only while the L2 prefetch budget is not spent
+      // (every popped task is reserved for this CTA, so popping far ahead
+      // delays the last tasks of an operator)
+      if (la_count >= 1 && pf_ahead >= p.pf_bytes) break;
+      pop_one();
+    }
+    __syncwarp();
+  };
 
   while (true) {
-    uint32_t ticket = __shfl_sync(0xffffffffu, next, 0);
-    const bool done = static_cast<int>(ticket) >= n_launch;
-    if (!done && lane == 0) next = atomicAdd(p.sync + S_QUEUE, 1u);
-
+    top_up(kLook);
     int okl = 1;
     if (lane == 0) okl = wait_mbar(p, ctl, &ctl->slot_empty[ts], ts_par ^ 1u, 0xfff00000u, 2);
     ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
     if (!ok) break;
 
     Slot &S = slots[ts];
-    if (done) {
+    if (la_count == 0) {  // queue drained
       if (lane == 0) {
         S.t.type = T_END;
         mbar_arrive(&ctl->slot_full[ts]);
       }
       break;
     }
-    const int tix = p.task_begin + static_cast<int>(ticket);
-    Task t = p.tasks[tix];
+    const Task t = la[la_head].t;
+    const int tix = la[la_head].tix;
+    pf_ahead -= la[la_head].pf;
+    la_head = (la_head + 1) % kLook;
+    --la_count;
     Slot info;
     info.t = t;
     info.idx = tix;
     info.b = -1;
     if (t.type == T_ATTN) attn_resolve(p, B, static_cast<int>(t.aux), info);
+    __syncwarp();
     if (lane == 0) {
       S = info;
       mbar_arrive(&ctl->slot_full[ts]);
@@ -453,8 +552,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     }
 
     // ---- stream the task's operands into the page ring ----
-    if (t.type == T_QKV || t.type == T_OPROJ || t.type == T_GATEUP || t.type == T_DOWN ||
-        t.type == T_LMHEAD) {
+    if (is_gemv(t.type)) {
       const Geo geo = gemv_geo(p, t, B);
       const int pitch = row_pitch_bytes(geo.kp);
       for (int xc0 = 0; xc0 < geo.K && ok; xc0 += geo.kx) {
@@ -481,6 +579,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
               pi = 0;
               pe_par ^= 1u;
             }
+            top_up(1);
           }
         }
       }
@@ -520,6 +619,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
           pi = 0;
           pe_par ^= 1u;
         }
+        top_up(1);
       }
     }
     if (lane == 0) trace_mark(p, tix, 2);
@@ -529,6 +629,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   if (!ok) {
     // Abandoning the step: no bulk copy may still be landing in shared
     // memory when this CTA exits.  Wait (bounded) for every page's last copy.
+    // (L2 prefetches carry no completion and write no shared memory.)
     ctl->cta_abort = 1;
     if (lane == 0) {
       for (int q = 0; q < p.n_pages; ++q) {
@@ -551,47 +652,70 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
 // One weight page (16 rows x nc columns) against the staged activation.
 // Lane (g, q): rows g and g+8, columns c..c+7 of each 32-column group; the
 // 8 columns feed both k16 steps of the mma (a fixed permutation of k that the
-// activation fragment follows as well).
+// activation fragment follows as well).  The staged activation holds, per
+// 8-column block, 8 bf16 "hi" values then 8 bf16 "lo" values (hi + lo == x to
+// ~2^-16), so a fragment is two 16-byte loads.
 template <int NN>
-__device__ __forceinline__ void page_mma(float (&acc)[NN][4], uint32_t pg, int pitch, int nc,
-                                         uint32_t xhi, uint32_t xlo, int xpitch, int xcol0, int B,
-                                         int warp, int lane) {
+__device__ __forceinline__ void page_mma(float (&acc)[NN][4], const uint8_t *pg, int pitch, int nc,
+                                         const uint8_t *xs, int xpitch, int xcol0, int B, int warp,
+                                         int lane) {
   const int g = lane >> 2, q = lane & 3;
   const int groups = (nc + 31) >> 5;
+  // four independent accumulator chains (k-step 0/1 x hi/lo) so consecutive
+  // mma instructions do not wait on each other; summed in a fixed order
+  float c1[NN][4], c2[NN][4], c3[NN][4];
+#pragma unroll
+  for (int nt = 0; nt < NN; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c1[nt][e] = c2[nt][e] = c3[nt][e] = 0.f;
+  const uint8_t *wrow0 = pg + g * pitch + q * 16;
+  const uint8_t *wrow1 = wrow0 + 8 * pitch;
+#pragma unroll 2
   for (int grp = warp; grp < groups; grp += kComputeWarps) {
     const int c = grp * 32 + q * 8;
     const bool valid = c < nc;
     uint4 wa = make_uint4(0, 0, 0, 0), wb = make_uint4(0, 0, 0, 0);
     if (valid) {
-      wa = lds128(pg + g * pitch + c * 2);
-      wb = lds128(pg + (g + 8) * pitch + c * 2);
+      wa = *reinterpret_cast<const uint4 *>(wrow0 + grp * 64);
+      wb = *reinterpret_cast<const uint4 *>(wrow1 + grp * 64);
     }
 #pragma unroll
     for (int nt = 0; nt < NN; ++nt) {
       const int b = nt * 8 + g;
       uint4 xh = make_uint4(0, 0, 0, 0), xl = make_uint4(0, 0, 0, 0);
       if (valid && b < B) {
-        const uint32_t off = b * xpitch + (xcol0 + c) * 2;
-        xh = lds128(xhi + off);
-        xl = lds128(xlo + off);
+        const uint8_t *blk = xs + b * xpitch + (xcol0 + c) * 4;
+        xh = *reinterpret_cast<const uint4 *>(blk);
+        xl = *reinterpret_cast<const uint4 *>(blk + 16);
       }
       mma_bf16(acc[nt], wa.x, wb.x, wa.y, wb.y, xh.x, xh.y);
-      mma_bf16(acc[nt], wa.z, wb.z, wa.w, wb.w, xh.z, xh.w);
-      mma_bf16(acc[nt], wa.x, wb.x, wa.y, wb.y, xl.x, xl.y);
-      mma_bf16(acc[nt], wa.z, wb.z, wa.w, wb.w, xl.z, xl.w);
+      mma_bf16(c1[nt], wa.z, wb.z, wa.w, wb.w, xh.z, xh.w);
+      mma_bf16(c2[nt], wa.x, wb.x, wa.y, wb.y, xl.x, xl.y);
+      mma_bf16(c3[nt], wa.z, wb.z, wa.w, wb.w, xl.z, xl.w);
     }
   }
+#pragma unroll
+  for (int nt = 0; nt < NN; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] += (c1[nt][e] + c2[nt][e]) + c3[nt][e];
 }
 
-// Stage activation columns [xc0, xc0 + xlen) of every sequence as bf16 hi/lo
-// pairs.  For normed inputs (QKV, gate/up, LM head) x = h * rs[b] * gain with
-// rs computed over the full width at the first chunk of the task.
-__device__ void stage_x(const Params &p, Ctl *ctl, uint8_t *smem, const Task &t, const Geo &geo,
-                        int xc0, int xlen, int B, int ctid) {
-  const float *src;
-  const __nv_bfloat16 *gain = nullptr;
-  int stride;
+struct ComputeState {
+  int pi = 0;
+  uint32_t pg_par = 0;
+  uint32_t x_par = 0;            // phase of the activation-copy barrier
+  uint32_t xkey = 0xffffffffu;   // (layer, type) of the staged activation
+  uint32_t sat_ev = kNoEvent;    // last (event, count) known satisfied
+  uint32_t sat_cnt = 0;
+  GroupSync gs;
+};
+
+// Activation source of a GEMV task: row stride, and the RMSNorm gain for the
+// normed inputs (QKV, gate/up, LM head read the residual stream h).
+__device__ __forceinline__ void gemv_source(const Params &p, const Task &t, const float *&src,
+                                            int &stride, const __nv_bfloat16 *&gain) {
   const LayerW &lw = p.layers[t.layer < p.L ? t.layer : 0];
+  gain = nullptr;
   switch (t.type) {
     case T_QKV: src = p.h; gain = lw.attn_norm; stride = p.H; break;
     case T_GATEUP: src = p.h; gain = lw.mlp_norm; stride = p.H; break;
@@ -599,73 +723,112 @@ __device__ void stage_x(const Params &p, Ctl *ctl, uint8_t *smem, const Task &t,
     case T_OPROJ: src = p.o; stride = p.Hq * p.d; break;
     default: src = p.u; stride = p.F; break;
   }
+}
+
+// Stage activation columns [xc0, xc0 + xlen) of every sequence in shared
+// memory as fp32 rows: the leader issues one bulk copy per sequence right
+// after the input event (one L2 round trip for the whole operand).  For
+// normed inputs each sequence's sum of squares over the chunk is added to
+// ss[b] by one warp in a fixed order; the RMSNorm scale is applied to the
+// task's outputs, since W (x * g * r) = r * W (x * g).
+__device__ bool stage_x(const Params &p, Ctl *ctl, uint8_t *smem, const Task &t, int xc0,
+                        int xlen, int xpitch, int B, int ctid, ComputeState &st) {
+  const float *src;
+  int stride;
+  const __nv_bfloat16 *gain;
+  gemv_source(p, t, src, stride, gain);
+  bool okl = true;
+  if (ctid == 0) {
+    // the rows were written by other SMs (generic proxy) and acquired by this
+    // thread; order them, and this CTA's earlier reads of the area, before
+    // the bulk copy (async proxy)
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive_expect_tx(&ctl->xbar, static_cast<uint32_t>(B * xlen * 4));
+    for (int b = 0; b < B; ++b)
+      bulk_load_plain(smem + p.off_x + b * xpitch, src + static_cast<size_t>(b) * stride + xc0,
+                      static_cast<uint32_t>(xlen * 4), &ctl->xbar);
+    okl = wait_mbar(p, ctl, &ctl->xbar, st.x_par, 0xfff80000u, 2);
+    if (!okl) {
+      // leaving on an abort: let the copy land before this CTA can exit
+      const uint64_t t0 = gtimer();
+      while (!mbar_try_wait(&ctl->xbar, st.x_par)) {
+        if (gtimer() - t0 > static_cast<uint64_t>(p.wait_limit_ns) * 4) break;
+      }
+    }
+  }
+  if (!st.gs.share(ctl, ctid, okl)) return false;
+  mbar_try_wait(&ctl->xbar, st.x_par);
+  st.x_par ^= 1u;
   const int warp = ctid >> 5, lane = ctid & 31;
-  if (gain != nullptr && xc0 == 0) {
-    for (int b = 0; b < B; ++b) {
+  if (gain != nullptr) {
+    // sum of squares of the raw rows (before the gain), one warp per sequence
+    for (int b = warp; b < B; b += kComputeWarps) {
+      const float4 *row = reinterpret_cast<const float4 *>(smem + p.off_x + b * xpitch);
       float s = 0.f;
-      for (int i = ctid * 8; i < geo.K; i += kComputeThreads * 8) {
-        const float4 a = __ldcg(reinterpret_cast<const float4 *>(src + b * stride + i));
-        const float4 c = __ldcg(reinterpret_cast<const float4 *>(src + b * stride + i + 4));
-        s += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
-        s += c.x * c.x + c.y * c.y + c.z * c.z + c.w * c.w;
+      for (int i = lane; i < xlen / 4; i += 32) {
+        const float4 v = row[i];
+        s += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
       }
       s = warp_sum(s);
-      if (lane == 0) ctl->red8[warp][b] = s;
-    }
-    compute_bar();
-    if (ctid < B) {
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < kComputeWarps; ++w) s += ctl->red8[w][ctid];
-      ctl->rs[ctid] = 1.0f / sqrtf(s / static_cast<float>(geo.K) + p.eps);
+      if (lane == 0) ctl->ss[b] = (xc0 == 0 ? 0.f : ctl->ss[b]) + s;
     }
     compute_bar();
   }
-  const int xpitch = row_pitch_bytes(geo.kx);
-  const uint32_t xhi = smem_u32(smem + p.off_x);
-  const uint32_t xlo = xhi + B * xpitch;
-  for (int b = 0; b < B; ++b) {
-    const float r = gain != nullptr ? ctl->rs[b] : 1.f;
-    for (int i = ctid * 8; i < xlen; i += kComputeThreads * 8) {
-      const float *s = src + b * stride + xc0 + i;
-      const float4 a = __ldcg(reinterpret_cast<const float4 *>(s));
-      const float4 c = __ldcg(reinterpret_cast<const float4 *>(s + 4));
-      float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-      if (gain != nullptr) {
-        const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gain + xc0 + i));
-        const uint32_t gg[4] = {gw.x, gw.y, gw.z, gw.w};
+  // each thread turns whole 8-element blocks (32 bytes of fp32) into
+  // [8 x bf16 hi | 8 x bf16 lo] in place; blocks are independent
+  const int nblk = xlen / 8;
+  for (int i0 = ctid; i0 < B * nblk; i0 += 2 * kComputeThreads) {
+    float v[2][8];
+    uint4 gw[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int it = i0 + u * kComputeThreads;
+      if (it < B * nblk) {
+        const int b = it / nblk, k = it % nblk;
+        const float4 *blk = reinterpret_cast<const float4 *>(smem + p.off_x + b * xpitch + k * 32);
+        const float4 x0 = blk[0], x1 = blk[1];
+        v[u][0] = x0.x; v[u][1] = x0.y; v[u][2] = x0.z; v[u][3] = x0.w;
+        v[u][4] = x1.x; v[u][5] = x1.y; v[u][6] = x1.z; v[u][7] = x1.w;
+        if (gain != nullptr) gw[u] = __ldg(reinterpret_cast<const uint4 *>(gain + xc0 + k * 8));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int it = i0 + u * kComputeThreads;
+      if (it < B * nblk) {
+        const int b = it / nblk, k = it % nblk;
+        if (gain != nullptr) {
+          const uint32_t gg[4] = {gw[u].x, gw[u].y, gw[u].z, gw[u].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            v[u][2 * e] *= bf_lo(gg[e]);
+            v[u][2 * e + 1] *= bf_hi(gg[e]);
+          }
+        }
+        uint32_t hw[4], lw4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          v[2 * e] = v[2 * e] * r * bf_lo(gg[e]);
-          v[2 * e + 1] = v[2 * e + 1] * r * bf_hi(gg[e]);
+          __nv_bfloat16 h0, l0, h1, l1;
+          split_bf16(v[u][2 * e], h0, l0);
+          split_bf16(v[u][2 * e + 1], h1, l1);
+          hw[e] = pack2(h0, h1);
+          lw4[e] = pack2(l0, l1);
         }
+        uint4 *blk = reinterpret_cast<uint4 *>(smem + p.off_x + b * xpitch + k * 32);
+        blk[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        blk[1] = make_uint4(lw4[0], lw4[1], lw4[2], lw4[3]);
       }
-      uint32_t hw[4], lw4[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        __nv_bfloat16 h0, l0, h1, l1;
-        split_bf16(v[2 * e], h0, l0);
-        split_bf16(v[2 * e + 1], h1, l1);
-        hw[e] = pack2(h0, h1);
-        lw4[e] = pack2(l0, l1);
-      }
-      sts128(xhi + b * xpitch + i * 2, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-      sts128(xlo + b * xpitch + i * 2, make_uint4(lw4[0], lw4[1], lw4[2], lw4[3]));
     }
   }
   compute_bar();
+  return true;
 }
 
-struct ComputeState {
-  int pi = 0;
-  uint32_t pg_par = 0;
-  uint32_t xkey = 0xffffffffu;   // (layer, type) of the staged activation
-  uint32_t sat_ev = kNoEvent;    // last (event, count) known satisfied
-  uint32_t sat_cnt = 0;
-  GroupSync gs;
-};
-
-template <int NN>
+// NN = batch n-tiles (1: B <= 8, 2: B <= 16).  With two n-tiles a task holds
+// at most kMaxMTiles/2 row tiles (the plan caps rows per task) so that the
+// accumulators stay in registers.
+template <int NN, int MT = (NN == 1 ? kMaxMTiles : kMaxMTiles / 2)>
 __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
                           ComputeState &st, float *out, int ctid) {
   const Task &t = S.t;
@@ -673,11 +836,14 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   const int warp = ctid >> 5, lane = ctid & 31;
   const Geo geo = gemv_geo(p, t, B);
   const int pitch = row_pitch_bytes(geo.kp);
-  const int xpitch = row_pitch_bytes(geo.kx);
-  const uint32_t pages = smem_u32(smem + p.off_pages);
-  const uint32_t xhi = smem_u32(smem + p.off_x);
-  const uint32_t xlo = xhi + B * xpitch;
+  const int xstride = x_row_bytes(geo.kx) / 4;
+  const uint8_t *pages = smem + p.off_pages;
+  const uint8_t *xs = smem + p.off_x;
   const uint32_t key = (static_cast<uint32_t>(t.layer) << 8) | t.type;
+  const float *src;
+  int stride;
+  const __nv_bfloat16 *gain;
+  gemv_source(p, t, src, stride, gain);
 
   if (t.dep_event != st.sat_ev || t.dep_count != st.sat_cnt) {
     bool okl = true;
@@ -688,9 +854,9 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   }
   if (ctid == 0) trace_mark(p, S.idx, 4);
 
-  float acc[kMaxMTiles][NN][4];
+  float acc[MT][NN][4];
 #pragma unroll
-  for (int m = 0; m < kMaxMTiles; ++m)
+  for (int m = 0; m < MT; ++m)
 #pragma unroll
     for (int n = 0; n < NN; ++n)
 #pragma unroll
@@ -699,7 +865,7 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   for (int xc0 = 0; xc0 < geo.K; xc0 += geo.kx) {
     const int xend = min(geo.K, xc0 + geo.kx);
     if (!(geo.whole && st.xkey == key)) {
-      stage_x(p, ctl, smem, t, geo, xc0, xend - xc0, B, ctid);
+      if (!stage_x(p, ctl, smem, t, xc0, xend - xc0, xstride * 4, B, ctid, st)) return false;
       st.xkey = geo.whole ? key : 0xffffffffu;
     }
     if (ctid == 0 && xc0 == 0) trace_mark(p, S.idx, 5);
@@ -710,11 +876,13 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
         if (ctid == 0) okl = wait_mbar(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff30000u, 2);
         if (!st.gs.share(ctl, ctid, okl)) return false;
         mbar_try_wait(&ctl->full[st.pi], st.pg_par);  // completed: acquire for this thread
-        const uint32_t pg = pages + st.pi * p.page_bytes;
+        const uint8_t *pg = pages + static_cast<size_t>(st.pi) * p.page_bytes;
         switch (m) {
-#define MK_PAGE_CASE(M)                                                                    \
-  case M:                                                                                  \
-    page_mma<NN>(acc[M], pg, pitch, nc, xhi, xlo, xpitch, c0 - xc0, B, warp, lane); \
+#define MK_PAGE_CASE(M)                                                                      \
+  case M:                                                                                    \
+    if (M < MT)                                                                              \
+      page_mma<NN>(acc[M < MT ? M : 0], pg, pitch, nc, xs, xstride * 4, c0 - xc0, B, warp, \
+                   lane);                                                                    \
     break;
           MK_PAGE_CASE(0)
           MK_PAGE_CASE(1)
@@ -737,12 +905,16 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     }
   }
 
+  if (gain != nullptr) {
+    if (ctid < B) ctl->rs[ctid] = 1.0f / sqrtf(ctl->ss[ctid] / static_cast<float>(geo.K) + p.eps);
+    compute_bar();
+  }
   // cross-warp reduction, one 16-row tile at a time, fixed warp order
   float *red = reinterpret_cast<float *>(smem + p.off_red);
   constexpr int NC = NN * 8;
   const int g = lane >> 2, q = lane & 3;
 #pragma unroll
-  for (int m = 0; m < kMaxMTiles; ++m) {
+  for (int m = 0; m < MT; ++m) {
     if (m >= t.n_m) break;
 #pragma unroll
     for (int nt = 0; nt < NN; ++nt) {
@@ -754,12 +926,12 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
       r1[1] = acc[m][nt][3];
     }
     compute_bar();
-    if (ctid < 16 * NC) {
-      const int row = ctid / NC, n = ctid % NC;
+    for (int e = ctid; e < 16 * NC; e += kComputeThreads) {
+      const int row = e / NC, n = e % NC;
       float s = 0.f;
 #pragma unroll
       for (int w = 0; w < kComputeWarps; ++w) s += red[(w * 16 + row) * NC + n];
-      if (n < B) out[n * (16 * kMaxMTiles) + m * 16 + row] = s;
+      if (n < B) out[n * (16 * kMaxMTiles) + m * 16 + row] = gain != nullptr ? s * ctl->rs[n] : s;
     }
     compute_bar();
   }
@@ -818,7 +990,6 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     if (ctid == 0) okl = wait_mbar(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff40000u, 2);
     if (!st.gs.share(ctl, ctid, okl)) return false;
     mbar_try_wait(&ctl->full[st.pi], st.pg_par);
-    uint8_t *pg = smem + p.off_pages + static_cast<size_t>(st.pi) * p.page_bytes;
     const uint32_t kbase = pages + st.pi * p.page_bytes;
     const uint32_t vbase = kbase + p.tpp * d * 2;
     // The current token's K/V were appended by this step's QKV epilogue and
@@ -838,30 +1009,101 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
       }
       compute_bar();
     }
-    for (int j = warp; j < ntok; j += kComputeWarps) {
-      float kf[DL], vf[DL];
-      const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(pg) + j * d + lane * DL;
-      const __nv_bfloat16 *vr =
-          reinterpret_cast<const __nv_bfloat16 *>(pg + static_cast<size_t>(p.tpp) * d * 2) + j * d +
-          lane * DL;
+    // Each warp takes 4 tokens at a time (tokens 4w..4w+3, then +32): the
+    // 4*G dot products reduce over the warp as independent shuffle chains,
+    // then one online-softmax update per head covers the 4 tokens.
+    constexpr int TB = 2;
+    for (int j0 = warp * TB; j0 < ntok; j0 += kComputeWarps * TB) {
+      float kf[TB][DL], vf[TB][DL];
 #pragma unroll
-      for (int i = 0; i < DL; ++i) {
-        kf[i] = __bfloat162float(kr[i]);
-        vf[i] = __bfloat162float(vr[i]);
+      for (int u = 0; u < TB; ++u) {
+        const int j = j0 + u;
+        const bool in = j < ntok;
+        const uint32_t ko = kbase + (j * d + lane * DL) * 2;
+        const uint32_t vo = vbase + (j * d + lane * DL) * 2;
+        uint32_t kw[DL > 1 ? DL / 2 : 1], vw[DL > 1 ? DL / 2 : 1];
+        if (DL == 1) {
+          // one bf16 per lane (d = 32)
+          uint16_t kh = 0, vh = 0;
+          if (in) {
+            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(kh) : "r"(ko));
+            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(vh) : "r"(vo));
+          }
+          kf[u][0] = __uint_as_float(static_cast<uint32_t>(kh) << 16);
+          vf[u][0] = __uint_as_float(static_cast<uint32_t>(vh) << 16);
+        } else {
+#pragma unroll
+          for (int i = 0; i < DL / 2; ++i) {
+            kw[i] = 0u;
+            vw[i] = 0u;
+          }
+          if (in) {
+            if (DL == 2) {
+              asm volatile("ld.shared.b32 %0, [%1];" : "=r"(kw[0]) : "r"(ko));
+              asm volatile("ld.shared.b32 %0, [%1];" : "=r"(vw[0]) : "r"(vo));
+            } else if (DL == 4) {
+              asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(kw[0]), "=r"(kw[1]) : "r"(ko));
+              asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(vw[0]), "=r"(vw[1]) : "r"(vo));
+            } else {
+#pragma unroll
+              for (int i = 0; i < DL / 8; ++i) {
+                const uint4 a = lds128(ko + i * 16), c = lds128(vo + i * 16);
+                kw[4 * i] = a.x; kw[4 * i + 1] = a.y; kw[4 * i + 2] = a.z; kw[4 * i + 3] = a.w;
+                vw[4 * i] = c.x; vw[4 * i + 1] = c.y; vw[4 * i + 2] = c.z; vw[4 * i + 3] = c.w;
+              }
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < DL / 2; ++i) {
+            kf[u][2 * i] = bf_lo(kw[i]);
+            kf[u][2 * i + 1] = bf_hi(kw[i]);
+            vf[u][2 * i] = bf_lo(vw[i]);
+            vf[u][2 * i + 1] = bf_hi(vw[i]);
+          }
+        }
       }
+      float sc[kMaxGroup][TB];
+#pragma unroll
+      for (int h = 0; h < kMaxGroup; ++h)
+#pragma unroll
+        for (int u = 0; u < TB; ++u) {
+          float s = 0.f;
+#pragma unroll
+          for (int i = 0; i < DL; ++i) s += qv[h][i] * kf[u][i];
+          sc[h][u] = s;
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+#pragma unroll
+          for (int u = 0; u < TB; ++u)
+            if (h < G) sc[h][u] += __shfl_xor_sync(0xffffffffu, sc[h][u], o);
 #pragma unroll
       for (int h = 0; h < kMaxGroup; ++h) {
         if (h >= G) break;
-        float s = 0.f;
+        float mn = mrun[h];
 #pragma unroll
-        for (int i = 0; i < DL; ++i) s += qv[h][i] * kf[i];
-        s = warp_sum(s);
-        const float mn = fmaxf(mrun[h], s);
+        for (int u = 0; u < TB; ++u) {
+          if (j0 + u >= ntok) sc[h][u] = -INFINITY;
+          mn = fmaxf(mn, sc[h][u]);
+        }
         const float corr = exp2f(mrun[h] - mn);
-        const float pr = exp2f(s - mn);
-        lrun[h] = lrun[h] * corr + pr;
+        float pr[TB];
+        float lsum = 0.f;
 #pragma unroll
-        for (int i = 0; i < DL; ++i) acc[h][i] = acc[h][i] * corr + pr * vf[i];
+        for (int u = 0; u < TB; ++u) {
+          pr[u] = exp2f(sc[h][u] - mn);
+          lsum += pr[u];
+        }
+        lrun[h] = lrun[h] * corr + lsum;
+#pragma unroll
+        for (int i = 0; i < DL; ++i) {
+          float a = acc[h][i] * corr;
+#pragma unroll
+          for (int u = 0; u < TB; ++u) a += pr[u] * vf[u][i];
+          acc[h][i] = a;
+        }
         mrun[h] = mn;
       }
     }
@@ -874,8 +1116,9 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     }
   }
 
-  // merge the 8 warps' running (max, sum, acc) in fixed order
-  const int rw = d + 2;
+  // merge the warps' running (max, sum, acc) in fixed order; the chunk's
+  // partial goes straight to global memory: row h = (acc[0..d), m, l, pad)
+  const int rw = d + 4;
 #pragma unroll
   for (int h = 0; h < kMaxGroup; ++h) {
     if (h >= G) break;
@@ -888,6 +1131,7 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     }
   }
   compute_bar();
+  float *part = p.attn_part + static_cast<size_t>(t.aux) * G * rw;
   for (int e = ctid; e < G * rw; e += kComputeThreads) {
     const int h = e / rw, i = e % rw;
     float M = -INFINITY;
@@ -902,16 +1146,77 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
       }
     } else if (i == d) {
       s = M;
-    } else {
+    } else if (i == d + 1) {
 #pragma unroll
       for (int w = 0; w < kComputeWarps; ++w) {
         const float mw = wsc[(w * G + h) * rw + d];
         if (mw != -INFINITY) s += exp2f(mw - M) * wsc[(w * G + h) * rw + d + 1];
       }
     }
-    out[e] = s;
+    __stcg(part + e, s);
   }
   compute_bar();
+
+  // The chunk that completes (b, g) merges all of its chunks by log-sum-exp
+  // and writes o for the G query heads.  The bar above orders every thread's
+  // partial before thread 0's release; thread 0's acquire orders the other
+  // chunks' partials before the reads below.
+  uint32_t *ctr = p.comb_ctr + b * p.Hkv + g;
+  bool last_l = false;
+  if (ctid == 0) last_l = atom_add_acq_rel(ctr, 1u) + 1u == static_cast<uint32_t>(S.n_chunks);
+  if (!st.gs.share(ctl, ctid, last_l)) return true;
+  const int nch = S.n_chunks;
+  float *ms = wsc;                     // [nch][G] chunk maxima, then weights
+  float *ls = wsc + nch * G;           // [nch][G] chunk sums
+  float *MD = ls + nch * G;            // [G] max, [G] 1/denominator
+  for (int e = ctid; e < nch * G; e += kComputeThreads) {
+    const int c = e / G, h = e % G;
+    const float *pc = p.attn_part + (static_cast<size_t>(S.first_slot + c) * G + h) * rw;
+    ms[e] = __ldcg(pc + d);
+    ls[e] = __ldcg(pc + d + 1);
+  }
+  compute_bar();
+  if (ctid < G) {
+    float M = -INFINITY;
+    for (int c = 0; c < nch; ++c) M = fmaxf(M, ms[c * G + ctid]);
+    float den = 0.f;
+    for (int c = 0; c < nch; ++c) den += exp2f(ms[c * G + ctid] - M) * ls[c * G + ctid];
+    MD[ctid] = M;
+    MD[G + ctid] = 1.0f / den;
+  }
+  compute_bar();
+  for (int e = ctid; e < nch * G; e += kComputeThreads) ms[e] = exp2f(ms[e] - MD[e % G]);
+  compute_bar();
+  const int q4 = d / 4;
+  for (int e = ctid; e < G * q4; e += kComputeThreads) {
+    const int h = e / q4, i = (e % q4) * 4;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    int c = 0;
+    for (; c + 4 <= nch; c += 4) {
+      float4 a[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        a[u] = __ldcg(reinterpret_cast<const float4 *>(
+            p.attn_part + (static_cast<size_t>(S.first_slot + c + u) * G + h) * rw + i));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float wgt = ms[(c + u) * G + h];
+        num.x += wgt * a[u].x; num.y += wgt * a[u].y; num.z += wgt * a[u].z; num.w += wgt * a[u].w;
+      }
+    }
+    for (; c < nch; ++c) {
+      const float4 a = __ldcg(reinterpret_cast<const float4 *>(
+          p.attn_part + (static_cast<size_t>(S.first_slot + c) * G + h) * rw + i));
+      const float wgt = ms[c * G + h];
+      num.x += wgt * a.x; num.y += wgt * a.y; num.z += wgt * a.z; num.w += wgt * a.w;
+    }
+    const float r = MD[G + h];
+    __stcg(reinterpret_cast<float4 *>(p.o + static_cast<size_t>(b) * p.Hq * d + (g * G + h) * d + i),
+           make_float4(num.x * r, num.y * r, num.z * r, num.w * r));
+  }
+  compute_bar();
+  if (ctid == 0) *ctr = 0u;   // rearm for the next layer / step
+  (void)out;
   return true;
 }
 
@@ -981,7 +1286,7 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
             case 1: tok = attn_task<1>(p, ctl, smem, S, st, out, ctid); break;
             case 2: tok = attn_task<2>(p, ctl, smem, S, st, out, ctid); break;
             case 4: tok = attn_task<4>(p, ctl, smem, S, st, out, ctid); break;
-            default: tok = attn_task<8>(p, ctl, smem, S, st, out, ctid); break;
+            default: tok = attn_task<4>(p, ctl, smem, S, st, out, ctid); break;
           }
         }
         break;
@@ -1021,6 +1326,9 @@ __device__ __forceinline__ void signal(const Params &p, uint32_t ev) {
 }
 
 // QK-norm + RoPE of one head for every sequence, then K/V append or q store.
+// Lane l holds elements 4l..4l+3 of the head (d/4 active lanes); the RoPE
+// partner of element i (i + d/2) sits d/8 lanes away, fetched by shuffle.
+// All loads of a sequence are issued before any is used.
 __device__ void rope_head(const Params &p, const Task &t, int lane) {
   const int d = p.d, half = d / 2, l = t.layer, B = p.batch;
   const int mat = static_cast<int>(t.aux);
@@ -1028,71 +1336,63 @@ __device__ void rope_head(const Params &p, const Task &t, int lane) {
   const int local = mat == 0 ? head : (mat == 1 ? head - p.Hq : head - p.Hq - p.Hkv);
   const int col0 = head * d;  // rows of q, then k, then v are contiguous in qkv
   const LayerW &lw = p.layers[l];
+  const bool active = lane < d / 4;
+  const int e0 = lane * 4;                         // first element held
+  const bool first_half = e0 < half;
+  const int pair0 = first_half ? e0 : e0 - half;   // RoPE pair index
+  const int xo = d / 8;                            // lane distance to the partner
+  const __nv_bfloat16 *gain = mat == 0 ? lw.q_norm : lw.k_norm;
   for (int b = 0; b < B; ++b) {
-    const float *y = p.qkv + static_cast<size_t>(b) * p.NQKV + col0;
     const int pos = p.pos[b];
     if (pos < 0 || pos >= p.max_pos) continue;  // reported by the embedding task
-    float rs = 1.f;
-    if (mat != 2 && p.qk_norm) {
-      float s = 0.f;
-      for (int i = lane; i < d; i += 32) {
-        const float v = __ldcg(y + i);
-        s += v * v;
-      }
-      s = warp_sum(s);
-      rs = 1.0f / sqrtf(s / static_cast<float>(d) + p.eps);
-    }
-    const __nv_bfloat16 *gain = mat == 0 ? lw.q_norm : lw.k_norm;
-    __nv_bfloat16 *dst = nullptr;
-    if (mat != 0) {
-      const int ph = kv_phys_page(p, b, pos / p.page_size);
-      if (ph < 0) continue;
-      dst = (mat == 1 ? p.k_pages[l] : p.v_pages[l]) +
-            ((static_cast<size_t>(ph) * p.Hkv + local) * p.page_size + pos % p.page_size) * d;
-    }
-    for (int i = lane; i < half; i += 32) {
-      float a = __ldcg(y + i), c = __ldcg(y + i + half);
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+    float g4[4] = {1.f, 1.f, 1.f, 1.f};
+    float2 cs[4];
+    if (active) {
+      y = __ldcg(reinterpret_cast<const float4 *>(p.qkv + static_cast<size_t>(b) * p.NQKV + col0 + e0));
       if (mat != 2) {
         if (p.qk_norm) {
-          a = a * rs * __bfloat162float(gain[i]);
-          c = c * rs * __bfloat162float(gain[i + half]);
+          const uint2 gw = *reinterpret_cast<const uint2 *>(gain + e0);
+          g4[0] = bf_lo(gw.x); g4[1] = bf_hi(gw.x); g4[2] = bf_lo(gw.y); g4[3] = bf_hi(gw.y);
         }
-        const float2 cs = p.rope_cs[static_cast<size_t>(pos) * half + i];
-        const float ra = a * cs.x - c * cs.y;
-        const float rc = c * cs.x + a * cs.y;
-        a = ra;
-        c = rc;
-      }
-      if (mat == 0) {
-        float *q = p.qrot + (static_cast<size_t>(b) * p.Hq + local) * d;
-        __stcg(q + i, a);
-        __stcg(q + i + half, c);
-      } else {
-        dst[i] = __float2bfloat16_rn(a);
-        dst[i + half] = __float2bfloat16_rn(c);
+        const float2 *tab = p.rope_cs + static_cast<size_t>(pos) * half + pair0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) cs[k] = tab[k];
       }
     }
-  }
-}
-
-// Merge the chunks of (b, g) by log-sum-exp and write o for its G heads.
-__device__ void attn_combine(const Params &p, const Slot &S, int lane) {
-  const int d = p.d, G = p.G, rw = d + 2;
-  for (int e = lane; e < G * d; e += 32) {
-    const int h = e / d, i = e % d;
-    float M = -INFINITY;
-    for (int c = 0; c < S.n_chunks; ++c) {
-      const float *pc = p.attn_part + (static_cast<size_t>(S.first_slot + c) * G + h) * rw;
-      M = fmaxf(M, __ldcg(pc + d));
+    float v[4] = {y.x, y.y, y.z, y.w};
+    if (mat != 2) {
+      float rs = 1.f;
+      if (p.qk_norm) {
+        float s = v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
+        s = warp_sum(s);
+        rs = 1.0f / sqrtf(s / static_cast<float>(d) + p.eps);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[k] = v[k] * rs * g4[k];
+      }
+      float w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) w[k] = __shfl_xor_sync(0xffffffffu, v[k], xo);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        // first half: (a, c) = (v, w) -> a cos - c sin; second half: c cos + a sin
+        v[k] = first_half ? v[k] * cs[k].x - w[k] * cs[k].y : v[k] * cs[k].x + w[k] * cs[k].y;
+      }
     }
-    float num = 0.f, den = 0.f;
-    for (int c = 0; c < S.n_chunks; ++c) {
-      const float *pc = p.attn_part + (static_cast<size_t>(S.first_slot + c) * G + h) * rw;
-      const float w = exp2f(__ldcg(pc + d) - M);
-      num += w * __ldcg(pc + i);
-      den += w * __ldcg(pc + d + 1);
+    if (!active) continue;
+    if (mat == 0) {
+      float *q = p.qrot + (static_cast<size_t>(b) * p.Hq + local) * d + e0;
+      __stcg(reinterpret_cast<float4 *>(q), make_float4(v[0], v[1], v[2], v[3]));
+    } else {
+      const int ph = kv_phys_page(p, b, pos / p.page_size);
+      if (ph < 0) continue;
+      __nv_bfloat16 *dst = (mat == 1 ? p.k_pages[l] : p.v_pages[l]) +
+                           ((static_cast<size_t>(ph) * p.Hkv + local) * p.page_size +
+                            pos % p.page_size) * d + e0;
+      const uint2 pk = make_uint2(pack2(__float2bfloat16_rn(v[0]), __float2bfloat16_rn(v[1])),
+                                  pack2(__float2bfloat16_rn(v[2]), __float2bfloat16_rn(v[3])));
+      *reinterpret_cast<uint2 *>(dst) = pk;
     }
-    __stcg(p.o + static_cast<size_t>(S.b) * p.Hq * d + (S.g * G + h) * d + i, num / den);
   }
 }
 
@@ -1102,6 +1402,10 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
   return (static_cast<unsigned long long>(u) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(idx));
 }
 
+// Ordering: every lane's global writes are followed by __syncwarp(), after
+// which lane 0's release (red.release / atom.acq_rel) publishes them; a last
+// arriver's acquire (atom.acq_rel) is followed by __syncwarp() before any lane
+// reads what the other arrivers published.  No full fences are needed.
 __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const float *out,
                                 int lane) {
   const Task &t = S.t;
@@ -1118,7 +1422,6 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
       for (int b = 0; b < B; ++b)
         for (int r = lane; r < static_cast<int>(t.nrows); r += 32)
           __stcg(p.qkv + static_cast<size_t>(b) * p.NQKV + base + t.row0 + r, out[b * OS + r]);
-      __threadfence();
       __syncwarp();
       const int head = static_cast<int>(t.aux2 & 0xffffu);
       const uint32_t need = t.aux2 >> 16;
@@ -1126,9 +1429,8 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
       if (lane == 0) old = atom_add_acq_rel(p.head_ctr + t.layer * (p.Hq + 2 * p.Hkv) + head, 1u);
       old = __shfl_sync(0xffffffffu, old, 0);
       if (old + 1u == need) {
-        fence_acq_rel();
+        __syncwarp();
         rope_head(p, t, lane);
-        __threadfence();
         __syncwarp();
         if (lane == 0) {
           p.head_ctr[t.layer * (p.Hq + 2 * p.Hkv) + head] = 0u;
@@ -1139,25 +1441,8 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
       break;
     }
     case T_ATTN: {
-      if (S.b >= 0) {
-        const int n = p.G * (p.d + 2);
-        float *dst = p.attn_part + static_cast<size_t>(t.aux) * n;
-        for (int e = lane; e < n; e += 32) __stcg(dst + e, out[e]);
-        __threadfence();
-        __syncwarp();
-        uint32_t old = 0;
-        uint32_t *ctr = p.comb_ctr + S.b * p.Hkv + S.g;
-        if (lane == 0) old = atom_add_acq_rel(ctr, 1u);
-        old = __shfl_sync(0xffffffffu, old, 0);
-        if (old + 1u == static_cast<uint32_t>(S.n_chunks)) {
-          fence_acq_rel();
-          attn_combine(p, S, lane);
-          __threadfence();
-          __syncwarp();
-          if (lane == 0) *ctr = 0u;
-        }
-      }
-      __syncwarp();
+      // the compute warps wrote the chunk partial (and, for the chunk that
+      // completed its (sequence, KV head), the merged o) before handing over
       if (lane == 0) signal(p, t.out_event);
       break;
     }
@@ -1171,7 +1456,6 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
           if (t.type == T_DOWN && p.hidden_dump != nullptr)
             p.hidden_dump[(static_cast<size_t>(t.layer) * B + b) * p.H + t.row0 + r] = v;
         }
-      __threadfence();
       __syncwarp();
       if (lane == 0) signal(p, t.out_event);
       break;
@@ -1184,7 +1468,6 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
           const float up = out[b * OS + nh16 + r];
           __stcg(p.u + static_cast<size_t>(b) * p.F + t.row0 + r, gt / (1.0f + __expf(-gt)) * up);
         }
-      __threadfence();
       __syncwarp();
       if (lane == 0) signal(p, t.out_event);
       break;
@@ -1213,13 +1496,12 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
         }
         if (lane == 0) atomicMax(p.argmax + b, argmax_key(best, bi));
       }
-      __threadfence();
       __syncwarp();
       uint32_t old = 0;
       if (lane == 0) old = atom_add_acq_rel(p.sync + S_LMCTR, 1u);
       old = __shfl_sync(0xffffffffu, old, 0);
       if (old + 1u == static_cast<uint32_t>(p.n_lm_tasks)) {
-        fence_acq_rel();
+        __syncwarp();
         if (lane < B) {
           const unsigned long long k = ld_relaxed_u64(p.argmax + lane);
           p.out_ids[lane] = static_cast<int32_t>(~static_cast<uint32_t>(k & 0xffffffffull));
@@ -1292,6 +1574,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       mbar_init(&ctl->out_full[i], 1);
       mbar_init(&ctl->out_empty[i], 1);
     }
+    mbar_init(&ctl->xbar, 1);
     ctl->cta_abort = 0;
     ctl->flag[0] = ctl->flag[1] = 0;
     // a device error from an earlier step is sticky until the host resets

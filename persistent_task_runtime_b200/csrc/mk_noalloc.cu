@@ -67,7 +67,7 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
   const int F = c.ffn, V = c.vocab, P = kv_page_size, B = a->batch;
   if (L < 1 || L > MK_MAX_LAYERS || H <= 0 || Hq <= 0 || Hkv <= 0 || F <= 0 || V <= 0 ||
       c.max_seq_len <= 0 || Hq % Hkv || Hq / Hkv > mk::kMaxGroup ||
-      (d != 32 && d != 64 && d != 128 && d != 256) || H % 8 || F % 8 || (Hq * d) % 8)
+      (d != 32 && d != 64 && d != 128) || H % 8 || F % 8 || (Hq * d) % 8)
     return nfail(MK_ERR_UNSUPPORTED, "model shape not supported (see mk_model_config)");
   if (P < 16 || P % 16) return nfail(MK_ERR_INVALID_ARG, "kv_page_size must be a multiple of 16");
   if (B < 1 || B > MK_MAX_BATCH) return nfail(MK_ERR_INVALID_ARG, "batch outside 1..16");
@@ -102,7 +102,11 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
 
   // ---- shared-memory carve-up (same rules as a plan built for max_batch = B)
   const int Kmax = std::max(H, std::max(Hq * d, F));
-  const int att_need = G * d * 4 + mk::kComputeWarps * G * (d + 2) * 4;
+  // attention scratch in the staging area: q [G][d] plus either the warps'
+  // running states [warps][G][d+4] or the combine's per-chunk (m, l) pairs
+  const int max_chunks = (c.max_seq_len + P - 1) / P;
+  const int att_need = G * d * 4 + std::max(mk::kComputeWarps * G * (d + 4),
+                                            2 * max_chunks * G + 2 * G) * 4;
   const int chunk_need = 2 * maxB * mk::row_pitch_bytes(std::min(1024, align_up_i(Kmax, 32)));
   int x_cap = std::min(std::max(2 * mk::row_pitch_bytes(Kmax), chunk_need), 64 * 1024);
   x_cap = std::max(x_cap, att_need);
@@ -127,10 +131,11 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
   }
   tpp = std::min(tpp, 16 * P);
   const int smem_max = std::min(smem_optin, mk::kMaxSmem);
-  const int off_slots = 1024;
+  const int off_look = 1024;   // loader lookahead (8 x 48 B)
+  const int off_slots = off_look + 512;
   const int off_red = align_up_i(off_slots + mk::kTaskSlots * 64, 128);
   const int off_out = align_up_i(off_red + mk::kComputeWarps * 16 * (maxB > 8 ? 16 : 8) * 4, 128);
-  const int out_bytes = align_up_i(std::max(maxB * 16 * mk::kMaxMTiles * 4, G * (d + 2) * 4), 128);
+  const int out_bytes = align_up_i(maxB * 16 * mk::kMaxMTiles * 4, 128);
   const int off_x = align_up_i(off_out + mk::kOutSlots * out_bytes, 128);
   const int off_pages = align_up_i(off_x + x_cap, 128);
   const int n_pages = std::min(mk::kMaxPages, (smem_max - off_pages) / page_bytes);
@@ -149,6 +154,7 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
   p.x_cap = x_cap;
   p.page_bytes = page_bytes;
   p.n_pages = n_pages;
+  p.off_look = off_look;
   p.off_slots = off_slots;
   p.off_red = off_red;
   p.off_out = off_out;
@@ -158,6 +164,7 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
   p.attn_target = grid;
   p.attn_slots = grid + maxB * Hkv;
   p.wait_limit_ns = 2000000000LL;
+  p.pf_bytes = 0u;
   p.ev_embed = 0;
   p.ev_layer0 = 1;
   p.ev_per_layer = Hkv + 4;
@@ -272,7 +279,7 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
   const size_t o_h = carve(sizeof(float) * maxB * H);
   const size_t o_qkv = carve(sizeof(float) * maxB * NQKV);
   const size_t o_qrot = carve(sizeof(float) * maxB * Hq * d);
-  const size_t o_part = carve(sizeof(float) * static_cast<size_t>(p.attn_slots) * G * (d + 2));
+  const size_t o_part = carve(sizeof(float) * static_cast<size_t>(p.attn_slots) * G * (d + 4));
   const size_t o_o = carve(sizeof(float) * maxB * Hq * d);
   const size_t o_u = carve(sizeof(float) * maxB * F);
   const size_t o_arg = carve(sizeof(unsigned long long) * maxB);
