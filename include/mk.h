@@ -132,6 +132,11 @@ typedef struct {
   int l2_prefetch_kb;     /* per-CTA budget of upcoming weights requested
                              into L2 ahead of the shared-memory ring, in
                              KB; 0 = off (the default)                      */
+  int prefetch_distance;  /* when task t is dispatched, the operands of task
+                             t + prefetch_distance (queue order) are
+                             requested into L2; 0 = off, negative = off    */
+  int prefetch_task_kb;   /* cap on what one such request covers, in KB
+                             (0 = 256)                                      */
 } mk_plan_options;
 
 typedef struct mk_plan mk_plan;

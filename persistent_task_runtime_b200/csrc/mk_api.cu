@@ -76,8 +76,10 @@ struct mk_plan {
 
 namespace {
 
+// Rows per task: small enough that every CTA gets ~16 tasks of an operator,
+// so the dynamic queue evens out the operator's tail across SMs.
 int choose_mtiles(int tiles, int nsm, int cap) {
-  int nm = tiles / (2 * nsm);
+  int nm = tiles / (16 * nsm);
   return std::max(1, std::min(cap, nm));
 }
 
@@ -178,10 +180,12 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
 
   // ---- shared-memory carve-up ------------------------------------------------
   const int Kmax = std::max(H, std::max(Hq * d, F));
-  // attention scratch in the staging area: q [G][d] plus either the warps'
-  // running states [warps][G][d+4] or the combine's per-chunk (m, l) pairs
+  // attention scratch in the staging area: q [G][d] plus either the page's
+  // scores [G][tokens per page] and per-head statistics, or the combine's
+  // per-chunk (m, l) pairs
   const int max_chunks = (c.max_seq_len + P - 1) / P;
-  const int att_need = G * d * 4 + std::max(mk::kComputeWarps * G * (d + 4),
+  const int tpp_bound = std::min(16 * P, 16 * mk::row_pitch_bytes(1024) / (4 * d));
+  const int att_need = G * d * 4 + std::max(G * tpp_bound + 3 * mk::kMaxGroup,
                                             2 * max_chunks * G + 2 * G) * 4;
   // activation staging: the whole widest input of one sequence, or a
   // 1024-column chunk of every sequence, whichever is larger (<= 64 KB)
@@ -255,6 +259,8 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   p.attn_slots = grid + maxB * Hkv;
   p.wait_limit_ns = o.wait_limit_ns;
   p.pf_bytes = o.l2_prefetch_kb > 0 ? 1024u * static_cast<uint32_t>(o.l2_prefetch_kb) : 0u;
+  p.pf_distance = o.prefetch_distance > 0 ? o.prefetch_distance : 0;
+  p.pf_task_bytes = 1024u * static_cast<uint32_t>(o.prefetch_task_kb > 0 ? o.prefetch_task_kb : 256);
   p.ev_embed = 0;
   p.ev_layer0 = 1;
   p.ev_per_layer = Hkv + 4;

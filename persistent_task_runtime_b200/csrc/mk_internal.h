@@ -100,6 +100,8 @@ struct Params {
   int page_bytes, n_pages;
   int off_look, off_slots, off_red, off_out, out_bytes, off_x, off_pages;  // smem carve-up
   uint32_t pf_bytes;                  // L2 prefetch budget per CTA (0 = off)
+  int pf_distance;                    // dispatching task t prefetches task t + this (0 = off)
+  uint32_t pf_task_bytes;             // cap on the bytes prefetched for one task
   int n_tasks;
   int ev_embed, ev_layer0, ev_per_layer;   // event numbering
   int n_lm_tasks;

@@ -551,6 +551,36 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       ts_par ^= 1u;
     }
 
+    // ---- warm L2 for the task pf_distance places later in the queue ----
+    // Nothing is reserved: whichever CTA later pops that task finds its
+    // operands in L2, and HBM keeps streaming while this CTA's compute warps
+    // wait at an operator boundary.
+    if (p.pf_distance > 0) {
+      const int fut = tix + p.pf_distance;
+      if (fut < p.task_end) {
+        const Task ft = p.tasks[fut];
+        if (is_gemv(ft.type)) {
+          l2_prefetch_task(p, ft, p.pf_task_bytes, lane);
+        } else if (ft.type == T_ATTN) {
+          Slot fi;
+          fi.b = -1;
+          attn_resolve(p, B, static_cast<int>(ft.aux), fi);
+          if (fi.b >= 0) {
+            const int P = p.page_size;
+            const size_t kvpage_elems = static_cast<size_t>(P) * p.d;
+            const int npg = (fi.t1 - fi.t0 + P - 1) / P;
+            for (int j = lane; j < 2 * npg; j += 32) {
+              const int ph = kv_phys_page(p, fi.b, fi.t0 / P + (j >> 1));
+              if (ph < 0) continue;
+              const __nv_bfloat16 *base = (j & 1) ? p.v_pages[ft.layer] : p.k_pages[ft.layer];
+              prefetch_l2(base + (static_cast<size_t>(ph) * p.Hkv + fi.g) * kvpage_elems,
+                          static_cast<uint32_t>(kvpage_elems * 2));
+            }
+          }
+        }
+      }
+    }
+
     // ---- stream the task's operands into the page ring ----
     if (is_gemv(t.type)) {
       const Geo geo = gemv_geo(p, t, B);
@@ -942,16 +972,31 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
 // compute warps: attention over one chunk of one (sequence, KV head)
 // ============================================================================
 
-template <int DL>
+// Attention for one chunk of one (sequence, KV head): scores for the G query
+// heads over the chunk's tokens, softmax statistics, and the unnormalised
+// P.V, all in three parallel phases per shared-memory page:
+//   1. thread <- (token, head): full dot product q.k over d, reading the
+//      8-element column blocks in a rotated order (block (c + t) mod d/8) so
+//      the 32 lanes of a warp hit distinct banks;
+//   2. warp <- head: running max m, rescale factor, p = 2^(s - m), running sum;
+//   3. thread <- (head, 4 columns of d): acc = acc * rescale + sum_t p v.
+// Scores are in log2 units (q is pre-scaled by log2(e)/sqrt(d)).
+template <int D>
 __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
                           ComputeState &st, float *out, int ctid) {
   const Task &t = S.t;
   const int warp = ctid >> 5, lane = ctid & 31;
-  const int d = p.d, G = p.G, l = t.layer;
+  const int G = p.G, l = t.layer;
   const int b = S.b, g = S.g;
-  float *qs = reinterpret_cast<float *>(smem + p.off_x);        // [G][d]
-  float *wsc = qs + G * d;                                      // [8][G][d+2]
-  st.xkey = 0xffffffffu;                                        // x area reused
+  constexpr int NB = D / 8;                 // 8-element column blocks per row
+  constexpr int Q4 = D / 4;                 // 4-column slices per head
+  constexpr int MAXP = (kMaxGroup * Q4 + kComputeThreads - 1) / kComputeThreads;
+  float *qs = reinterpret_cast<float *>(smem + p.off_x);   // [G][D]
+  float *sc = qs + G * D;                                   // [G][tpp] scores, then p
+  float *mst = sc + G * p.tpp;                              // [G] running max
+  float *lst = mst + kMaxGroup;                             // [G] running sum
+  float *cor = lst + kMaxGroup;                             // [G] rescale of this page
+  st.xkey = 0xffffffffu;                                    // staging area reused
 
   {
     const uint32_t ev = static_cast<uint32_t>(ev_attn_ready(p, l, g));
@@ -960,151 +1005,108 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     if (!st.gs.share(ctl, ctid, okl)) return false;
     if (ctid == 0) trace_mark(p, S.idx, 4);
   }
-  // q (normed, rotated) for the G query heads of KV head g, pre-scaled so
-  // that scores are in log2 units: s = q.k / sqrt(d) * log2(e).
-  const float qscale = rsqrtf(static_cast<float>(d)) * 1.4426950408889634f;
-  for (int i = ctid; i < G * d; i += kComputeThreads)
-    qs[i] = __ldcg(p.qrot + (static_cast<size_t>(b) * p.Hq + g * G) * d + i) * qscale;
+  const float qscale = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;
+  for (int i = ctid; i < G * D; i += kComputeThreads)
+    qs[i] = __ldcg(p.qrot + (static_cast<size_t>(b) * p.Hq + g * G) * D + i) * qscale;
+  if (ctid < G) {
+    mst[ctid] = -INFINITY;
+    lst[ctid] = 0.f;
+  }
   compute_bar();
   if (ctid == 0) trace_mark(p, S.idx, 5);
 
-  float qv[kMaxGroup][DL];
-  float mrun[kMaxGroup], lrun[kMaxGroup], acc[kMaxGroup][DL];
+  float acc[MAXP][4];
 #pragma unroll
-  for (int h = 0; h < kMaxGroup; ++h) {
-    mrun[h] = -INFINITY;
-    lrun[h] = 0.f;
-#pragma unroll
-    for (int i = 0; i < DL; ++i) {
-      acc[h][i] = 0.f;
-      qv[h][i] = h < G ? qs[h * d + lane * DL + i] : 0.f;
-    }
-  }
+  for (int k = 0; k < MAXP; ++k) acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
 
   const int P = p.page_size;
   const int cur = p.pos[b];
-  const uint32_t pages = smem_u32(smem + p.off_pages);
   for (int tok0 = S.t0; tok0 < S.t1; tok0 += p.tpp) {
     const int ntok = min(p.tpp, S.t1 - tok0);
     bool okl = true;
     if (ctid == 0) okl = wait_mbar(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff40000u, 2);
     if (!st.gs.share(ctl, ctid, okl)) return false;
     mbar_try_wait(&ctl->full[st.pi], st.pg_par);
-    const uint32_t kbase = pages + st.pi * p.page_bytes;
-    const uint32_t vbase = kbase + p.tpp * d * 2;
+    uint8_t *kpg = smem + p.off_pages + static_cast<size_t>(st.pi) * p.page_bytes;
+    uint8_t *vpg = kpg + static_cast<size_t>(p.tpp) * D * 2;
     // The current token's K/V were appended by this step's QKV epilogue and
     // may have been copied into the page before they landed: reload them.
     const bool has_cur = cur >= tok0 && cur < tok0 + ntok;
     if (has_cur) {
       const int ph = kv_phys_page(p, b, cur / P);
-      const size_t src = ((static_cast<size_t>(ph < 0 ? 0 : ph) * p.Hkv + g) * P + cur % P) * d;
+      const size_t src = ((static_cast<size_t>(ph < 0 ? 0 : ph) * p.Hkv + g) * P + cur % P) * D;
       const int j = cur - tok0;
-      const int nvec = d / 8;
-      if (ctid < 2 * nvec) {
-        const bool isv = ctid >= nvec;
-        const int e = (isv ? ctid - nvec : ctid) * 8;
-        const __nv_bfloat16 *gsrc = (isv ? p.v_pages[l] : p.k_pages[l]) + src + e;
-        const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(gsrc));
-        sts128((isv ? vbase : kbase) + (j * d + e) * 2, v);
+      if (ctid < 2 * NB) {
+        const bool isv = ctid >= NB;
+        const int e = (isv ? ctid - NB : ctid) * 8;
+        const uint4 v = __ldcg(reinterpret_cast<const uint4 *>((isv ? p.v_pages[l] : p.k_pages[l]) + src + e));
+        *reinterpret_cast<uint4 *>((isv ? vpg : kpg) + (j * D + e) * 2) = v;
       }
       compute_bar();
     }
-    // Each warp takes 4 tokens at a time (tokens 4w..4w+3, then +32): the
-    // 4*G dot products reduce over the warp as independent shuffle chains,
-    // then one online-softmax update per head covers the 4 tokens.
-    constexpr int TB = 2;
-    for (int j0 = warp * TB; j0 < ntok; j0 += kComputeWarps * TB) {
-      float kf[TB][DL], vf[TB][DL];
-#pragma unroll
-      for (int u = 0; u < TB; ++u) {
-        const int j = j0 + u;
-        const bool in = j < ntok;
-        const uint32_t ko = kbase + (j * d + lane * DL) * 2;
-        const uint32_t vo = vbase + (j * d + lane * DL) * 2;
-        uint32_t kw[DL > 1 ? DL / 2 : 1], vw[DL > 1 ? DL / 2 : 1];
-        if (DL == 1) {
-          // one bf16 per lane (d = 32)
-          uint16_t kh = 0, vh = 0;
-          if (in) {
-            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(kh) : "r"(ko));
-            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(vh) : "r"(vo));
-          }
-          kf[u][0] = __uint_as_float(static_cast<uint32_t>(kh) << 16);
-          vf[u][0] = __uint_as_float(static_cast<uint32_t>(vh) << 16);
-        } else {
-#pragma unroll
-          for (int i = 0; i < DL / 2; ++i) {
-            kw[i] = 0u;
-            vw[i] = 0u;
-          }
-          if (in) {
-            if (DL == 2) {
-              asm volatile("ld.shared.b32 %0, [%1];" : "=r"(kw[0]) : "r"(ko));
-              asm volatile("ld.shared.b32 %0, [%1];" : "=r"(vw[0]) : "r"(vo));
-            } else if (DL == 4) {
-              asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(kw[0]), "=r"(kw[1]) : "r"(ko));
-              asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(vw[0]), "=r"(vw[1]) : "r"(vo));
-            } else {
-#pragma unroll
-              for (int i = 0; i < DL / 8; ++i) {
-                const uint4 a = lds128(ko + i * 16), c = lds128(vo + i * 16);
-                kw[4 * i] = a.x; kw[4 * i + 1] = a.y; kw[4 * i + 2] = a.z; kw[4 * i + 3] = a.w;
-                vw[4 * i] = c.x; vw[4 * i + 1] = c.y; vw[4 * i + 2] = c.z; vw[4 * i + 3] = c.w;
-              }
-            }
-          }
-#pragma unroll
-          for (int i = 0; i < DL / 2; ++i) {
-            kf[u][2 * i] = bf_lo(kw[i]);
-            kf[u][2 * i + 1] = bf_hi(kw[i]);
-            vf[u][2 * i] = bf_lo(vw[i]);
-            vf[u][2 * i + 1] = bf_hi(vw[i]);
-          }
-        }
+    // phase 1: scores
+    for (int pp = ctid; pp < ntok * G; pp += kComputeThreads) {
+      const int tk = pp % ntok, h = pp / ntok;
+      const uint8_t *krow = kpg + tk * D * 2;
+      const float *qh = qs + h * D;
+      float s = 0.f;
+#pragma unroll 4
+      for (int c = 0; c < NB; ++c) {
+        const int cc = (c + tk) & (NB - 1);
+        const uint4 kw = *reinterpret_cast<const uint4 *>(krow + cc * 16);
+        const float4 q0 = *reinterpret_cast<const float4 *>(qh + cc * 8);
+        const float4 q1 = *reinterpret_cast<const float4 *>(qh + cc * 8 + 4);
+        s += q0.x * bf_lo(kw.x) + q0.y * bf_hi(kw.x) + q0.z * bf_lo(kw.y) + q0.w * bf_hi(kw.y);
+        s += q1.x * bf_lo(kw.z) + q1.y * bf_hi(kw.z) + q1.z * bf_lo(kw.w) + q1.w * bf_hi(kw.w);
       }
-      float sc[kMaxGroup][TB];
+      sc[h * p.tpp + tk] = s;
+    }
+    compute_bar();
+    // phase 2: softmax statistics, one warp per head
+    for (int h = warp; h < G; h += kComputeWarps) {
+      float *row = sc + h * p.tpp;
+      float mx = -INFINITY;
+      for (int tk = lane; tk < ntok; tk += 32) mx = fmaxf(mx, row[tk]);
 #pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h)
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float mold = mst[h];
+      const float mnew = fmaxf(mold, mx);
+      float sum = 0.f;
+      for (int tk = lane; tk < ntok; tk += 32) {
+        const float pr = exp2f(row[tk] - mnew);
+        row[tk] = pr;
+        sum += pr;
+      }
+      sum = warp_sum(sum);
+      __syncwarp();
+      if (lane == 0) {
+        const float c = exp2f(mold - mnew);   // 0 on the first page (mold = -inf)
+        cor[h] = c;
+        lst[h] = lst[h] * c + sum;
+        mst[h] = mnew;
+      }
+    }
+    compute_bar();
+    // phase 3: acc = acc * rescale + sum_t p_t v_t
 #pragma unroll
-        for (int u = 0; u < TB; ++u) {
-          float s = 0.f;
-#pragma unroll
-          for (int i = 0; i < DL; ++i) s += qv[h][i] * kf[u][i];
-          sc[h][u] = s;
+    for (int k = 0; k < MAXP; ++k) {
+      const int pq = ctid + k * kComputeThreads;
+      if (pq < G * Q4) {
+        const int h = pq / Q4, i4 = pq % Q4;
+        const float c = cor[h];
+        float a0 = acc[k][0] * c, a1 = acc[k][1] * c, a2 = acc[k][2] * c, a3 = acc[k][3] * c;
+        const float *prow = sc + h * p.tpp;
+        const uint8_t *vcol = vpg + i4 * 8;
+#pragma unroll 4
+        for (int tk = 0; tk < ntok; ++tk) {
+          const float pr = prow[tk];
+          const uint2 vw = *reinterpret_cast<const uint2 *>(vcol + tk * D * 2);
+          a0 += pr * bf_lo(vw.x);
+          a1 += pr * bf_hi(vw.x);
+          a2 += pr * bf_lo(vw.y);
+          a3 += pr * bf_hi(vw.y);
         }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h)
-#pragma unroll
-          for (int u = 0; u < TB; ++u)
-            if (h < G) sc[h][u] += __shfl_xor_sync(0xffffffffu, sc[h][u], o);
-#pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) {
-        if (h >= G) break;
-        float mn = mrun[h];
-#pragma unroll
-        for (int u = 0; u < TB; ++u) {
-          if (j0 + u >= ntok) sc[h][u] = -INFINITY;
-          mn = fmaxf(mn, sc[h][u]);
-        }
-        const float corr = exp2f(mrun[h] - mn);
-        float pr[TB];
-        float lsum = 0.f;
-#pragma unroll
-        for (int u = 0; u < TB; ++u) {
-          pr[u] = exp2f(sc[h][u] - mn);
-          lsum += pr[u];
-        }
-        lrun[h] = lrun[h] * corr + lsum;
-#pragma unroll
-        for (int i = 0; i < DL; ++i) {
-          float a = acc[h][i] * corr;
-#pragma unroll
-          for (int u = 0; u < TB; ++u) a += pr[u] * vf[u][i];
-          acc[h][i] = a;
-        }
-        mrun[h] = mn;
+        acc[k][0] = a0; acc[k][1] = a1; acc[k][2] = a2; acc[k][3] = a3;
       }
     }
     if (has_cur) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -1114,48 +1116,28 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
       st.pi = 0;
       st.pg_par ^= 1u;
     }
+    compute_bar();   // sc is rewritten by the next page
   }
 
-  // merge the warps' running (max, sum, acc) in fixed order; the chunk's
-  // partial goes straight to global memory: row h = (acc[0..d), m, l, pad)
-  const int rw = d + 4;
-#pragma unroll
-  for (int h = 0; h < kMaxGroup; ++h) {
-    if (h >= G) break;
-    float *w = wsc + (warp * G + h) * rw;
-#pragma unroll
-    for (int i = 0; i < DL; ++i) w[lane * DL + i] = acc[h][i];
-    if (lane == 0) {
-      w[d] = mrun[h];
-      w[d + 1] = lrun[h];
-    }
-  }
-  compute_bar();
+  // the chunk's partial goes straight to global memory: row h = (acc, m, l, pad)
+  const int rw = D + 4;
   float *part = p.attn_part + static_cast<size_t>(t.aux) * G * rw;
-  for (int e = ctid; e < G * rw; e += kComputeThreads) {
-    const int h = e / rw, i = e % rw;
-    float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, wsc[(w * G + h) * rw + d]);
-    float s = 0.f;
-    if (i < d) {
-#pragma unroll
-      for (int w = 0; w < kComputeWarps; ++w) {
-        const float mw = wsc[(w * G + h) * rw + d];
-        if (mw != -INFINITY) s += exp2f(mw - M) * wsc[(w * G + h) * rw + i];
-      }
-    } else if (i == d) {
-      s = M;
-    } else if (i == d + 1) {
-#pragma unroll
-      for (int w = 0; w < kComputeWarps; ++w) {
-        const float mw = wsc[(w * G + h) * rw + d];
-        if (mw != -INFINITY) s += exp2f(mw - M) * wsc[(w * G + h) * rw + d + 1];
-      }
+  for (int k = 0; k < MAXP; ++k) {
+    const int pq = ctid + k * kComputeThreads;
+    if (pq < G * Q4) {
+      const int h = pq / Q4, i4 = pq % Q4;
+      __stcg(reinterpret_cast<float4 *>(part + h * rw + i4 * 4),
+             make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]));
     }
-    __stcg(part + e, s);
+  }
+  if (ctid < G) {
+    __stcg(part + ctid * rw + D, mst[ctid]);
+    __stcg(part + ctid * rw + D + 1, lst[ctid]);
   }
   compute_bar();
+  const int d = D;
+  float *wsc = sc;   // combine scratch (reuses the score area)
 
   // The chunk that completes (b, g) merges all of its chunks by log-sum-exp
   // and writes o for the G query heads.  The bar above orders every thread's
@@ -1283,10 +1265,9 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       case T_ATTN:
         if (S.b >= 0) {
           switch (p.d >> 5) {
-            case 1: tok = attn_task<1>(p, ctl, smem, S, st, out, ctid); break;
-            case 2: tok = attn_task<2>(p, ctl, smem, S, st, out, ctid); break;
-            case 4: tok = attn_task<4>(p, ctl, smem, S, st, out, ctid); break;
-            default: tok = attn_task<4>(p, ctl, smem, S, st, out, ctid); break;
+            case 1: tok = attn_task<32>(p, ctl, smem, S, st, out, ctid); break;
+            case 2: tok = attn_task<64>(p, ctl, smem, S, st, out, ctid); break;
+            default: tok = attn_task<128>(p, ctl, smem, S, st, out, ctid); break;
           }
         }
         break;

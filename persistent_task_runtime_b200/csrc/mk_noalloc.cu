@@ -49,7 +49,7 @@ inline size_t align_up_z(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int pick_mtiles(int tiles, int nsm, int cap) {
-  return std::max(1, std::min(cap, tiles / (2 * nsm)));
+  return std::max(1, std::min(cap, tiles / (16 * nsm)));
 }
 
 }  // namespace
@@ -102,10 +102,12 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
 
   // ---- shared-memory carve-up (same rules as a plan built for max_batch = B)
   const int Kmax = std::max(H, std::max(Hq * d, F));
-  // attention scratch in the staging area: q [G][d] plus either the warps'
-  // running states [warps][G][d+4] or the combine's per-chunk (m, l) pairs
+  // attention scratch in the staging area: q [G][d] plus either the page's
+  // scores [G][tokens per page] and per-head statistics, or the combine's
+  // per-chunk (m, l) pairs
   const int max_chunks = (c.max_seq_len + P - 1) / P;
-  const int att_need = G * d * 4 + std::max(mk::kComputeWarps * G * (d + 4),
+  const int tpp_bound = std::min(16 * P, 16 * mk::row_pitch_bytes(1024) / (4 * d));
+  const int att_need = G * d * 4 + std::max(G * tpp_bound + 3 * mk::kMaxGroup,
                                             2 * max_chunks * G + 2 * G) * 4;
   const int chunk_need = 2 * maxB * mk::row_pitch_bytes(std::min(1024, align_up_i(Kmax, 32)));
   int x_cap = std::min(std::max(2 * mk::row_pitch_bytes(Kmax), chunk_need), 64 * 1024);
@@ -165,6 +167,8 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
   p.attn_slots = grid + maxB * Hkv;
   p.wait_limit_ns = 2000000000LL;
   p.pf_bytes = 0u;
+  p.pf_distance = 0;
+  p.pf_task_bytes = 256u * 1024u;
   p.ev_embed = 0;
   p.ev_layer0 = 1;
   p.ev_per_layer = Hkv + 4;
