@@ -129,14 +129,10 @@ typedef struct {
                              task waits for one completion more than can
                              ever happen, so the step must end in
                              MK_ERR_TIMEOUT after wait_limit_ns             */
-  int l2_prefetch_kb;     /* per-CTA budget of upcoming weights requested
-                             into L2 ahead of the shared-memory ring, in
-                             KB; 0 = off (the default)                      */
-  int prefetch_distance;  /* when task t is dispatched, the operands of task
-                             t + prefetch_distance (queue order) are
-                             requested into L2; 0 = off, negative = off    */
-  int prefetch_task_kb;   /* cap on what one such request covers, in KB
-                             (0 = 256)                                      */
+  int max_page_cols;      /* widest weight page, in columns: 32 .. 2048, a
+                             multiple of 32; 0 = 2048.  A page is 16 weight
+                             rows; wider pages mean fewer ring hand-offs
+                             per byte, narrower ones more pages in flight  */
 } mk_plan_options;
 
 typedef struct mk_plan mk_plan;

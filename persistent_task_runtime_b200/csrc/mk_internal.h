@@ -6,6 +6,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstring>
+#include <string>
+#include <vector>
+
 #include "../../include/mk.h"
 
 namespace mk {
@@ -21,7 +25,8 @@ constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kTaskSlots = 4;                     // tasks in flight per CTA
 constexpr int kOutSlots = 4;                      // compute -> storer buffers
 constexpr int kMaxPages = 16;                     // ring entries (upper bound)
-constexpr int kMaxMTiles = 8;                     // 16-row tiles per GEMV task
+constexpr int kMaxMTiles = 8;                     // 16-row tiles per GEMV task (B <= 4)
+constexpr int kMaxPageCols = 2048;                // widest weight page (16 rows)
 constexpr int kMaxGroup = 8;                      // query heads per KV head
 constexpr int kMaxSmem = 232448;                  // opt-in smem per CTA (B200)
 
@@ -42,7 +47,9 @@ struct alignas(16) Task {
   uint8_t n_m;        // 16-row tiles (GEMV); gate/up: gate tiles + up tiles
   uint16_t layer;
   uint32_t row0;      // first output row within its matrix
-  uint32_t nrows;     // valid output rows (<= 16 * n_m; gate/up: per matrix)
+  uint16_t nrows;     // valid output rows (<= 16 * n_m; gate/up: per matrix)
+  uint8_t ksplit;     // split-K part of this task (O / down projections)
+  uint8_t nsplit;     // number of split-K parts of its row tile (0 or 1: none)
   uint32_t dep_event; // event this task waits on (kNoEvent = none)
   uint32_t dep_count; // completions of dep_event per step
   uint32_t out_event; // event incremented once the task's output is visible
@@ -82,7 +89,7 @@ struct Params {
   float *h;                     // [maxB][H]      residual stream
   float *qkv;                   // [maxB][NQKV]   raw projections
   float *qrot;                  // [maxB][Hq][d]  q after norm + RoPE
-  float *attn_part;             // [slots][G][d+2] chunk partials (acc, m, l)
+  float *attn_part;             // [slots][G][d+4] chunk partials (acc, m, l, pad)
   float *o;                     // [maxB][Hq*d]   attention output
   float *u;                     // [maxB][F]      SwiGLU output
   unsigned long long *argmax;   // [maxB]         packed (value, ~index)
@@ -96,14 +103,16 @@ struct Params {
   int max_batch, page_size, max_pos, num_kv_pages, max_pages_per_seq;
   int attn_slots, attn_target, tpp;   // slots per layer, chunk target, tokens per smem page
   int kp[4];                          // page columns per op class
+  int kchunk[4];                      // split-K columns per op class (0 = unsplit)
+  float *kpart;                       // [splits][maxB][H] split-K partial sums
+  uint32_t *tile_ctr;                 // [H/16 + 1] split-K parts done per row tile
   int x_cap;                          // bytes of the activation staging area
   int page_bytes, n_pages;
   int off_look, off_slots, off_red, off_out, out_bytes, off_x, off_pages;  // smem carve-up
-  uint32_t pf_bytes;                  // L2 prefetch budget per CTA (0 = off)
-  int pf_distance;                    // dispatching task t prefetches task t + this (0 = off)
-  uint32_t pf_task_bytes;             // cap on the bytes prefetched for one task
+  int out_stride;                     // floats per sequence in an output buffer (16 x row tiles)
   int n_tasks;
   int ev_embed, ev_layer0, ev_per_layer;   // event numbering
+  int n_ffn_parts;                         // gate/up events per layer (split-K parts of down)
   int n_lm_tasks;
   long long wait_limit_ns;
 
@@ -131,19 +140,62 @@ __host__ __device__ inline int ev_o_ready(const Params &p, int l) {
 __host__ __device__ inline int ev_oproj(const Params &p, int l) {
   return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + 1;
 }
-__host__ __device__ inline int ev_gateup(const Params &p, int l) {
-  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + 2;
+// gate/up rows of down-projection part `part` (its K range) are complete
+__host__ __device__ inline int ev_gateup(const Params &p, int l, int part) {
+  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + 2 + part;
 }
 __host__ __device__ inline int ev_down(const Params &p, int l) {
-  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + 3;
+  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + 2 + p.n_ffn_parts;
 }
 
-// smem pitch of one 16-row weight page row / one activation row, in bytes:
-// rounded to 128 and offset by 64 so rows g and g+1 fall in opposite halves
-// of the 32 banks (conflict-free 16-byte fragment loads).
+// Batch n-tiles of a GEMV: each mma n-tile carries 4 sequences, the bf16
+// high parts of their activations in columns 0..3 and the low parts in
+// columns 4..7, so one mma covers both halves.  Row tiles per task shrink as
+// n-tiles grow, which keeps the accumulators in registers.
+__host__ __device__ inline int n_tiles_for(int batch) { return batch <= 4 ? 1 : (batch <= 8 ? 2 : 4); }
+__host__ __device__ inline int max_mtiles_for(int batch) { return kMaxMTiles / n_tiles_for(batch); }
+
+// smem pitch of one row of a 16-row weight page, in bytes: rounded to 128
+// and offset by 64 so rows g and g+1 fall in opposite halves of the 32 banks
+// (conflict-free 16-byte fragment loads).
 __host__ __device__ inline int row_pitch_bytes(int cols) {
   return ((cols * 2 + 127) / 128) * 128 + 64;
 }
+
+// Staged activation: fp32 rows, pitch rounded to 128 B and offset by 16 B so
+// the fragments of consecutive sequences fall on complementary banks.
+__host__ __device__ inline int x_row_bytes(int cols) { return ((cols * 4 + 127) / 128) * 128 + 16; }
+
+// ---- plan layout (mk_layout.cu) --------------------------------------------
+struct LayoutOptions {
+  int max_batch = 1;
+  int page_size = 16;
+  int num_ctas = 0;             // 0: one per SM
+  int max_page_cols = 0;        // 0: kMaxPageCols
+  int rows_per_task[5] = {0, 0, 0, 0, 0};
+  long long wait_limit_ns = 2000000000LL;
+  bool debug_unsatisfiable_dep = false;
+};
+struct OpRange {
+  int begin, end;   // task indices of one operator (per-operator launches)
+};
+struct Layout {
+  Params p;                     // static kernel parameters (no pointers bound)
+  int grid = 0, smem = 0, n_events = 0;
+  int rows[5] = {0, 0, 0, 0, 0};   // rows per task: QKV, O, gate/up, down, LM head
+  std::vector<Task> tasks;
+  std::vector<OpRange> ops;
+  std::vector<float2> rope;     // [max_seq_len][d/2] (cos, sin)
+  // workspace byte offsets and size; counter words
+  size_t o_h = 0, o_qkv = 0, o_qrot = 0, o_part = 0, o_o = 0, o_u = 0, o_arg = 0, o_kpart = 0;
+  size_t ws_bytes = 0;
+  size_t head_words = 0, comb_words = 0, tile_words = 0, sync_words = 0;
+};
+int validate_config(const mk_model_config &c, std::string &err);
+int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int smem_optin,
+                 Layout &out, std::string &err);
+void bind_workspace(const Layout &lay, char *ws, uint32_t *sync, Params &p);
+std::vector<LayerW> layer_table(const mk_model_config &c, const mk_weights &w);
 
 cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative,
                         cudaStream_t stream);

@@ -197,6 +197,7 @@ struct Ctl {
   uint64_t out_empty[kOutSlots];
   uint64_t xbar;                    // activation bulk copy landed
   volatile int cta_abort;
+  volatile int cbad;                // a compute warp gave up (written by compute only)
   int skip;
   int flag[2];
   float rs[MK_MAX_BATCH];           // RMSNorm scale per sequence
@@ -211,7 +212,7 @@ struct Slot {
   int b, g, t0, t1;          // attention: sequence, KV head, token range
   int first_slot, n_chunks;  // attention: partial slots of (b, g)
   int idx;                   // task index (for error reports)
-  int pad;
+  int dep_ok;                // the loader saw the input event complete
 };
 static_assert(sizeof(Slot) == 64, "slot must be 64 bytes");
 
@@ -301,16 +302,14 @@ struct GroupSync {
 // ============================================================================
 
 struct Geo {
-  int K;        // input width
+  int K;        // full input width (row length of the weight matrix)
+  int k0, Kt;   // the task's columns: [k0, k0 + Kt) (split-K parts cover a range)
   int kp;       // columns per weight page
   int kx;       // columns per staged activation chunk
-  int whole;    // kx == K: the staged activation can be reused by later tasks
+  int whole;    // kx == Kt: the staged activation can be reused by later tasks
   int cls;      // OpK
 };
 
-// Staged activation: fp32 rows, pitch rounded to 128 B and offset by 16 B so
-// the fragments of consecutive sequences fall on complementary banks.
-__device__ __forceinline__ int x_row_bytes(int cols) { return ((cols * 4 + 127) / 128) * 128 + 16; }
 __device__ __forceinline__ int x_bytes(int B, int cols) { return B * x_row_bytes(cols); }
 
 __device__ Geo gemv_geo(const Params &p, const Task &t, int B) {
@@ -322,11 +321,18 @@ __device__ Geo gemv_geo(const Params &p, const Task &t, int B) {
     default: g.K = p.H; g.cls = K_HID; break;
   }
   g.kp = p.kp[g.cls];
-  if (x_bytes(B, g.K) <= p.x_cap) {
-    g.kx = g.K;
+  if (t.nsplit > 1) {
+    g.k0 = t.ksplit * p.kchunk[g.cls];
+    g.Kt = min(g.K, g.k0 + p.kchunk[g.cls]) - g.k0;
+  } else {
+    g.k0 = 0;
+    g.Kt = g.K;
+  }
+  if (x_bytes(B, g.Kt) <= p.x_cap) {
+    g.kx = g.Kt;
     g.whole = 1;
   } else {
-    int n = g.K / g.kp;
+    int n = g.Kt / g.kp;
     while (n > 1 && x_bytes(B, n * g.kp) > p.x_cap) --n;
     g.kx = n * g.kp;
     g.whole = 0;
@@ -368,18 +374,19 @@ __device__ __forceinline__ int seq_len(const Params &p, int b) {
   return n < 1 ? 1 : (n > p.max_pos ? p.max_pos : n);
 }
 
-__device__ int attn_chunk_pages(const Params &p, int B) {
-  int total = 0;
-  for (int b = 0; b < B; ++b) total += (seq_len(p, b) + p.tpp - 1) / p.tpp;
-  total *= p.Hkv;
-  const int c = (total + p.attn_target - 1) / p.attn_target;
-  return c < 1 ? 1 : c;
+// Tokens per attention chunk: a whole number of KV pages, sized so the
+// chunks of all (sequence, KV head) pairs number about one per CTA.
+__device__ int attn_span(const Params &p, int B) {
+  const int P = p.page_size;
+  int units = 0;
+  for (int b = 0; b < B; ++b) units += (seq_len(p, b) + P - 1) / P;
+  units *= p.Hkv;
+  const int c = (units + p.attn_target - 1) / p.attn_target;
+  return (c < 1 ? 1 : c) * P;
 }
 
-// Slot s -> (b, g, chunk token range, first slot of (b, g), chunks of (b, g)).
 __device__ bool attn_resolve(const Params &p, int B, int s, Slot &o) {
-  const int cp = attn_chunk_pages(p, B);
-  const int span = cp * p.tpp;
+  const int span = attn_span(p, B);
   int base = 0;
   for (int b = 0; b < B; ++b) {
     const int len = seq_len(p, b);
@@ -416,40 +423,12 @@ __device__ __forceinline__ bool is_gemv(uint8_t type) {
          type == T_LMHEAD;
 }
 
-__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// Ask L2 for (up to `budget` bytes of) a GEMV task's weight rows: each task
-// covers whole rows, so its weights are one contiguous region per matrix.
-// Lanes issue 32 KB pieces.  Returns the bytes requested.
-__device__ uint32_t l2_prefetch_task(const Params &p, const Task &t, uint32_t budget, int lane) {
-  if (!is_gemv(t.type) || budget == 0) return 0;
-  const int K = t.type == T_OPROJ ? p.Hq * p.d : (t.type == T_DOWN ? p.F : p.H);
-  const int regions = t.type == T_GATEUP ? 2 : 1;
-  const uint32_t bytes = t.nrows * static_cast<uint32_t>(K) * 2u;
-  uint32_t want = min(budget, bytes * regions);
-  uint32_t done = 0;
-  for (int r = 0; r < regions && done < want; ++r) {
-    const __nv_bfloat16 *W;
-    int row, rv;
-    gemv_tile(p, t, r == 0 ? 0 : (t.n_m >> 1), W, row, rv);
-    const char *base = reinterpret_cast<const char *>(W + static_cast<size_t>(row) * K);
-    const uint32_t n = min(bytes, want - done);
-    for (uint32_t off = static_cast<uint32_t>(lane) * 32768u; off < n; off += 32u * 32768u)
-      prefetch_l2(base + off, min(32768u, n - off));
-    done += n;
-  }
-  return done;
-}
-
 // Tasks popped from the queue but not yet handed to the compute warps.
 constexpr int kLook = 8;
 struct Look {
   Task t;
   int tix;
-  uint32_t pf;   // bytes of its weights already requested into L2
-  int pad[2];
+  int pad[3];
 };
 static_assert(sizeof(Look) == 48, "lookahead entry size");
 
@@ -473,11 +452,12 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   if (lane == 0) next = atomicAdd(p.sync + S_QUEUE, 1u);
   int la_head = 0, la_count = 0;
   bool exhausted = false;
-  uint32_t pf_ahead = 0;
+  uint32_t la_ev = 0;   // lane 0: input-event counter read when the task was popped
 
-  // Pop one task into the lookahead (warp-uniform).  With an L2 budget the
-  // loader keeps up to p.pf_bytes of future weights requested into L2, so
-  // HBM keeps streaming while the compute warps wait at a dependency.
+  // Pop one task into the lookahead (warp-uniform).  The next ticket is
+  // always requested one pop ahead, so a pop waits only for the descriptor.
+  // Lane 0 also starts reading the GEMV task's input-event counter; the
+  // value is looked at only when the task is handed over, a task later.
   auto pop_one = [&]() {
     const uint32_t ticket = __shfl_sync(0xffffffffu, next, 0);
     if (static_cast<int>(ticket) >= n_launch) {
@@ -487,24 +467,19 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     if (lane == 0) next = atomicAdd(p.sync + S_QUEUE, 1u);
     const int tix = p.task_begin + static_cast<int>(ticket);
     const Task t = p.tasks[tix];
-    const uint32_t room = p.pf_bytes > pf_ahead ? p.pf_bytes - pf_ahead : 0u;
-    const uint32_t pf = l2_prefetch_task(p, t, room, lane);
     const int e = (la_head + la_count) % kLook;
     if (lane == 0) {
       la[e].t = t;
       la[e].tix = tix;
-      la[e].pf = pf;
+      if (is_gemv(t.type) && t.dep_event != kNoEvent) la_ev = ld_relaxed(p.sync + S_EVENTS + t.dep_event);
     }
     ++la_count;
-    pf_ahead += pf;
   };
   auto top_up = [&](int max_pops) {
     for (int k = 0; k < max_pops; ++k) {
-      if (exhausted || la_count == kLook) break;
-      // one task ahead; more only while the L2 prefetch budget is not spent
-      // (every popped task is reserved for this CTA, so popping far ahead
-      // delays the last tasks of an operator)
-      if (la_count >= 1 && pf_ahead >= p.pf_bytes) break;
+      // one task ahead: every popped task is reserved for this CTA, so
+      // popping further ahead would delay the last tasks of an operator
+      if (exhausted || la_count >= 1) break;
       pop_one();
     }
     __syncwarp();
@@ -527,16 +502,24 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     }
     const Task t = la[la_head].t;
     const int tix = la[la_head].tix;
-    pf_ahead -= la[la_head].pf;
     la_head = (la_head + 1) % kLook;
     --la_count;
     Slot info;
     info.t = t;
     info.idx = tix;
     info.b = -1;
+    info.dep_ok = 0;
     if (t.type == T_ATTN) attn_resolve(p, B, static_cast<int>(t.aux), info);
     __syncwarp();
     if (lane == 0) {
+      // an input event already complete when the task was popped: order its
+      // producers' writes before the hand-over (the slot barrier publishes
+      // them to the compute warps), which then skip their own wait
+      if (is_gemv(t.type) && t.dep_event != kNoEvent &&
+          static_cast<int32_t>(la_ev - p.epoch * t.dep_count) >= 0) {
+        fence_acq_rel();
+        info.dep_ok = 1;
+      }
       S = info;
       mbar_arrive(&ctl->slot_full[ts]);
       if (p.trace != nullptr) {
@@ -551,42 +534,12 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       ts_par ^= 1u;
     }
 
-    // ---- warm L2 for the task pf_distance places later in the queue ----
-    // Nothing is reserved: whichever CTA later pops that task finds its
-    // operands in L2, and HBM keeps streaming while this CTA's compute warps
-    // wait at an operator boundary.
-    if (p.pf_distance > 0) {
-      const int fut = tix + p.pf_distance;
-      if (fut < p.task_end) {
-        const Task ft = p.tasks[fut];
-        if (is_gemv(ft.type)) {
-          l2_prefetch_task(p, ft, p.pf_task_bytes, lane);
-        } else if (ft.type == T_ATTN) {
-          Slot fi;
-          fi.b = -1;
-          attn_resolve(p, B, static_cast<int>(ft.aux), fi);
-          if (fi.b >= 0) {
-            const int P = p.page_size;
-            const size_t kvpage_elems = static_cast<size_t>(P) * p.d;
-            const int npg = (fi.t1 - fi.t0 + P - 1) / P;
-            for (int j = lane; j < 2 * npg; j += 32) {
-              const int ph = kv_phys_page(p, fi.b, fi.t0 / P + (j >> 1));
-              if (ph < 0) continue;
-              const __nv_bfloat16 *base = (j & 1) ? p.v_pages[ft.layer] : p.k_pages[ft.layer];
-              prefetch_l2(base + (static_cast<size_t>(ph) * p.Hkv + fi.g) * kvpage_elems,
-                          static_cast<uint32_t>(kvpage_elems * 2));
-            }
-          }
-        }
-      }
-    }
-
     // ---- stream the task's operands into the page ring ----
     if (is_gemv(t.type)) {
       const Geo geo = gemv_geo(p, t, B);
       const int pitch = row_pitch_bytes(geo.kp);
-      for (int xc0 = 0; xc0 < geo.K && ok; xc0 += geo.kx) {
-        const int xend = min(geo.K, xc0 + geo.kx);
+      for (int xc0 = geo.k0; xc0 < geo.k0 + geo.Kt && ok; xc0 += geo.kx) {
+        const int xend = min(geo.k0 + geo.Kt, xc0 + geo.kx);
         for (int m = 0; m < t.n_m && ok; ++m) {
           const __nv_bfloat16 *W;
           int row, rv;
@@ -659,7 +612,6 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   if (!ok) {
     // Abandoning the step: no bulk copy may still be landing in shared
     // memory when this CTA exits.  Wait (bounded) for every page's last copy.
-    // (L2 prefetches carry no completion and write no shared memory.)
     ctl->cta_abort = 1;
     if (lane == 0) {
       for (int q = 0; q < p.n_pages; ++q) {
@@ -684,20 +636,22 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
 // 8 columns feed both k16 steps of the mma (a fixed permutation of k that the
 // activation fragment follows as well).  The staged activation holds, per
 // 8-column block, 8 bf16 "hi" values then 8 bf16 "lo" values (hi + lo == x to
-// ~2^-16), so a fragment is two 16-byte loads.
+// ~2^-16).  n-tile nt serves sequences 4nt..4nt+3: lanes with g < 4 supply
+// the hi block of sequence 4nt+g (mma column g), lanes with g >= 4 the lo
+// block of sequence 4nt+g-4 (column g), so one mma per k-step covers both
+// halves and the epilogue adds column n+4 to column n.
 template <int NN>
 __device__ __forceinline__ void page_mma(float (&acc)[NN][4], const uint8_t *pg, int pitch, int nc,
                                          const uint8_t *xs, int xpitch, int xcol0, int B, int warp,
                                          int lane) {
   const int g = lane >> 2, q = lane & 3;
   const int groups = (nc + 31) >> 5;
-  // four independent accumulator chains (k-step 0/1 x hi/lo) so consecutive
-  // mma instructions do not wait on each other; summed in a fixed order
-  float c1[NN][4], c2[NN][4], c3[NN][4];
+  const int xhalf = (g >> 2) * 16;   // 0: hi block, 16: lo block
+  float c1[NN][4];                   // second k-step: an independent chain
 #pragma unroll
   for (int nt = 0; nt < NN; ++nt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) c1[nt][e] = c2[nt][e] = c3[nt][e] = 0.f;
+    for (int e = 0; e < 4; ++e) c1[nt][e] = 0.f;
   const uint8_t *wrow0 = pg + g * pitch + q * 16;
   const uint8_t *wrow1 = wrow0 + 8 * pitch;
 #pragma unroll 2
@@ -711,23 +665,29 @@ __device__ __forceinline__ void page_mma(float (&acc)[NN][4], const uint8_t *pg,
     }
 #pragma unroll
     for (int nt = 0; nt < NN; ++nt) {
-      const int b = nt * 8 + g;
-      uint4 xh = make_uint4(0, 0, 0, 0), xl = make_uint4(0, 0, 0, 0);
-      if (valid && b < B) {
-        const uint8_t *blk = xs + b * xpitch + (xcol0 + c) * 4;
-        xh = *reinterpret_cast<const uint4 *>(blk);
-        xl = *reinterpret_cast<const uint4 *>(blk + 16);
-      }
-      mma_bf16(acc[nt], wa.x, wb.x, wa.y, wb.y, xh.x, xh.y);
-      mma_bf16(c1[nt], wa.z, wb.z, wa.w, wb.w, xh.z, xh.w);
-      mma_bf16(c2[nt], wa.x, wb.x, wa.y, wb.y, xl.x, xl.y);
-      mma_bf16(c3[nt], wa.z, wb.z, wa.w, wb.w, xl.z, xl.w);
+      const int b = nt * 4 + (g & 3);
+      uint4 xv = make_uint4(0, 0, 0, 0);
+      if (valid && b < B)
+        xv = *reinterpret_cast<const uint4 *>(xs + b * xpitch + (xcol0 + c) * 4 + xhalf);
+      mma_bf16(acc[nt], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
+      mma_bf16(c1[nt], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
     }
   }
 #pragma unroll
   for (int nt = 0; nt < NN; ++nt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[nt][e] += (c1[nt][e] + c2[nt][e]) + c3[nt][e];
+    for (int e = 0; e < 4; ++e) acc[nt][e] += c1[nt][e];
+}
+
+// All lanes of a compute warp wait (bounded) for a full ring page; the
+// result is warp-uniform.
+__device__ __forceinline__ bool warp_wait_page(const Params &p, Ctl *ctl, uint64_t *bar,
+                                               uint32_t parity, uint32_t where) {
+  const bool done = mbar_try_wait(bar, parity);
+  if (__all_sync(0xffffffffu, done)) return true;
+  int ok = 1;
+  if (!done) ok = wait_mbar(p, ctl, bar, parity, where, 2) ? 1 : 0;
+  return __all_sync(0xffffffffu, ok) != 0;
 }
 
 struct ComputeState {
@@ -762,7 +722,7 @@ __device__ __forceinline__ void gemv_source(const Params &p, const Task &t, cons
 // ss[b] by one warp in a fixed order; the RMSNorm scale is applied to the
 // task's outputs, since W (x * g * r) = r * W (x * g).
 __device__ bool stage_x(const Params &p, Ctl *ctl, uint8_t *smem, const Task &t, int xc0,
-                        int xlen, int xpitch, int B, int ctid, ComputeState &st) {
+                        int xlen, int xpitch, int B, int ctid, ComputeState &st, bool first) {
   const float *src;
   int stride;
   const __nv_bfloat16 *gain;
@@ -801,7 +761,7 @@ __device__ bool stage_x(const Params &p, Ctl *ctl, uint8_t *smem, const Task &t,
         s += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
       }
       s = warp_sum(s);
-      if (lane == 0) ctl->ss[b] = (xc0 == 0 ? 0.f : ctl->ss[b]) + s;
+      if (lane == 0) ctl->ss[b] = (first ? 0.f : ctl->ss[b]) + s;
     }
     compute_bar();
   }
@@ -855,10 +815,10 @@ __device__ bool stage_x(const Params &p, Ctl *ctl, uint8_t *smem, const Task &t,
   return true;
 }
 
-// NN = batch n-tiles (1: B <= 8, 2: B <= 16).  With two n-tiles a task holds
-// at most kMaxMTiles/2 row tiles (the plan caps rows per task) so that the
+// NN = batch n-tiles (1: B <= 4, 2: B <= 8, 4: B <= 16).  A task holds at
+// most kMaxMTiles / NN row tiles (the plan caps rows per task) so that the
 // accumulators stay in registers.
-template <int NN, int MT = (NN == 1 ? kMaxMTiles : kMaxMTiles / 2)>
+template <int NN, int MT = kMaxMTiles / NN>
 __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
                           ComputeState &st, float *out, int ctid) {
   const Task &t = S.t;
@@ -869,19 +829,20 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   const int xstride = x_row_bytes(geo.kx) / 4;
   const uint8_t *pages = smem + p.off_pages;
   const uint8_t *xs = smem + p.off_x;
-  const uint32_t key = (static_cast<uint32_t>(t.layer) << 8) | t.type;
+  const uint32_t key = (static_cast<uint32_t>(t.layer) << 16) | (static_cast<uint32_t>(t.type) << 8) |
+                       t.ksplit;
   const float *src;
   int stride;
   const __nv_bfloat16 *gain;
   gemv_source(p, t, src, stride, gain);
 
-  if (t.dep_event != st.sat_ev || t.dep_count != st.sat_cnt) {
+  if (!S.dep_ok && (t.dep_event != st.sat_ev || t.dep_count != st.sat_cnt)) {
     bool okl = true;
     if (ctid == 0) okl = wait_event(p, ctl, t.dep_event, t.dep_count, S.idx);
     if (!st.gs.share(ctl, ctid, okl)) return false;
-    st.sat_ev = t.dep_event;
-    st.sat_cnt = t.dep_count;
   }
+  st.sat_ev = t.dep_event;
+  st.sat_cnt = t.dep_count;
   if (ctid == 0) trace_mark(p, S.idx, 4);
 
   float acc[MT][NN][4];
@@ -892,20 +853,36 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[m][n][e] = 0.f;
 
-  for (int xc0 = 0; xc0 < geo.K; xc0 += geo.kx) {
-    const int xend = min(geo.K, xc0 + geo.kx);
+  bool bad = false;   // this warp gave up waiting for a page (warp-uniform)
+  for (int xc0 = geo.k0; xc0 < geo.k0 + geo.Kt; xc0 += geo.kx) {
+    const int xend = min(geo.k0 + geo.Kt, xc0 + geo.kx);
     if (!(geo.whole && st.xkey == key)) {
-      if (!stage_x(p, ctl, smem, t, xc0, xend - xc0, xstride * 4, B, ctid, st)) return false;
+      if (!stage_x(p, ctl, smem, t, xc0, xend - xc0, xstride * 4, B, ctid, st, xc0 == geo.k0))
+        return false;
       st.xkey = geo.whole ? key : 0xffffffffu;
     }
-    if (ctid == 0 && xc0 == 0) trace_mark(p, S.idx, 5);
+    if (ctid == 0 && xc0 == geo.k0) trace_mark(p, S.idx, 5);
+    // Each warp waits for a page by itself (bounded) and releases its share
+    // of it, so warps are not locked together page by page.  A warp whose
+    // wait fails stops computing, flags the CTA, and the warps agree on the
+    // outcome once, after the last page.
     for (int m = 0; m < t.n_m; ++m) {
       for (int c0 = xc0; c0 < xend; c0 += geo.kp) {
         const int nc = min(geo.kp, xend - c0);
-        bool okl = true;
-        if (ctid == 0) okl = wait_mbar(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff30000u, 2);
-        if (!st.gs.share(ctl, ctid, okl)) return false;
-        mbar_try_wait(&ctl->full[st.pi], st.pg_par);  // completed: acquire for this thread
+        if (!bad && !warp_wait_page(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff30000u)) {
+          bad = true;
+          if (lane == 0) {
+            ctl->cbad = 1;
+            ctl->cta_abort = 1;
+          }
+        }
+        if (bad) {
+          if (++st.pi == p.n_pages) {
+            st.pi = 0;
+            st.pg_par ^= 1u;
+          }
+          continue;
+        }
         const uint8_t *pg = pages + static_cast<size_t>(st.pi) * p.page_bytes;
         switch (m) {
 #define MK_PAGE_CASE(M)                                                                      \
@@ -935,11 +912,15 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     }
   }
 
+  // every warp has passed all pages (or given up): one uniform decision
+  compute_bar();
+  if (ctl->cbad != 0) return false;
   if (gain != nullptr) {
     if (ctid < B) ctl->rs[ctid] = 1.0f / sqrtf(ctl->ss[ctid] / static_cast<float>(geo.K) + p.eps);
     compute_bar();
   }
-  // cross-warp reduction, one 16-row tile at a time, fixed warp order
+  // cross-warp reduction, one 16-row tile at a time, fixed warp order; for
+  // sequence b = 4 nt + j a warp contributes its columns j (hi) and j + 4 (lo)
   float *red = reinterpret_cast<float *>(smem + p.off_red);
   constexpr int NC = NN * 8;
   const int g = lane >> 2, q = lane & 3;
@@ -956,12 +937,16 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
       r1[1] = acc[m][nt][3];
     }
     compute_bar();
-    for (int e = ctid; e < 16 * NC; e += kComputeThreads) {
-      const int row = e / NC, n = e % NC;
+    for (int e = ctid; e < 16 * 4 * NN; e += kComputeThreads) {
+      const int row = e / (4 * NN), b = e % (4 * NN);
+      const int col = (b >> 2) * 8 + (b & 3);
       float s = 0.f;
 #pragma unroll
-      for (int w = 0; w < kComputeWarps; ++w) s += red[(w * 16 + row) * NC + n];
-      if (n < B) out[n * (16 * kMaxMTiles) + m * 16 + row] = gain != nullptr ? s * ctl->rs[n] : s;
+      for (int w = 0; w < kComputeWarps; ++w) {
+        const float *rr = red + (w * 16 + row) * NC + col;
+        s += rr[0] + rr[4];
+      }
+      if (b < B) out[b * p.out_stride + m * 16 + row] = gain != nullptr ? s * ctl->rs[b] : s;
     }
     compute_bar();
   }
@@ -1272,8 +1257,9 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
         }
         break;
       default:
-        tok = p.batch > 8 ? gemv_task<2>(p, ctl, smem, S, st, out, ctid)
-                          : gemv_task<1>(p, ctl, smem, S, st, out, ctid);
+        tok = p.batch > 8   ? gemv_task<4>(p, ctl, smem, S, st, out, ctid)
+              : p.batch > 4 ? gemv_task<2>(p, ctl, smem, S, st, out, ctid)
+                            : gemv_task<1>(p, ctl, smem, S, st, out, ctid);
         break;
     }
     if (!tok) {
@@ -1391,7 +1377,7 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
                                 int lane) {
   const Task &t = S.t;
   const int B = p.batch;
-  constexpr int OS = 16 * kMaxMTiles;
+  const int OS = p.out_stride;
   switch (t.type) {
     case T_EMBED: {
       __syncwarp();
@@ -1429,6 +1415,38 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
     }
     case T_OPROJ:
     case T_DOWN: {
+      if (t.nsplit > 1) {
+        // split-K part: publish the partial; the part that completes the row
+        // tile sums all parts in a fixed order and applies the residual
+        const size_t sp = static_cast<size_t>(p.max_batch) * p.H;
+        for (int b = 0; b < B; ++b)
+          for (int r = lane; r < static_cast<int>(t.nrows); r += 32)
+            __stcg(p.kpart + t.ksplit * sp + static_cast<size_t>(b) * p.H + t.row0 + r, out[b * OS + r]);
+        __syncwarp();
+        uint32_t *tc = p.tile_ctr + t.row0 / 16;
+        uint32_t old = 0;
+        if (lane == 0) old = atom_add_acq_rel(tc, 1u);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old + 1u != static_cast<uint32_t>(t.nsplit)) break;
+        __syncwarp();
+        for (int b = 0; b < B; ++b)
+          for (int r = lane; r < static_cast<int>(t.nrows); r += 32) {
+            const size_t o = static_cast<size_t>(b) * p.H + t.row0 + r;
+            float sum = 0.f;
+            for (int k = 0; k < t.nsplit; ++k) sum += __ldcg(p.kpart + k * sp + o);
+            float *hp = p.h + o;
+            const float v = __ldcg(hp) + sum;
+            __stcg(hp, v);
+            if (t.type == T_DOWN && p.hidden_dump != nullptr)
+              p.hidden_dump[(static_cast<size_t>(t.layer) * B + b) * p.H + t.row0 + r] = v;
+          }
+        __syncwarp();
+        if (lane == 0) {
+          *tc = 0u;
+          signal(p, t.out_event);
+        }
+        break;
+      }
       for (int b = 0; b < B; ++b)
         for (int r = lane; r < static_cast<int>(t.nrows); r += 32) {
           float *hp = p.h + static_cast<size_t>(b) * p.H + t.row0 + r;
@@ -1557,6 +1575,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     }
     mbar_init(&ctl->xbar, 1);
     ctl->cta_abort = 0;
+    ctl->cbad = 0;
     ctl->flag[0] = ctl->flag[1] = 0;
     // a device error from an earlier step is sticky until the host resets
     ctl->skip = (ld_relaxed(p.sync + S_STATUS) != 0u || ld_relaxed(p.sync + S_ABORT) != 0u);
