@@ -25,6 +25,7 @@ ranks produced divided by that time.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -51,6 +52,9 @@ def parse_workload(name: str) -> dict:
         return dict(model="1.5b", batch=1, lengths=[256], prefill="decode")
     if name == "8b_b1_ctx512":
         return dict(model="8b", batch=1, lengths=[512], prefill="decode")
+    if name == "8b4l_b1_ctx512":
+        # profiling case: 8B-shaped layers, 4 of them, same kernel (not a bench line)
+        return dict(model="8b", layers=4, batch=1, lengths=[512], prefill="synthetic")
     if name.startswith("8b_b") and name.endswith("_ctx1024"):
         B = int(name[len("8b_b"):-len("_ctx1024")])
         return dict(model="8b", batch=B, lengths=[1024] * B, prefill="synthetic")
@@ -58,6 +62,57 @@ def parse_workload(name: str) -> dict:
         return dict(model="8b", batch=16, lengths=synth.ragged_lengths(16, 32, 8192, seed=2),
                     prefill="synthetic")
     raise SystemExit(f"unknown workload {name}")
+
+
+def model_config(wl: dict) -> dict:
+    cfg = dict(synth.CONFIGS[wl["model"]])
+    if "layers" in wl:
+        cfg["n_layers"] = wl["layers"]
+    return cfg
+
+
+def source_digest() -> str:
+    """sha256 over the kernel and plan sources (the code a DRAM capture covers)."""
+    h = hashlib.sha256()
+    cdir = os.path.join(ROOT, "persistent_task_runtime_b200", "csrc")
+    for name in sorted(os.listdir(cdir)):
+        if name.endswith((".cu", ".h")):
+            with open(os.path.join(cdir, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    with open(os.path.join(ROOT, "include", "mk.h"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    or None when there is none or the kernel sources changed since."""
+    path = os.path.join(ROOT, "profiles", f"mk_decode_step_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("- ") and " = " in line:
+                k, v = line[2:].split(" = ", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256") != source_digest() or "dram_bytes_per_launch" not in vals:
+        return None
+    return int(vals["dram_bytes_per_launch"])
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest value of x over all ranks (x itself on one rank)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, batch: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job tokens/s: every rank decodes `batch` tokens per step (replicas)."""
+    return world * batch * steps / (elapsed_ms / 1e3)
 
 
 def measured_peaks() -> dict:
@@ -142,7 +197,7 @@ def run_mk(args, rank: int, world: int, local_rank: int) -> dict:
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = parse_workload(args.workload)
-    cfg = synth.CONFIGS[wl["model"]]
+    cfg = model_config(wl)
     B, lengths = wl["batch"], list(wl["lengths"])
     W, K = args.warmup, args.steps
     horizon = W + K + max(args.e2e_steps, 0) + 8
@@ -212,10 +267,7 @@ def run_mk(args, rank: int, world: int, local_rank: int) -> dict:
     print(f"[bench] rank {rank}: {K} steps in {elapsed_ms:.3f} ms "
           f"({1e3 * elapsed_ms / K:.1f} us/step)", file=sys.stderr, flush=True)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
 
     # algorithmic bytes of one step: weights (+ one embedding row per sequence)
     # + KV read over positions 0..pos of every sequence, averaged over the
@@ -246,11 +298,7 @@ def run_mk(args, rank: int, world: int, local_rank: int) -> dict:
                 raise RuntimeError(f"host step failed: {rc}")
             h_ids.copy_(h_out)
             h_pos += 1
-        e2e_s = time.perf_counter() - w0
-        if world > 1:
-            tt = torch.tensor([e2e_s], device=dev)
-            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-            e2e_s = float(tt.item())
+        e2e_s = max_over_ranks(time.perf_counter() - w0, world, dev)
         e2e = {"value": world * B * n / e2e_s, "unit": UNIT,
                "h2d_bytes_per_step": 2 * 4 * B, "d2h_bytes_per_step": 4 * B + 4,
                "us_per_step": 1e6 * e2e_s / n, "steps": n}
@@ -314,7 +362,7 @@ def cores_used() -> int:
 
 def run_reference(args) -> dict:
     wl = parse_workload(args.workload)
-    cfg = synth.CONFIGS[wl["model"]]
+    cfg = model_config(wl)
     B, lengths = wl["batch"], list(wl["lengths"])
     w = cpu_weights_sample(cfg)
     head_s, _, L = oracle_layer_timing(cfg, B, lengths, w)
@@ -347,7 +395,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     wl = parse_workload(args.workload)
-    cfg = synth.CONFIGS[wl["model"]]
+    cfg = model_config(wl)
     config = {"workload": args.workload, "model_shape": wl["model"], "batch": wl["batch"],
               "context": wl["lengths"] if len(set(wl["lengths"])) > 1 else wl["lengths"][0],
               "kv_page": 16, "weights": "random N(0,0.02) bf16", "ids": "uniform random",
@@ -383,13 +431,12 @@ def main():
     r = run_mk(args, rank, world, local_rank)
     K = args.steps
     ms_per_step = r["elapsed_ms"] / K
-    tokens = world * r["B"] * K
-    value = tokens / (r["elapsed_ms"] / 1e3)
+    value = job_throughput(world, r["B"], K, r["elapsed_ms"])
     peaks = measured_peaks()
     achieved = r["step_bytes"] / (r["mean_launch_ms"] / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": None, "peak_source": peaks["source"],
+                "traffic": profiled_traffic(args.workload), "peak_source": peaks["source"],
                 "bytes_per_step": int(r["step_bytes"]), "kernel_us": 1e3 * r["mean_launch_ms"],
                 "vs_8tbs": round(achieved / 8000.0, 4)}
     line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,

@@ -47,6 +47,11 @@ SHAPES = {
     # head_dim 32, MHA (G = 1)
     "d32_mha": dict(n_layers=1, hidden=128, n_q_heads=4, n_kv_heads=4, head_dim=32,
                     ffn=256, vocab=512, rms_eps=1e-6, rope_theta=1e6, qk_norm=True),
+    # 3 KV groups of 4 x 128: the O projection splits along K into parts of
+    # whole groups (2 + 1), the down projection into 2 parts
+    "o_split_3groups": dict(n_layers=2, hidden=1024, n_q_heads=12, n_kv_heads=3,
+                            head_dim=128, ffn=2816, vocab=2048, rms_eps=1e-6,
+                            rope_theta=1e6, qk_norm=True),
 }
 
 
