@@ -133,6 +133,10 @@ typedef struct {
                              multiple of 32; 0 = 2048.  A page is 16 weight
                              rows; wider pages mean fewer ring hand-offs
                              per byte, narrower ones more pages in flight  */
+  int o_split;            /* nonzero: split the O projection along K into two
+                             parts of whole KV groups, each waiting only for
+                             the attention of its groups (needs >= 2 KV heads
+                             and >= 1024 columns per part); 0 = one part   */
 } mk_plan_options;
 
 typedef struct mk_plan mk_plan;

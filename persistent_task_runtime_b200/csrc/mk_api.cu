@@ -119,6 +119,7 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   lo.page_size = o.kv_page_size == 0 ? 16 : o.kv_page_size;
   lo.num_ctas = o.num_ctas;
   lo.max_page_cols = o.max_page_cols;
+  lo.o_split = o.o_split != 0;
   for (int i = 0; i < 5; ++i) lo.rows_per_task[i] = o.rows_per_task[i];
   lo.wait_limit_ns = o.wait_limit_ns == 0 ? 2000000000LL : o.wait_limit_ns;
   lo.debug_unsatisfiable_dep = o.debug_unsatisfiable_dep != 0;

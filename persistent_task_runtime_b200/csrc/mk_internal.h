@@ -101,7 +101,7 @@ struct Params {
   float eps;
   int qk_norm;
   int max_batch, page_size, max_pos, num_kv_pages, max_pages_per_seq;
-  int attn_slots, attn_target, tpp;   // slots per layer, chunk target, tokens per smem page
+  int attn_slots, attn_spg, tpp;      // slots per layer, slots per KV group, tokens per smem page
   int kp[4];                          // page columns per op class
   int kchunk[4];                      // split-K columns per op class (0 = unsplit)
   float *kpart;                       // [splits][maxB][H] split-K partial sums
@@ -113,6 +113,7 @@ struct Params {
   int n_tasks;
   int ev_embed, ev_layer0, ev_per_layer;   // event numbering
   int n_ffn_parts;                         // gate/up events per layer (split-K parts of down)
+  int n_o_parts, o_groups;                 // split-K parts of the O projection, KV groups per part
   int n_lm_tasks;
   long long wait_limit_ns;
 
@@ -134,18 +135,19 @@ struct Params {
 __host__ __device__ inline int ev_attn_ready(const Params &p, int l, int g) {
   return p.ev_layer0 + l * p.ev_per_layer + g;
 }
-__host__ __device__ inline int ev_o_ready(const Params &p, int l) {
-  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv;
+// attention of the KV groups of O-projection part `part` is complete (o ready)
+__host__ __device__ inline int ev_o_ready(const Params &p, int l, int part) {
+  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + part;
 }
 __host__ __device__ inline int ev_oproj(const Params &p, int l) {
-  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + 1;
+  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + p.n_o_parts;
 }
 // gate/up rows of down-projection part `part` (its K range) are complete
 __host__ __device__ inline int ev_gateup(const Params &p, int l, int part) {
-  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + 2 + part;
+  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + p.n_o_parts + 1 + part;
 }
 __host__ __device__ inline int ev_down(const Params &p, int l) {
-  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + 2 + p.n_ffn_parts;
+  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + p.n_o_parts + 1 + p.n_ffn_parts;
 }
 
 // Batch n-tiles of a GEMV: each mma n-tile carries 4 sequences, the bf16
@@ -172,6 +174,7 @@ struct LayoutOptions {
   int page_size = 16;
   int num_ctas = 0;             // 0: one per SM
   int max_page_cols = 0;        // 0: kMaxPageCols
+  bool o_split = false;         // O projection in two K parts of whole KV groups
   int rows_per_task[5] = {0, 0, 0, 0, 0};
   long long wait_limit_ns = 2000000000LL;
   bool debug_unsatisfiable_dep = false;

@@ -374,35 +374,39 @@ __device__ __forceinline__ int seq_len(const Params &p, int b) {
   return n < 1 ? 1 : (n > p.max_pos ? p.max_pos : n);
 }
 
-// Tokens per attention chunk: a whole number of KV pages, sized so the
-// chunks of all (sequence, KV head) pairs number about one per CTA.
+// Tokens per attention chunk: a whole number of KV pages, sized so each KV
+// group's chunks over all sequences fit its block of slots (one partial
+// chunk per sequence is allowed for).
 __device__ int attn_span(const Params &p, int B) {
   const int P = p.page_size;
   int units = 0;
   for (int b = 0; b < B; ++b) units += (seq_len(p, b) + P - 1) / P;
-  units *= p.Hkv;
-  const int c = (units + p.attn_target - 1) / p.attn_target;
+  const int target = p.attn_spg - B;
+  const int c = (units + target - 1) / target;
   return (c < 1 ? 1 : c) * P;
 }
 
+// Slot s of a layer -> (sequence, KV head, token range).  Slots come in one
+// block per KV group; inside a block, the chunks of sequence 0, then 1, ...
 __device__ bool attn_resolve(const Params &p, int B, int s, Slot &o) {
   const int span = attn_span(p, B);
+  const int g = s / p.attn_spg;
+  const int r = s - g * p.attn_spg;
   int base = 0;
   for (int b = 0; b < B; ++b) {
     const int len = seq_len(p, b);
     const int nb = (len + span - 1) / span;
-    if (s < base + p.Hkv * nb) {
-      const int r = s - base;
+    if (r < base + nb) {
+      const int c = r - base;
       o.b = b;
-      o.g = r / nb;
-      const int c = r % nb;
+      o.g = g;
       o.t0 = c * span;
       o.t1 = min(len, o.t0 + span);
-      o.first_slot = base + o.g * nb;
+      o.first_slot = g * p.attn_spg + base;
       o.n_chunks = nb;
       return true;
     }
-    base += p.Hkv * nb;
+    base += nb;
   }
   o.b = -1;
   return false;

@@ -98,7 +98,12 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   const int R_o = std::min(rows_opt(1, 16 * choose_mtiles(H / 16, grid, mt_cap)), 16 * mt_cap);
   const int gu_cap = std::max(1, mt_cap / 2);   // gate and up tiles share a task
   const int R_gu = std::min(rows_opt(2, 16 * choose_mtiles(F / 16, grid, gu_cap)), 16 * gu_cap);
-  const int R_d = std::min(rows_opt(3, 16 * choose_mtiles(H / 16, grid, mt_cap)), 16 * mt_cap);
+  // a split down projection has a third or less of the columns per task:
+  // two row tiles per task keep its per-task costs (dependency check,
+  // restaging at each part) small against its pages
+  const bool ffn_split = F > std::max(H, Hq * d);
+  const int nm_d = std::max(choose_mtiles(H / 16, grid, mt_cap), ffn_split ? std::min(2, mt_cap) : 1);
+  const int R_d = std::min(rows_opt(3, 16 * nm_d), 16 * mt_cap);
   const int R_lm = std::min(rows_opt(4, 16 * choose_mtiles(V / 16, grid, mt_cap)), 16 * mt_cap);
 
   // ---- split-K of the down projection --------------------------------------------
@@ -119,6 +124,17 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     }
   }
   if (n_ksplit > 255) return lfail(err, MK_ERR_UNSUPPORTED, "ffn too wide for the split-K layout");
+
+  // ---- split-K of the O projection (option) ---------------------------------------------
+  // Two parts of whole KV groups: a part waits only for the attention of its
+  // groups, so the first part can stream while later groups still attend.
+  // Only where a part is at least 1024 columns wide (narrower parts make
+  // tasks too small to pay for their staging).  Off by default: on the 8B
+  // shape every group's attention ends within a few microseconds of the
+  // others, so the overlap does not pay for the extra tasks.
+  int o_groups = (o.o_split && Hkv >= 2) ? cdiv(Hkv, 2) : Hkv;
+  if (o_groups * G * d < 1024) o_groups = Hkv;
+  const int n_o_parts = cdiv(Hkv, o_groups);
 
   // ---- shared memory: activation staging and the weight-page ring ------------------
   // Activation staging holds fp32 rows of every sequence: a whole input when
@@ -146,7 +162,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
       return align_up_i(cdiv(K, cdiv(K, kpmax)), 32);
     };
     g.kp[K_HID] = page_cols(H);
-    g.kp[K_ATT] = page_cols(Hq * d);
+    g.kp[K_ATT] = page_cols(n_o_parts > 1 ? o_groups * G * d : Hq * d);
     g.kp[K_FFN] = page_cols(kchunk_ffn);
     g.kp[K_LM] = page_cols(H);
     const int kp_big = std::max(std::max(g.kp[0], g.kp[1]), g.kp[2]);
@@ -222,13 +238,20 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   p.out_stride = out_stride;
   p.off_x = off_x;
   p.off_pages = geo.off_pages;
-  p.attn_target = grid;
-  p.attn_slots = grid + maxB * Hkv;
+  // attention slots: a fixed block per KV group (so each group's completion
+  // is a static count), enough for about one chunk per CTA in all plus one
+  // partial chunk per sequence
+  p.attn_spg = cdiv(grid, Hkv) + maxB;
+  p.attn_slots = Hkv * p.attn_spg;
+  p.n_o_parts = n_o_parts;
+  p.o_groups = o_groups;
+  p.kchunk[K_ATT] = n_o_parts > 1 ? o_groups * G * d : 0;
   p.wait_limit_ns = o.wait_limit_ns;
   p.n_ffn_parts = n_ksplit;
   p.ev_embed = 0;
   p.ev_layer0 = 1;
-  p.ev_per_layer = Hkv + 3 + n_ksplit;   // attn_ready[Hkv], o_ready, oproj, gateup[parts], down
+  // attn_ready[Hkv], o_ready[O parts], oproj, gateup[down parts], down
+  p.ev_per_layer = Hkv + n_o_parts + 2 + n_ksplit;
   const int n_events = 1 + L * p.ev_per_layer;
 
   // ---- task graph -----------------------------------------------------------------------
@@ -287,15 +310,22 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
       t.type = T_ATTN;
       t.layer = static_cast<uint16_t>(l);
       t.dep_event = kNoEvent;  // resolved at run time: attn_ready(l, g)
-      t.out_event = ev_o_ready(p, l);
+      t.out_event = ev_o_ready(p, l, (s / p.attn_spg) / o_groups);
       t.aux = s;
       T.push_back(t);
     }
     out.ops.push_back({b0, static_cast<int>(T.size())});
     b0 = static_cast<int>(T.size());
-    for (int r0 = 0; r0 < H; r0 += R_o) {
-      const int nr = std::min(R_o, H - r0);
-      T.push_back(gemv(T_OPROJ, l, r0, nr, cdiv(nr, 16), ev_o_ready(p, l), p.attn_slots, ev_oproj(p, l)));
+    for (int k = 0; k < n_o_parts; ++k) {
+      const int groups = std::min(o_groups, Hkv - k * o_groups);
+      for (int r0 = 0; r0 < H; r0 += R_o) {
+        const int nr = std::min(R_o, H - r0);
+        Task t = gemv(T_OPROJ, l, r0, nr, cdiv(nr, 16), ev_o_ready(p, l, k),
+                      static_cast<uint32_t>(groups * p.attn_spg), ev_oproj(p, l));
+        t.ksplit = static_cast<uint8_t>(k);
+        t.nsplit = static_cast<uint8_t>(n_o_parts);
+        T.push_back(t);
+      }
     }
     out.ops.push_back({b0, static_cast<int>(T.size())});
     b0 = static_cast<int>(T.size());
@@ -352,7 +382,8 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   out.o_o = carve(sizeof(float) * maxB * Hq * d);
   out.o_u = carve(sizeof(float) * maxB * F);
   out.o_arg = carve(sizeof(unsigned long long) * maxB);
-  out.o_kpart = carve(sizeof(float) * static_cast<size_t>(n_ksplit > 1 ? n_ksplit : 0) * maxB * H);
+  const int kparts = std::max(n_ksplit > 1 ? n_ksplit : 0, n_o_parts > 1 ? n_o_parts : 0);
+  out.o_kpart = carve(sizeof(float) * static_cast<size_t>(kparts) * maxB * H);
   out.ws_bytes = off;
   out.n_events = n_events;
   out.head_words = static_cast<size_t>(L) * (Hq + 2 * Hkv);

@@ -68,7 +68,8 @@ class mk_kv_cache(C.Structure):
 class mk_plan_options(C.Structure):
     _fields_ = [("max_batch", C.c_int), ("kv_page_size", C.c_int), ("num_ctas", C.c_int),
                 ("wait_limit_ns", C.c_int64), ("rows_per_task", C.c_int * 5),
-                ("debug_unsatisfiable_dep", C.c_int), ("max_page_cols", C.c_int)]
+                ("debug_unsatisfiable_dep", C.c_int), ("max_page_cols", C.c_int),
+                ("o_split", C.c_int)]
 
 
 class mk_step_args(C.Structure):
@@ -167,7 +168,7 @@ class Plan:
     def __init__(self, cfg: Dict, weights: Dict, max_batch: int = 1, page_size: int = 16,
                  max_seq_len: int = 4096, num_ctas: int = 0, wait_limit_ns: int = 0,
                  rows_per_task: Sequence[int] = (0, 0, 0, 0, 0), debug_unsatisfiable_dep=False,
-                 max_page_cols: int = 0):
+                 max_page_cols: int = 0, o_split: bool = False):
         lib = load_library()
         self.cfg = dict(cfg)
         self.max_batch = max_batch
@@ -187,7 +188,7 @@ class Plan:
                              _ptr(weights["lm_head"]))
         opts = mk_plan_options(max_batch, page_size, num_ctas, wait_limit_ns,
                                (C.c_int * 5)(*rows_per_task), 1 if debug_unsatisfiable_dep else 0,
-                               max_page_cols)
+                               max_page_cols, 1 if o_split else 0)
         h = C.c_void_p()
         _check(lib.mk_plan_create_ex(C.byref(self._c), C.byref(self._w), C.byref(opts),
                                      C.byref(h)))

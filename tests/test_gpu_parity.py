@@ -58,7 +58,8 @@ SHAPES = {
 @pytest.mark.parametrize("name", sorted(SHAPES))
 def test_odd_shapes(cuda_device, name):
     cfg = SHAPES[name]
-    pair = Pair(cfg, _weights(cfg, seed=3, gain="random"), 1, [40])
+    pair = Pair(cfg, _weights(cfg, seed=3, gain="random"), 1, [40],
+                o_split=name.startswith("o_split"))
     ids = synth.make_ids(cfg["vocab"], (40,), seed=4).tolist()
     rep = StepReport()
     for t in range(40):
