@@ -54,7 +54,7 @@ struct alignas(16) Task {
   uint32_t dep_count; // completions of dep_event per step
   uint32_t out_event; // event incremented once the task's output is visible
   uint32_t aux;       // QKV: matrix (0 q, 1 k, 2 v); ATTN: slot index
-  uint32_t aux2;      // QKV: global head index; epilogue count in high 16 bits
+  uint32_t aux2;      // QKV: global head index (q heads, then k, then v)
 };
 static_assert(sizeof(Task) == 32, "task descriptor must be 32 bytes");
 constexpr uint32_t kNoEvent = 0xffffffffu;
@@ -88,13 +88,11 @@ struct Params {
   const float2 *rope_cs;        // [max_seq_len][d/2] (cos, sin)
   float *h;                     // [maxB][H]      residual stream
   float *qkv;                   // [maxB][NQKV]   raw projections
-  float *qrot;                  // [maxB][Hq][d]  q after norm + RoPE
   float *attn_part;             // [slots][G][d+4] chunk partials (acc, m, l, pad)
   float *o;                     // [maxB][Hq*d]   attention output
   float *u;                     // [maxB][F]      SwiGLU output
   unsigned long long *argmax;   // [maxB]         packed (value, ~index)
   uint32_t *sync;               // counters
-  uint32_t *head_ctr;           // [L][Hq+2Hkv]   QKV tasks done per head
   uint32_t *comb_ctr;           // [maxB][Hkv]    attention chunks done
 
   int L, H, Hq, Hkv, d, F, V, G, NQKV;
@@ -102,6 +100,7 @@ struct Params {
   int qk_norm;
   int max_batch, page_size, max_pos, num_kv_pages, max_pages_per_seq;
   int attn_slots, attn_spg, tpp;      // slots per layer, slots per KV group, tokens per smem page
+  int qkv_tasks_per_group;            // QKV tasks of one KV group's heads (G q + k + v)
   int kp[4];                          // page columns per op class
   int kchunk[4];                      // split-K columns per op class (0 = unsplit)
   float *kpart;                       // [splits][maxB][H] split-K partial sums
@@ -190,9 +189,9 @@ struct Layout {
   std::vector<OpRange> ops;
   std::vector<float2> rope;     // [max_seq_len][d/2] (cos, sin)
   // workspace byte offsets and size; counter words
-  size_t o_h = 0, o_qkv = 0, o_qrot = 0, o_part = 0, o_o = 0, o_u = 0, o_arg = 0, o_kpart = 0;
+  size_t o_h = 0, o_qkv = 0, o_part = 0, o_o = 0, o_u = 0, o_arg = 0, o_kpart = 0;
   size_t ws_bytes = 0;
-  size_t head_words = 0, comb_words = 0, tile_words = 0, sync_words = 0;
+  size_t comb_words = 0, tile_words = 0, sync_words = 0;
 };
 int validate_config(const mk_model_config &c, std::string &err);
 int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int smem_optin,

@@ -719,14 +719,71 @@ __device__ __forceinline__ void gemv_source(const Params &p, const Task &t, cons
   }
 }
 
+// RMSNorm gain blocks (8 bf16 each) a compute thread scales while staging:
+// column blocks ctid, ctid + kComputeThreads, ...  Gains are static weights,
+// so they are requested before the task waits for its input and arrive
+// during the wait.
+constexpr int kGainPre = 4;   // covers inputs up to 4 x 192 x 8 = 6144 columns
+struct GainPre {
+  uint4 g[kGainPre];
+};
+
+__device__ __forceinline__ void prefetch_gain(const __nv_bfloat16 *gain, int xc0, int xlen,
+                                              int ctid, GainPre &gp) {
+  const int nblk = xlen / 8;
+#pragma unroll
+  for (int j = 0; j < kGainPre; ++j) {
+    const int k = ctid + j * kComputeThreads;
+    gp.g[j] = (gain != nullptr && k < nblk)
+                  ? __ldg(reinterpret_cast<const uint4 *>(gain + xc0 + k * 8))
+                  : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// One staged 8-column block: 8 fp32 values -> [8 x bf16 hi | 8 x bf16 lo] of
+// x * g (hi + lo == x * g to ~2^-16), in place.  Returns the sum of squares of
+// the raw values (before the gain).
+__device__ __forceinline__ float stage_block(uint8_t *blk8, bool has_gain, uint4 gw) {
+  float4 *blk = reinterpret_cast<float4 *>(blk8);
+  const float4 x0 = blk[0], x1 = blk[1];
+  float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s += v[e] * v[e];
+  if (has_gain) {
+    const uint32_t gg[4] = {gw.x, gw.y, gw.z, gw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] *= bf_lo(gg[e]);
+      v[2 * e + 1] *= bf_hi(gg[e]);
+    }
+  }
+  uint32_t hw[4], lw[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat16 h0, l0, h1, l1;
+    split_bf16(v[2 * e], h0, l0);
+    split_bf16(v[2 * e + 1], h1, l1);
+    hw[e] = pack2(h0, h1);
+    lw[e] = pack2(l0, l1);
+  }
+  uint4 *o = reinterpret_cast<uint4 *>(blk8);
+  o[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  o[1] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  return s;
+}
+
 // Stage activation columns [xc0, xc0 + xlen) of every sequence in shared
-// memory as fp32 rows: the leader issues one bulk copy per sequence right
-// after the input event (one L2 round trip for the whole operand).  For
-// normed inputs each sequence's sum of squares over the chunk is added to
-// ss[b] by one warp in a fixed order; the RMSNorm scale is applied to the
-// task's outputs, since W (x * g * r) = r * W (x * g).
+// memory: the leader issues one bulk copy per sequence right after the input
+// event (one L2 round trip for the whole operand); then one parallel pass
+// turns each 8-column block into bf16 hi/lo of x * g and, for normed inputs,
+// adds each sequence's sum of squares over the chunk to ss[b] (per-warp
+// partials summed in warp order).  The RMSNorm scale is applied to the
+// task's outputs, since W (x * g * r) = r * W (x * g).  `gp`, when given,
+// holds this thread's gain blocks for the chunk.
 __device__ bool stage_x(const Params &p, Ctl *ctl, uint8_t *smem, const Task &t, int xc0,
-                        int xlen, int xpitch, int B, int ctid, ComputeState &st, bool first) {
+                        int xlen, int xpitch, int B, int ctid, ComputeState &st, bool first,
+                        const GainPre *gp) {
   const float *src;
   int stride;
   const __nv_bfloat16 *gain;
@@ -755,64 +812,38 @@ __device__ bool stage_x(const Params &p, Ctl *ctl, uint8_t *smem, const Task &t,
   mbar_try_wait(&ctl->xbar, st.x_par);
   st.x_par ^= 1u;
   const int warp = ctid >> 5, lane = ctid & 31;
-  if (gain != nullptr) {
-    // sum of squares of the raw rows (before the gain), one warp per sequence
-    for (int b = warp; b < B; b += kComputeWarps) {
-      const float4 *row = reinterpret_cast<const float4 *>(smem + p.off_x + b * xpitch);
-      float s = 0.f;
-      for (int i = lane; i < xlen / 4; i += 32) {
-        const float4 v = row[i];
-        s += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-      }
-      s = warp_sum(s);
-      if (lane == 0) ctl->ss[b] = (first ? 0.f : ctl->ss[b]) + s;
-    }
-    compute_bar();
-  }
-  // each thread turns whole 8-element blocks (32 bytes of fp32) into
-  // [8 x bf16 hi | 8 x bf16 lo] in place; blocks are independent
+  const bool has_gain = gain != nullptr;
   const int nblk = xlen / 8;
-  for (int i0 = ctid; i0 < B * nblk; i0 += 2 * kComputeThreads) {
-    float v[2][8];
-    uint4 gw[2];
+  for (int b = 0; b < B; ++b) {
+    uint8_t *row = smem + p.off_x + b * xpitch;
+    float s = 0.f;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int it = i0 + u * kComputeThreads;
-      if (it < B * nblk) {
-        const int b = it / nblk, k = it % nblk;
-        const float4 *blk = reinterpret_cast<const float4 *>(smem + p.off_x + b * xpitch + k * 32);
-        const float4 x0 = blk[0], x1 = blk[1];
-        v[u][0] = x0.x; v[u][1] = x0.y; v[u][2] = x0.z; v[u][3] = x0.w;
-        v[u][4] = x1.x; v[u][5] = x1.y; v[u][6] = x1.z; v[u][7] = x1.w;
-        if (gain != nullptr) gw[u] = __ldg(reinterpret_cast<const uint4 *>(gain + xc0 + k * 8));
+    for (int j = 0; j < kGainPre; ++j) {
+      const int k = ctid + j * kComputeThreads;
+      if (k < nblk) {
+        const uint4 gw = !has_gain ? make_uint4(0, 0, 0, 0)
+                         : gp != nullptr ? gp->g[j]
+                                         : __ldg(reinterpret_cast<const uint4 *>(gain + xc0 + k * 8));
+        s += stage_block(row + k * 32, has_gain, gw);
       }
     }
+    for (int k = ctid + kGainPre * kComputeThreads; k < nblk; k += kComputeThreads) {
+      const uint4 gw = has_gain ? __ldg(reinterpret_cast<const uint4 *>(gain + xc0 + k * 8))
+                                : make_uint4(0, 0, 0, 0);
+      s += stage_block(row + k * 32, has_gain, gw);
+    }
+    if (has_gain) {
+      s = warp_sum(s);
+      if (lane == 0) ctl->red8[warp][b] = s;
+    }
+  }
+  if (has_gain) {
+    compute_bar();
+    if (ctid < B) {
+      float s = 0.f;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int it = i0 + u * kComputeThreads;
-      if (it < B * nblk) {
-        const int b = it / nblk, k = it % nblk;
-        if (gain != nullptr) {
-          const uint32_t gg[4] = {gw[u].x, gw[u].y, gw[u].z, gw[u].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            v[u][2 * e] *= bf_lo(gg[e]);
-            v[u][2 * e + 1] *= bf_hi(gg[e]);
-          }
-        }
-        uint32_t hw[4], lw4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          __nv_bfloat16 h0, l0, h1, l1;
-          split_bf16(v[u][2 * e], h0, l0);
-          split_bf16(v[u][2 * e + 1], h1, l1);
-          hw[e] = pack2(h0, h1);
-          lw4[e] = pack2(l0, l1);
-        }
-        uint4 *blk = reinterpret_cast<uint4 *>(smem + p.off_x + b * xpitch + k * 32);
-        blk[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        blk[1] = make_uint4(lw4[0], lw4[1], lw4[2], lw4[3]);
-      }
+      for (int w = 0; w < kComputeWarps; ++w) s += ctl->red8[w][ctid];
+      ctl->ss[ctid] = (first ? 0.f : ctl->ss[ctid]) + s;
     }
   }
   compute_bar();
@@ -839,6 +870,9 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   int stride;
   const __nv_bfloat16 *gain;
   gemv_source(p, t, src, stride, gain);
+  const bool restage = !(geo.whole && st.xkey == key);
+  GainPre gp;
+  if (gain != nullptr && restage) prefetch_gain(gain, geo.k0, min(geo.kx, geo.Kt), ctid, gp);
 
   if (!S.dep_ok && (t.dep_event != st.sat_ev || t.dep_count != st.sat_cnt)) {
     bool okl = true;
@@ -861,7 +895,12 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   for (int xc0 = geo.k0; xc0 < geo.k0 + geo.Kt; xc0 += geo.kx) {
     const int xend = min(geo.k0 + geo.Kt, xc0 + geo.kx);
     if (!(geo.whole && st.xkey == key)) {
-      if (!stage_x(p, ctl, smem, t, xc0, xend - xc0, xstride * 4, B, ctid, st, xc0 == geo.k0))
+      // a later chunk overwrites the staging area: every compute warp must be
+      // done with the previous chunk's pages (warps move through the pages
+      // independently)
+      if (xc0 != geo.k0) compute_bar();
+      if (!stage_x(p, ctl, smem, t, xc0, xend - xc0, xstride * 4, B, ctid, st, xc0 == geo.k0,
+                   (gain != nullptr && xc0 == geo.k0) ? &gp : nullptr))
         return false;
       st.xkey = geo.whole ? key : 0xffffffffu;
     }
@@ -961,6 +1000,51 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
 // compute warps: attention over one chunk of one (sequence, KV head)
 // ============================================================================
 
+// One head of raw projection values (fp32, d elements at src): optionally an
+// RMSNorm over d times `gain`, then optionally RoPE with the table row `cs`
+// (pairs (i, i + d/2)).  Lane l < d/4 returns elements 4l..4l+3; the RoPE
+// partner of element i sits d/8 lanes away and is fetched by shuffle.  All
+// 32 lanes must call it.
+template <int D>
+__device__ __forceinline__ void head_norm_rope(const float *src, const __nv_bfloat16 *gain,
+                                               bool norm, bool rope, const float2 *cs, float eps,
+                                               int lane, float (&v)[4]) {
+  constexpr int half = D / 2, xo = D / 8;
+  const bool active = lane < D / 4;
+  const int e0 = lane * 4;
+  float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (active) y = __ldcg(reinterpret_cast<const float4 *>(src + e0));
+  v[0] = y.x; v[1] = y.y; v[2] = y.z; v[3] = y.w;
+  if (norm) {
+    float g4[4] = {1.f, 1.f, 1.f, 1.f};
+    if (active) {
+      const uint2 gw = *reinterpret_cast<const uint2 *>(gain + e0);
+      g4[0] = bf_lo(gw.x); g4[1] = bf_hi(gw.x); g4[2] = bf_lo(gw.y); g4[3] = bf_hi(gw.y);
+    }
+    const float s = warp_sum(v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3]);
+    const float rs = 1.0f / sqrtf(s / static_cast<float>(D) + eps);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = v[k] * rs * g4[k];
+  }
+  if (rope) {
+    const bool first_half = e0 < half;
+    const int pair0 = first_half ? e0 : e0 - half;
+    float2 c[4] = {make_float2(1.f, 0.f), make_float2(1.f, 0.f), make_float2(1.f, 0.f),
+                   make_float2(1.f, 0.f)};
+    if (active) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) c[k] = cs[pair0 + k];
+    }
+    float w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w[k] = __shfl_xor_sync(0xffffffffu, v[k], xo);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      // first half: (a, c) = (v, w) -> a cos - c sin; second half: c cos + a sin
+      v[k] = first_half ? v[k] * c[k].x - w[k] * c[k].y : v[k] * c[k].x + w[k] * c[k].y;
+  }
+}
+
 // Attention for one chunk of one (sequence, KV head): scores for the G query
 // heads over the chunk's tokens, softmax statistics, and the unnormalised
 // P.V, all in three parallel phases per shared-memory page:
@@ -985,18 +1069,58 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   float *mst = sc + G * p.tpp;                              // [G] running max
   float *lst = mst + kMaxGroup;                             // [G] running sum
   float *cor = lst + kMaxGroup;                             // [G] rescale of this page
+  __nv_bfloat16 *kvcur = reinterpret_cast<__nv_bfloat16 *>(cor + kMaxGroup);  // [2][D] K, V at pos
   st.xkey = 0xffffffffu;                                    // staging area reused
 
   {
     const uint32_t ev = static_cast<uint32_t>(ev_attn_ready(p, l, g));
     bool okl = true;
-    if (ctid == 0) okl = wait_event(p, ctl, ev, static_cast<uint32_t>(G + 2), S.idx);
+    if (ctid == 0) okl = wait_event(p, ctl, ev, static_cast<uint32_t>(p.qkv_tasks_per_group), S.idx);
     if (!st.gs.share(ctl, ctid, okl)) return false;
     if (ctid == 0) trace_mark(p, S.idx, 4);
   }
-  const float qscale = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;
-  for (int i = ctid; i < G * D; i += kComputeThreads)
-    qs[i] = __ldcg(p.qrot + (static_cast<size_t>(b) * p.Hq + g * G) * D + i) * qscale;
+  // From this step's raw projections, one warp per head: the G query heads
+  // (QK-norm, RoPE, pre-scaled by log2(e)/sqrt(d) for the exp2 softmax) and,
+  // in the chunk that holds the current position, K (QK-norm, RoPE) and V of
+  // the current token, rounded to bf16 and appended to the cache.
+  const int P = p.page_size;
+  const int cur = p.pos[b];
+  const bool own_cur = cur >= S.t0 && cur < S.t1;
+  {
+    const float qscale = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;
+    const LayerW &lw = p.layers[l];
+    // a position outside 0..max_pos-1 is reported by the embedding task; the
+    // table row stays in range regardless
+    const int cpos = cur < 0 ? 0 : (cur >= p.max_pos ? p.max_pos - 1 : cur);
+    const float2 *cs = p.rope_cs + static_cast<size_t>(cpos) * (D / 2);
+    const float *raw = p.qkv + static_cast<size_t>(b) * p.NQKV;
+    const int nh = G + (own_cur ? 2 : 0);
+    for (int h = warp; h < nh; h += kComputeWarps) {
+      const int mat = h < G ? 0 : h - G + 1;   // 0 q, 1 k, 2 v
+      const int col = mat == 0 ? (g * G + h) * D
+                               : (mat == 1 ? (p.Hq + g) * D : (p.Hq + p.Hkv + g) * D);
+      float v[4];
+      head_norm_rope<D>(raw + col, mat == 0 ? lw.q_norm : lw.k_norm, p.qk_norm != 0 && mat != 2,
+                        mat != 2, cs, p.eps, lane, v);
+      if (lane < D / 4) {
+        const int e0 = lane * 4;
+        if (mat == 0) {
+          *reinterpret_cast<float4 *>(qs + h * D + e0) =
+              make_float4(v[0] * qscale, v[1] * qscale, v[2] * qscale, v[3] * qscale);
+        } else {
+          const uint2 pk = make_uint2(pack2(__float2bfloat16_rn(v[0]), __float2bfloat16_rn(v[1])),
+                                      pack2(__float2bfloat16_rn(v[2]), __float2bfloat16_rn(v[3])));
+          *reinterpret_cast<uint2 *>(kvcur + (mat - 1) * D + e0) = pk;
+          const int ph = kv_phys_page(p, b, cur / P);
+          if (ph >= 0) {
+            __nv_bfloat16 *dst = (mat == 1 ? p.k_pages[l] : p.v_pages[l]) +
+                                 ((static_cast<size_t>(ph) * p.Hkv + g) * P + cur % P) * D + e0;
+            *reinterpret_cast<uint2 *>(dst) = pk;
+          }
+        }
+      }
+    }
+  }
   if (ctid < G) {
     mst[ctid] = -INFINITY;
     lst[ctid] = 0.f;
@@ -1008,8 +1132,6 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
 #pragma unroll
   for (int k = 0; k < MAXP; ++k) acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
 
-  const int P = p.page_size;
-  const int cur = p.pos[b];
   for (int tok0 = S.t0; tok0 < S.t1; tok0 += p.tpp) {
     const int ntok = min(p.tpp, S.t1 - tok0);
     bool okl = true;
@@ -1018,18 +1140,16 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     mbar_try_wait(&ctl->full[st.pi], st.pg_par);
     uint8_t *kpg = smem + p.off_pages + static_cast<size_t>(st.pi) * p.page_bytes;
     uint8_t *vpg = kpg + static_cast<size_t>(p.tpp) * D * 2;
-    // The current token's K/V were appended by this step's QKV epilogue and
-    // may have been copied into the page before they landed: reload them.
+    // The page was copied from the cache before this step's K/V of the
+    // current token were formed: put them into its slot.
     const bool has_cur = cur >= tok0 && cur < tok0 + ntok;
     if (has_cur) {
-      const int ph = kv_phys_page(p, b, cur / P);
-      const size_t src = ((static_cast<size_t>(ph < 0 ? 0 : ph) * p.Hkv + g) * P + cur % P) * D;
       const int j = cur - tok0;
       if (ctid < 2 * NB) {
         const bool isv = ctid >= NB;
         const int e = (isv ? ctid - NB : ctid) * 8;
-        const uint4 v = __ldcg(reinterpret_cast<const uint4 *>((isv ? p.v_pages[l] : p.k_pages[l]) + src + e));
-        *reinterpret_cast<uint4 *>((isv ? vpg : kpg) + (j * D + e) * 2) = v;
+        *reinterpret_cast<uint4 *>((isv ? vpg : kpg) + (j * D + e) * 2) =
+            *reinterpret_cast<const uint4 *>(kvcur + (isv ? D : 0) + e);
       }
       compute_bar();
     }
@@ -1296,76 +1416,6 @@ __device__ __forceinline__ void signal(const Params &p, uint32_t ev) {
   red_add_release(p.sync + S_EVENTS + ev, 1u);
 }
 
-// QK-norm + RoPE of one head for every sequence, then K/V append or q store.
-// Lane l holds elements 4l..4l+3 of the head (d/4 active lanes); the RoPE
-// partner of element i (i + d/2) sits d/8 lanes away, fetched by shuffle.
-// All loads of a sequence are issued before any is used.
-__device__ void rope_head(const Params &p, const Task &t, int lane) {
-  const int d = p.d, half = d / 2, l = t.layer, B = p.batch;
-  const int mat = static_cast<int>(t.aux);
-  const int head = static_cast<int>(t.aux2 & 0xffffu);
-  const int local = mat == 0 ? head : (mat == 1 ? head - p.Hq : head - p.Hq - p.Hkv);
-  const int col0 = head * d;  // rows of q, then k, then v are contiguous in qkv
-  const LayerW &lw = p.layers[l];
-  const bool active = lane < d / 4;
-  const int e0 = lane * 4;                         // first element held
-  const bool first_half = e0 < half;
-  const int pair0 = first_half ? e0 : e0 - half;   // RoPE pair index
-  const int xo = d / 8;                            // lane distance to the partner
-  const __nv_bfloat16 *gain = mat == 0 ? lw.q_norm : lw.k_norm;
-  for (int b = 0; b < B; ++b) {
-    const int pos = p.pos[b];
-    if (pos < 0 || pos >= p.max_pos) continue;  // reported by the embedding task
-    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-    float g4[4] = {1.f, 1.f, 1.f, 1.f};
-    float2 cs[4];
-    if (active) {
-      y = __ldcg(reinterpret_cast<const float4 *>(p.qkv + static_cast<size_t>(b) * p.NQKV + col0 + e0));
-      if (mat != 2) {
-        if (p.qk_norm) {
-          const uint2 gw = *reinterpret_cast<const uint2 *>(gain + e0);
-          g4[0] = bf_lo(gw.x); g4[1] = bf_hi(gw.x); g4[2] = bf_lo(gw.y); g4[3] = bf_hi(gw.y);
-        }
-        const float2 *tab = p.rope_cs + static_cast<size_t>(pos) * half + pair0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) cs[k] = tab[k];
-      }
-    }
-    float v[4] = {y.x, y.y, y.z, y.w};
-    if (mat != 2) {
-      float rs = 1.f;
-      if (p.qk_norm) {
-        float s = v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
-        s = warp_sum(s);
-        rs = 1.0f / sqrtf(s / static_cast<float>(d) + p.eps);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = v[k] * rs * g4[k];
-      }
-      float w[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) w[k] = __shfl_xor_sync(0xffffffffu, v[k], xo);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        // first half: (a, c) = (v, w) -> a cos - c sin; second half: c cos + a sin
-        v[k] = first_half ? v[k] * cs[k].x - w[k] * cs[k].y : v[k] * cs[k].x + w[k] * cs[k].y;
-      }
-    }
-    if (!active) continue;
-    if (mat == 0) {
-      float *q = p.qrot + (static_cast<size_t>(b) * p.Hq + local) * d + e0;
-      __stcg(reinterpret_cast<float4 *>(q), make_float4(v[0], v[1], v[2], v[3]));
-    } else {
-      const int ph = kv_phys_page(p, b, pos / p.page_size);
-      if (ph < 0) continue;
-      __nv_bfloat16 *dst = (mat == 1 ? p.k_pages[l] : p.v_pages[l]) +
-                           ((static_cast<size_t>(ph) * p.Hkv + local) * p.page_size +
-                            pos % p.page_size) * d + e0;
-      const uint2 pk = make_uint2(pack2(__float2bfloat16_rn(v[0]), __float2bfloat16_rn(v[1])),
-                                  pack2(__float2bfloat16_rn(v[2]), __float2bfloat16_rn(v[3])));
-      *reinterpret_cast<uint2 *>(dst) = pk;
-    }
-  }
-}
 
 __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
   uint32_t u = __float_as_uint(v);
@@ -1389,25 +1439,17 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
       break;
     }
     case T_QKV: {
+      // raw projection rows; QK-norm, RoPE and the KV append happen in the
+      // attention tasks of the head's KV group
       const int base = t.aux == 0 ? 0 : (t.aux == 1 ? p.Hq * p.d : (p.Hq + p.Hkv) * p.d);
       for (int b = 0; b < B; ++b)
         for (int r = lane; r < static_cast<int>(t.nrows); r += 32)
           __stcg(p.qkv + static_cast<size_t>(b) * p.NQKV + base + t.row0 + r, out[b * OS + r]);
       __syncwarp();
-      const int head = static_cast<int>(t.aux2 & 0xffffu);
-      const uint32_t need = t.aux2 >> 16;
-      uint32_t old = 0;
-      if (lane == 0) old = atom_add_acq_rel(p.head_ctr + t.layer * (p.Hq + 2 * p.Hkv) + head, 1u);
-      old = __shfl_sync(0xffffffffu, old, 0);
-      if (old + 1u == need) {
-        __syncwarp();
-        rope_head(p, t, lane);
-        __syncwarp();
-        if (lane == 0) {
-          p.head_ctr[t.layer * (p.Hq + 2 * p.Hkv) + head] = 0u;
-          const int g = t.aux == 0 ? head / p.G : (t.aux == 1 ? head - p.Hq : head - p.Hq - p.Hkv);
-          signal(p, static_cast<uint32_t>(ev_attn_ready(p, t.layer, g)));
-        }
+      if (lane == 0) {
+        const int head = static_cast<int>(t.aux2);
+        const int g = t.aux == 0 ? head / p.G : (t.aux == 1 ? head - p.Hq : head - p.Hq - p.Hkv);
+        signal(p, static_cast<uint32_t>(ev_attn_ready(p, t.layer, g)));
       }
       break;
     }

@@ -178,9 +178,10 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     }
     g.tpp = std::min(tpp, 16 * P);
     // attention scratch in the staging area: q [G][d] plus either the page's
-    // scores [G][tpp] and per-head statistics, or the combine's per-chunk
-    // (m, l) pairs
-    const int att_need = G * d * 4 + std::max(G * g.tpp + 3 * kMaxGroup, 2 * max_chunks * G + 2 * G) * 4;
+    // scores [G][tpp], per-head statistics and the current token's K and V
+    // (bf16), or the combine's per-chunk (m, l) pairs
+    const int att_need = G * d * 4 + std::max((G * g.tpp + 3 * kMaxGroup) * 4 + 2 * d * 2,
+                                              (2 * max_chunks * G + 2 * G) * 4);
     g.x_cap = std::max(x_cap, att_need);
     g.off_pages = align_up_i(off_x + g.x_cap, 1024);
     g.n_pages = std::min(kMaxPages, (smem_max - g.off_pages) / g.page_bytes);
@@ -272,6 +273,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     return t;
   };
   const int n_o = cdiv(H, R_o), n_down = cdiv(H, R_d), n_lm = cdiv(V, R_lm);
+  p.qkv_tasks_per_group = (G + 2) * (d / R_qkv);
   // gate/up tasks per split-K part of the down projection
   std::vector<uint32_t> gu_per_part(n_ksplit, 0);
   for (int r0 = 0; r0 < F; r0 += R_gu) gu_per_part[n_ksplit > 1 ? r0 / kchunk_ffn : 0] += 1;
@@ -290,7 +292,6 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     // in KV-group order (the G query heads, then the K and V heads of group
     // 0, then group 1, ...), so each group's attention can start while the
     // later groups are still being projected
-    const int per_head = d / R_qkv;
     for (int kvg = 0; kvg < Hkv; ++kvg)
       for (int j = 0; j < G + 2; ++j) {
         const int mat = j < G ? 0 : j - G + 1;          // 0 q, 1 k, 2 v
@@ -299,7 +300,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
         for (int r0 = 0; r0 < d; r0 += R_qkv) {
           Task t = gemv(T_QKV, l, hh * d + r0, R_qkv, R_qkv / 16, dep, cnt, kNoEvent);
           t.aux = mat;
-          t.aux2 = static_cast<uint32_t>(head) | (static_cast<uint32_t>(per_head) << 16);
+          t.aux2 = static_cast<uint32_t>(head);
           T.push_back(t);
         }
       }
@@ -377,7 +378,6 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   };
   out.o_h = carve(sizeof(float) * maxB * H);
   out.o_qkv = carve(sizeof(float) * maxB * NQKV);
-  out.o_qrot = carve(sizeof(float) * maxB * Hq * d);
   out.o_part = carve(sizeof(float) * static_cast<size_t>(p.attn_slots) * G * (d + 4));
   out.o_o = carve(sizeof(float) * maxB * Hq * d);
   out.o_u = carve(sizeof(float) * maxB * F);
@@ -386,10 +386,9 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   out.o_kpart = carve(sizeof(float) * static_cast<size_t>(kparts) * maxB * H);
   out.ws_bytes = off;
   out.n_events = n_events;
-  out.head_words = static_cast<size_t>(L) * (Hq + 2 * Hkv);
   out.comb_words = static_cast<size_t>(maxB) * Hkv;
   out.tile_words = static_cast<size_t>(H) / 16 + 1;
-  out.sync_words = S_EVENTS + n_events + out.head_words + out.comb_words + out.tile_words;
+  out.sync_words = S_EVENTS + n_events + out.comb_words + out.tile_words;
 
   out.grid = grid;
   out.smem = smem;
@@ -404,15 +403,13 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
 void bind_workspace(const Layout &lay, char *ws, uint32_t *sync, Params &p) {
   p.h = reinterpret_cast<float *>(ws + lay.o_h);
   p.qkv = reinterpret_cast<float *>(ws + lay.o_qkv);
-  p.qrot = reinterpret_cast<float *>(ws + lay.o_qrot);
   p.attn_part = reinterpret_cast<float *>(ws + lay.o_part);
   p.o = reinterpret_cast<float *>(ws + lay.o_o);
   p.u = reinterpret_cast<float *>(ws + lay.o_u);
   p.argmax = reinterpret_cast<unsigned long long *>(ws + lay.o_arg);
   p.kpart = reinterpret_cast<float *>(ws + lay.o_kpart);
   p.sync = sync;
-  p.head_ctr = sync + S_EVENTS + lay.n_events;
-  p.comb_ctr = p.head_ctr + lay.head_words;
+  p.comb_ctr = sync + S_EVENTS + lay.n_events;
   p.tile_ctr = p.comb_ctr + lay.comb_words;
 }
 
