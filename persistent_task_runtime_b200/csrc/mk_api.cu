@@ -56,7 +56,7 @@ struct mk_plan {
   int max_batch = 1;
   uint32_t epoch = 0;
   mk::Layout lay;           // tasks, per-operator ranges, workspace layout
-  void *d_tasks = nullptr, *d_layers = nullptr, *d_rope = nullptr, *d_ws = nullptr;
+  void *d_tasks = nullptr, *d_rope = nullptr, *d_ws = nullptr;
   uint32_t *d_sync = nullptr;
   size_t sync_words = 0;
   int32_t *d_host_ids = nullptr, *d_host_pos = nullptr, *d_host_out = nullptr;
@@ -157,9 +157,8 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
     if (e != cudaSuccess) return fail(MK_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
     return MK_OK;
   };
-  const std::vector<mk::LayerW> lw = mk::layer_table(*cfg, *w);
+  mk::bind_task_operands(*cfg, *w, lay.tasks);
   if ((rc = upload(&plan->d_tasks, lay.tasks.data(), lay.tasks.size() * sizeof(Task), "task array")) ||
-      (rc = upload(&plan->d_layers, lw.data(), lw.size() * sizeof(mk::LayerW), "weight table")) ||
       (rc = upload(&plan->d_rope, lay.rope.data(), lay.rope.size() * sizeof(float2), "RoPE table")))
     return cleanup_fail(rc);
   cudaError_t e = cudaMalloc(&plan->d_ws, lay.ws_bytes);
@@ -171,7 +170,6 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   plan->sync_words = lay.sync_words;
   mk::bind_workspace(lay, static_cast<char *>(plan->d_ws), plan->d_sync, p);
   p.tasks = static_cast<const Task *>(plan->d_tasks);
-  p.layers = static_cast<const mk::LayerW *>(plan->d_layers);
   p.embed = static_cast<const __nv_bfloat16 *>(w->embed);
   p.final_norm = static_cast<const __nv_bfloat16 *>(w->final_norm);
   p.lm_head = static_cast<const __nv_bfloat16 *>(w->lm_head);
@@ -365,7 +363,6 @@ void mk_plan_destroy(mk_plan *plan) {
   if (plan == nullptr) return;
   cudaDeviceSynchronize();
   cudaFree(plan->d_tasks);
-  cudaFree(plan->d_layers);
   cudaFree(plan->d_rope);
   cudaFree(plan->d_ws);
   cudaFree(plan->d_sync);

@@ -23,6 +23,8 @@ constexpr int kStorerWarp = 1 + kComputeWarps;    // epilogues + signalling
 constexpr int kThreads = 32 * (kComputeWarps + 2);
 constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kTaskSlots = 4;                     // tasks in flight per CTA
+constexpr int kSlotBytes = 96;                    // one task slot in shared memory
+constexpr int kLookBytes = 512;                   // loader lookahead area
 constexpr int kOutSlots = 4;                      // compute -> storer buffers
 constexpr int kMaxPages = 16;                     // ring entries (upper bound)
 constexpr int kMaxMTiles = 8;                     // 16-row tiles per GEMV task (B <= 4)
@@ -30,7 +32,7 @@ constexpr int kMaxPageCols = 2048;                // widest weight page (16 rows
 constexpr int kMaxGroup = 8;                      // query heads per KV head
 constexpr int kMaxSmem = 232448;                  // opt-in smem per CTA (B200)
 
-// ---- task descriptor (32 bytes, two 16-byte loads) ----------------------------
+// ---- task descriptor (64 bytes, four 16-byte loads) ---------------------------
 enum TaskType : uint8_t {
   T_EMBED = 1,
   T_QKV = 2,
@@ -55,15 +57,14 @@ struct alignas(16) Task {
   uint32_t out_event; // event incremented once the task's output is visible
   uint32_t aux;       // QKV: matrix (0 q, 1 k, 2 v); ATTN: slot index
   uint32_t aux2;      // QKV: global head index (q heads, then k, then v)
+  // operands, filled in by the plan so that no task looks up a layer table:
+  const __nv_bfloat16 *w0;    // GEMV: the weight matrix (gate/up: gate); ATTN: q-norm gain
+  const __nv_bfloat16 *w1;    // gate/up: the up matrix; ATTN: k-norm gain
+  const __nv_bfloat16 *gain;  // RMSNorm gain of the task's input (QKV, gate/up, LM head)
+  uint64_t pad;
 };
-static_assert(sizeof(Task) == 32, "task descriptor must be 32 bytes");
+static_assert(sizeof(Task) == 64, "task descriptor must be 64 bytes");
 constexpr uint32_t kNoEvent = 0xffffffffu;
-
-// ---- per-layer weight pointers (device table) ------------------------------
-struct LayerW {
-  const __nv_bfloat16 *attn_norm, *wq, *wk, *wv, *q_norm, *k_norm, *wo,
-      *mlp_norm, *w_gate, *w_up, *w_down;
-};
 
 // ---- counters region (uint32 words) ----------------------------------------
 enum SyncWord : int {
@@ -83,7 +84,6 @@ enum OpK : int { K_HID = 0, K_ATT = 1, K_FFN = 2, K_LM = 3 };
 struct Params {
   // plan (static)
   const Task *tasks;
-  const LayerW *layers;
   const __nv_bfloat16 *embed, *final_norm, *lm_head;
   const float2 *rope_cs;        // [max_seq_len][d/2] (cos, sin)
   float *h;                     // [maxB][H]      residual stream
@@ -197,7 +197,8 @@ int validate_config(const mk_model_config &c, std::string &err);
 int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int smem_optin,
                  Layout &out, std::string &err);
 void bind_workspace(const Layout &lay, char *ws, uint32_t *sync, Params &p);
-std::vector<LayerW> layer_table(const mk_model_config &c, const mk_weights &w);
+// Fill every task's operand pointers (weights, norm gains) from `w`.
+void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vector<Task> &tasks);
 
 cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative,
                         cudaStream_t stream);

@@ -214,7 +214,7 @@ struct Slot {
   int idx;                   // task index (for error reports)
   int dep_ok;                // the loader saw the input event complete
 };
-static_assert(sizeof(Slot) == 64, "slot must be 64 bytes");
+static_assert(sizeof(Slot) == kSlotBytes, "slot size");
 
 // ============================================================================
 // errors and bounded waits
@@ -343,21 +343,13 @@ __device__ Geo gemv_geo(const Params &p, const Task &t, int B) {
 // Row `m`-tile of a GEMV task: weight matrix base, first row, valid rows.
 __device__ __forceinline__ void gemv_tile(const Params &p, const Task &t, int m,
                                           const __nv_bfloat16 *&W, int &row, int &rows_valid) {
-  const LayerW &lw = p.layers[t.layer < p.L ? t.layer : 0];
   int mm = m;
-  switch (t.type) {
-    case T_QKV: W = t.aux == 0 ? lw.wq : (t.aux == 1 ? lw.wk : lw.wv); break;
-    case T_OPROJ: W = lw.wo; break;
-    case T_DOWN: W = lw.w_down; break;
-    case T_LMHEAD: W = p.lm_head; break;
-    default: {  // gate/up: first half of the tiles read w_gate, second w_up
-      const int nh = t.n_m >> 1;
-      if (m < nh) {
-        W = lw.w_gate;
-      } else {
-        W = lw.w_up;
-        mm = m - nh;
-      }
+  W = t.w0;
+  if (t.type == T_GATEUP) {  // first half of the tiles read w_gate, second w_up
+    const int nh = t.n_m >> 1;
+    if (m >= nh) {
+      W = t.w1;
+      mm = m - nh;
     }
   }
   row = static_cast<int>(t.row0) + 16 * mm;
@@ -428,13 +420,13 @@ __device__ __forceinline__ bool is_gemv(uint8_t type) {
 }
 
 // Tasks popped from the queue but not yet handed to the compute warps.
-constexpr int kLook = 8;
 struct Look {
   Task t;
   int tix;
   int pad[3];
 };
-static_assert(sizeof(Look) == 48, "lookahead entry size");
+constexpr int kLook = kLookBytes / static_cast<int>(sizeof(Look));
+static_assert(sizeof(Look) == 80 && kLook >= 2, "lookahead entry size");
 
 __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   const int lane = threadIdx.x & 31;
@@ -708,12 +700,11 @@ struct ComputeState {
 // normed inputs (QKV, gate/up, LM head read the residual stream h).
 __device__ __forceinline__ void gemv_source(const Params &p, const Task &t, const float *&src,
                                             int &stride, const __nv_bfloat16 *&gain) {
-  const LayerW &lw = p.layers[t.layer < p.L ? t.layer : 0];
-  gain = nullptr;
+  gain = t.gain;
   switch (t.type) {
-    case T_QKV: src = p.h; gain = lw.attn_norm; stride = p.H; break;
-    case T_GATEUP: src = p.h; gain = lw.mlp_norm; stride = p.H; break;
-    case T_LMHEAD: src = p.h; gain = p.final_norm; stride = p.H; break;
+    case T_QKV:
+    case T_GATEUP:
+    case T_LMHEAD: src = p.h; stride = p.H; break;
     case T_OPROJ: src = p.o; stride = p.Hq * p.d; break;
     default: src = p.u; stride = p.F; break;
   }
@@ -1088,7 +1079,6 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   const bool own_cur = cur >= S.t0 && cur < S.t1;
   {
     const float qscale = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;
-    const LayerW &lw = p.layers[l];
     // a position outside 0..max_pos-1 is reported by the embedding task; the
     // table row stays in range regardless
     const int cpos = cur < 0 ? 0 : (cur >= p.max_pos ? p.max_pos - 1 : cur);
@@ -1100,7 +1090,7 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
       const int col = mat == 0 ? (g * G + h) * D
                                : (mat == 1 ? (p.Hq + g) * D : (p.Hq + p.Hkv + g) * D);
       float v[4];
-      head_norm_rope<D>(raw + col, mat == 0 ? lw.q_norm : lw.k_norm, p.qk_norm != 0 && mat != 2,
+      head_norm_rope<D>(raw + col, mat == 0 ? t.w0 : t.w1, p.qk_norm != 0 && mat != 2,
                         mat != 2, cs, p.eps, lane, v);
       if (lane < D / 4) {
         const int e0 = lane * 4;

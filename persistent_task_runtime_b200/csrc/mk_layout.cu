@@ -145,9 +145,9 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   const int red_bytes = kComputeWarps * 16 * 8 * n_tiles_for(maxB) * 4;
   const int out_stride = 16 * mt_cap;
   const int out_bytes = align_up_i(maxB * out_stride * 4, 128);
-  const int off_look = 1024;   // loader lookahead (8 x 48 B)
-  const int off_slots = off_look + 512;
-  const int off_red = align_up_i(off_slots + kTaskSlots * 64, 128);
+  const int off_look = 1024;   // loader lookahead
+  const int off_slots = off_look + kLookBytes;
+  const int off_red = align_up_i(off_slots + kTaskSlots * kSlotBytes, 128);
   const int off_out = align_up_i(off_red + red_bytes, 128);
   const int off_x = align_up_i(off_out + kOutSlots * out_bytes, 128);
 
@@ -413,15 +413,36 @@ void bind_workspace(const Layout &lay, char *ws, uint32_t *sync, Params &p) {
   p.tile_ctr = p.comb_ctr + lay.comb_words;
 }
 
-std::vector<LayerW> layer_table(const mk_model_config &c, const mk_weights &w) {
-  std::vector<LayerW> lw(c.n_layers);
+void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vector<Task> &tasks) {
   auto bf = [](const void *q) { return static_cast<const __nv_bfloat16 *>(q); };
-  for (int l = 0; l < c.n_layers; ++l) {
-    const mk_layer_weights &s = w.layers[l];
-    lw[l] = {bf(s.attn_norm), bf(s.wq), bf(s.wk), bf(s.wv), bf(s.q_norm), bf(s.k_norm),
-             bf(s.wo), bf(s.mlp_norm), bf(s.w_gate), bf(s.w_up), bf(s.w_down)};
+  for (Task &t : tasks) {
+    t.w0 = t.w1 = t.gain = nullptr;
+    if (t.type == T_EMBED || t.type == T_END) continue;
+    if (t.type == T_LMHEAD) {
+      t.w0 = bf(w.lm_head);
+      t.gain = bf(w.final_norm);
+      continue;
+    }
+    const mk_layer_weights &lw = w.layers[t.layer < c.n_layers ? t.layer : 0];
+    switch (t.type) {
+      case T_QKV:
+        t.w0 = bf(t.aux == 0 ? lw.wq : (t.aux == 1 ? lw.wk : lw.wv));
+        t.gain = bf(lw.attn_norm);
+        break;
+      case T_ATTN:
+        t.w0 = bf(lw.q_norm);
+        t.w1 = bf(lw.k_norm);
+        break;
+      case T_OPROJ: t.w0 = bf(lw.wo); break;
+      case T_GATEUP:
+        t.w0 = bf(lw.w_gate);
+        t.w1 = bf(lw.w_up);
+        t.gain = bf(lw.mlp_norm);
+        break;
+      case T_DOWN: t.w0 = bf(lw.w_down); break;
+      default: break;
+    }
   }
-  return lw;
 }
 
 }  // namespace mk

@@ -104,7 +104,7 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
   if (rc) return nfail(rc, err.c_str());
   Params p = lay.p;
   const int grid = lay.grid, smem = lay.smem;
-  const std::vector<mk::LayerW> lw = mk::layer_table(c, *w);
+  mk::bind_task_operands(c, *w, lay.tasks);
 
   // ---- layout inside the static array -------------------------------------
   size_t off = 0;
@@ -114,7 +114,6 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
     return at;
   };
   const size_t o_tasks = carve(lay.tasks.size() * sizeof(Task));
-  const size_t o_layers = carve(L * sizeof(mk::LayerW));
   const size_t o_rope = carve(lay.rope.size() * sizeof(float2));
   const size_t o_ws = carve(lay.ws_bytes);
   const size_t o_sync = carve(lay.sync_words * sizeof(uint32_t));
@@ -149,8 +148,6 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemcpyAsync(base + o_tasks, lay.tasks.data(), lay.tasks.size() * sizeof(Task),
                       cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(base + o_layers, lw.data(), L * sizeof(mk::LayerW), cudaMemcpyHostToDevice,
-                      s) != cudaSuccess ||
       cudaMemcpyAsync(base + o_rope, lay.rope.data(), lay.rope.size() * sizeof(float2),
                       cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemsetAsync(base + o_ws + lay.o_arg, 0, sizeof(unsigned long long) * B, s) != cudaSuccess ||
@@ -158,7 +155,6 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
     return nfail(MK_ERR_CUDA, "uploading the step's tables into the scratch array failed");
 
   p.tasks = reinterpret_cast<const Task *>(base + o_tasks);
-  p.layers = reinterpret_cast<const mk::LayerW *>(base + o_layers);
   p.rope_cs = reinterpret_cast<const float2 *>(base + o_rope);
   mk::bind_workspace(lay, base + o_ws, reinterpret_cast<uint32_t *>(base + o_sync), p);
   p.embed = static_cast<const __nv_bfloat16 *>(w->embed);
