@@ -29,6 +29,7 @@ constexpr int kOutSlots = 4;                      // compute -> storer buffers
 constexpr int kMaxPages = 16;                     // ring entries (upper bound)
 constexpr int kMaxMTiles = 8;                     // 16-row tiles per GEMV task (B <= 4)
 constexpr int kMaxPageCols = 2048;                // widest weight page (16 rows)
+constexpr int kXWholeMax = 72 * 1024;             // largest activation staged whole (all sequences)
 constexpr int kMaxGroup = 8;                      // query heads per KV head
 constexpr int kMaxSmem = 232448;                  // opt-in smem per CTA (B200)
 

@@ -90,28 +90,33 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     const int r = o.rows_per_task[i];
     return r > 0 ? std::max(16, r / 16 * 16) : dflt;
   };
-  // QKV tasks never straddle heads (the last task of a head runs its RoPE)
-  int nm_qkv = choose_mtiles(NQKV / 16, grid, mt_cap);
+  // When the inputs of every sequence do not fit the staging area whole, each
+  // task restages its input chunk by chunk: then every task takes as many
+  // row tiles as its accumulators allow, so a staged chunk serves more rows.
+  const int kx_limit = std::max(H, Hq * d);
+  const bool chunked = maxB * x_row_bytes(kx_limit) > kXWholeMax;
+  auto pick = [&](int tiles, int cap) { return chunked ? cap : choose_mtiles(tiles, grid, cap); };
+  // QKV tasks never straddle heads (a head's rows belong to one KV group)
+  int nm_qkv = pick(NQKV / 16, mt_cap);
   while ((d / 16) % nm_qkv) --nm_qkv;
   int R_qkv = rows_opt(0, 16 * nm_qkv);
   if (R_qkv > d || d % R_qkv || R_qkv > 16 * mt_cap) R_qkv = 16;
-  const int R_o = std::min(rows_opt(1, 16 * choose_mtiles(H / 16, grid, mt_cap)), 16 * mt_cap);
+  const int R_o = std::min(rows_opt(1, 16 * pick(H / 16, mt_cap)), 16 * mt_cap);
   const int gu_cap = std::max(1, mt_cap / 2);   // gate and up tiles share a task
-  const int R_gu = std::min(rows_opt(2, 16 * choose_mtiles(F / 16, grid, gu_cap)), 16 * gu_cap);
+  const int R_gu = std::min(rows_opt(2, 16 * pick(F / 16, gu_cap)), 16 * gu_cap);
   // a split down projection has a third or less of the columns per task:
   // two row tiles per task keep its per-task costs (dependency check,
   // restaging at each part) small against its pages
-  const bool ffn_split = F > std::max(H, Hq * d);
-  const int nm_d = std::max(choose_mtiles(H / 16, grid, mt_cap), ffn_split ? std::min(2, mt_cap) : 1);
+  const bool ffn_split = F > kx_limit;
+  const int nm_d = std::max(pick(H / 16, mt_cap), ffn_split ? std::min(2, mt_cap) : 1);
   const int R_d = std::min(rows_opt(3, 16 * nm_d), 16 * mt_cap);
-  const int R_lm = std::min(rows_opt(4, 16 * choose_mtiles(V / 16, grid, mt_cap)), 16 * mt_cap);
+  const int R_lm = std::min(rows_opt(4, 16 * pick(V / 16, mt_cap)), 16 * mt_cap);
 
   // ---- split-K of the down projection --------------------------------------------
   // Parts of at most kx_limit columns (the widest other input), so the down
   // projection's input stages like every other operator's.  A part's columns
   // are whole gate/up tasks' rows, so each part waits only on the gate/up
   // tasks that produce its slice of u.
-  const int kx_limit = std::max(H, Hq * d);
   int n_ksplit = F > kx_limit ? cdiv(F, kx_limit) : 1;
   int kchunk_ffn = F;
   if (n_ksplit > 1) {
@@ -138,8 +143,9 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
 
   // ---- shared memory: activation staging and the weight-page ring ------------------
   // Activation staging holds fp32 rows of every sequence: a whole input when
-  // the widest input other than the FFN's fits in 64 KB (staged once, reused
-  // by the operator's later tasks on this SM), else one page-wide chunk.
+  // the widest input other than the FFN's fits in kXWholeMax (staged once,
+  // reused by the operator's later tasks on this SM), else one page-wide
+  // chunk (<= 64 KB).
   const int max_chunks = cdiv(c.max_seq_len, P);
   const int x_whole = maxB * x_row_bytes(kx_limit);
   const int red_bytes = kComputeWarps * 16 * 8 * n_tiles_for(maxB) * 4;
@@ -167,8 +173,8 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     g.kp[K_LM] = page_cols(H);
     const int kp_big = std::max(std::max(g.kp[0], g.kp[1]), g.kp[2]);
     const int x_chunk = maxB * x_row_bytes(kp_big);
-    if (x_chunk > 64 * 1024) return false;
-    int x_cap = x_whole <= 64 * 1024 ? std::max(x_whole, x_chunk) : x_chunk;
+    if (x_chunk > kXWholeMax) return false;
+    int x_cap = x_whole <= kXWholeMax ? std::max(x_whole, x_chunk) : x_chunk;
     g.page_bytes = 16 * row_pitch_bytes(kp_big);
     // attention pages hold tpp tokens of K and V (4 d bytes per token)
     int tpp = (g.page_bytes / (4 * d)) / P * P;
@@ -199,10 +205,12 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   int best_ring = 0;
   for (const Geom &g : cands)
     if (g.n_pages >= 3) best_ring = std::max(best_ring, g.ring);
+  // (with chunked staging every chunk is restaged per task: the widest pages
+  // that leave 3 in flight, whatever the ring size)
   Geom geo{};
   bool have = false;
   for (const Geom &g : cands)
-    if (g.n_pages >= 3 && 10LL * g.ring >= 9LL * best_ring) {
+    if (g.n_pages >= 3 && (chunked || 10LL * g.ring >= 9LL * best_ring)) {
       geo = g;
       have = true;
       break;
