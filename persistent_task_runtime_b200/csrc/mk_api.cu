@@ -171,8 +171,6 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   mk::bind_workspace(lay, static_cast<char *>(plan->d_ws), plan->d_sync, p);
   p.tasks = static_cast<const Task *>(plan->d_tasks);
   p.embed = static_cast<const __nv_bfloat16 *>(w->embed);
-  p.final_norm = static_cast<const __nv_bfloat16 *>(w->final_norm);
-  p.lm_head = static_cast<const __nv_bfloat16 *>(w->lm_head);
   p.rope_cs = static_cast<const float2 *>(plan->d_rope);
 
   e = cudaMalloc(&plan->d_host_ids, 3 * sizeof(int32_t) * MK_MAX_BATCH);

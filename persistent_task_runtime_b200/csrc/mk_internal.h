@@ -85,7 +85,7 @@ enum OpK : int { K_HID = 0, K_ATT = 1, K_FFN = 2, K_LM = 3 };
 struct Params {
   // plan (static)
   const Task *tasks;
-  const __nv_bfloat16 *embed, *final_norm, *lm_head;
+  const __nv_bfloat16 *embed;   // token embedding [V][H]
   const float2 *rope_cs;        // [max_seq_len][d/2] (cos, sin)
   float *h;                     // [maxB][H]      residual stream
   float *qkv;                   // [maxB][NQKV]   raw projections

@@ -357,10 +357,9 @@ __device__ __forceinline__ void gemv_tile(const Params &p, const Task &t, int m,
   rows_valid = left < 16 ? (left > 0 ? left : 0) : 16;
 }
 
-// Attention split: how many smem pages per chunk so that this step's whole
-// KV length, over all (sequence, KV head), fills about `attn_target` chunks.
-// Lengths are clamped to [1, max_pos] so bad positions cannot blow it up
-// (they are reported by the embedding task).
+// Tokens attended by sequence b this step (positions 0..pos), clamped to
+// [1, max_pos] so a bad position cannot blow up the attention split (bad
+// positions are reported by the embedding task).
 __device__ __forceinline__ int seq_len(const Params &p, int b) {
   int n = p.pos[b] + 1;
   return n < 1 ? 1 : (n > p.max_pos ? p.max_pos : n);

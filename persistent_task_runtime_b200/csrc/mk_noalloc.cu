@@ -158,8 +158,6 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
   p.rope_cs = reinterpret_cast<const float2 *>(base + o_rope);
   mk::bind_workspace(lay, base + o_ws, reinterpret_cast<uint32_t *>(base + o_sync), p);
   p.embed = static_cast<const __nv_bfloat16 *>(w->embed);
-  p.final_norm = static_cast<const __nv_bfloat16 *>(w->final_norm);
-  p.lm_head = static_cast<const __nv_bfloat16 *>(w->lm_head);
 
   p.epoch = 1;  // counters were just zeroed
   p.batch = B;

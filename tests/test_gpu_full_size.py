@@ -6,7 +6,8 @@ synthetic: the GPU cache and the oracle's cache receive the same bf16 values,
 so one decode step can be checked without replaying a long prompt.  At batch
 16 with ragged contexts up to 8192 tokens, all 16 sequences run in one GPU
 step and the oracle recomputes three of them (the shortest, the median and
-the longest).  Decode treats sequences independently, so every sampled
+the longest); the batch sweep at context 1024 (4 and 8 sequences) is checked
+the same way.  Decode treats sequences independently, so every sampled
 output has a plain reference value.  Tolerances are those of
 tests/gpu_harness.py.
 
@@ -41,12 +42,22 @@ def test_full_size_batch1(cuda_device, name, ctx, steps):
     assert_report(rep)
 
 
-def test_full_size_8b_batch16_ragged_sampled(cuda_device):
+SAMPLED = {
+    # the batch sweep at context 1024 (two sequences recomputed) and the
+    # ragged batch of 16 (shortest, median, longest recomputed)
+    "b4_ctx1024": (4, lambda: [1024] * 4),
+    "b8_ctx1024": (8, lambda: [1024] * 8),
+    "b16_ragged": (16, lambda: synth.ragged_lengths(16, 32, 8192, seed=2)),
+}
+
+
+@pytest.mark.parametrize("case", sorted(SAMPLED))
+def test_full_size_8b_batched_sampled(cuda_device, case):
     cfg = synth.CONFIGS["8b"]
-    B = 16
-    lengths = synth.ragged_lengths(B, 32, 8192, seed=2)     # the benchmark's contexts
+    B, make_lengths = SAMPLED[case]
+    lengths = make_lengths()                                  # the benchmark's contexts
     order = np.argsort(lengths, kind="stable")
-    pick = [int(order[0]), int(order[B // 2]), int(order[-1])]
+    pick = sorted({int(order[0]), int(order[B // 2]), int(order[-1])})
     w = synth.make_weights(cfg, seed=0, device="cuda")
     plan = mk.Plan(cfg, w, max_batch=B, page_size=16, max_seq_len=max(lengths) + 17)
     kv = PagedKVCache(cfg, B, [n + 2 for n in lengths], page=16,
