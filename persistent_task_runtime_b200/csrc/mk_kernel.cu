@@ -470,11 +470,25 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     }
     ++la_count;
   };
+  // A handed-over GEMV task whose input was not yet complete blocks further
+  // pops until that input completes, so a CTA waiting at an operator
+  // boundary does not reserve more of the next operator's tasks.
+  bool blocked = false;
+  uint32_t blk_ev = kNoEvent, blk_cnt = 0;
+  int blk_tix = 0;   // the blocked task (named in a timeout report)
+  auto may_pop = [&]() {
+    if (!blocked) return true;
+    int ok = 0;
+    if (lane == 0) ok = static_cast<int32_t>(ld_relaxed(p.sync + S_EVENTS + blk_ev) - p.epoch * blk_cnt) >= 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) blocked = false;
+    return ok != 0;
+  };
   auto top_up = [&](int max_pops) {
     for (int k = 0; k < max_pops; ++k) {
       // one task ahead: every popped task is reserved for this CTA, so
       // popping further ahead would delay the last tasks of an operator
-      if (exhausted || la_count >= 1) break;
+      if (exhausted || la_count >= 1 || !may_pop()) break;
       pop_one();
     }
     __syncwarp();
@@ -482,6 +496,16 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
 
   while (true) {
     top_up(kLook);
+    if (la_count == 0 && !exhausted && blocked) {
+      int okw = 1;
+      if (lane == 0) okw = wait_event(p, ctl, blk_ev, blk_cnt, static_cast<uint32_t>(blk_tix));
+      if (__shfl_sync(0xffffffffu, okw, 0) == 0) {
+        ok = false;
+        break;
+      }
+      blocked = false;
+      top_up(kLook);
+    }
     int okl = 1;
     if (lane == 0) okl = wait_mbar(p, ctl, &ctl->slot_empty[ts], ts_par ^ 1u, 0xfff00000u, 2);
     ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
@@ -522,6 +546,15 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
             blockIdx.x | (static_cast<unsigned long long>(t.type) << 32) |
             (static_cast<unsigned long long>(t.layer) << 40);
         trace_mark(p, tix, 1);
+      }
+    }
+    {
+      const int dok = __shfl_sync(0xffffffffu, info.dep_ok, 0);
+      if (is_gemv(t.type) && t.dep_event != kNoEvent && !dok) {
+        blocked = true;
+        blk_ev = t.dep_event;
+        blk_cnt = t.dep_count;
+        blk_tix = tix;
       }
     }
     if (++ts == kTaskSlots) {
