@@ -470,9 +470,10 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     }
     ++la_count;
   };
-  // A handed-over GEMV task whose input was not yet complete blocks further
-  // pops until that input completes, so a CTA waiting at an operator
-  // boundary does not reserve more of the next operator's tasks.
+  // A handed-over GEMV task whose input was not yet complete, or an
+  // attention chunk, blocks further pops until its input completes, so a CTA
+  // waiting at an operator boundary does not reserve more of the next
+  // operator's tasks.
   bool blocked = false;
   uint32_t blk_ev = kNoEvent, blk_cnt = 0;
   int blk_tix = 0;   // the blocked task (named in a timeout report)
@@ -554,6 +555,13 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
         blocked = true;
         blk_ev = t.dep_event;
         blk_cnt = t.dep_count;
+        blk_tix = tix;
+      } else if (t.type == T_ATTN && info.b >= 0) {
+        // an attention chunk waits for its KV group's projections: one such
+        // chunk per CTA, so a group's chunks run on as many SMs as it has
+        blocked = true;
+        blk_ev = static_cast<uint32_t>(ev_attn_ready(p, t.layer, info.g));
+        blk_cnt = static_cast<uint32_t>(p.qkv_tasks_per_group);
         blk_tix = tix;
       }
     }
