@@ -216,8 +216,38 @@ typedef struct {
   int page_cols[4];       /* columns per weight page: K=H, K=Hq*d, K=F, LM  */
   int64_t weight_bytes;   /* bytes of weights one step streams (excluding the
                              embedding rows)                                */
+  /* task-graph facts (event k of layer l is 1 + l*events_per_layer + k:
+     attn_ready[n_kv_heads], o_ready[o_parts], oproj, gateup[ffn_parts],
+     down; event 0 is the embedding)                                      */
+  int events_per_layer;
+  int attn_slots_per_group; /* attention slots of one KV group per layer   */
+  int qkv_tasks_per_group;  /* QKV tasks whose rows one KV group attends   */
+  int ffn_parts, ffn_part_cols; /* split-K parts of the down projection and
+                             columns per part (1 part: ffn_part_cols = ffn) */
+  int o_parts, o_part_cols; /* the same for the O projection               */
 } mk_plan_info_t;
 MK_API int mk_plan_info(const mk_plan *plan, mk_plan_info_t *info);
+
+/* Task records returned by mk_plan_describe (MK_TASK_RECORD_BYTES each;
+ * for tests and tools, the layout may change between versions):
+ *   byte 0 type (1 embed, 2 QKV, 3 attention, 4 O, 5 gate/up, 6 down,
+ *   7 LM head), 1 row tiles, 2-3 layer, 4-7 first output row, 8-9 rows,
+ *   10 split-K part, 11 split-K parts (0/1: none), 12-15 input event
+ *   (0xffffffff: none; attention: resolved at run time), 16-19 completions
+ *   of the input event per step, 20-23 output event (0xffffffff: none; a QKV
+ *   task signals attn_ready of its head's KV group), 24-27 aux (QKV: 0 q,
+ *   1 k, 2 v; attention: slot), 28-31 aux2 (QKV: head index over q, k, v),
+ *   32-63 operand pointers (NULL in a described plan). */
+#define MK_TASK_RECORD_BYTES 64
+
+/* Describe, without any GPU, the plan mk_plan_create_ex(cfg, weights, opts)
+ * would build on a device with `num_sms` SMs and `smem_optin` bytes of
+ * opt-in shared memory per block: fills *info and, when `tasks` is not NULL
+ * and `max_tasks` >= info->n_tasks, copies the task records.  Returns MK_OK,
+ * or the error mk_plan_create_ex would return for the shape and options. */
+MK_API int mk_plan_describe(const mk_model_config *cfg, const mk_plan_options *opts,
+                            int num_sms, int smem_optin, mk_plan_info_t *info,
+                            void *tasks, int64_t max_tasks);
 
 /* Message of the last error on the calling thread ("" if none). */
 MK_API const char *mk_last_error(void);

@@ -87,6 +87,50 @@ int validate_weights(const mk_model_config *c, const mk_weights *w) {
   return MK_OK;
 }
 
+// Plan options -> layout options (defaults filled in).
+int layout_options(const mk_plan_options *opts, mk::LayoutOptions &lo) {
+  mk_plan_options o{};
+  if (opts) o = *opts;
+  if (o.wait_limit_ns < 0) return fail(MK_ERR_INVALID_ARG, "wait_limit_ns < 0");
+  lo.max_batch = o.max_batch == 0 ? 1 : o.max_batch;
+  lo.page_size = o.kv_page_size == 0 ? 16 : o.kv_page_size;
+  lo.num_ctas = o.num_ctas;
+  lo.max_page_cols = o.max_page_cols;
+  lo.o_split = o.o_split != 0;
+  for (int i = 0; i < 5; ++i) lo.rows_per_task[i] = o.rows_per_task[i];
+  lo.wait_limit_ns = o.wait_limit_ns == 0 ? 2000000000LL : o.wait_limit_ns;
+  lo.debug_unsatisfiable_dep = o.debug_unsatisfiable_dep != 0;
+  return MK_OK;
+}
+
+void fill_info(const mk::Layout &lay, const mk_model_config &c, mk_plan_info_t &I) {
+  const Params &p = lay.p;
+  const int L = c.n_layers, H = c.hidden, d = c.head_dim, F = c.ffn, V = c.vocab;
+  I = mk_plan_info_t{};
+  I.num_ctas = lay.grid;
+  I.threads_per_cta = mk::kThreads;
+  I.smem_bytes = lay.smem;
+  I.n_pages = p.n_pages;
+  I.page_bytes = p.page_bytes;
+  I.n_tasks = p.n_tasks;
+  I.n_events = lay.n_events;
+  I.attn_slots = p.attn_slots;
+  I.tokens_per_smem_page = p.tpp;
+  for (int i = 0; i < 5; ++i) I.rows_per_task[i] = lay.rows[i];
+  for (int i = 0; i < 4; ++i) I.page_cols[i] = p.kp[i];
+  I.weight_bytes = 2LL * L *
+                       (static_cast<long long>(p.NQKV) * H + static_cast<long long>(H) * c.n_q_heads * d +
+                        3LL * F * H) +
+                   2LL * V * H;
+  I.events_per_layer = p.ev_per_layer;
+  I.attn_slots_per_group = p.attn_spg;
+  I.qkv_tasks_per_group = p.qkv_tasks_per_group;
+  I.ffn_parts = p.n_ffn_parts;
+  I.ffn_part_cols = p.kchunk[mk::K_FFN] > 0 ? p.kchunk[mk::K_FFN] : F;
+  I.o_parts = p.n_o_parts;
+  I.o_part_cols = p.kchunk[mk::K_ATT] > 0 ? p.kchunk[mk::K_ATT] : c.n_q_heads * d;
+}
+
 }  // namespace
 
 extern "C" {
@@ -111,18 +155,9 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   if (rc) return rc;
   rc = validate_weights(cfg, w);
   if (rc) return rc;
-  mk_plan_options o{};
-  if (opts) o = *opts;
-  if (o.wait_limit_ns < 0) return fail(MK_ERR_INVALID_ARG, "wait_limit_ns < 0");
   mk::LayoutOptions lo;
-  lo.max_batch = o.max_batch == 0 ? 1 : o.max_batch;
-  lo.page_size = o.kv_page_size == 0 ? 16 : o.kv_page_size;
-  lo.num_ctas = o.num_ctas;
-  lo.max_page_cols = o.max_page_cols;
-  lo.o_split = o.o_split != 0;
-  for (int i = 0; i < 5; ++i) lo.rows_per_task[i] = o.rows_per_task[i];
-  lo.wait_limit_ns = o.wait_limit_ns == 0 ? 2000000000LL : o.wait_limit_ns;
-  lo.debug_unsatisfiable_dep = o.debug_unsatisfiable_dep != 0;
+  rc = layout_options(opts, lo);
+  if (rc) return rc;
 
   int dev = 0, nsm = 0, smem_optin = 0, coop = 0;
   MK_CUDA(cudaGetDevice(&dev));
@@ -181,24 +216,7 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   e = mk::configure_kernel(lay.smem);
   if (e != cudaSuccess) return cleanup_fail(fail(MK_ERR_CUDA, "kernel attribute: %s", cudaGetErrorString(e)));
 
-  // ---- facts ------------------------------------------------------------------
-  const int L = cfg->n_layers, H = cfg->hidden, d = cfg->head_dim, F = cfg->ffn, V = cfg->vocab;
-  mk_plan_info_t &I = plan->info;
-  I.num_ctas = lay.grid;
-  I.threads_per_cta = mk::kThreads;
-  I.smem_bytes = lay.smem;
-  I.n_pages = p.n_pages;
-  I.page_bytes = p.page_bytes;
-  I.n_tasks = p.n_tasks;
-  I.n_events = lay.n_events;
-  I.attn_slots = p.attn_slots;
-  I.tokens_per_smem_page = p.tpp;
-  for (int i = 0; i < 5; ++i) I.rows_per_task[i] = lay.rows[i];
-  for (int i = 0; i < 4; ++i) I.page_cols[i] = p.kp[i];
-  I.weight_bytes = 2LL * L *
-                       (static_cast<long long>(p.NQKV) * H + static_cast<long long>(H) * cfg->n_q_heads * d +
-                        3LL * F * H) +
-                   2LL * V * H;
+  fill_info(lay, *cfg, plan->info);
   *out = plan;
   return MK_OK;
 }
@@ -354,6 +372,27 @@ int mk_plan_reset(mk_plan *plan) {
 int mk_plan_info(const mk_plan *plan, mk_plan_info_t *info) {
   if (plan == nullptr || info == nullptr) return fail(MK_ERR_INVALID_ARG, "plan or info is NULL");
   *info = plan->info;
+  return MK_OK;
+}
+
+int mk_plan_describe(const mk_model_config *cfg, const mk_plan_options *opts, int num_sms,
+                     int smem_optin, mk_plan_info_t *info, void *tasks, int64_t max_tasks) {
+  g_err.clear();
+  if (cfg == nullptr || info == nullptr) return fail(MK_ERR_INVALID_ARG, "cfg or info is NULL");
+  if (num_sms < 1 || smem_optin < 1)
+    return fail(MK_ERR_INVALID_ARG, "num_sms and smem_optin must be positive");
+  int rc = mk::validate_config(*cfg, g_err);
+  if (rc) return rc;
+  mk::LayoutOptions lo;
+  rc = layout_options(opts, lo);
+  if (rc) return rc;
+  mk::Layout lay;
+  rc = mk::build_layout(*cfg, lo, num_sms, smem_optin, lay, g_err);
+  if (rc) return rc;
+  fill_info(lay, *cfg, *info);
+  static_assert(sizeof(Task) == MK_TASK_RECORD_BYTES, "task record size");
+  if (tasks != nullptr && max_tasks >= static_cast<int64_t>(lay.tasks.size()))
+    std::memcpy(tasks, lay.tasks.data(), lay.tasks.size() * sizeof(Task));
   return MK_OK;
 }
 

@@ -36,7 +36,8 @@ ERROR_NAMES = {MK_OK: "MK_OK", MK_ERR_INVALID_ARG: "MK_ERR_INVALID_ARG",
 #: every symbol include/mk.h declares
 EXPORTS = ["mk_plan_create", "mk_plan_create_ex", "mk_decode_step", "mk_decode_step_ex",
            "mk_decode_step_host", "mk_plan_status", "mk_plan_error_info", "mk_plan_reset",
-           "mk_plan_info", "mk_last_error", "mk_plan_destroy", "mk_decode_step_noalloc"]
+           "mk_plan_info", "mk_last_error", "mk_plan_destroy", "mk_decode_step_noalloc",
+           "mk_plan_describe"]
 
 #: bytes of the library's static scratch array used by mk_decode_step_noalloc
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -84,7 +85,10 @@ class mk_plan_info_t(C.Structure):
                 ("n_pages", C.c_int), ("page_bytes", C.c_int), ("n_tasks", C.c_int),
                 ("n_events", C.c_int), ("attn_slots", C.c_int),
                 ("tokens_per_smem_page", C.c_int), ("rows_per_task", C.c_int * 5),
-                ("page_cols", C.c_int * 4), ("weight_bytes", C.c_int64)]
+                ("page_cols", C.c_int * 4), ("weight_bytes", C.c_int64),
+                ("events_per_layer", C.c_int), ("attn_slots_per_group", C.c_int),
+                ("qkv_tasks_per_group", C.c_int), ("ffn_parts", C.c_int),
+                ("ffn_part_cols", C.c_int), ("o_parts", C.c_int), ("o_part_cols", C.c_int)]
 
 
 _lib = None
@@ -111,6 +115,8 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
     lib.mk_plan_error_info.argtypes = [P, C.POINTER(C.c_int32)]
     lib.mk_plan_reset.argtypes = [P]
     lib.mk_plan_info.argtypes = [P, C.POINTER(mk_plan_info_t)]
+    lib.mk_plan_describe.argtypes = [C.POINTER(mk_model_config), C.POINTER(mk_plan_options),
+                                     C.c_int, C.c_int, C.POINTER(mk_plan_info_t), P, C.c_int64]
     lib.mk_last_error.restype = C.c_char_p
     lib.mk_last_error.argtypes = []
     lib.mk_plan_destroy.argtypes = [P]
@@ -162,6 +168,50 @@ class KVCacheView:
                                   block_table.shape[1])
 
 
+#: one task record of mk_plan_describe (see include/mk.h)
+TASK_RECORD_DTYPE = [("type", "u1"), ("n_m", "u1"), ("layer", "<u2"), ("row0", "<u4"),
+                     ("nrows", "<u2"), ("ksplit", "u1"), ("nsplit", "u1"), ("dep_event", "<u4"),
+                     ("dep_count", "<u4"), ("out_event", "<u4"), ("aux", "<u4"), ("aux2", "<u4"),
+                     ("operands", "<u8", (4,))]
+TASK_TYPES = {1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead"}
+NO_EVENT = 0xFFFFFFFF
+
+
+def _info_dict(i: "mk_plan_info_t") -> dict:
+    out = {k: getattr(i, k) for k, _ in mk_plan_info_t._fields_}
+    out["rows_per_task"] = list(i.rows_per_task)
+    out["page_cols"] = list(i.page_cols)
+    return out
+
+
+def _config(cfg: Dict, max_seq_len: int) -> mk_model_config:
+    return mk_model_config(cfg["n_layers"], cfg["hidden"], cfg["n_q_heads"], cfg["n_kv_heads"],
+                           cfg["head_dim"], cfg["ffn"], cfg["vocab"], cfg.get("rms_eps", 1e-6),
+                           cfg.get("rope_theta", 1e6), 1 if cfg.get("qk_norm", True) else 0,
+                           max_seq_len)
+
+
+def describe(cfg: Dict, max_batch: int = 1, page_size: int = 16, max_seq_len: int = 4096,
+             num_sms: int = 148, smem_optin: int = 232448, rows_per_task=(0, 0, 0, 0, 0),
+             max_page_cols: int = 0, o_split: bool = False):
+    """The plan mk_plan_create_ex would build, without a GPU: (info, task records).
+
+    The task records are a numpy structured array (TASK_RECORD_DTYPE)."""
+    import numpy as np
+    lib = load_library()
+    c = _config(cfg, max_seq_len)
+    opts = mk_plan_options(max_batch, page_size, 0, 0, (C.c_int * 5)(*rows_per_task), 0,
+                           max_page_cols, 1 if o_split else 0)
+    info = mk_plan_info_t()
+    _check(lib.mk_plan_describe(C.byref(c), C.byref(opts), num_sms, smem_optin, C.byref(info),
+                                None, 0))
+    tasks = np.zeros(info.n_tasks, dtype=TASK_RECORD_DTYPE)
+    assert tasks.itemsize == 64
+    _check(lib.mk_plan_describe(C.byref(c), C.byref(opts), num_sms, smem_optin, C.byref(info),
+                                tasks.ctypes.data, info.n_tasks))
+    return _info_dict(info), tasks
+
+
 class Plan:
     """A decode plan over caller-owned bf16 weights (see include/mk.h)."""
 
@@ -172,10 +222,7 @@ class Plan:
         lib = load_library()
         self.cfg = dict(cfg)
         self.max_batch = max_batch
-        self._c = mk_model_config(cfg["n_layers"], cfg["hidden"], cfg["n_q_heads"],
-                                  cfg["n_kv_heads"], cfg["head_dim"], cfg["ffn"], cfg["vocab"],
-                                  cfg.get("rms_eps", 1e-6), cfg.get("rope_theta", 1e6),
-                                  1 if cfg.get("qk_norm", True) else 0, max_seq_len)
+        self._c = _config(cfg, max_seq_len)
         L = cfg["n_layers"]
         self._weights = weights  # keep the tensors alive
         lw = (mk_layer_weights * L)()
@@ -198,10 +245,7 @@ class Plan:
     def info(self) -> dict:
         i = mk_plan_info_t()
         _check(self._lib.mk_plan_info(self._h, C.byref(i)))
-        out = {k: getattr(i, k) for k, _ in mk_plan_info_t._fields_}
-        out["rows_per_task"] = list(i.rows_per_task)
-        out["page_cols"] = list(i.page_cols)
-        return out
+        return _info_dict(i)
 
     def step(self, ids: torch.Tensor, pos: torch.Tensor, kv: KVCacheView, out_ids: torch.Tensor,
              out_logits: Optional[torch.Tensor] = None, out_pos: Optional[torch.Tensor] = None,
@@ -278,10 +322,7 @@ class ModelRef:
     mk_decode_step_noalloc)."""
 
     def __init__(self, cfg: Dict, weights: Dict, max_seq_len: int = 4096):
-        self._c = mk_model_config(cfg["n_layers"], cfg["hidden"], cfg["n_q_heads"],
-                                  cfg["n_kv_heads"], cfg["head_dim"], cfg["ffn"], cfg["vocab"],
-                                  cfg.get("rms_eps", 1e-6), cfg.get("rope_theta", 1e6),
-                                  1 if cfg.get("qk_norm", True) else 0, max_seq_len)
+        self._c = _config(cfg, max_seq_len)
         L = cfg["n_layers"]
         self._weights = weights
         lw = (mk_layer_weights * L)()

@@ -1,0 +1,200 @@
+"""CPU tests of the plan builder (mk_plan_describe): the task graph the
+persistent kernel runs, checked without a GPU.
+
+A step runs tasks in queue order on whichever SM asks first.  A task runs
+once the event it names has been signalled `dep_count` times in the current
+step.  The graph must therefore satisfy, for every shape and option:
+  * every event receives, per step, exactly the completions its waiters
+    require (else a wait never ends or ends early);
+  * every producer of an event sits earlier in the queue than every task
+    waiting on it (the in-order queue then cannot deadlock: the earliest
+    unfinished task has all its inputs done);
+  * the tasks of an operator cover its output rows (and split-K parts cover
+    its columns) exactly once;
+  * the shared-memory carve-up fits the device, and tasks stay within the
+    row tiles the accumulators hold.
+"""
+
+from collections import Counter, defaultdict
+
+import numpy as np
+import pytest
+
+from persistent_task_runtime_b200 import build, mk, synth
+
+SHAPES = {
+    "tiny": synth.CONFIGS["tiny"],
+    "1.5b": synth.CONFIGS["1.5b"],
+    "8b": synth.CONFIGS["8b"],
+    # ragged rows, no QK-norm, G = 3
+    "ragged": dict(n_layers=2, hidden=200, n_q_heads=3, n_kv_heads=1, head_dim=64, ffn=344,
+                   vocab=1000, rms_eps=1e-6, rope_theta=1e4, qk_norm=False),
+    # three KV groups of 4 x 128 (an O projection that can split into 2 + 1 groups)
+    "3groups": dict(n_layers=2, hidden=1024, n_q_heads=12, n_kv_heads=3, head_dim=128,
+                    ffn=2816, vocab=2048, rms_eps=1e-6, rope_theta=1e6, qk_norm=True),
+    # head_dim 32, MHA
+    "d32": dict(n_layers=1, hidden=128, n_q_heads=4, n_kv_heads=4, head_dim=32, ffn=256,
+                vocab=512, rms_eps=1e-6, rope_theta=1e6, qk_norm=True),
+}
+SMEM = 232448
+T_EMBED, T_QKV, T_ATTN, T_OPROJ, T_GATEUP, T_DOWN, T_LMHEAD = 1, 2, 3, 4, 5, 6, 7
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+def n_tiles_for(batch):
+    return 1 if batch <= 4 else (2 if batch <= 8 else 4)
+
+
+def check_plan(cfg, info, t, max_batch):
+    H, Hq, Hkv, d = cfg["hidden"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["head_dim"]
+    F, V, L = cfg["ffn"], cfg["vocab"], cfg["n_layers"]
+    G = Hq // Hkv
+    epl, spg = info["events_per_layer"], info["attn_slots_per_group"]
+    o_parts, ffn_parts = info["o_parts"], info["ffn_parts"]
+    n_events = info["n_events"]
+    assert n_events == 1 + L * epl
+    assert epl == Hkv + o_parts + 2 + ffn_parts
+
+    def ev_attn_ready(l, g):
+        return 1 + l * epl + g
+
+    def ev_gateup(l, part):
+        return 1 + l * epl + Hkv + o_parts + 1 + part
+
+    # ---- resources -------------------------------------------------------------------
+    assert info["smem_bytes"] <= SMEM
+    assert info["n_pages"] >= 2
+    assert info["n_pages"] * info["page_bytes"] < info["smem_bytes"]
+    max_mt = 8 // n_tiles_for(max_batch)
+
+    # ---- who signals what, per step ----------------------------------------------------
+    signals = Counter()
+    producers = defaultdict(list)        # event -> task indices that signal it
+    split_tiles = set()
+    for i, r in enumerate(t):
+        ty = int(r["type"])
+        if ty == T_QKV:
+            head, mat = int(r["aux2"]), int(r["aux"])
+            g = head // G if mat == 0 else (head - Hq if mat == 1 else head - Hq - Hkv)
+            assert 0 <= g < Hkv
+            ev = ev_attn_ready(int(r["layer"]), g)
+        elif ty in (T_OPROJ, T_DOWN) and r["nsplit"] > 1:
+            # the part that completes a row tile signals once for the tile
+            key = (ty, int(r["layer"]), int(r["row0"]))
+            if key in split_tiles:
+                producers[int(r["out_event"])].append(i)
+                continue
+            split_tiles.add(key)
+            ev = int(r["out_event"])
+        else:
+            ev = int(r["out_event"])
+        if ev == mk.NO_EVENT:
+            continue
+        assert 0 <= ev < n_events
+        signals[ev] += 1
+        producers[ev].append(i)
+
+    # ---- every wait is satisfied exactly, by earlier tasks ------------------------------
+    for i, r in enumerate(t):
+        ty = int(r["type"])
+        if ty == T_ATTN:
+            g = int(r["aux"]) // spg
+            ev = ev_attn_ready(int(r["layer"]), g)
+            need = info["qkv_tasks_per_group"]
+        else:
+            ev, need = int(r["dep_event"]), int(r["dep_count"])
+            if ev == mk.NO_EVENT:
+                assert ty == T_EMBED
+                continue
+        assert signals[ev] == need, (i, ty, ev, signals[ev], need)
+        assert max(producers[ev]) < i, (i, ty, ev)
+
+    # ---- coverage of output rows (and split-K columns) ----------------------------------
+    for l in range(L):
+        lay = t[t["layer"] == l]
+        qkv = lay[lay["type"] == T_QKV]
+        for mat, rows in ((0, Hq * d), (1, Hkv * d), (2, Hkv * d)):
+            m = qkv[qkv["aux"] == mat]
+            cover = np.zeros(rows, dtype=int)
+            for r in m:
+                r0, n = int(r["row0"]), int(r["nrows"])
+                assert r0 // d == (r0 + n - 1) // d          # never straddles heads
+                cover[r0:r0 + n] += 1
+            assert (cover == 1).all()
+        for ty, rows, parts in ((T_OPROJ, H, max(o_parts, 1)), (T_DOWN, H, max(ffn_parts, 1))):
+            m = lay[lay["type"] == ty]
+            for ks in range(parts):
+                cover = np.zeros(rows, dtype=int)
+                for r in m[m["ksplit"] == ks]:
+                    cover[int(r["row0"]):int(r["row0"]) + int(r["nrows"])] += 1
+                assert (cover == 1).all(), (l, ty, ks)
+        gu = lay[lay["type"] == T_GATEUP]
+        cover = np.zeros(F, dtype=int)
+        cols = info["ffn_part_cols"]
+        for r in gu:
+            r0, n = int(r["row0"]), int(r["nrows"])
+            cover[r0:r0 + n] += 1
+            part = r0 // cols if ffn_parts > 1 else 0
+            assert (r0 + n - 1) // cols == r0 // cols or ffn_parts == 1
+            assert int(r["out_event"]) == ev_gateup(l, part)
+            assert int(r["n_m"]) % 2 == 0 and 16 * (int(r["n_m"]) // 2) >= n
+        assert (cover == 1).all()
+    assert ffn_parts * info["ffn_part_cols"] >= F > (ffn_parts - 1) * info["ffn_part_cols"]
+    assert o_parts * info["o_part_cols"] >= Hq * d > (o_parts - 1) * info["o_part_cols"]
+    lm = t[t["type"] == T_LMHEAD]
+    cover = np.zeros(V, dtype=int)
+    for r in lm:
+        cover[int(r["row0"]):int(r["row0"]) + int(r["nrows"])] += 1
+    assert (cover == 1).all()
+
+    # ---- row tiles within the accumulators ------------------------------------------------
+    gemv = t[np.isin(t["type"], [T_QKV, T_OPROJ, T_GATEUP, T_DOWN, T_LMHEAD])]
+    assert int(gemv["n_m"].max()) <= max_mt
+    ng = gemv[gemv["type"] != T_GATEUP]
+    assert (16 * ng["n_m"].astype(int) >= ng["nrows"].astype(int)).all()
+
+    # ---- attention slots: one block per KV group ------------------------------------------
+    att = t[t["type"] == T_ATTN]
+    assert len(att) == L * Hkv * spg == L * info["attn_slots"]
+
+
+CASES = [(name, b, split) for name in SHAPES for b in (1, 3, 4, 8, 16) for split in (False, True)]
+
+
+@pytest.mark.parametrize("name,batch,o_split", CASES)
+def test_task_graph_invariants(name, batch, o_split):
+    cfg = SHAPES[name]
+    info, t = mk.describe(cfg, max_batch=batch, max_seq_len=2048 if name == "8b" else 600,
+                          o_split=o_split)
+    check_plan(cfg, info, t, batch)
+
+
+@pytest.mark.parametrize("cols", [256, 1024, 2048])
+def test_page_width_option(cols):
+    cfg = SHAPES["8b"]
+    info, t = mk.describe(cfg, max_batch=1, max_seq_len=1024, max_page_cols=cols)
+    assert max(info["page_cols"]) <= cols
+    check_plan(cfg, info, t, 1)
+
+
+def test_batch1_8b_plan_facts():
+    """The benchmark's plan: 3 ring pages of 16 x 2048 bf16, the down
+    projection in 3 parts of 4096 columns, one O part."""
+    info, _ = mk.describe(SHAPES["8b"], max_batch=1, max_seq_len=600)
+    assert info["n_pages"] == 3 and info["page_cols"] == [2048, 2048, 2048, 2048]
+    assert (info["ffn_parts"], info["ffn_part_cols"]) == (3, 4096)
+    assert info["o_parts"] == 1
+
+
+def test_describe_rejects_what_create_rejects():
+    cfg = dict(SHAPES["tiny"], head_dim=96)
+    with pytest.raises(mk.MkError):
+        mk.describe(cfg)
+    with pytest.raises(mk.MkError):
+        mk.describe(SHAPES["tiny"], max_page_cols=100)
+    with pytest.raises(mk.MkError):
+        mk.describe(SHAPES["tiny"], max_batch=17)
