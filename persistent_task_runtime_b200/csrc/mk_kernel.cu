@@ -9,15 +9,15 @@
 //                        the next tasks while the compute warps still wait for
 //                        a dependency (MPK write-up, "3.2 任务预取与流水线":
 //                        the next task's pre-load overlaps the current task).
-//   warps 1..8  compute: wait for the task's input event (in-GPU event
+//   warps 1..6  compute: wait for the task's input event (in-GPU event
 //                        counters, MPK write-up "2.1 Mega-Kernel执行模型":
 //                        trigger count vs. required count), stage the
 //                        activation, and consume the pages (bf16 mma.sync for
-//                        the projections, warp-shuffle online softmax for
-//                        attention).
-//   warp 9      storer : epilogues (residual add, SwiGLU, QK-norm + RoPE + KV
-//                        append, split-attention combine, argmax) and the
-//                        release of the task's output event.
+//                        the projections; for attention: QK-norm + RoPE of the
+//                        step's q and K, the KV append, online softmax over the
+//                        chunk's pages and the split-attention combine).
+//   warp 7      storer : epilogues (residual add, split-K sums, SwiGLU,
+//                        argmax) and the release of the task's output event.
 // (Loader / consumer / storer roles: Ada-MK summary, "Methodik", Phase II.)
 //
 // Shared-memory pages are a ring guarded by mbarriers (full: TMA bytes landed;
@@ -1076,6 +1076,41 @@ __device__ __forceinline__ void head_norm_rope(const float *src, const __nv_bflo
   }
 }
 
+// Split-attention merge, one batch of up to kCombRegs chunk partials for one
+// (head, 4 columns): row c of `ph` (stride `cstride` floats) holds the
+// chunk's unnormalised sum over d columns, then its max m and sum l (log2
+// units).  Folds the batch into the running (M, den, num).
+constexpr int kCombRegs = 17;
+template <int D>
+__device__ __forceinline__ void comb_batch(const float *ph, size_t cstride, int i, int n, float &M,
+                                           float &den, float4 &num) {
+  float2 ml[kCombRegs];
+  float4 a[kCombRegs];
+#pragma unroll
+  for (int c = 0; c < kCombRegs; ++c) {
+    if (c < n) {
+      ml[c] = __ldcg(reinterpret_cast<const float2 *>(ph + c * cstride + D));
+      a[c] = __ldcg(reinterpret_cast<const float4 *>(ph + c * cstride + i));
+    } else {
+      ml[c] = make_float2(-INFINITY, 0.f);
+      a[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  float Mb = M;
+#pragma unroll
+  for (int c = 0; c < kCombRegs; ++c) Mb = fmaxf(Mb, ml[c].x);
+  const float sc = exp2f(M - Mb);   // 0 before the first batch (M = -inf)
+  den *= sc;
+  num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
+#pragma unroll
+  for (int c = 0; c < kCombRegs; ++c) {
+    const float wgt = exp2f(ml[c].x - Mb);   // 0 for the padding entries
+    den += wgt * ml[c].y;
+    num.x += wgt * a[c].x; num.y += wgt * a[c].y; num.z += wgt * a[c].z; num.w += wgt * a[c].w;
+  }
+  M = Mb;
+}
+
 // Attention for one chunk of one (sequence, KV head): scores for the G query
 // heads over the chunk's tokens, softmax statistics, and the unnormalised
 // P.V, all in three parallel phases per shared-memory page:
@@ -1276,7 +1311,6 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   }
   compute_bar();
   const int d = D;
-  float *wsc = sc;   // combine scratch (reuses the score area)
 
   // The chunk that completes (b, g) merges all of its chunks by log-sum-exp
   // and writes o for the G query heads.  The bar above orders every thread's
@@ -1286,52 +1320,25 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   bool last_l = false;
   if (ctid == 0) last_l = atom_add_acq_rel(ctr, 1u) + 1u == static_cast<uint32_t>(S.n_chunks);
   if (!st.gs.share(ctl, ctid, last_l)) return true;
+  // Each (head, 4 columns) thread merges the chunks in batches of kCombRegs:
+  // a batch's (m, l) pairs and 4-column partial sums are loaded into
+  // registers with all loads in flight together, so a batch costs one L2
+  // round trip; the running maximum rescales the earlier batches.  17 is the
+  // largest batch that measured no slower elsewhere in the kernel (register
+  // pressure); decode at one sequence per 148 SMs splits a head's context
+  // into at most about 20 chunks.  The first batch is straight-line code.
   const int nch = S.n_chunks;
-  float *ms = wsc;                     // [nch][G] chunk maxima, then weights
-  float *ls = wsc + nch * G;           // [nch][G] chunk sums
-  float *MD = ls + nch * G;            // [G] max, [G] 1/denominator
-  for (int e = ctid; e < nch * G; e += kComputeThreads) {
-    const int c = e / G, h = e % G;
-    const float *pc = p.attn_part + (static_cast<size_t>(S.first_slot + c) * G + h) * rw;
-    ms[e] = __ldcg(pc + d);
-    ls[e] = __ldcg(pc + d + 1);
-  }
-  compute_bar();
-  if (ctid < G) {
-    float M = -INFINITY;
-    for (int c = 0; c < nch; ++c) M = fmaxf(M, ms[c * G + ctid]);
-    float den = 0.f;
-    for (int c = 0; c < nch; ++c) den += exp2f(ms[c * G + ctid] - M) * ls[c * G + ctid];
-    MD[ctid] = M;
-    MD[G + ctid] = 1.0f / den;
-  }
-  compute_bar();
-  for (int e = ctid; e < nch * G; e += kComputeThreads) ms[e] = exp2f(ms[e] - MD[e % G]);
-  compute_bar();
+  const size_t cstride = static_cast<size_t>(G) * rw;
+  const float *p0 = p.attn_part + static_cast<size_t>(S.first_slot) * cstride;
   const int q4 = d / 4;
   for (int e = ctid; e < G * q4; e += kComputeThreads) {
     const int h = e / q4, i = (e % q4) * 4;
+    float M = -INFINITY, den = 0.f;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    int c = 0;
-    for (; c + 4 <= nch; c += 4) {
-      float4 a[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        a[u] = __ldcg(reinterpret_cast<const float4 *>(
-            p.attn_part + (static_cast<size_t>(S.first_slot + c + u) * G + h) * rw + i));
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float wgt = ms[(c + u) * G + h];
-        num.x += wgt * a[u].x; num.y += wgt * a[u].y; num.z += wgt * a[u].z; num.w += wgt * a[u].w;
-      }
-    }
-    for (; c < nch; ++c) {
-      const float4 a = __ldcg(reinterpret_cast<const float4 *>(
-          p.attn_part + (static_cast<size_t>(S.first_slot + c) * G + h) * rw + i));
-      const float wgt = ms[c * G + h];
-      num.x += wgt * a.x; num.y += wgt * a.y; num.z += wgt * a.z; num.w += wgt * a.w;
-    }
-    const float r = MD[G + h];
+    comb_batch<D>(p0 + h * rw, cstride, i, nch, M, den, num);
+    for (int c0 = kCombRegs; c0 < nch; c0 += kCombRegs)
+      comb_batch<D>(p0 + c0 * cstride + h * rw, cstride, i, nch - c0, M, den, num);
+    const float r = 1.0f / den;
     __stcg(reinterpret_cast<float4 *>(p.o + static_cast<size_t>(b) * p.Hq * d + (g * G + h) * d + i),
            make_float4(num.x * r, num.y * r, num.z * r, num.w * r));
   }

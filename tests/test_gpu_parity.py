@@ -85,6 +85,22 @@ def test_batch_ragged_history(cuda_device):
     assert_report(rep)
 
 
+def test_long_context_many_attention_chunks(cuda_device):
+    """One sequence over a 1100-token history with 2 KV heads: each head's
+    context splits into about 70 one-page chunks, so the split-attention
+    merge runs over several register batches of chunk partials."""
+    cfg = synth.CONFIGS["tiny"]
+    n = 1100
+    pair = Pair(cfg, _weights(cfg, seed=13), 1, [n + 3])
+    pair.load_history(synth.make_kv_history(cfg, [n], seed=14), [n])
+    ids = synth.make_ids(cfg["vocab"], (3, 1), seed=15)
+    rep = StepReport()
+    for s in range(3):
+        pair.compare(ids[s].tolist(), [n + s], rep)
+    pair.close()
+    assert_report(rep)
+
+
 def test_large_batch_chunked_activations(cuda_device):
     """B = 16 (two mma n-tiles) with activations too wide for one staging
     buffer, so every projection stages its input in column chunks."""
