@@ -2,12 +2,16 @@
 """Decode-step benchmark of the persistent megakernel.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--mode mega|perop] [--impl mk|reference]
+                    [--mode mega|perop|perop-graph] [--impl mk|reference]
 
 A *step* is one greedy decode step of the whole decoder (every layer, LM head
 and argmax) for the workload's batch, i.e. one megakernel launch.  Inputs are
 synthetic (seeded random-init weights and token ids, see
 persistent_task_runtime_b200/synth.py).  Prints ONE JSON line on rank 0.
+
+``--mode perop`` times the comparison build: the same task code launched once
+per operator (embedding, 5 per layer, LM head) on one stream.
+``--mode perop-graph`` replays those launches from a CUDA graph recorded once.
 
 Workloads (default ``8b_b1_ctx512``):
   tiny_b1_p16        2-layer tiny decoder, batch 1, 16-token prompt
@@ -211,7 +215,10 @@ def run_mk(args, rank: int, world: int, local_rank: int) -> dict:
     ids = torch.zeros(B, dtype=torch.int32, device=dev)
     pos = torch.zeros(B, dtype=torch.int32, device=dev)
     nids, npos = torch.zeros_like(ids), torch.zeros_like(pos)
-    mode = mk.MODE_PER_OP if args.mode == "perop" else mk.MODE_MEGAKERNEL
+    mode = {"mega": mk.MODE_MEGAKERNEL, "perop": mk.MODE_PER_OP,
+            "perop-graph": mk.MODE_PER_OP_GRAPH}[args.mode]
+    if mode == mk.MODE_PER_OP_GRAPH:
+        torch.cuda.set_stream(torch.cuda.Stream(dev))   # graph capture needs a created stream
     stream = torch.cuda.current_stream(dev)
 
     if wl["prefill"] == "decode":
@@ -386,7 +393,7 @@ def main():
     ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--workload", default="8b_b1_ctx512")
-    ap.add_argument("--mode", choices=["mega", "perop"], default="mega")
+    ap.add_argument("--mode", choices=["mega", "perop", "perop-graph"], default="mega")
     ap.add_argument("--impl", choices=["mk", "reference"], default="mk")
     ap.add_argument("--e2e-steps", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -156,6 +156,15 @@ MK_API int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *weigh
                                 (embed, then per layer QKV, attention, O,
                                 gate/up, down, then LM head), ordered by the
                                 stream instead of by in-GPU counters        */
+#define MK_MODE_PER_OP_GRAPH 2 /* MK_MODE_PER_OP recorded once as a CUDA graph
+                                and replayed.  The plan keeps the graphs of
+                                the two most recent argument sets (pointers,
+                                batch) and stream, and records a new one for
+                                any other; every replay patches the step
+                                counter into its kernel nodes.  Needs a
+                                created stream (not the legacy default one);
+                                a stream that is being captured is refused
+                                by CUDA (MK_ERR_CUDA).                      */
 
 /* Everything one step reads and writes. */
 typedef struct {

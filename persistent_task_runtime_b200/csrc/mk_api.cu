@@ -47,6 +47,20 @@ namespace mk {
 void set_last_error(const char *msg) { g_err = msg; }
 }  // namespace mk
 
+// A per-operator step recorded as a CUDA graph (MK_MODE_PER_OP_GRAPH): the
+// launches of one set of step arguments on one stream.  A replay patches the
+// step counter into every kernel node.
+struct OpGraph {
+  Params key{};                  // the step's parameters, step counter zeroed
+  cudaStream_t stream = nullptr;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  std::vector<cudaGraphNode_t> nodes;       // kernel nodes
+  std::vector<cudaKernelNodeParams> kp;     // their launch configurations
+  std::vector<Params> params;               // their parameters
+  uint64_t used = 0;                        // last use (least recently used is replaced)
+};
+
 struct mk_plan {
   mk_model_config cfg;
   Params base;  // static part of the kernel parameters
@@ -62,6 +76,8 @@ struct mk_plan {
   int32_t *d_host_ids = nullptr, *d_host_pos = nullptr, *d_host_out = nullptr;
   float *d_host_logits = nullptr;
   mk_plan_info_t info{};
+  OpGraph graphs[2];   // two argument sets: a caller may alternate input/output buffers
+  uint64_t graph_clock = 0;
 };
 
 namespace {
@@ -237,6 +253,88 @@ static int validate_kv(const mk_plan *plan, const mk_kv_cache *kv) {
   return MK_OK;
 }
 
+namespace {
+
+void release_graph(OpGraph &g) {
+  if (g.exec != nullptr) cudaGraphExecDestroy(g.exec);
+  if (g.graph != nullptr) cudaGraphDestroy(g.graph);
+  g = OpGraph{};
+}
+
+// Record the per-operator launches of `p` on `s` into `g`.
+int record_graph(mk_plan *plan, const Params &p, cudaStream_t s, OpGraph &g) {
+  release_graph(g);
+  MK_CUDA(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal));
+  Params q = p;
+  for (const mk::OpRange &r : plan->lay.ops) {
+    q.task_begin = r.begin;
+    q.task_end = r.end;
+    const cudaError_t e = mk::launch_step(q, std::min(plan->grid, r.end - r.begin), plan->smem,
+                                          false, s);
+    if (e != cudaSuccess) {
+      cudaGraph_t partial = nullptr;
+      cudaStreamEndCapture(s, &partial);
+      if (partial != nullptr) cudaGraphDestroy(partial);
+      return fail(MK_ERR_CUDA, "per-op graph capture: %s", cudaGetErrorString(e));
+    }
+  }
+  MK_CUDA(cudaStreamEndCapture(s, &g.graph));
+  MK_CUDA(cudaGraphInstantiate(&g.exec, g.graph, 0));
+  size_t n = 0;
+  MK_CUDA(cudaGraphGetNodes(g.graph, nullptr, &n));
+  std::vector<cudaGraphNode_t> all(n);
+  MK_CUDA(cudaGraphGetNodes(g.graph, all.data(), &n));
+  for (cudaGraphNode_t node : all) {
+    cudaGraphNodeType type;
+    MK_CUDA(cudaGraphNodeGetType(node, &type));
+    if (type != cudaGraphNodeTypeKernel) continue;
+    cudaKernelNodeParams kp{};
+    MK_CUDA(cudaGraphKernelNodeGetParams(node, &kp));
+    g.nodes.push_back(node);
+    g.params.push_back(*static_cast<const Params *>(kp.kernelParams[0]));
+    kp.kernelParams = nullptr;
+    kp.extra = nullptr;
+    g.kp.push_back(kp);
+  }
+  if (g.nodes.size() != plan->lay.ops.size()) {
+    release_graph(g);
+    return fail(MK_ERR_CUDA, "per-op graph holds an unexpected number of kernels");
+  }
+  g.key = p;
+  g.key.epoch = 0;
+  g.stream = s;
+  return MK_OK;
+}
+
+// Replay the per-operator graph for `p` on `s`, recording it first if no
+// recorded graph matches the step's arguments and stream.
+int replay_graph(mk_plan *plan, const Params &p, cudaStream_t s) {
+  Params key = p;
+  key.epoch = 0;
+  OpGraph *g = nullptr;
+  for (OpGraph &c : plan->graphs)
+    if (c.exec != nullptr && c.stream == s && std::memcmp(&c.key, &key, sizeof(Params)) == 0) g = &c;
+  if (g == nullptr) {
+    g = &plan->graphs[0];
+    for (OpGraph &c : plan->graphs)
+      if (c.used < g->used) g = &c;
+    const int rc = record_graph(plan, p, s, *g);
+    if (rc) return rc;
+  }
+  g->used = ++plan->graph_clock;
+  for (size_t i = 0; i < g->nodes.size(); ++i) {
+    g->params[i].epoch = p.epoch;
+    void *args[] = {&g->params[i]};
+    cudaKernelNodeParams kp = g->kp[i];
+    kp.kernelParams = args;
+    MK_CUDA(cudaGraphExecKernelNodeSetParams(g->exec, g->nodes[i], &kp));
+  }
+  MK_CUDA(cudaGraphLaunch(g->exec, s));
+  return MK_OK;
+}
+
+}  // namespace
+
 int mk_decode_step_ex(mk_plan *plan, const mk_step_args *a, void *stream) {
   g_err.clear();
   if (plan == nullptr || a == nullptr) return fail(MK_ERR_INVALID_ARG, "plan or args is NULL");
@@ -244,8 +342,10 @@ int mk_decode_step_ex(mk_plan *plan, const mk_step_args *a, void *stream) {
     return fail(MK_ERR_INVALID_ARG, "batch %d outside 1..max_batch %d", a->batch, plan->max_batch);
   if (a->d_ids == nullptr || a->d_pos == nullptr || a->d_out_ids == nullptr)
     return fail(MK_ERR_INVALID_ARG, "d_ids, d_pos and d_out_ids must not be NULL");
-  if (a->mode != MK_MODE_MEGAKERNEL && a->mode != MK_MODE_PER_OP)
+  if (a->mode != MK_MODE_MEGAKERNEL && a->mode != MK_MODE_PER_OP && a->mode != MK_MODE_PER_OP_GRAPH)
     return fail(MK_ERR_INVALID_ARG, "unknown mode %d", a->mode);
+  if (a->mode == MK_MODE_PER_OP_GRAPH && stream == nullptr)
+    return fail(MK_ERR_INVALID_ARG, "graph mode needs a created stream, not the legacy default stream");
   int rc = validate_kv(plan, a->kv);
   if (rc) return rc;
 
@@ -278,6 +378,12 @@ int mk_decode_step_ex(mk_plan *plan, const mk_step_args *a, void *stream) {
     if (e != cudaSuccess) {
       plan->epoch -= 1;
       return fail(MK_ERR_CUDA, "megakernel launch: %s", cudaGetErrorString(e));
+    }
+  } else if (a->mode == MK_MODE_PER_OP_GRAPH) {
+    const int rc2 = replay_graph(plan, p, s);
+    if (rc2) {
+      plan->epoch -= 1;
+      return rc2;
     }
   } else {
     for (const mk::OpRange &r : plan->lay.ops) {
@@ -399,6 +505,7 @@ int mk_plan_describe(const mk_model_config *cfg, const mk_plan_options *opts, in
 void mk_plan_destroy(mk_plan *plan) {
   if (plan == nullptr) return;
   cudaDeviceSynchronize();
+  for (OpGraph &g : plan->graphs) release_graph(g);
   cudaFree(plan->d_tasks);
   cudaFree(plan->d_rope);
   cudaFree(plan->d_ws);

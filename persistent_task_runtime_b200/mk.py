@@ -27,6 +27,7 @@ MK_MAX_LAYERS = 128
 MK_MAX_BATCH = 16
 MODE_MEGAKERNEL = 0
 MODE_PER_OP = 1
+MODE_PER_OP_GRAPH = 2
 
 ERROR_NAMES = {MK_OK: "MK_OK", MK_ERR_INVALID_ARG: "MK_ERR_INVALID_ARG",
                MK_ERR_UNSUPPORTED: "MK_ERR_UNSUPPORTED", MK_ERR_CUDA: "MK_ERR_CUDA",

@@ -123,29 +123,34 @@ def test_large_batch_chunked_activations(cuda_device):
 
 
 def test_megakernel_equals_per_operator_launches(cuda_device):
-    """Same task code, two schedules: one persistent launch vs one launch per
-    operator.  Results must be bit-identical."""
+    """Same task code, three schedules: one persistent launch, one launch per
+    operator, and the per-operator launches replayed from a CUDA graph (one
+    recording, then replays with the step counter patched in).  Results must
+    be bit-identical."""
     cfg = synth.CONFIGS["tiny"]
     w = _weights(cfg, seed=11)
     B, lengths, steps = 3, [5, 33, 64], 4
     outs = []
-    for mode in (mk.MODE_MEGAKERNEL, mk.MODE_PER_OP):
-        pair = Pair(cfg, w, B, [n + steps for n in lengths])
-        pair.load_history(synth.make_kv_history(cfg, lengths, seed=12), lengths)
-        ids = synth.make_ids(cfg["vocab"], (steps, B), seed=13)
-        rec = []
-        for s in range(steps):
-            rec.append(pair.gpu_step(ids[s].tolist(), [n + s for n in lengths], mode=mode))
-        kvs = [t.clone() for t in pair.kv.k + pair.kv.v]
-        outs.append((rec, kvs))
-        pair.close()
-    (ra, ka), (rb, kb) = outs
-    for (ia, la, ha), (ib, lb, hb) in zip(ra, rb):
-        assert np.array_equal(ia, ib)
-        assert np.array_equal(la, lb)
-        assert np.array_equal(ha, hb)
-    for x, y in zip(ka, kb):
-        assert torch.equal(x, y)
+    stream = torch.cuda.Stream()   # graph capture needs a created stream
+    with torch.cuda.stream(stream):
+        for mode in (mk.MODE_MEGAKERNEL, mk.MODE_PER_OP, mk.MODE_PER_OP_GRAPH):
+            pair = Pair(cfg, w, B, [n + steps for n in lengths])
+            pair.load_history(synth.make_kv_history(cfg, lengths, seed=12), lengths)
+            ids = synth.make_ids(cfg["vocab"], (steps, B), seed=13)
+            rec = []
+            for s in range(steps):
+                rec.append(pair.gpu_step(ids[s].tolist(), [n + s for n in lengths], mode=mode))
+            kvs = [t.clone() for t in pair.kv.k + pair.kv.v]
+            outs.append((rec, kvs))
+            pair.close()
+    (ra, ka) = outs[0]
+    for rb, kb in outs[1:]:
+        for (ia, la, ha), (ib, lb, hb) in zip(ra, rb):
+            assert np.array_equal(ia, ib)
+            assert np.array_equal(la, lb)
+            assert np.array_equal(ha, hb)
+        for x, y in zip(ka, kb):
+            assert torch.equal(x, y)
 
 
 def test_closed_loop_greedy_on_device(cuda_device):
@@ -244,6 +249,11 @@ def test_host_argument_errors(cuda_device):
     pair = Pair(cfg, _weights(cfg, seed=19), 2, [16, 16])
     with pytest.raises(mk.MkError) as e:
         pair.plan.step(pair.d_ids, pair.d_pos, pair.kv.view, pair.d_out, batch=3)
+    assert e.value.code == mk.MK_ERR_INVALID_ARG
+    # graph replay cannot record on the legacy default stream
+    with pytest.raises(mk.MkError) as e:
+        pair.plan.step(pair.d_ids, pair.d_pos, pair.kv.view, pair.d_out, batch=1,
+                       mode=mk.MODE_PER_OP_GRAPH, stream=torch.cuda.default_stream())
     assert e.value.code == mk.MK_ERR_INVALID_ARG
     with pytest.raises(mk.MkError):
         mk.Plan(cfg, _weights(cfg), max_batch=17)
