@@ -116,7 +116,17 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
   return v;
 }
 
-__device__ __forceinline__ void fence_acq_rel() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+// Acquire load.  Re-reading a counter with acquire after a relaxed poll saw it
+// complete orders the producers' writes (published by their release
+// increments) before this thread's later accesses.  It costs a load round
+// trip, where a GPU-scope fence also waits for this thread's outstanding
+// memory operations: 4% of an 8B decode step when both dependency paths
+// used the fence.
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
 __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
   uint32_t old;
@@ -268,7 +278,7 @@ __device__ bool wait_event(const Params &p, Ctl *ctl, uint32_t ev, uint32_t coun
   for (uint32_t it = 0;; ++it) {
     const uint32_t v = ld_relaxed(ctr);
     if (static_cast<int32_t>(v - target) >= 0) {
-      fence_acq_rel();
+      (void)ld_acquire(ctr);
       return true;
     }
     if ((it & 3u) == 3u) {
@@ -532,12 +542,13 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     if (t.type == T_ATTN) attn_resolve(p, B, static_cast<int>(t.aux), info);
     __syncwarp();
     if (lane == 0) {
-      // an input event already complete when the task was popped: order its
-      // producers' writes before the hand-over (the slot barrier publishes
-      // them to the compute warps), which then skip their own wait
+      // an input event already complete when the task was popped: acquire
+      // its producers' writes before the hand-over (the slot barrier, a
+      // CTA-scope release/acquire pair, carries them on to the compute
+      // warps), which then skip their own wait
       if (is_gemv(t.type) && t.dep_event != kNoEvent &&
           static_cast<int32_t>(la_ev - p.epoch * t.dep_count) >= 0) {
-        fence_acq_rel();
+        (void)ld_acquire(p.sync + S_EVENTS + t.dep_event);
         info.dep_ok = 1;
       }
       S = info;
