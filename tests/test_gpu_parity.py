@@ -153,6 +153,57 @@ def test_megakernel_equals_per_operator_launches(cuda_device):
             assert torch.equal(x, y)
 
 
+def test_lm_head_argmax_planted_ties_and_last_tile_maximum(cuda_device):
+    """The argmax over the LM-head tiles picks the lowest index among equal
+    logits, across tiles and inside one, and finds a maximum planted in the
+    last row tile.  The plan reads the weights in place, so rows of the LM
+    head are rewritten between steps.  Copies of a row give bit-equal logits;
+    a row scaled by a power of 2 (exact in bf16) scales the logit exactly."""
+    cfg = synth.CONFIGS["tiny"]
+    V = cfg["vocab"]
+    w = _weights(cfg, seed=21)
+    pair = Pair(cfg, w, 2, [4, 4])
+    ids, pos = [17, 3001], [0, 0]
+    lm = w["lm_head"]
+    orig = lm.clone()
+
+    g_ids, g_logits, _ = pair.gpu_step(ids, pos)
+    top = int(g_ids[0])
+    assert g_logits[0, top] > 0
+    # plant the winner at row 100: 4x the winning row
+    win, nb = 100, 101          # rows 100 and 101 share a row tile and task
+    lm[win] = orig[top] * 4
+    g_ids, g_logits, _ = pair.gpu_step(ids, pos)
+    assert int(g_ids[0]) == win
+    assert g_logits[0, win] == 4 * g_logits[0, top]
+    planted = lm[win].clone()
+
+    # ties: copies of the winning row in the first row, its neighbour and the last row
+    for r in (0, nb, V - 1):
+        lm[r] = planted
+    g_ids, g_logits, _ = pair.gpu_step(ids, pos)
+    for b in range(2):
+        assert int(g_ids[b]) == int(np.argmax(g_logits[b]))
+        for r in (0, nb, V - 1):
+            assert g_logits[b, r] == g_logits[b, win]
+    assert int(g_ids[0]) == 0
+
+    # a tie inside one tile only
+    lm[0] = orig[0]
+    lm[V - 1] = orig[V - 1]
+    g_ids, g_logits, _ = pair.gpu_step(ids, pos)
+    assert g_logits[0, nb] == g_logits[0, win]
+    assert int(g_ids[0]) == win
+
+    # a strict maximum in the last row tile
+    lm[V - 1] = planted * 2
+    g_ids, g_logits, _ = pair.gpu_step(ids, pos)
+    assert g_logits[0, V - 1] == 2 * g_logits[0, win]
+    assert int(g_ids[0]) == V - 1
+    assert int(g_ids[1]) == int(np.argmax(g_logits[1]))
+    pair.close()
+
+
 def test_closed_loop_greedy_on_device(cuda_device):
     """out_ids and out_pos fed straight back as the next step's inputs (no host
     round trip); the token sequence must follow the oracle's greedy decode up
