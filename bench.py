@@ -29,6 +29,7 @@ ranks produced divided by that time.
 from __future__ import annotations
 
 import argparse
+import contextlib
 import hashlib
 import json
 import math
@@ -369,6 +370,16 @@ def cores_used() -> int:
         return os.cpu_count() or 1
 
 
+def oracle_threads(n: int):
+    """(context that limits the oracle's BLAS/OpenMP and torch threads to n,
+    threads used); n <= 0 keeps every core of the process's affinity."""
+    if n <= 0:
+        return contextlib.nullcontext(), cores_used()
+    from threadpoolctl import threadpool_limits
+    torch.set_num_threads(n)
+    return threadpool_limits(limits=n), n
+
+
 def run_reference(args) -> dict:
     wl = parse_workload(args.workload)
     cfg = model_config(wl)
@@ -397,6 +408,8 @@ def main():
     ap.add_argument("--impl", choices=["mk", "reference"], default="mk")
     ap.add_argument("--e2e-steps", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-threads", type=int, default=0,
+                    help="threads for the CPU oracle (0: every core of the affinity mask)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -416,9 +429,10 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        r = run_reference(args)
+        ctx, cores = oracle_threads(args.oracle_threads)
+        with ctx:
+            r = run_reference(args)
         val = r["B"] / r["step_s"]
-        cores = cores_used()
         sample = (f"per step: one decoder layer of one {wl['model']} decode step "
                   f"(batch {r['B']}) timed, x{r['L']} layers + embedding/final-norm/LM-head "
                   f"timed once")
@@ -457,10 +471,12 @@ def main():
             "gpu_launches": K * r["launches_per_step"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         w = cpu_weights_sample(cfg)
-        head_s, layer_s, L = oracle_layer_timing(cfg, r["B"], r["lengths"], w)
+        ctx, cores = oracle_threads(args.oracle_threads)
+        with ctx:
+            head_s, layer_s, L = oracle_layer_timing(cfg, r["B"], r["lengths"], w)
         step_s = head_s + L * layer_s
         line["cpu_baseline"] = {
-            "value": r["B"] / step_s, "unit": UNIT, "cores": cores_used(), "kind": "oracle",
+            "value": r["B"] / step_s, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": (f"one decoder layer + embedding/final-norm/LM-head of one decode step "
                        f"(batch {r['B']}), scaled to {L} layers")}
     if world > 1:
