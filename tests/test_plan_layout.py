@@ -198,3 +198,34 @@ def test_describe_rejects_what_create_rejects():
         mk.describe(SHAPES["tiny"], max_page_cols=100)
     with pytest.raises(mk.MkError):
         mk.describe(SHAPES["tiny"], max_batch=17)
+
+
+def test_describe_argument_errors_and_short_buffer():
+    """NULL config or info and non-positive device sizes are host errors; a
+    task buffer shorter than the plan is left untouched while info is filled."""
+    import ctypes as C
+
+    lib = mk.load_library()
+    cfg = SHAPES["tiny"]
+    c = mk._config(cfg, 64)
+    opts = mk.mk_plan_options(1, 16, 0, 0, (C.c_int * 5)(0, 0, 0, 0, 0), 0, 0, 0)
+    info = mk.mk_plan_info_t()
+    assert lib.mk_plan_describe(None, C.byref(opts), 148, SMEM, C.byref(info), None, 0) == \
+        mk.MK_ERR_INVALID_ARG
+    assert lib.mk_plan_describe(C.byref(c), C.byref(opts), 148, SMEM, None, None, 0) == \
+        mk.MK_ERR_INVALID_ARG
+    assert lib.mk_plan_describe(C.byref(c), C.byref(opts), 0, SMEM, C.byref(info), None, 0) == \
+        mk.MK_ERR_INVALID_ARG
+    assert lib.mk_plan_describe(C.byref(c), C.byref(opts), 148, 0, C.byref(info), None, 0) == \
+        mk.MK_ERR_INVALID_ARG
+    # NULL options take the defaults
+    assert lib.mk_plan_describe(C.byref(c), None, 148, SMEM, C.byref(info), None, 0) == mk.MK_OK
+    n = info.n_tasks
+    buf = np.full(n - 1, 0xAB, dtype=np.uint8).repeat(64)
+    assert lib.mk_plan_describe(C.byref(c), C.byref(opts), 148, SMEM, C.byref(info),
+                                buf.ctypes.data, n - 1) == mk.MK_OK
+    assert info.n_tasks == n and (buf == 0xAB).all()
+    # a smaller device gives fewer CTAs and still a valid graph
+    info2, t2 = mk.describe(cfg, max_batch=2, num_sms=20, max_seq_len=64)
+    assert info2["num_ctas"] == 20
+    check_plan(cfg, info2, t2, 2)
