@@ -14,8 +14,9 @@ Times are GPU global-timer nanoseconds.
 
 from __future__ import annotations
 
+import json
 from collections import defaultdict
-from typing import Dict
+from typing import Dict, Optional
 
 import numpy as np
 
@@ -70,3 +71,31 @@ def summarize(raw: np.ndarray) -> str:
                 parts.append(f"{name} {a:.1f}-{b:.1f}")
         lines.append(f"  L{l}: " + ", ".join(parts))
     return "\n".join(lines)
+
+
+PHASES = (("wait", 2, 3), ("stage", 3, 4), ("pages", 4, 5), ("store", 5, 6))
+
+
+def to_chrome_trace(raw: np.ndarray, path: Optional[str] = None) -> dict:
+    """Chrome trace-event JSON of a step's timeline (open in Perfetto or
+    chrome://tracing): one track per CTA, one complete event per task phase
+    (compute: input wait, staging, pages; storer: release), times in us from
+    the first traced event.  Tasks with an unrecorded mark are left out.
+    Written to `path` when given; returned either way."""
+    d = decode(raw)
+    t, ty, layer, cta, valid = d["t"], d["type"], d["layer"], d["cta"], d["valid"]
+    events = []
+    for i in np.nonzero(valid)[0]:
+        name = TYPE_NAMES.get(int(ty[i]), f"type{int(ty[i])}")
+        for phase, a, b in PHASES:
+            dur = (t[i, b] - t[i, a]) / 1e3
+            if dur <= 0:
+                continue
+            events.append({"name": f"{name} {phase}", "cat": name, "ph": "X",
+                           "ts": t[i, a] / 1e3, "dur": dur, "pid": 0, "tid": int(cta[i]),
+                           "args": {"task": int(i), "layer": int(layer[i])}})
+    doc = {"traceEvents": events, "displayTimeUnit": "ns"}
+    if path is not None:
+        with open(path, "w") as f:
+            json.dump(doc, f)
+    return doc
