@@ -372,10 +372,12 @@ def cores_used() -> int:
 
 def oracle_threads(n: int):
     """(context that limits the oracle's BLAS/OpenMP and torch threads to n,
-    threads used); n <= 0 keeps every core of the process's affinity."""
+    threads used); n <= 0 keeps the process's thread pools as they are and
+    reports their size (torchrun, for one, sets OMP_NUM_THREADS=1)."""
+    from threadpoolctl import threadpool_info, threadpool_limits
     if n <= 0:
-        return contextlib.nullcontext(), cores_used()
-    from threadpoolctl import threadpool_limits
+        pools = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        return contextlib.nullcontext(), max(pools) if pools else cores_used()
     torch.set_num_threads(n)
     return threadpool_limits(limits=n), n
 
@@ -409,7 +411,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-threads", type=int, default=0,
-                    help="threads for the CPU oracle (0: every core of the affinity mask)")
+                    help="threads for the CPU oracle (0: the process's BLAS thread pool as set up)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -15,11 +15,39 @@ def test_oracle_threads_limits_blas_and_reports_the_count():
         assert all(p["num_threads"] == 1 for p in pools)
 
 
-def test_oracle_threads_default_is_every_core():
+def test_oracle_threads_default_reports_the_blas_pool():
     ctx, cores = bench.oracle_threads(0)
-    assert cores == bench.cores_used() >= 1
+    blas = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+    assert cores == (max(blas) if blas else bench.cores_used()) >= 1
     with ctx:
         pass
+
+
+def test_reference_arm_under_torchrun_prints_one_line_from_rank0(tmp_path):
+    """--impl reference under torchrun: rank 0 times the oracle and prints the
+    JSON line, the other rank exits 0 without work."""
+    import json
+    import os
+    import socket
+    import subprocess
+    import sys
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.join(root, "bench.py"), "--impl", "reference", "--workload", "tiny_b1_p16",
+           "--steps", "2", "--warmup", "3", "--gpus", "2"]
+    r = subprocess.run(cmd, cwd=str(tmp_path), capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
 
 
 @pytest.mark.parametrize("name,batch,model", [("8b_b1_ctx512", 1, "8b"),
