@@ -90,3 +90,32 @@ def test_argument_errors_before_any_launch(lib):
     assert lib.mk_plan_status(None) == mk.MK_ERR_INVALID_ARG
     assert lib.mk_plan_reset(None) == mk.MK_ERR_INVALID_ARG
     lib.mk_plan_destroy(None)   # no-op
+
+
+def test_noalloc_argument_errors_before_any_device_call(lib):
+    """mk_decode_step_noalloc checks its arguments on the host first."""
+    cfg = mk.mk_model_config(2, 256, 4, 2, 64, 688, 4096, 1e-6, 1e6, 1, 64)
+    w = mk.mk_weights()
+    lw = (mk.mk_layer_weights * 2)()
+    w.layers = lw
+    kv = mk.mk_kv_cache()
+    a = mk.mk_step_args()
+    a.kv = C.pointer(kv)
+    a.batch = 1
+    E = mk.MK_ERR_INVALID_ARG
+    assert lib.mk_decode_step_noalloc(None, C.byref(w), 16, C.byref(a), None) == E
+    assert lib.mk_decode_step_noalloc(C.byref(cfg), C.byref(w), 16, None, None) == E
+    assert lib.mk_decode_step_noalloc(C.byref(cfg), C.byref(w), 8, C.byref(a), None) == E
+    assert b"kv_page_size" in lib.mk_last_error()
+    a.batch = 0
+    assert lib.mk_decode_step_noalloc(C.byref(cfg), C.byref(w), 16, C.byref(a), None) == E
+    a.batch = 1
+    a.mode = mk.MODE_PER_OP
+    assert lib.mk_decode_step_noalloc(C.byref(cfg), C.byref(w), 16, C.byref(a), None) == E
+    assert b"MK_MODE_MEGAKERNEL" in lib.mk_last_error()
+    a.mode = mk.MODE_MEGAKERNEL
+    # NULL ids / positions / outputs / KV pointers
+    assert lib.mk_decode_step_noalloc(C.byref(cfg), C.byref(w), 16, C.byref(a), None) == E
+    bad = mk.mk_model_config(2, 256, 4, 2, 48, 688, 4096, 1e-6, 1e6, 1, 64)   # head_dim 48
+    assert lib.mk_decode_step_noalloc(C.byref(bad), C.byref(w), 16, C.byref(a), None) == \
+        mk.MK_ERR_UNSUPPORTED
