@@ -321,6 +321,89 @@ def pin_brute_force_micro(O):
         np.testing.assert_allclose(out["logits"][0], ref[t], rtol=1e-10, atol=1e-12)
 
 
+def pin_greedy_decode_hand_loop(O):
+    """greedy_decode against two things it must equal on tiny inputs:
+    a hand-written loop over decode_step (teacher-forced prompt at positions
+    0..n-1, first token = argmax after the last prompt token, token s-1 fed
+    at position n+s-1), and the brute-force scalar decoder run over the
+    prompt followed by the generated tokens (its logits at positions
+    n-1 .. n+steps-2 are the greedy steps' logits)."""
+    for base, seed in ((MICRO, 31), (synth.CONFIGS["tiny"], 32)):
+        d = dict(base)
+        cfg = _cfg(O, d)
+        w, W = _weights(O, d, seed=seed)
+        n, steps = 5, 4
+        prompts = [synth.make_ids(d["vocab"], (n,), seed=seed + 1).tolist(),
+                   synth.make_ids(d["vocab"], (n,), seed=seed + 2).tolist()]
+        got = O.greedy_decode(cfg, W, prompts, steps)
+        assert got["logits"].shape == (steps, 2, d["vocab"])
+        # hand loop, one sequence at a time
+        for b, prompt in enumerate(prompts):
+            cache = O.KVCache(cfg, 1, n + steps)
+            for t in range(n):
+                out = O.decode_step(cfg, W, cache, [prompt[t]], [t])
+            toks, logits = [], []
+            for s in range(steps):
+                logits.append(out["logits"][0])
+                tok = int(np.argmax(out["logits"][0]))
+                toks.append(tok)
+                if s + 1 < steps:
+                    out = O.decode_step(cfg, W, cache, [tok], [n + s])
+            np.testing.assert_allclose(got["logits"][:, b], np.stack(logits), rtol=1e-10,
+                                       atol=1e-11)
+            assert got["tokens"][:, b].tolist() == toks
+            np.testing.assert_allclose(got["margins"][:, b],
+                                       [np.sort(x)[-1] - np.sort(x)[-2] for x in logits],
+                                       rtol=0, atol=1e-12)
+            if base is MICRO:
+                # scalar-loop decoder over prompt + generated tokens
+                ref = _bf_decoder(w, d, prompt + toks[:-1])
+                np.testing.assert_allclose(got["logits"][:, b], ref[n - 1:], rtol=1e-10,
+                                           atol=1e-12)
+        # forced tokens replace the fed ones
+        force = np.array([[1, 2], [3, 4], [5, 6]])
+        fz = O.greedy_decode(cfg, W, prompts, steps, force=force)
+        np.testing.assert_allclose(fz["logits"][0], got["logits"][0], rtol=0, atol=0)
+        if base is MICRO:
+            for b, prompt in enumerate(prompts):
+                ref = _bf_decoder(w, d, prompt + force[:, b].tolist())
+                np.testing.assert_allclose(fz["logits"][:, b], ref[n - 1:], rtol=1e-10,
+                                           atol=1e-12)
+
+
+def pin_prefill_equals_incremental(O):
+    """prefill (whole-sequence pass installed into a cache) against feeding
+    the prompt one decode step at a time: the same bf16 K/V at every cached
+    position, the same last-position logits, and a later decode step from
+    either cache gives the same result.  Two prompts of different lengths."""
+    d = dict(synth.CONFIGS["tiny"])
+    cfg = _cfg(O, d)
+    _, W = _weights(O, d, seed=33)
+    prompts = [synth.make_ids(d["vocab"], (7,), seed=34).tolist(),
+               synth.make_ids(d["vocab"], (4,), seed=35).tolist()]
+    cap = 12
+    cache, last, outs = O.prefill(cfg, W, prompts, cap)
+    assert last.shape == (2, d["vocab"]) and len(outs) == 2
+    for b, prompt in enumerate(prompts):
+        inc = O.KVCache(cfg, 1, cap)
+        for t, tok in enumerate(prompt):
+            out = O.decode_step(cfg, W, inc, [tok], [t])
+        n = len(prompt)
+        assert cache.length[b] == n
+        np.testing.assert_allclose(last[b], out["logits"][0], rtol=1e-10, atol=1e-11)
+        for l in range(cfg.n_layers):
+            np.testing.assert_allclose(cache.k[l][b][:, :n], inc.k[l][0][:, :n], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(cache.v[l][b][:, :n], inc.v[l][0][:, :n], rtol=0, atol=1e-12)
+            # nothing beyond the prompt is written
+            assert not np.any(cache.k[l][b][:, n:]) and not np.any(cache.v[l][b][:, n:])
+        nxt_a = O.decode_step(cfg, W, inc, [9], [n])
+        one = O.KVCache(cfg, 1, cap)
+        for l in range(cfg.n_layers):
+            one.load_history(l, 0, cache.k[l][b][:, :n], cache.v[l][b][:, :n])
+        nxt_b = O.decode_step(cfg, W, one, [9], [n])
+        np.testing.assert_allclose(nxt_a["logits"], nxt_b["logits"], rtol=1e-10, atol=1e-11)
+
+
 # ------------------------------------------ torch library composition ------
 
 
@@ -385,7 +468,7 @@ ALL_PINS = [
     pin_round_bf16, pin_rms_norm, pin_rope, pin_silu_softmax, pin_attend, pin_top2_argmax,
     pin_incremental_equals_full, pin_causality, pin_batch_rows_independent,
     pin_gqa_head_mapping, pin_mha_equals_expanded_gqa, pin_brute_force_micro,
-    pin_torch_composition_tiny,
+    pin_torch_composition_tiny, pin_greedy_decode_hand_loop, pin_prefill_equals_incremental,
 ]
 
 

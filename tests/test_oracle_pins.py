@@ -42,6 +42,12 @@ MUTATIONS = {
     "qk_norm_dropped": ("if cfg.qk_norm:", "if False:"),
     "silu_sign": ("z / (1.0 + np.exp(-z))", "z / (1.0 + np.exp(z))"),
     "softmax_no_norm": ("e / np.sum(e, axis=-1, keepdims=True)", "e"),
+    "greedy_position_off_by_one": ("[n + s - 1] * len(prompts)", "[n + s] * len(prompts)"),
+    "greedy_first_token_wrong_row": ('last.append(out["logits"][-1])',
+                                     'last.append(out["logits"][-2])'),
+    "prefill_drops_last_position": ("cache.load_history(l, b, out[\"k\"][l], out[\"v\"][l])",
+                                    "cache.load_history(l, b, out[\"k\"][l][:, :-1], "
+                                    "out[\"v\"][l][:, :-1])"),
 }
 
 
