@@ -61,6 +61,10 @@ def parse_workload(name: str) -> dict:
     if name == "8b4l_b1_ctx512":
         # profiling case: 8B-shaped layers, 4 of them, same kernel (not a bench line)
         return dict(model="8b", layers=4, batch=1, lengths=[512], prefill="synthetic")
+    if name.startswith("8b4l_b") and name.endswith("_ctx1024"):
+        # profiling case: 8B-shaped layers, 4 of them, batch B at context 1024
+        B = int(name[len("8b4l_b"):-len("_ctx1024")])
+        return dict(model="8b", layers=4, batch=B, lengths=[1024] * B, prefill="synthetic")
     if name.startswith("8b_b") and name.endswith("_ctx1024"):
         B = int(name[len("8b_b"):-len("_ctx1024")])
         return dict(model="8b", batch=B, lengths=[1024] * B, prefill="synthetic")
@@ -461,7 +465,11 @@ def main():
     achieved = r["step_bytes"] / (r["mean_launch_ms"] / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": profiled_traffic(args.workload), "peak_source": peaks["source"],
+                "traffic": profiled_traffic(args.workload),
+                "traffic_source": ("ncu DRAM bytes of one launch, read from the committed "
+                                   f"profiles/mk_decode_step_{args.workload}.md, used only while "
+                                   "the kernel sources hash to the digest recorded there"),
+                "peak_source": peaks["source"],
                 "bytes_per_step": int(r["step_bytes"]), "kernel_us": 1e3 * r["mean_launch_ms"],
                 "vs_8tbs": round(achieved / 8000.0, 4)}
     line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,

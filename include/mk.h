@@ -276,11 +276,17 @@ MK_API void mk_plan_destroy(mk_plan *plan);
  *
  * The caller passes the model, the weights, the KV page size and the step
  * exactly as for a plan built with max_batch = args->batch; args->mode must
- * be MK_MODE_MEGAKERNEL.  Each call rebuilds and uploads the tables, zeroes
- * the counters, launches on `stream`, synchronizes it and returns the device
- * status (MK_OK, MK_ERR_RANGE, MK_ERR_TIMEOUT) or a host error code.  A shape,
- * batch or max_seq_len whose scratch would exceed the array is rejected with
- * MK_ERR_UNSUPPORTED and a message in mk_last_error().
+ * be MK_MODE_MEGAKERNEL and args->d_trace NULL (MK_ERR_INVALID_ARG
+ * otherwise: a trace buffer is sized by a plan's task count).  A call builds
+ * the plan layout on the host and uploads its task array and RoPE table into
+ * the array, unless the previous call on this device had the same model,
+ * weight pointers, batch and page size (then both are reused; building them
+ * costs tens of milliseconds of host time for an 8B-shaped model).  Every
+ * call zeroes the counters, launches on `stream`, synchronizes it and
+ * returns the device status (MK_OK, MK_ERR_RANGE, MK_ERR_TIMEOUT) or a host
+ * error code.  A shape, batch or max_seq_len whose scratch would exceed the
+ * array is rejected with MK_ERR_UNSUPPORTED and a message in
+ * mk_last_error().
  *
  * Every call uses the same array and leaves the previous call's contents
  * behind: calls that overlap on the GPU (several streams or threads) race

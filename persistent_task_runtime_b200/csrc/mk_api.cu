@@ -229,7 +229,7 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   plan->d_host_pos = plan->d_host_ids + MK_MAX_BATCH;
   plan->d_host_out = plan->d_host_pos + MK_MAX_BATCH;
 
-  e = mk::configure_kernel(lay.smem);
+  e = mk::configure_kernel(smem_optin);
   if (e != cudaSuccess) return cleanup_fail(fail(MK_ERR_CUDA, "kernel attribute: %s", cudaGetErrorString(e)));
 
   fill_info(lay, *cfg, plan->info);

@@ -203,7 +203,8 @@ void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vect
 
 cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative,
                         cudaStream_t stream);
-cudaError_t configure_kernel(int smem);
+// Allow the kernel the device's opt-in shared memory (capped at kMaxSmem).
+cudaError_t configure_kernel(int smem_optin);
 void set_last_error(const char *msg);  // message returned by mk_last_error()
 
 }  // namespace mk

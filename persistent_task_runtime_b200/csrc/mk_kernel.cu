@@ -1698,8 +1698,14 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   }
 }
 
-cudaError_t configure_kernel(int smem) {
-  return cudaFuncSetAttribute(mk_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+// The kernel's dynamic shared-memory limit on the current device is set to
+// the most any layout may use there (every layout stays within
+// min(device opt-in, kMaxSmem)), never to one plan's own size: plans of
+// different shapes and the no-allocation entry point share the kernel, and a
+// later, smaller setting would fail the launches of an earlier, larger one.
+cudaError_t configure_kernel(int smem_optin) {
+  const int lim = smem_optin < kMaxSmem ? smem_optin : kMaxSmem;
+  return cudaFuncSetAttribute(mk_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
 }
 
 cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative, cudaStream_t stream) {

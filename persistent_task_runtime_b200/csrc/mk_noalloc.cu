@@ -10,9 +10,11 @@
 // GPU which loads this library keeps until the process exits.
 //
 // The step runs the same persistent kernel as mk_decode_step(); only the
-// place its scratch comes from differs.  Each call rebuilds the task array on
-// the host, uploads it and the tables into the array, zeroes the counters and
-// the argmax slots, launches, synchronizes and returns the device status.
+// place its scratch comes from differs.  A call builds the plan layout on the
+// host and uploads the task array and the RoPE table into the array unless
+// the previous upload on this device was for the same model, weights, batch,
+// page size and device (then it reuses them); every call zeroes the counters
+// and the argmax slots, launches, synchronizes and returns the device status.
 // Calls share the one array, so calls that overlap on the GPU (two streams,
 // two threads) race and must not be issued.  The first call on a device looks
 // up the array's device address (cudaGetSymbolAddress) and sets the kernel's
@@ -37,7 +39,30 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[MK_NOALLOC_SCRATCH_BYT
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_scratch_addr[kMaxDevices] = {};
-int g_scratch_smem[kMaxDevices] = {};
+bool g_configured[kMaxDevices] = {};
+
+// What the array holds on one device: the layout last uploaded into it and
+// the inputs it was built from.  A call with the same key reuses the task
+// array and the RoPE table already in the array.
+struct Uploaded {
+  bool valid = false;
+  mk_model_config cfg{};
+  int page = 0, batch = 0, nsm = 0, smem_optin = 0;
+  std::vector<const void *> ptrs;   // every weight pointer, in a fixed order
+  mk::Layout lay;
+  size_t o_tasks = 0, o_rope = 0, o_ws = 0, o_sync = 0;
+};
+Uploaded g_up[kMaxDevices];
+
+std::vector<const void *> weight_ptrs(const mk_model_config &c, const mk_weights &w) {
+  std::vector<const void *> v = {w.embed, w.final_norm, w.lm_head};
+  for (int l = 0; l < c.n_layers; ++l) {
+    const mk_layer_weights &s = w.layers[l];
+    v.insert(v.end(), {s.attn_norm, s.wq, s.wk, s.wv, s.q_norm, s.k_norm, s.wo, s.mlp_norm,
+                       s.w_gate, s.w_up, s.w_down});
+  }
+  return v;
+}
 
 int nfail(int code, const char *msg) {
   mk::set_last_error(msg);
@@ -68,6 +93,9 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
   if (B < 1 || B > MK_MAX_BATCH) return nfail(MK_ERR_INVALID_ARG, "batch outside 1..16");
   if (a->mode != MK_MODE_MEGAKERNEL)
     return nfail(MK_ERR_INVALID_ARG, "only MK_MODE_MEGAKERNEL is available without allocation");
+  if (a->d_trace != nullptr)
+    return nfail(MK_ERR_INVALID_ARG,
+                 "d_trace is not available without a plan (its size is the plan's task count)");
   if (a->d_ids == nullptr || a->d_pos == nullptr || a->d_out_ids == nullptr ||
       a->kv->k_pages == nullptr || a->kv->v_pages == nullptr || a->kv->block_table == nullptr ||
       a->kv->num_pages < 1 || a->kv->max_pages_per_seq < 1)
@@ -94,65 +122,81 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
           cudaSuccess)
     return nfail(MK_ERR_CUDA, "device attribute query failed");
 
-  // the layout of a plan built for max_batch = B with default options
-  mk::LayoutOptions lo;
-  lo.max_batch = B;
-  lo.page_size = P;
-  mk::Layout lay;
-  std::string err;
-  int rc = mk::build_layout(c, lo, nsm, smem_optin, lay, err);
-  if (rc) return nfail(rc, err.c_str());
+  std::lock_guard<std::mutex> lock(g_mu);
+  // ---- once per device: the array's device address, the kernel's smem cap
+  if (g_scratch_addr[dev] == nullptr) {
+    void *ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr)
+      return nfail(MK_ERR_CUDA, "cudaGetSymbolAddress of the scratch array failed");
+    g_scratch_addr[dev] = ptr;
+  }
+  if (!g_configured[dev]) {
+    if (mk::configure_kernel(smem_optin) != cudaSuccess)
+      return nfail(MK_ERR_CUDA, "setting the kernel's shared-memory limit failed");
+    g_configured[dev] = true;
+  }
+  char *base = static_cast<char *>(g_scratch_addr[dev]);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // ---- the layout of a plan built for max_batch = B with default options:
+  // built and uploaded unless the array already holds it
+  Uploaded &up = g_up[dev];
+  std::vector<const void *> ptrs = weight_ptrs(c, *w);
+  const bool same = up.valid && std::memcmp(&up.cfg, &c, sizeof(c)) == 0 && up.page == P &&
+                    up.batch == B && up.nsm == nsm && up.smem_optin == smem_optin &&
+                    up.ptrs == ptrs;
+  if (!same) {
+    up.valid = false;
+    mk::LayoutOptions lo;
+    lo.max_batch = B;
+    lo.page_size = P;
+    std::string err;
+    const int rc = mk::build_layout(c, lo, nsm, smem_optin, up.lay, err);
+    if (rc) return nfail(rc, err.c_str());
+    mk::bind_task_operands(c, *w, up.lay.tasks);
+    // ---- layout inside the static array -----------------------------------
+    size_t off = 0;
+    auto carve = [&](size_t bytes) {
+      const size_t at = off;
+      off = align_up_z(off + bytes, 256);
+      return at;
+    };
+    up.o_tasks = carve(up.lay.tasks.size() * sizeof(Task));
+    up.o_rope = carve(up.lay.rope.size() * sizeof(float2));
+    up.o_ws = carve(up.lay.ws_bytes);
+    up.o_sync = carve(up.lay.sync_words * sizeof(uint32_t));
+    if (off > MK_NOALLOC_SCRATCH_BYTES) {
+      char msg[256];
+      snprintf(msg, sizeof(msg),
+               "this model/batch/max_seq_len needs %zu bytes of scratch; the no-allocation entry "
+               "point has %u (MK_NOALLOC_SCRATCH_BYTES)",
+               off, static_cast<unsigned>(MK_NOALLOC_SCRATCH_BYTES));
+      return nfail(MK_ERR_UNSUPPORTED, msg);
+    }
+    if (cudaMemcpyAsync(base + up.o_tasks, up.lay.tasks.data(), up.lay.tasks.size() * sizeof(Task),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(base + up.o_rope, up.lay.rope.data(), up.lay.rope.size() * sizeof(float2),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return nfail(MK_ERR_CUDA, "uploading the step's tables into the scratch array failed");
+    up.cfg = c;
+    up.page = P;
+    up.batch = B;
+    up.nsm = nsm;
+    up.smem_optin = smem_optin;
+    up.ptrs = std::move(ptrs);
+    up.valid = true;
+  }
+  const mk::Layout &lay = up.lay;
   Params p = lay.p;
   const int grid = lay.grid, smem = lay.smem;
-  mk::bind_task_operands(c, *w, lay.tasks);
-
-  // ---- layout inside the static array -------------------------------------
-  size_t off = 0;
-  auto carve = [&](size_t bytes) {
-    const size_t at = off;
-    off = align_up_z(off + bytes, 256);
-    return at;
-  };
-  const size_t o_tasks = carve(lay.tasks.size() * sizeof(Task));
-  const size_t o_rope = carve(lay.rope.size() * sizeof(float2));
-  const size_t o_ws = carve(lay.ws_bytes);
-  const size_t o_sync = carve(lay.sync_words * sizeof(uint32_t));
-  if (off > MK_NOALLOC_SCRATCH_BYTES) {
-    char msg[256];
-    snprintf(msg, sizeof(msg),
-             "this model/batch/max_seq_len needs %zu bytes of scratch; the no-allocation entry "
-             "point has %u (MK_NOALLOC_SCRATCH_BYTES)",
-             off, static_cast<unsigned>(MK_NOALLOC_SCRATCH_BYTES));
-    return nfail(MK_ERR_UNSUPPORTED, msg);
+  const size_t o_tasks = up.o_tasks, o_rope = up.o_rope, o_ws = up.o_ws, o_sync = up.o_sync;
+  // the counters and the argmax slots start every call at zero
+  if (cudaMemsetAsync(base + o_ws + lay.o_arg, 0, sizeof(unsigned long long) * B, s) != cudaSuccess ||
+      cudaMemsetAsync(base + o_sync, 0, lay.sync_words * sizeof(uint32_t), s) != cudaSuccess) {
+    up.valid = false;
+    return nfail(MK_ERR_CUDA, "clearing the counters in the scratch array failed");
   }
-
-  // ---- once per device: the array's device address, the kernel's smem cap
-  char *base = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-      void *ptr = nullptr;
-      const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-      if (e != cudaSuccess || ptr == nullptr)
-        return nfail(MK_ERR_CUDA, "cudaGetSymbolAddress of the scratch array failed");
-      g_scratch_addr[dev] = ptr;
-    }
-    if (g_scratch_smem[dev] < smem) {
-      if (mk::configure_kernel(smem) != cudaSuccess)
-        return nfail(MK_ERR_CUDA, "setting the kernel's shared-memory limit failed");
-      g_scratch_smem[dev] = smem;
-    }
-    base = static_cast<char *>(g_scratch_addr[dev]);
-  }
-
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(base + o_tasks, lay.tasks.data(), lay.tasks.size() * sizeof(Task),
-                      cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(base + o_rope, lay.rope.data(), lay.rope.size() * sizeof(float2),
-                      cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemsetAsync(base + o_ws + lay.o_arg, 0, sizeof(unsigned long long) * B, s) != cudaSuccess ||
-      cudaMemsetAsync(base + o_sync, 0, lay.sync_words * sizeof(uint32_t), s) != cudaSuccess)
-    return nfail(MK_ERR_CUDA, "uploading the step's tables into the scratch array failed");
 
   p.tasks = reinterpret_cast<const Task *>(base + o_tasks);
   p.rope_cs = reinterpret_cast<const float2 *>(base + o_rope);

@@ -302,7 +302,8 @@ class Plan:
 
 def decode_step_noalloc(plan_like: "Plan", ids: torch.Tensor, pos: torch.Tensor, kv: KVCacheView,
                         out_ids: torch.Tensor, out_logits: Optional[torch.Tensor] = None,
-                        page_size: int = 16, stream=None) -> int:
+                        page_size: int = 16, stream=None,
+                        trace: Optional[torch.Tensor] = None) -> int:
     """mk_decode_step_noalloc: one step with no device allocation by the library.
 
     ``plan_like`` only supplies the model config and weight pointers (its
@@ -310,7 +311,7 @@ def decode_step_noalloc(plan_like: "Plan", ids: torch.Tensor, pos: torch.Tensor,
     the device status (raises on host-side errors)."""
     lib = load_library()
     a = mk_step_args(_ptr(ids), _ptr(pos), C.pointer(kv.struct), ids.shape[0], _ptr(out_ids),
-                     _ptr(out_logits), None, None, MODE_MEGAKERNEL, None)
+                     _ptr(out_logits), None, None, MODE_MEGAKERNEL, _ptr(trace))
     rc = lib.mk_decode_step_noalloc(C.byref(plan_like._c), C.byref(plan_like._w), page_size,
                                     C.byref(a), _stream_handle(stream))
     if rc in (MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_CUDA):

@@ -155,7 +155,20 @@ class Pair:
         self.plan.close()
 
 
+#: Every report checked in this process, with the test that produced it; the
+#: session summary (tests/conftest.py) prints them, so the margins left under
+#: the tolerances are visible in a passing run's log.
+REPORTS: List[tuple] = []
+
+
+def record(rep: StepReport):
+    import os
+    name = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    REPORTS.append((name, rep))
+
+
 def assert_report(rep: StepReport):
+    record(rep)
     assert rep.max_hidden_rel <= HIDDEN_RTOL, rep
     assert rep.max_logit_err <= LOGITS_ATOL, rep
     assert rep.token_mismatch == 0, rep

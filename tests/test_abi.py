@@ -114,6 +114,10 @@ def test_noalloc_argument_errors_before_any_device_call(lib):
     assert lib.mk_decode_step_noalloc(C.byref(cfg), C.byref(w), 16, C.byref(a), None) == E
     assert b"MK_MODE_MEGAKERNEL" in lib.mk_last_error()
     a.mode = mk.MODE_MEGAKERNEL
+    a.d_trace = 0x1000   # a trace buffer is sized by a plan's task count
+    assert lib.mk_decode_step_noalloc(C.byref(cfg), C.byref(w), 16, C.byref(a), None) == E
+    assert b"d_trace" in lib.mk_last_error()
+    a.d_trace = None
     # NULL ids / positions / outputs / KV pointers
     assert lib.mk_decode_step_noalloc(C.byref(cfg), C.byref(w), 16, C.byref(a), None) == E
     bad = mk.mk_model_config(2, 256, 4, 2, 48, 688, 4096, 1e-6, 1e6, 1, 64)   # head_dim 48

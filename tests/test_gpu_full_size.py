@@ -6,8 +6,8 @@ synthetic: the GPU cache and the oracle's cache receive the same bf16 values,
 so one decode step can be checked without replaying a long prompt.  At batch
 16 with ragged contexts up to 8192 tokens, all 16 sequences run in one GPU
 step and the oracle recomputes three of them (the shortest, the median and
-the longest); the batch sweep at context 1024 (4 and 8 sequences) is checked
-the same way.  Decode treats sequences independently, so every sampled
+the longest); the batch sweep at context 1024 (1, 2, 4, 8 and 16 sequences)
+is checked the same way.  Decode treats sequences independently, so every sampled
 output has a plain reference value.  Tolerances are those of
 tests/gpu_harness.py.
 
@@ -45,8 +45,11 @@ def test_full_size_batch1(cuda_device, name, ctx, steps):
 SAMPLED = {
     # the batch sweep at context 1024 (two sequences recomputed) and the
     # ragged batch of 16 (shortest, median, longest recomputed)
+    "b1_ctx1024": (1, lambda: [1024]),
+    "b2_ctx1024": (2, lambda: [1024] * 2),
     "b4_ctx1024": (4, lambda: [1024] * 4),
     "b8_ctx1024": (8, lambda: [1024] * 8),
+    "b16_ctx1024": (16, lambda: [1024] * 16),
     "b16_ragged": (16, lambda: synth.ragged_lengths(16, 32, 8192, seed=2)),
 }
 
