@@ -215,7 +215,8 @@ def run_mk(args, rank: int, world: int, local_rank: int) -> dict:
     weights = synth.make_weights(cfg, seed=0, device=dev)
     cap = [n + horizon for n in lengths]
     kv = PagedKVCache(cfg, B, cap, page=16, device=dev)
-    plan = mk.Plan(cfg, weights, max_batch=B, page_size=16, max_seq_len=max(cap) + 16)
+    plan = mk.Plan(cfg, weights, max_batch=B, page_size=16, max_seq_len=max(cap) + 16,
+                   gemv_path=args.gemv_path, schedule=args.schedule)
     info = plan.info()
     ids = torch.zeros(B, dtype=torch.int32, device=dev)
     pos = torch.zeros(B, dtype=torch.int32, device=dev)
@@ -318,6 +319,7 @@ def run_mk(args, rank: int, world: int, local_rank: int) -> dict:
                "us_per_step": 1e6 * e2e_s / n, "steps": n}
     plan.close()
     return dict(elapsed_ms=elapsed_ms, mean_launch_ms=mean_launch_ms, step_bytes=step_bytes,
+                launch_ms=launch_ms,
                 kv_bytes=kvb, weight_bytes=info["weight_bytes"], info=info, clocks=clk.summary(),
                 e2e=e2e, cfg=cfg, B=B, lengths=lengths, mode=args.mode, start_pos=start_pos,
                 launches_per_step=(1 if mode == mk.MODE_MEGAKERNEL else
@@ -413,6 +415,10 @@ def main():
     ap.add_argument("--mode", choices=["mega", "perop", "perop-graph"], default="mega")
     ap.add_argument("--impl", choices=["mk", "reference"], default="mk")
     ap.add_argument("--e2e-steps", type=int, default=32)
+    ap.add_argument("--gemv-path", type=int, default=0, choices=[0, 1, 2],
+                    help="projections: 0 automatic, 1 mma.sync pages, 2 tcgen05 tiles")
+    ap.add_argument("--schedule", type=int, default=0, choices=[0, 1],
+                    help="0 dynamic ticket queue, 1 solidified per-CTA task lists")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-threads", type=int, default=0,
                     help="threads for the CPU oracle (0: the process's BLAS thread pool as set up)")
@@ -477,6 +483,14 @@ def main():
             "us_per_step": round(1e3 * ms_per_step, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": config, "mode": r["mode"],
+            "plan": {"gemv_path": r["info"]["gemv_path"], "schedule": r["info"]["schedule"],
+                     "n_tasks": r["info"]["n_tasks"]},
+            "step_us": {"mean": round(1e3 * statistics.mean(r["launch_ms"]), 1),
+                        "p50": round(1e3 * statistics.median(r["launch_ms"]), 1),
+                        "min": round(1e3 * min(r["launch_ms"]), 1),
+                        "max": round(1e3 * max(r["launch_ms"]), 1),
+                        "std": round(1e3 * (statistics.pstdev(r["launch_ms"])
+                                            if len(r["launch_ms"]) > 1 else 0.0), 2)},
             "roofline": roofline, "clocks": r["clocks"], "e2e": r["e2e"],
             "gpu_launches": K * r["launches_per_step"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

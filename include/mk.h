@@ -136,7 +136,27 @@ typedef struct {
   int o_split;            /* nonzero: split the O projection along K into two
                              parts of whole KV groups, each waiting only for
                              the attention of its groups (needs >= 2 KV heads
-                             and >= 1024 columns per part); 0 = one part   */
+                             and >= 1024 columns per part); 0 = one part.
+                             mma.sync path only                             */
+  int gemv_path;          /* how the projections run: 0 = automatic (tensor
+                             cores when max_batch >= 5 and the shape allows),
+                             1 = CUDA-core mma.sync over 16-row weight pages,
+                             2 = tcgen05 tensor cores over 128-row tiles: the
+                             weights arrive by TMA tensor copies in the
+                             swizzled layout the MMA reads, the activation is
+                             staged as bf16 high/low halves, accumulators sit
+                             in tensor memory.  2 needs head_dim 128 and
+                             hidden, ffn and n_q_heads*head_dim multiples of
+                             64 (else MK_ERR_UNSUPPORTED); rows_per_task,
+                             max_page_cols and o_split apply to path 1 only */
+  int schedule;           /* 0 = dynamic: every CTA takes the next task from
+                             one in-GPU ticket queue; 1 = solidified: the
+                             plan assigns each CTA its task list offline (list
+                             scheduling in queue order under a cost model of
+                             weight bytes per task; the Ada-MK summary's
+                             offline path solidification) and each CTA runs
+                             its list in order.  Per-operator modes always
+                             use the queue                                  */
 } mk_plan_options;
 
 typedef struct mk_plan mk_plan;
@@ -234,6 +254,10 @@ typedef struct {
   int ffn_parts, ffn_part_cols; /* split-K parts of the down projection and
                              columns per part (1 part: ffn_part_cols = ffn) */
   int o_parts, o_part_cols; /* the same for the O projection               */
+  int gemv_path;          /* the path the plan uses: 1 mma.sync, 2 tcgen05  */
+  int schedule;           /* 0 dynamic queue, 1 solidified per-CTA lists    */
+  int qkv_parts, gateup_parts; /* split-K parts of the QKV and gate/up
+                             projections (tensor-core path; 1 otherwise)   */
 } mk_plan_info_t;
 MK_API int mk_plan_info(const mk_plan *plan, mk_plan_info_t *info);
 
@@ -246,7 +270,8 @@ MK_API int mk_plan_info(const mk_plan *plan, mk_plan_info_t *info);
  *   of the input event per step, 20-23 output event (0xffffffff: none; a QKV
  *   task signals attn_ready of its head's KV group), 24-27 aux (QKV: 0 q,
  *   1 k, 2 v; attention: slot), 28-31 aux2 (QKV: head index over q, k, v),
- *   32-63 operand pointers (NULL in a described plan). */
+ *   32-55 operand pointers (NULL in a described plan), 56-59 and 60-63
+ *   tensor-map indices of the task's matrices (tensor-core path). */
 #define MK_TASK_RECORD_BYTES 64
 
 /* Describe, without any GPU, the plan mk_plan_create_ex(cfg, weights, opts)
@@ -257,6 +282,16 @@ MK_API int mk_plan_info(const mk_plan *plan, mk_plan_info_t *info);
 MK_API int mk_plan_describe(const mk_model_config *cfg, const mk_plan_options *opts,
                             int num_sms, int smem_optin, mk_plan_info_t *info,
                             void *tasks, int64_t max_tasks);
+
+/* The CTA each task of that plan runs on under a solidified schedule
+ * (opts->schedule == 1), without any GPU: cta_of_task[i] for i < n_tasks,
+ * or -1 for every task when the plan uses the dynamic queue.  Each CTA runs
+ * its tasks in ascending index order.  MK_ERR_INVALID_ARG if max_tasks is
+ * below the plan's task count. */
+MK_API int mk_plan_describe_schedule(const mk_model_config *cfg,
+                                     const mk_plan_options *opts, int num_sms,
+                                     int smem_optin, int32_t *cta_of_task,
+                                     int64_t max_tasks);
 
 /* Message of the last error on the calling thread ("" if none). */
 MK_API const char *mk_last_error(void);

@@ -70,7 +70,8 @@ struct mk_plan {
   int max_batch = 1;
   uint32_t epoch = 0;
   mk::Layout lay;           // tasks, per-operator ranges, workspace layout
-  void *d_tasks = nullptr, *d_rope = nullptr, *d_ws = nullptr;
+  void *d_tasks = nullptr, *d_rope = nullptr, *d_ws = nullptr, *d_maps = nullptr;
+  void *d_sched = nullptr;   // solidified schedule: offsets [grid + 1], then task indices
   uint32_t *d_sync = nullptr;
   size_t sync_words = 0;
   int32_t *d_host_ids = nullptr, *d_host_pos = nullptr, *d_host_out = nullptr;
@@ -113,6 +114,8 @@ int layout_options(const mk_plan_options *opts, mk::LayoutOptions &lo) {
   lo.num_ctas = o.num_ctas;
   lo.max_page_cols = o.max_page_cols;
   lo.o_split = o.o_split != 0;
+  lo.gemv_path = o.gemv_path;
+  lo.schedule = o.schedule;
   for (int i = 0; i < 5; ++i) lo.rows_per_task[i] = o.rows_per_task[i];
   lo.wait_limit_ns = o.wait_limit_ns == 0 ? 2000000000LL : o.wait_limit_ns;
   lo.debug_unsatisfiable_dep = o.debug_unsatisfiable_dep != 0;
@@ -145,6 +148,14 @@ void fill_info(const mk::Layout &lay, const mk_model_config &c, mk_plan_info_t &
   I.ffn_part_cols = p.kchunk[mk::K_FFN] > 0 ? p.kchunk[mk::K_FFN] : F;
   I.o_parts = p.n_o_parts;
   I.o_part_cols = p.kchunk[mk::K_ATT] > 0 ? p.kchunk[mk::K_ATT] : c.n_q_heads * d;
+  if (p.tc) {
+    I.o_part_cols = p.tc_kt[mk::T_OPROJ] > 0 ? p.tc_kt[mk::T_OPROJ] : c.n_q_heads * d;
+    I.ffn_part_cols = p.tc_kt[mk::T_DOWN] > 0 ? p.tc_kt[mk::T_DOWN] : F;
+  }
+  I.gemv_path = p.tc ? 2 : 1;
+  I.schedule = lay.sched.empty() ? 0 : 1;
+  I.qkv_parts = lay.splits[0];
+  I.gateup_parts = lay.splits[2];
 }
 
 }  // namespace
@@ -212,6 +223,18 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   if ((rc = upload(&plan->d_tasks, lay.tasks.data(), lay.tasks.size() * sizeof(Task), "task array")) ||
       (rc = upload(&plan->d_rope, lay.rope.data(), lay.rope.size() * sizeof(float2), "RoPE table")))
     return cleanup_fail(rc);
+  if (!lay.sched.empty()) {
+    std::vector<int> both(lay.sched_off);
+    both.insert(both.end(), lay.sched.begin(), lay.sched.end());
+    if ((rc = upload(&plan->d_sched, both.data(), both.size() * sizeof(int), "schedule")))
+      return cleanup_fail(rc);
+  }
+  if (lay.n_maps > 0) {
+    std::vector<unsigned char> maps;
+    rc = mk::encode_weight_maps(*cfg, *w, lay, maps, g_err);
+    if (rc) return cleanup_fail(rc);
+    if ((rc = upload(&plan->d_maps, maps.data(), maps.size(), "tensor maps"))) return cleanup_fail(rc);
+  }
   cudaError_t e = cudaMalloc(&plan->d_ws, lay.ws_bytes);
   if (e == cudaSuccess) e = cudaMemset(plan->d_ws, 0, lay.ws_bytes);
   if (e != cudaSuccess) return cleanup_fail(fail(MK_ERR_CUDA, "workspace: %s", cudaGetErrorString(e)));
@@ -223,6 +246,11 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   p.tasks = static_cast<const Task *>(plan->d_tasks);
   p.embed = static_cast<const __nv_bfloat16 *>(w->embed);
   p.rope_cs = static_cast<const float2 *>(plan->d_rope);
+  p.tmaps = plan->d_maps;
+  if (plan->d_sched != nullptr) {
+    p.sched_off = static_cast<const int *>(plan->d_sched);
+    p.sched = p.sched_off + lay.sched_off.size();
+  }
 
   e = cudaMalloc(&plan->d_host_ids, 3 * sizeof(int32_t) * MK_MAX_BATCH);
   if (e != cudaSuccess) return cleanup_fail(fail(MK_ERR_CUDA, "cudaMalloc staging: %s", cudaGetErrorString(e)));
@@ -371,6 +399,11 @@ int mk_decode_step_ex(mk_plan *plan, const mk_step_args *a, void *stream) {
     p.v_pages[l] = static_cast<__nv_bfloat16 *>(a->kv->v_pages[l]);
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (a->mode != MK_MODE_MEGAKERNEL) {
+    // per-operator launches take their operator's tasks from the queue
+    p.sched = nullptr;
+    p.sched_off = nullptr;
+  }
   if (a->mode == MK_MODE_MEGAKERNEL) {
     p.task_begin = 0;
     p.task_end = p.n_tasks;
@@ -502,12 +535,40 @@ int mk_plan_describe(const mk_model_config *cfg, const mk_plan_options *opts, in
   return MK_OK;
 }
 
+int mk_plan_describe_schedule(const mk_model_config *cfg, const mk_plan_options *opts,
+                              int num_sms, int smem_optin, int32_t *cta_of_task,
+                              int64_t max_tasks) {
+  g_err.clear();
+  if (cfg == nullptr || cta_of_task == nullptr)
+    return fail(MK_ERR_INVALID_ARG, "cfg or cta_of_task is NULL");
+  if (num_sms < 1 || smem_optin < 1)
+    return fail(MK_ERR_INVALID_ARG, "num_sms and smem_optin must be positive");
+  int rc = mk::validate_config(*cfg, g_err);
+  if (rc) return rc;
+  mk::LayoutOptions lo;
+  rc = layout_options(opts, lo);
+  if (rc) return rc;
+  mk::Layout lay;
+  rc = mk::build_layout(*cfg, lo, num_sms, smem_optin, lay, g_err);
+  if (rc) return rc;
+  if (max_tasks < static_cast<int64_t>(lay.tasks.size()))
+    return fail(MK_ERR_INVALID_ARG, "cta_of_task holds %lld entries; the plan has %zu tasks",
+                static_cast<long long>(max_tasks), lay.tasks.size());
+  for (size_t i = 0; i < lay.tasks.size(); ++i) cta_of_task[i] = -1;
+  for (size_t c = 0; c + 1 < lay.sched_off.size(); ++c)
+    for (int k = lay.sched_off[c]; k < lay.sched_off[c + 1]; ++k)
+      cta_of_task[lay.sched[static_cast<size_t>(k)]] = static_cast<int32_t>(c);
+  return MK_OK;
+}
+
 void mk_plan_destroy(mk_plan *plan) {
   if (plan == nullptr) return;
   cudaDeviceSynchronize();
   for (OpGraph &g : plan->graphs) release_graph(g);
   cudaFree(plan->d_tasks);
   cudaFree(plan->d_rope);
+  cudaFree(plan->d_maps);
+  cudaFree(plan->d_sched);
   cudaFree(plan->d_ws);
   cudaFree(plan->d_sync);
   cudaFree(plan->d_host_ids);

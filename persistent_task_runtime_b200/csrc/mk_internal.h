@@ -25,13 +25,26 @@ constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kTaskSlots = 4;                     // tasks in flight per CTA
 constexpr int kSlotBytes = 96;                    // one task slot in shared memory
 constexpr int kLookBytes = 512;                   // loader lookahead area
-constexpr int kOutSlots = 4;                      // compute -> storer buffers
+constexpr int kOutSlots = 4;                      // compute -> storer buffers (upper bound)
 constexpr int kMaxPages = 16;                     // ring entries (upper bound)
 constexpr int kMaxMTiles = 8;                     // 16-row tiles per GEMV task (B <= 4)
 constexpr int kMaxPageCols = 2048;                // widest weight page (16 rows)
 constexpr int kXWholeMax = 72 * 1024;             // largest activation staged whole (all sequences)
 constexpr int kMaxGroup = 8;                      // query heads per KV head
 constexpr int kMaxSmem = 232448;                  // opt-in smem per CTA (B200)
+
+// ---- tensor-core GEMV path (tcgen05) -------------------------------------------
+// A task is one or two 128-row tiles of a weight matrix over a K range; the
+// weights arrive by TMA tensor copies in the 128-byte-swizzled K-major layout
+// the tensor core reads, the activation is staged as bf16 hi/lo rows in the
+// same layout, and the fp32 accumulators live in tensor memory.
+constexpr int kTcRows = 128;                      // MMA M: weight rows per tile
+constexpr int kTcAtomCols = 64;                   // columns of one 128-byte swizzle atom
+constexpr int kTcAtomBytes = kTcRows * 128;       // one weight atom: 128 rows x 128 B
+constexpr int kTcXBytes = 32 * 1024;              // one staged activation chunk buffer
+constexpr int kTcTmemCols = 128;                  // tensor-memory columns allocated per CTA
+constexpr int kTcAutoBatch = 5;                   // smallest max_batch that takes it by default
+constexpr int kTcMatsPerLayer = 7;                // tensor maps: wq wk wv wo w_gate w_up w_down
 
 // ---- task descriptor (64 bytes, four 16-byte loads) ---------------------------
 enum TaskType : uint8_t {
@@ -62,7 +75,7 @@ struct alignas(16) Task {
   const __nv_bfloat16 *w0;    // GEMV: the weight matrix (gate/up: gate); ATTN: q-norm gain
   const __nv_bfloat16 *w1;    // gate/up: the up matrix; ATTN: k-norm gain
   const __nv_bfloat16 *gain;  // RMSNorm gain of the task's input (QKV, gate/up, LM head)
-  uint64_t pad;
+  uint32_t map0, map1;        // tensor-core path: tensor maps of w0 / w1 (index into Params::tmaps)
 };
 static_assert(sizeof(Task) == 64, "task descriptor must be 64 bytes");
 constexpr uint32_t kNoEvent = 0xffffffffu;
@@ -104,8 +117,8 @@ struct Params {
   int qkv_tasks_per_group;            // QKV tasks of one KV group's heads (G q + k + v)
   int kp[4];                          // page columns per op class
   int kchunk[4];                      // split-K columns per op class (0 = unsplit)
-  float *kpart;                       // [splits][maxB][H] split-K partial sums
-  uint32_t *tile_ctr;                 // [H/16 + 1] split-K parts done per row tile
+  float *kpart;                       // [parts][maxB][rows] split-K partials: QKV, down
+  uint32_t *tile_ctr;                 // split-K parts done per 16-row tile: QKV, down
   int x_cap;                          // bytes of the activation staging area
   int page_bytes, n_pages;
   int off_look, off_slots, off_red, off_out, out_bytes, off_x, off_pages;  // smem carve-up
@@ -116,6 +129,27 @@ struct Params {
   int n_o_parts, o_groups;                 // split-K parts of the O projection, KV groups per part
   int n_lm_tasks;
   long long wait_limit_ns;
+  int n_out;                          // compute -> storer output buffers in use (<= kOutSlots)
+  int tile_rows;                      // rows per row tile: 16 (mma.sync) or kTcRows (tcgen05)
+
+  // tensor-core GEMV path (tc = 1): every GEMV task runs on tcgen05 tiles
+  int tc;
+  int tc_bpad;                        // sequences per half of the MMA's N (max_batch rounded to 8)
+  int tc_n;                           // MMA N = 2 * tc_bpad: bf16 hi rows, then lo rows
+  int tc_kc;                          // weight page columns (a multiple of 64)
+  int tc_kx;                          // staged activation chunk columns (a multiple of tc_kc)
+  int tc_kt[8];                       // split-K part columns per task type (0: unsplit)
+  const void *tmaps;                  // CUtensorMap[L * 7 + 1], 128 B each (LM head last)
+  float *ssq_attn;                    // [H/16][maxB] sums of h^2 per 16 rows: QKV / LM head input
+  float *ssq_mlp;                     // [H/16][maxB] the same for the gate/up input
+  float *kpart2;                      // [parts][maxB][2F] split-K partials of gate/up
+  uint32_t *tile_ctr2;                // [F/16 + 1] split-K parts done per gate/up row tile
+  // solidified schedule (NULL: the global ticket queue): CTA c runs tasks
+  // sched[sched_off[c] .. sched_off[c + 1]) in that (ascending) order
+  const int *sched;
+  const int *sched_off;
+  float *kpart_o;                     // [parts][maxB][H] split-K partials of the O projection
+  uint32_t *tile_ctr_o;               // [H/16 + 1] split-K parts done per O row tile
 
   // per step
   uint32_t epoch;
@@ -150,6 +184,10 @@ __host__ __device__ inline int ev_down(const Params &p, int l) {
   return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + p.n_o_parts + 1 + p.n_ffn_parts;
 }
 
+// Tensor map of weight matrix j (0 wq, 1 wk, 2 wv, 3 wo, 4 w_gate, 5 w_up,
+// 6 w_down) of layer l; the LM head's is the last.
+__host__ __device__ inline int tc_map_index(int l, int j) { return l * kTcMatsPerLayer + j; }
+
 // Batch n-tiles of a GEMV: each mma n-tile carries 4 sequences, the bf16
 // high parts of their activations in columns 0..3 and the low parts in
 // columns 4..7, so one mma covers both halves.  Row tiles per task shrink as
@@ -175,6 +213,8 @@ struct LayoutOptions {
   int num_ctas = 0;             // 0: one per SM
   int max_page_cols = 0;        // 0: kMaxPageCols
   bool o_split = false;         // O projection in two K parts of whole KV groups
+  int gemv_path = 0;            // 0 automatic, 1 mma.sync pages, 2 tcgen05 tiles
+  int schedule = 0;             // 0 dynamic ticket queue, 1 solidified per-CTA task lists
   int rows_per_task[5] = {0, 0, 0, 0, 0};
   long long wait_limit_ns = 2000000000LL;
   bool debug_unsatisfiable_dep = false;
@@ -191,8 +231,14 @@ struct Layout {
   std::vector<float2> rope;     // [max_seq_len][d/2] (cos, sin)
   // workspace byte offsets and size; counter words
   size_t o_h = 0, o_qkv = 0, o_part = 0, o_o = 0, o_u = 0, o_arg = 0, o_kpart = 0;
+  size_t o_kpart2 = 0, o_kpart_o = 0, o_ssq_attn = 0, o_ssq_mlp = 0;
   size_t ws_bytes = 0;
-  size_t comb_words = 0, tile_words = 0, sync_words = 0;
+  size_t comb_words = 0, tile_words = 0, tile2_words = 0, tile_o_words = 0, sync_words = 0;
+  int n_maps = 0;                      // tensor maps the tensor-core path needs (0: none)
+  // solidified schedule (empty: dynamic queue): task indices per CTA, and
+  // the CTA's first entry (grid + 1 offsets)
+  std::vector<int> sched, sched_off;
+  int splits[5] = {1, 1, 1, 1, 1};     // split-K parts: QKV, O, gate/up, down, LM head
 };
 int validate_config(const mk_model_config &c, std::string &err);
 int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int smem_optin,
@@ -200,6 +246,10 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
 void bind_workspace(const Layout &lay, char *ws, uint32_t *sync, Params &p);
 // Fill every task's operand pointers (weights, norm gains) from `w`.
 void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vector<Task> &tasks);
+// Encode the tensor maps of every weight matrix (lay.n_maps of them, 128
+// bytes each) into `out` for the tensor-core path.  Needs the CUDA driver.
+int encode_weight_maps(const mk_model_config &c, const mk_weights &w, const Layout &lay,
+                       std::vector<unsigned char> &out, std::string &err);
 
 cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative,
                         cudaStream_t stream);

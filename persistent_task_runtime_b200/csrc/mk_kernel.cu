@@ -98,6 +98,97 @@ __device__ __forceinline__ void bulk_load_plain(void *dst, const void *src, uint
       : "memory");
 }
 
+// ---- tensor-core path: TMA tensor copies and tcgen05 -------------------------
+
+// 2-D tensor copy of one box (tensor map `tmap`, coordinates {x = column,
+// y = row}) into this CTA's shared memory, completion on `bar`.  No cluster
+// multicast: the map covers this GPU's own memory only.
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, int y,
+                                            uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte
+// swizzled layout: 8-row groups 1024 bytes apart, rows 128 bytes apart.
+// Fields: start address >> 4 (bits 0-13), leading-dimension offset (unused
+// for this layout, 1), stride-dimension offset 1024 >> 4 (bits 32-45),
+// descriptor version 1 (bits 46-47), layout type 2 = 128-byte swizzle
+// (bits 61-63).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (1ull << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of a dense bf16 x bf16 -> fp32 MMA, both operands
+// K-major: D format f32 (bits 4-5 = 1), A and B format bf16 (bits 7-9 and
+// 10-12 = 1), N >> 3 (bits 17-22), M >> 4 (bits 24-28).
+__device__ __forceinline__ uint32_t mma_idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, M = 128, issued by one thread.
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+
+// Arrive on `bar` once every tcgen05 operation this thread issued so far has
+// completed.
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Warp-wide: allocate `ncols` tensor-memory columns; the base address is
+// written to shared memory at `dst`.
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// Warp-wide: 16 consecutive fp32 accumulator columns of this warp's 32 lanes
+// (lane i of the warp reads tensor-memory lane (taddr >> 16) + i).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ uint64_t gtimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -206,6 +297,10 @@ struct Ctl {
   uint64_t out_full[kOutSlots];
   uint64_t out_empty[kOutSlots];
   uint64_t xbar;                    // activation bulk copy landed
+  uint64_t x_full[2];               // tensor-core path: staged chunk buffer ready for the MMAs
+  uint64_t x_free[2];               // ... its MMAs completed (buffer may be restaged)
+  uint64_t acc_bar;                 // ... the task's MMAs completed (accumulators final)
+  uint32_t tmem;                    // tensor-memory base address of this CTA
   volatile int cta_abort;
   volatile int cbad;                // a compute warp gave up (written by compute only)
   int skip;
@@ -350,6 +445,24 @@ __device__ Geo gemv_geo(const Params &p, const Task &t, int B) {
   return g;
 }
 
+// Tensor-core path: a task's columns [k0, k0 + Kt) of its K-wide input.
+struct TcGeo {
+  int K, k0, Kt;
+};
+__device__ __forceinline__ TcGeo tc_geo(const Params &p, const Task &t) {
+  TcGeo g;
+  g.K = t.type == T_OPROJ ? p.Hq * p.d : (t.type == T_DOWN ? p.F : p.H);
+  const int kt = p.tc_kt[t.type];
+  if (t.nsplit > 1 && kt > 0) {
+    g.k0 = t.ksplit * kt;
+    g.Kt = min(g.K, g.k0 + kt) - g.k0;
+  } else {
+    g.k0 = 0;
+    g.Kt = g.K;
+  }
+  return g;
+}
+
 // Row `m`-tile of a GEMV task: weight matrix base, first row, valid rows.
 __device__ __forceinline__ void gemv_tile(const Params &p, const Task &t, int m,
                                           const __nv_bfloat16 *&W, int &row, int &rows_valid) {
@@ -452,9 +565,13 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   uint32_t ts_par = 0;
   bool ok = true;
 
-  const int n_launch = p.task_end - p.task_begin;
+  // the dynamic queue hands out tickets from one global counter; a
+  // solidified schedule walks this CTA's own list of task indices
+  const bool fixed = p.sched != nullptr;
+  const int s_begin = fixed ? p.sched_off[blockIdx.x] : 0;
+  const int n_launch = fixed ? p.sched_off[blockIdx.x + 1] - s_begin : p.task_end - p.task_begin;
   uint32_t next = 0;
-  if (lane == 0) next = atomicAdd(p.sync + S_QUEUE, 1u);
+  if (lane == 0 && !fixed) next = atomicAdd(p.sync + S_QUEUE, 1u);
   int la_head = 0, la_count = 0;
   bool exhausted = false;
   uint32_t la_ev = 0;   // lane 0: input-event counter read when the task was popped
@@ -469,8 +586,9 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       exhausted = true;
       return;
     }
-    if (lane == 0) next = atomicAdd(p.sync + S_QUEUE, 1u);
-    const int tix = p.task_begin + static_cast<int>(ticket);
+    if (lane == 0) next = fixed ? ticket + 1u : atomicAdd(p.sync + S_QUEUE, 1u);
+    const int tix = fixed ? p.sched[s_begin + static_cast<int>(ticket)]
+                          : p.task_begin + static_cast<int>(ticket);
     const Task t = p.tasks[tix];
     const int e = (la_head + la_count) % kLook;
     if (lane == 0) {
@@ -582,7 +700,37 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     }
 
     // ---- stream the task's operands into the page ring ----
-    if (is_gemv(t.type)) {
+    if (is_gemv(t.type) && p.tc) {
+      // tensor-core path: per activation chunk, per 128-row tile, pages of
+      // tc_kc columns, each one TMA box per 64-column swizzle atom
+      const TcGeo g = tc_geo(p, t);
+      const uint8_t *maps = static_cast<const uint8_t *>(p.tmaps);
+      for (int xc0 = g.k0; xc0 < g.k0 + g.Kt && ok; xc0 += p.tc_kx) {
+        const int xend = min(g.k0 + g.Kt, xc0 + p.tc_kx);
+        for (int m = 0; m < t.n_m && ok; ++m) {
+          const void *map = maps + static_cast<size_t>(m == 0 ? t.map0 : t.map1) * 128;
+          for (int c0 = xc0; c0 < xend; c0 += p.tc_kc) {
+            const int nc = min(p.tc_kc, xend - c0);
+            if (lane == 0) okl = wait_mbar(p, ctl, &ctl->empty[pi], pe_par ^ 1u, 0xfff10000u, 2);
+            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+            if (!ok) break;
+            uint8_t *pg = pages + static_cast<size_t>(pi) * p.page_bytes;
+            if (lane == 0) mbar_arrive_expect_tx(&ctl->full[pi], static_cast<uint32_t>(nc * kTcRows * 2));
+            __syncwarp();
+            if (lane < nc / kTcAtomCols)
+              tma_load_2d(pg + lane * kTcAtomBytes, map, c0 + lane * kTcAtomCols,
+                          static_cast<int>(t.row0), &ctl->full[pi], pol);
+            issued |= 1u << pi;
+            last_par = (last_par & ~(1u << pi)) | (pe_par << pi);
+            if (++pi == p.n_pages) {
+              pi = 0;
+              pe_par ^= 1u;
+            }
+            top_up(1);
+          }
+        }
+      }
+    } else if (is_gemv(t.type)) {
       const Geo geo = gemv_geo(p, t, B);
       const int pitch = row_pitch_bytes(geo.kp);
       for (int xc0 = geo.k0; xc0 < geo.k0 + geo.Kt && ok; xc0 += geo.kx) {
@@ -740,6 +888,8 @@ __device__ __forceinline__ bool warp_wait_page(const Params &p, Ctl *ctl, uint64
 struct ComputeState {
   int pi = 0;
   uint32_t pg_par = 0;
+  uint32_t xuse = 0;             // tensor-core path: staged chunks so far (buffer = xuse & 1)
+  uint32_t accuse = 0;           // tensor-core path: tasks whose accumulators were read
   uint32_t x_par = 0;            // phase of the activation-copy barrier
   uint32_t xkey = 0xffffffffu;   // (layer, type) of the staged activation
   uint32_t sat_ev = kNoEvent;    // last (event, count) known satisfied
@@ -1039,6 +1189,260 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
 }
 
 // ============================================================================
+// compute warps: GEMV on the tensor cores (tcgen05)
+// ============================================================================
+//
+// A task is n_m (1, or 2 for gate/up) tiles of 128 weight rows over its K
+// range.  Thread 0 issues the MMAs: D[128 x N] += W[128 x 16] * X[N x 16]^T
+// per 16 columns, accumulating in tensor memory (one N-column accumulator per
+// tile).  X holds the activation as bf16 rows: sequences 0..bpad-1 carry the
+// high parts of x * g and rows bpad..2*bpad-1 the low parts (hi + lo == x * g
+// to ~2^-16), so D[:, b] + D[:, bpad + b] is the fp32-accurate product.
+// Warps 2-6 stage the activation chunk by chunk into two buffers, one chunk
+// ahead of the MMAs.  After the last MMA, warps 1-4 (tensor-memory lane
+// quarters 1, 2, 3, 0) read the accumulators and hand the task's rows to the
+// storer, scaled by the RMSNorm factor for normed inputs.
+
+__device__ __forceinline__ void compute_stage_bar() {
+  asm volatile("bar.sync 2, %0;" ::"n"(kComputeThreads - 32) : "memory");
+}
+
+// 8 fp32 values times their gains -> 8 bf16 high parts and 8 low parts.
+__device__ __forceinline__ void split8(const float4 &x0, const float4 &x1, bool has_gain, uint4 gw,
+                                      uint4 &hw, uint4 &lw) {
+  float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+  if (has_gain) {
+    const uint32_t gg[4] = {gw.x, gw.y, gw.z, gw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] *= bf_lo(gg[e]);
+      v[2 * e + 1] *= bf_hi(gg[e]);
+    }
+  }
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat16 h0, l0, h1, l1;
+    split_bf16(v[2 * e], h0, l0);
+    split_bf16(v[2 * e + 1], h1, l1);
+    h[e] = pack2(h0, h1);
+    l[e] = pack2(l0, l1);
+  }
+  hw = make_uint4(h[0], h[1], h[2], h[3]);
+  lw = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Stage activation columns [xc0, xc0 + xlen) of every sequence into `xbuf`
+// (160 threads, sid 0..159) in the K-major 128-byte-swizzled layout: per
+// 64-column atom, rows of 128 bytes (hi rows 0..bpad-1, lo rows
+// bpad..2*bpad-1), the 16-byte chunk c of a row stored at chunk c XOR
+// (row address bits 7..9).  Sequences >= B are zeros.
+__device__ void stage_chunk_tc(const Params &p, const float *src, int stride,
+                               const __nv_bfloat16 *gain, int xc0, int xlen, uint8_t *xbuf, int B,
+                               int sid) {
+  const int bpad = p.tc_bpad;
+  const int nblk = xlen / 8;
+  const uint32_t xs = smem_u32(xbuf);
+  const uint32_t atom_bytes = static_cast<uint32_t>(p.tc_n) * 128u;
+  for (int u = sid; u < bpad * nblk; u += kComputeThreads - 32) {
+    const int b = u / nblk, j = u - b * nblk;
+    uint4 hw = make_uint4(0, 0, 0, 0), lw = make_uint4(0, 0, 0, 0);
+    if (b < B) {
+      const float4 *sp = reinterpret_cast<const float4 *>(src + static_cast<size_t>(b) * stride + xc0 + j * 8);
+      const float4 x0 = __ldcg(sp), x1 = __ldcg(sp + 1);
+      const uint4 gw = gain != nullptr ? __ldg(reinterpret_cast<const uint4 *>(gain + xc0 + j * 8))
+                                       : make_uint4(0, 0, 0, 0);
+      split8(x0, x1, gain != nullptr, gw, hw, lw);
+    }
+    const uint32_t atom = xs + static_cast<uint32_t>(j >> 3) * atom_bytes;
+    const uint32_t ch = static_cast<uint32_t>(j & 7);
+    const uint32_t rh = atom + static_cast<uint32_t>(b) * 128u;
+    const uint32_t rl = atom + static_cast<uint32_t>(bpad + b) * 128u;
+    sts128(rh + ((ch ^ ((rh >> 7) & 7u)) << 4), hw);
+    sts128(rl + ((ch ^ ((rl >> 7) & 7u)) << 4), lw);
+  }
+}
+
+template <int NT>   // accumulator columns / 16: 1 (N = 16, batch <= 8) or 2 (N = 32)
+__device__ bool gemv_task_tc(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
+                             ComputeState &st, float *out, int ctid) {
+  const Task &t = S.t;
+  const int B = p.batch;
+  const int warp = ctid >> 5, lane = ctid & 31;
+  const TcGeo g = tc_geo(p, t);
+  const float *src;
+  int stride;
+  const __nv_bfloat16 *gain;
+  gemv_source(p, t, src, stride, gain);
+  const bool normed = gain != nullptr;
+
+  if (!S.dep_ok && (t.dep_event != st.sat_ev || t.dep_count != st.sat_cnt)) {
+    bool okl = true;
+    if (ctid == 0) okl = wait_event(p, ctl, t.dep_event, t.dep_count, S.idx);
+    if (!st.gs.share(ctl, ctid, okl)) return false;
+  }
+  st.sat_ev = t.dep_event;
+  st.sat_cnt = t.dep_count;
+  if (ctid == 0) trace_mark(p, S.idx, 4);
+
+  // RMSNorm scale of each sequence from the per-16-row sums of h^2 that the
+  // producers of h wrote (fixed order: strided per lane, then a warp tree)
+  if (normed) {
+    const float *ssq = t.type == T_GATEUP ? p.ssq_mlp : p.ssq_attn;
+    const int n16 = p.H / 16;
+    for (int b = warp; b < B; b += kComputeWarps) {
+      float s = 0.f;
+      for (int i = lane; i < n16; i += 32) s += __ldcg(ssq + static_cast<size_t>(i) * p.max_batch + b);
+      s = warp_sum(s);
+      if (lane == 0) ctl->rs[b] = 1.0f / sqrtf(s / static_cast<float>(p.H) + p.eps);
+    }
+  }
+
+  const int nchunks = (g.Kt + p.tc_kx - 1) / p.tc_kx;
+  uint8_t *xbase = smem + p.off_x;
+  if (ctid >= 32) {
+    // ---- stagers: one chunk ahead of the MMAs, in two buffers ----
+    bool bad = false;
+    for (int c = 0; c < nchunks; ++c) {
+      const uint32_t u = st.xuse + c;
+      const int buf = static_cast<int>(u & 1u);
+      const uint32_t use = u >> 1;
+      const int xc0 = g.k0 + c * p.tc_kx;
+      const int xlen = min(p.tc_kx, g.k0 + g.Kt - xc0);
+      if (use > 0 && !bad &&
+          !warp_wait_page(p, ctl, &ctl->x_free[buf], (use - 1u) & 1u, 0xfff90000u)) {
+        bad = true;
+        if (lane == 0) {
+          ctl->cbad = 1;
+          ctl->cta_abort = 1;
+        }
+      }
+      // (the MMAs that last read this buffer did so through the async proxy)
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      if (!bad)
+        stage_chunk_tc(p, src, stride, gain, xc0, xlen, xbase + buf * kTcXBytes, B, ctid - 32);
+      // the tensor core reads the buffer through the async proxy
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      compute_stage_bar();
+      if (ctid == 32) mbar_arrive(&ctl->x_full[buf]);
+    }
+  } else if (ctid == 0) {
+    // ---- MMA issuer ----
+    const uint32_t idesc = mma_idesc_bf16(kTcRows, p.tc_n);
+    const uint32_t tmem = ctl->tmem;
+    const uint32_t pages = smem_u32(smem + p.off_pages);
+    const uint32_t xs0 = smem_u32(xbase);
+    const uint32_t xatom = static_cast<uint32_t>(p.tc_n) * 128u;
+    bool bad = false;
+    bool started0 = false, started1 = false;   // tile 0 / 1 has its first MMA
+    for (int c = 0; c < nchunks; ++c) {
+      const uint32_t u = st.xuse + c;
+      const int buf = static_cast<int>(u & 1u);
+      const int xc0 = g.k0 + c * p.tc_kx;
+      const int xlen = min(p.tc_kx, g.k0 + g.Kt - xc0);
+      if (!bad && !wait_mbar(p, ctl, &ctl->x_full[buf], (u >> 1) & 1u, 0xfffa0000u, 2)) bad = true;
+      tc_fence_after();
+      const uint32_t xb = xs0 + static_cast<uint32_t>(buf) * kTcXBytes;
+      for (int m = 0; m < t.n_m; ++m) {
+        for (int c0 = xc0; c0 < xc0 + xlen; c0 += p.tc_kc) {
+          const int nc = min(p.tc_kc, xc0 + xlen - c0);
+          if (!bad && !wait_mbar(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff30000u, 2)) bad = true;
+          if (!bad) {
+            tc_fence_after();
+            const uint32_t pg = pages + static_cast<uint32_t>(st.pi) * p.page_bytes;
+            const uint32_t xa0 = xb + static_cast<uint32_t>((c0 - xc0) / kTcAtomCols) * xatom;
+            for (int a = 0; a < nc / kTcAtomCols; ++a)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint64_t ad = sw128_desc(pg + a * kTcAtomBytes + j * 32);
+                const uint64_t bd = sw128_desc(xa0 + a * xatom + j * 32);
+                tc_mma(tmem + m * p.tc_n, ad, bd, idesc, m == 0 ? started0 : started1);
+                if (m == 0) started0 = true; else started1 = true;
+              }
+            tc_commit(&ctl->empty[st.pi]);   // the page is free once these MMAs complete
+          }
+          if (++st.pi == p.n_pages) {
+            st.pi = 0;
+            st.pg_par ^= 1u;
+          }
+        }
+      }
+      tc_commit(&ctl->x_free[buf]);
+    }
+    tc_commit(&ctl->acc_bar);
+    // wait for the accumulators (also after a failed wait: no MMA may still
+    // be running when the task returns)
+    if (!wait_mbar(p, ctl, &ctl->acc_bar, st.accuse & 1u, 0xfffb0000u, 4)) bad = true;
+    if (bad) {
+      ctl->cbad = 1;
+      ctl->cta_abort = 1;
+    }
+  }
+  if (ctid < 32 && ctid != 0) {
+    // the rest of the MMA warp: keep the page-ring position in step with thread 0
+    for (int c = 0; c < nchunks; ++c) {
+      const int xc0 = g.k0 + c * p.tc_kx;
+      const int xlen = min(p.tc_kx, g.k0 + g.Kt - xc0);
+      const int np = t.n_m * ((xlen + p.tc_kc - 1) / p.tc_kc);
+      for (int k = 0; k < np; ++k)
+        if (++st.pi == p.n_pages) {
+          st.pi = 0;
+          st.pg_par ^= 1u;
+        }
+    }
+  } else if (ctid >= 32) {
+    for (int c = 0; c < nchunks; ++c) {
+      const int xc0 = g.k0 + c * p.tc_kx;
+      const int xlen = min(p.tc_kx, g.k0 + g.Kt - xc0);
+      const int np = t.n_m * ((xlen + p.tc_kc - 1) / p.tc_kc);
+      for (int k = 0; k < np; ++k)
+        if (++st.pi == p.n_pages) {
+          st.pi = 0;
+          st.pg_par ^= 1u;
+        }
+    }
+  }
+  st.xuse += static_cast<uint32_t>(nchunks);
+  st.xkey = 0xffffffffu;   // the staging area no longer holds an mma.sync operand
+  __syncwarp();            // the MMA warp reconverges (thread 0 waited for the accumulators)
+  compute_bar();
+  if (ctl->cbad != 0) return false;
+  if (ctid == 0) trace_mark(p, S.idx, 5);
+  tc_fence_after();
+
+  // ---- epilogue: accumulators -> the output buffer ----
+  if (ctid < 128) {
+    const int q = (warp + 1) & 3;            // CTA warp warp+1 reads lanes 32q..32q+31
+    const int row = q * 32 + lane;
+    constexpr int BP = 8 * NT;               // tc_bpad of a plan with this NT
+    for (int m = 0; m < t.n_m; ++m) {
+      const uint32_t ta = ctl->tmem + (static_cast<uint32_t>(q * 32) << 16) +
+                          static_cast<uint32_t>(m * p.tc_n);
+      float v[NT][16];
+      tmem_ld16(ta, v[0]);
+      if (NT > 1) tmem_ld16(ta + 16, v[NT - 1]);
+      if (row < static_cast<int>(t.nrows)) {
+#pragma unroll
+        for (int b = 0; b < 8 * NT; ++b) {
+          if (b < B) {
+            // hi column b, lo column BP + b
+            const float hi = v[b / 16][b % 16];
+            const float lo = v[(BP + b) / 16][(BP + b) % 16];
+            float r = hi + lo;
+            if (normed) r *= ctl->rs[b];
+            out[b * p.out_stride + m * kTcRows + row] = r;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  compute_bar();
+  ++st.accuse;
+  return true;
+}
+
+// ============================================================================
 // compute warps: attention over one chunk of one (sequence, KV head)
 // ============================================================================
 
@@ -1296,12 +1700,14 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     }
     if (has_cur) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl->empty[st.pi]);
+    if (!p.tc && lane == 0) mbar_arrive(&ctl->empty[st.pi]);
+    compute_bar();   // sc is rewritten by the next page
+    // (tensor-core plans release a page once, after every warp is done with it)
+    if (p.tc && ctid == 0) mbar_arrive(&ctl->empty[st.pi]);
     if (++st.pi == p.n_pages) {
       st.pi = 0;
       st.pg_par ^= 1u;
     }
-    compute_bar();   // sc is rewritten by the next page
   }
 
   // the chunk's partial goes straight to global memory: row h = (acc, m, l, pad)
@@ -1385,6 +1791,22 @@ __device__ void embed_task(const Params &p, const Slot &S, int ctid) {
       __stcg(reinterpret_cast<float4 *>(p.h + b * H + i + 4), c);
     }
   }
+  if (p.tc) {
+    // sums of h^2 per 16 rows for the first QKV tasks' RMSNorm (tensor-core path)
+    const int n16 = H / 16;
+    for (int u = ctid; u < B * n16; u += kComputeThreads) {
+      const int b = u / n16, i = u - b * n16;
+      const int id = p.ids[b];
+      if (id < 0 || id >= p.V) continue;   // reported above
+      const uint4 *e = reinterpret_cast<const uint4 *>(p.embed + static_cast<size_t>(id) * H + i * 16);
+      const uint4 w0 = __ldg(e), w1 = __ldg(e + 1);
+      const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      float sq = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sq += bf_lo(ww[k]) * bf_lo(ww[k]) + bf_hi(ww[k]) * bf_hi(ww[k]);
+      __stcg(p.ssq_attn + static_cast<size_t>(i) * p.max_batch + b, sq);
+    }
+  }
   __threadfence();
 }
 
@@ -1429,9 +1851,13 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
         }
         break;
       default:
-        tok = p.batch > 8   ? gemv_task<4>(p, ctl, smem, S, st, out, ctid)
-              : p.batch > 4 ? gemv_task<2>(p, ctl, smem, S, st, out, ctid)
-                            : gemv_task<1>(p, ctl, smem, S, st, out, ctid);
+        if (p.tc)
+          tok = p.tc_n > 16 ? gemv_task_tc<2>(p, ctl, smem, S, st, out, ctid)
+                            : gemv_task_tc<1>(p, ctl, smem, S, st, out, ctid);
+        else
+          tok = p.batch > 8   ? gemv_task<4>(p, ctl, smem, S, st, out, ctid)
+                : p.batch > 4 ? gemv_task<2>(p, ctl, smem, S, st, out, ctid)
+                              : gemv_task<1>(p, ctl, smem, S, st, out, ctid);
         break;
     }
     if (!tok) {
@@ -1448,7 +1874,7 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       ts = 0;
       ts_par ^= 1u;
     }
-    if (++os == kOutSlots) {
+    if (++os == p.n_out) {
       os = 0;
       os_par ^= 1u;
     }
@@ -1486,82 +1912,110 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
       if (lane == 0) signal(p, t.out_event);
       break;
     }
-    case T_QKV: {
-      // raw projection rows; QK-norm, RoPE and the KV append happen in the
-      // attention tasks of the head's KV group
-      const int base = t.aux == 0 ? 0 : (t.aux == 1 ? p.Hq * p.d : (p.Hq + p.Hkv) * p.d);
-      for (int b = 0; b < B; ++b)
-        for (int r = lane; r < static_cast<int>(t.nrows); r += 32)
-          __stcg(p.qkv + static_cast<size_t>(b) * p.NQKV + base + t.row0 + r, out[b * OS + r]);
+    case T_QKV:
+    case T_OPROJ:
+    case T_DOWN:
+    case T_GATEUP: {
+      const int nr = static_cast<int>(t.nrows);
+      // the rows this task's output covers within its operator's row space
+      // (QKV: q rows, then k rows, then v rows; gate/up: gate rows then up
+      // rows, 2F in all)
+      const int qbase = t.aux == 0 ? 0 : (t.aux == 1 ? p.Hq * p.d : (p.Hq + p.Hkv) * p.d);
+      const int grow0 = static_cast<int>(t.row0) + (t.type == T_QKV ? qbase : 0);
+      const int up_off = (t.n_m >> 1) * p.tile_rows;   // gate/up: the up rows in `out`
+      float *kp = p.kpart;
+      int rstride = p.H;
+      uint32_t *ctr = p.tile_ctr;
+      if (t.type == T_QKV) {
+        rstride = p.NQKV;
+      } else if (t.type == T_OPROJ) {
+        kp = p.kpart_o;
+        ctr = p.tile_ctr_o;
+      } else if (t.type == T_GATEUP) {
+        kp = p.kpart2;
+        rstride = 2 * p.F;
+        ctr = p.tile_ctr2;
+      }
+      const size_t pstride = static_cast<size_t>(p.max_batch) * rstride;
+      const bool split = t.nsplit > 1;
+      if (split) {
+        // split-K part: publish the partial; the part that completes the row
+        // tile sums all parts in a fixed order and runs the epilogue
+        for (int b = 0; b < B; ++b)
+          for (int r = lane; r < nr; r += 32) {
+            float *dst = kp + t.ksplit * pstride + static_cast<size_t>(b) * rstride + grow0 + r;
+            __stcg(dst, out[b * OS + r]);
+            if (t.type == T_GATEUP) __stcg(dst + p.F, out[b * OS + up_off + r]);
+          }
+        __syncwarp();
+        ctr += grow0 / 16;
+        uint32_t old = 0;
+        if (lane == 0) old = atom_add_acq_rel(ctr, 1u);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old + 1u != static_cast<uint32_t>(t.nsplit)) break;
+        __syncwarp();
+      }
+      // the task's (summed) output of sequence b, row r (half 1: gate/up's up rows)
+      auto value = [&](int b, int r, int half) -> float {
+        if (!split) return out[b * OS + half * up_off + r];
+        const float *src = kp + static_cast<size_t>(b) * rstride + grow0 + half * p.F + r;
+        float sum = 0.f;
+        for (int k = 0; k < t.nsplit; ++k) sum += __ldcg(src + k * pstride);
+        return sum;
+      };
+      if (t.type == T_QKV) {
+        // raw projection rows; QK-norm, RoPE and the KV append happen in the
+        // attention tasks of the head's KV group
+        for (int b = 0; b < B; ++b)
+          for (int r = lane; r < nr; r += 32)
+            __stcg(p.qkv + static_cast<size_t>(b) * p.NQKV + grow0 + r, value(b, r, 0));
+      } else if (t.type == T_GATEUP) {
+        for (int b = 0; b < B; ++b)
+          for (int r = lane; r < nr; r += 32) {
+            const float gt = value(b, r, 0);
+            const float up = value(b, r, 1);
+            __stcg(p.u + static_cast<size_t>(b) * p.F + t.row0 + r, gt / (1.0f + __expf(-gt)) * up);
+          }
+      } else {
+        // residual add; on the tensor-core path also the sums of h^2 per 16
+        // rows that the next normed operator's RMSNorm reads
+        float *ssq = t.type == T_OPROJ ? p.ssq_mlp : p.ssq_attn;
+        for (int b = 0; b < B; ++b)
+          for (int r0 = 0; r0 < nr; r0 += 32) {
+            const int r = r0 + lane;
+            float v = 0.f;
+            if (r < nr) {
+              float *hp = p.h + static_cast<size_t>(b) * p.H + t.row0 + r;
+              v = __ldcg(hp) + value(b, r, 0);
+              __stcg(hp, v);
+              if (t.type == T_DOWN && p.hidden_dump != nullptr)
+                p.hidden_dump[(static_cast<size_t>(t.layer) * B + b) * p.H + t.row0 + r] = v;
+            }
+            if (p.tc) {
+              float sq = v * v;
+#pragma unroll
+              for (int o = 8; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+              if ((lane & 15) == 0 && r < nr)
+                __stcg(ssq + static_cast<size_t>((t.row0 + r) / 16) * p.max_batch + b, sq);
+            }
+          }
+      }
       __syncwarp();
       if (lane == 0) {
-        const int head = static_cast<int>(t.aux2);
-        const int g = t.aux == 0 ? head / p.G : (t.aux == 1 ? head - p.Hq : head - p.Hq - p.Hkv);
-        signal(p, static_cast<uint32_t>(ev_attn_ready(p, t.layer, g)));
+        if (split) *ctr = 0u;   // rearm for the next layer / step
+        if (t.type == T_QKV) {
+          const int head = static_cast<int>(t.aux2);
+          const int g = t.aux == 0 ? head / p.G : (t.aux == 1 ? head - p.Hq : head - p.Hq - p.Hkv);
+          signal(p, static_cast<uint32_t>(ev_attn_ready(p, t.layer, g)));
+        } else {
+          signal(p, t.out_event);
+        }
       }
       break;
     }
     case T_ATTN: {
       // the compute warps wrote the chunk partial (and, for the chunk that
       // completed its (sequence, KV head), the merged o) before handing over
-      if (lane == 0) signal(p, t.out_event);
-      break;
-    }
-    case T_OPROJ:
-    case T_DOWN: {
-      if (t.nsplit > 1) {
-        // split-K part: publish the partial; the part that completes the row
-        // tile sums all parts in a fixed order and applies the residual
-        const size_t sp = static_cast<size_t>(p.max_batch) * p.H;
-        for (int b = 0; b < B; ++b)
-          for (int r = lane; r < static_cast<int>(t.nrows); r += 32)
-            __stcg(p.kpart + t.ksplit * sp + static_cast<size_t>(b) * p.H + t.row0 + r, out[b * OS + r]);
-        __syncwarp();
-        uint32_t *tc = p.tile_ctr + t.row0 / 16;
-        uint32_t old = 0;
-        if (lane == 0) old = atom_add_acq_rel(tc, 1u);
-        old = __shfl_sync(0xffffffffu, old, 0);
-        if (old + 1u != static_cast<uint32_t>(t.nsplit)) break;
-        __syncwarp();
-        for (int b = 0; b < B; ++b)
-          for (int r = lane; r < static_cast<int>(t.nrows); r += 32) {
-            const size_t o = static_cast<size_t>(b) * p.H + t.row0 + r;
-            float sum = 0.f;
-            for (int k = 0; k < t.nsplit; ++k) sum += __ldcg(p.kpart + k * sp + o);
-            float *hp = p.h + o;
-            const float v = __ldcg(hp) + sum;
-            __stcg(hp, v);
-            if (t.type == T_DOWN && p.hidden_dump != nullptr)
-              p.hidden_dump[(static_cast<size_t>(t.layer) * B + b) * p.H + t.row0 + r] = v;
-          }
-        __syncwarp();
-        if (lane == 0) {
-          *tc = 0u;
-          signal(p, t.out_event);
-        }
-        break;
-      }
-      for (int b = 0; b < B; ++b)
-        for (int r = lane; r < static_cast<int>(t.nrows); r += 32) {
-          float *hp = p.h + static_cast<size_t>(b) * p.H + t.row0 + r;
-          const float v = __ldcg(hp) + out[b * OS + r];
-          __stcg(hp, v);
-          if (t.type == T_DOWN && p.hidden_dump != nullptr)
-            p.hidden_dump[(static_cast<size_t>(t.layer) * B + b) * p.H + t.row0 + r] = v;
-        }
-      __syncwarp();
-      if (lane == 0) signal(p, t.out_event);
-      break;
-    }
-    case T_GATEUP: {
-      const int nh16 = (t.n_m >> 1) * 16;
-      for (int b = 0; b < B; ++b)
-        for (int r = lane; r < static_cast<int>(t.nrows); r += 32) {
-          const float gt = out[b * OS + r];
-          const float up = out[b * OS + nh16 + r];
-          __stcg(p.u + static_cast<size_t>(b) * p.F + t.row0 + r, gt / (1.0f + __expf(-gt)) * up);
-        }
-      __syncwarp();
       if (lane == 0) signal(p, t.out_event);
       break;
     }
@@ -1638,7 +2092,7 @@ __device__ void storer_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       ts = 0;
       ts_par ^= 1u;
     }
-    if (++os == kOutSlots) {
+    if (++os == p.n_out) {
       os = 0;
       os_par ^= 1u;
     }
@@ -1657,8 +2111,15 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.n_pages; ++i) {
       mbar_init(&ctl->full[i], 1);
-      mbar_init(&ctl->empty[i], kComputeWarps);
+      // a page is released by each compute warp, or (tensor-core path) once:
+      // by the MMAs' commit, or by one thread after an attention page
+      mbar_init(&ctl->empty[i], p.tc ? 1 : kComputeWarps);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->x_full[i], 1);
+      mbar_init(&ctl->x_free[i], 1);
+    }
+    mbar_init(&ctl->acc_bar, 1);
     for (int i = 0; i < kTaskSlots; ++i) {
       mbar_init(&ctl->slot_full[i], 1);
       mbar_init(&ctl->slot_empty[i], 1);
@@ -1673,9 +2134,19 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     ctl->flag[0] = ctl->flag[1] = 0;
     // a device error from an earlier step is sticky until the host resets
     ctl->skip = (ld_relaxed(p.sync + S_STATUS) != 0u || ld_relaxed(p.sync + S_ABORT) != 0u);
+    // the swizzled operand layouts assume 1024-byte aligned shared memory
+    if (p.tc && (smem_u32(smem) & 1023u) != 0u) {
+      raise_error(p, MK_ERR_UNSUPPORTED, 0xfffffff0u, smem_u32(smem), 0u);
+      ctl->skip = 1;
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  const bool tmem_owner = p.tc && !ctl->skip && (threadIdx.x >> 5) == 1;
+  if (tmem_owner) tmem_alloc(&ctl->tmem, kTcTmemCols);
+  if (p.tc) tc_fence_before();
+  __syncthreads();
+  if (p.tc) tc_fence_after();
   if (!ctl->skip) {
     const int warp = threadIdx.x >> 5;
     if (warp == kLoaderWarp) {
@@ -1686,7 +2157,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       compute_main(p, ctl, smem);
     }
   }
+  if (p.tc) tc_fence_before();
   __syncthreads();
+  if (p.tc) tc_fence_after();
+  if (tmem_owner) tmem_dealloc(ctl->tmem, kTcTmemCols);
   if (threadIdx.x == 0) {
     __threadfence();
     const uint32_t old = atomicAdd(p.sync + S_EXIT, 1u);

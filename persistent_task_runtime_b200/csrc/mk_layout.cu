@@ -43,6 +43,72 @@ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 // operator, so the dynamic queue evens out the operator's tail across SMs.
 int choose_mtiles(int tiles, int nsm, int cap) { return std::max(1, std::min(cap, tiles / (16 * nsm))); }
 
+// Solidified schedule (the Ada-MK summary's "Offline-Suche und
+// Pfad-Solidifizierung": the execution order is fixed offline instead of by
+// run-time dispatch).  List scheduling over the task array in queue order:
+// each task goes to the CTA on which a cost model says it would start first,
+// after that CTA's previous task and after the event it waits on is complete
+// (the latest finish among the event's producers).  Costs: a projection task
+// streams its weight bytes at an SM's share of the HBM bandwidth, plus a
+// fixed per-task cost; an attention slot and the embedding task a fixed cost.
+// Each CTA then runs its tasks in ascending index order.  That order cannot
+// deadlock: the unfinished task with the smallest index has all of its
+// producers (smaller indices) finished, and every earlier task of its own CTA
+// too.
+void solidify_schedule(const Params &p, const std::vector<Task> &T, int grid,
+                       std::vector<int> &sched, std::vector<int> &off) {
+  const double per_sm_bytes_per_us = 6.5e6 / 148.0;   // ~6.5 TB/s over 148 SMs
+  const double task_us = 0.8, attn_us = 2.5;
+  const int n = static_cast<int>(T.size());
+  std::vector<double> ev_ready(static_cast<size_t>(1 + p.L * p.ev_per_layer), 0.0);
+  std::vector<double> cta_free(static_cast<size_t>(grid), 0.0);
+  std::vector<int> owner(static_cast<size_t>(n), 0);
+  for (int i = 0; i < n; ++i) {
+    const Task &t = T[static_cast<size_t>(i)];
+    double ready = 0.0, cost = attn_us;
+    uint32_t sig = t.out_event;
+    if (t.type == T_ATTN) {
+      const int g = static_cast<int>(t.aux) / p.attn_spg;
+      ready = ev_ready[static_cast<size_t>(ev_attn_ready(p, t.layer, g))];
+    } else if (t.dep_event != kNoEvent) {
+      ready = ev_ready[t.dep_event];
+    }
+    if (t.type != T_ATTN && t.type != T_EMBED) {
+      int K = t.type == T_OPROJ ? p.Hq * p.d : (t.type == T_DOWN ? p.F : p.H);
+      const int kt = p.tc ? p.tc_kt[t.type] : (t.type == T_DOWN ? p.kchunk[K_FFN]
+                                                : (t.type == T_OPROJ ? p.kchunk[K_ATT] : 0));
+      if (t.nsplit > 1 && kt > 0) K = std::min(K - t.ksplit * kt, kt);
+      const double rows = static_cast<double>(t.nrows) * (t.type == T_GATEUP ? 2 : 1);
+      cost = task_us + rows * K * 2.0 / per_sm_bytes_per_us;
+    }
+    if (t.type == T_QKV) {
+      const int head = static_cast<int>(t.aux2);
+      const int g = t.aux == 0 ? head / p.G
+                               : (t.aux == 1 ? head - p.Hq : head - p.Hq - p.Hkv);
+      sig = static_cast<uint32_t>(ev_attn_ready(p, t.layer, g));
+    }
+    int best = 0;
+    double best_start = 1e300;
+    for (int c = 0; c < grid; ++c) {
+      const double st = std::max(cta_free[static_cast<size_t>(c)], ready);
+      if (st < best_start) {
+        best_start = st;
+        best = c;
+      }
+    }
+    const double fin = best_start + cost;
+    cta_free[static_cast<size_t>(best)] = fin;
+    owner[static_cast<size_t>(i)] = best;
+    if (sig != kNoEvent) ev_ready[sig] = std::max(ev_ready[sig], fin);
+  }
+  off.assign(static_cast<size_t>(grid) + 1, 0);
+  for (int i = 0; i < n; ++i) off[static_cast<size_t>(owner[static_cast<size_t>(i)]) + 1] += 1;
+  for (int c = 0; c < grid; ++c) off[static_cast<size_t>(c) + 1] += off[static_cast<size_t>(c)];
+  sched.assign(static_cast<size_t>(n), 0);
+  std::vector<int> fill(off.begin(), off.end() - 1);
+  for (int i = 0; i < n; ++i) sched[static_cast<size_t>(fill[static_cast<size_t>(owner[static_cast<size_t>(i)])]++)] = i;
+}
+
 }  // namespace
 
 int validate_config(const mk_model_config &c, std::string &err) {
@@ -85,6 +151,29 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   const int smem_max = std::min(smem_optin, kMaxSmem);
   const int mt_cap = max_mtiles_for(maxB);
 
+  // ---- GEMV path: CUDA-core mma.sync pages, or tcgen05 tiles of 128 rows -------------
+  // The tensor-core path needs one 128-row tile per head (head_dim 128) and
+  // inputs whose width is a whole number of 64-column swizzle atoms.
+  const bool tc_ok = d == kTcRows && H % 64 == 0 && F % 64 == 0 && (Hq * d) % 64 == 0;
+  if (o.gemv_path < 0 || o.gemv_path > 2)
+    return lfail(err, MK_ERR_INVALID_ARG, "gemv_path %d: 0 automatic, 1 mma.sync, 2 tcgen05",
+                 o.gemv_path);
+  if (o.gemv_path == 2 && !tc_ok)
+    return lfail(err, MK_ERR_UNSUPPORTED,
+                 "the tensor-core GEMV path needs head_dim 128 and hidden, ffn and "
+                 "n_q_heads*head_dim multiples of 64");
+  if (o.gemv_path == 2 && o.o_split)
+    return lfail(err, MK_ERR_INVALID_ARG, "o_split is an option of the mma.sync path");
+  const bool tc = o.gemv_path == 2 || (o.gemv_path == 0 && tc_ok && !o.o_split &&
+                                       maxB >= kTcAutoBatch);
+  if (tc) {
+    for (int i = 0; i < 5; ++i)
+      if (o.rows_per_task[i] != 0)
+        return lfail(err, MK_ERR_INVALID_ARG, "rows_per_task is an option of the mma.sync path");
+    if (o.max_page_cols != 0)
+      return lfail(err, MK_ERR_INVALID_ARG, "max_page_cols is an option of the mma.sync path");
+  }
+
   // ---- rows per task ----------------------------------------------------------
   auto rows_opt = [&](int i, int dflt) {
     const int r = o.rows_per_task[i];
@@ -101,16 +190,16 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   while ((d / 16) % nm_qkv) --nm_qkv;
   int R_qkv = rows_opt(0, 16 * nm_qkv);
   if (R_qkv > d || d % R_qkv || R_qkv > 16 * mt_cap) R_qkv = 16;
-  const int R_o = std::min(rows_opt(1, 16 * pick(H / 16, mt_cap)), 16 * mt_cap);
+  int R_o = std::min(rows_opt(1, 16 * pick(H / 16, mt_cap)), 16 * mt_cap);
   const int gu_cap = std::max(1, mt_cap / 2);   // gate and up tiles share a task
-  const int R_gu = std::min(rows_opt(2, 16 * pick(F / 16, gu_cap)), 16 * gu_cap);
+  int R_gu = std::min(rows_opt(2, 16 * pick(F / 16, gu_cap)), 16 * gu_cap);
   // a split down projection has a third or less of the columns per task:
   // two row tiles per task keep its per-task costs (dependency check,
   // restaging at each part) small against its pages
   const bool ffn_split = F > kx_limit;
   const int nm_d = std::max(pick(H / 16, mt_cap), ffn_split ? std::min(2, mt_cap) : 1);
-  const int R_d = std::min(rows_opt(3, 16 * nm_d), 16 * mt_cap);
-  const int R_lm = std::min(rows_opt(4, 16 * pick(V / 16, mt_cap)), 16 * mt_cap);
+  int R_d = std::min(rows_opt(3, 16 * nm_d), 16 * mt_cap);
+  int R_lm = std::min(rows_opt(4, 16 * pick(V / 16, mt_cap)), 16 * mt_cap);
 
   // ---- split-K of the down projection --------------------------------------------
   // Parts of at most kx_limit columns (the widest other input), so the down
@@ -139,7 +228,46 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   // others, so the overlap does not pay for the extra tasks.
   int o_groups = (o.o_split && Hkv >= 2) ? cdiv(Hkv, 2) : Hkv;
   if (o_groups * G * d < 1024) o_groups = Hkv;
-  const int n_o_parts = cdiv(Hkv, o_groups);
+  int n_o_parts = cdiv(Hkv, o_groups);
+
+  // ---- tensor-core path: 128-row tiles, split along K for load balance ----------------
+  // A task is one 128-row tile (gate/up: the gate tile and the up tile of the
+  // same rows) over a K range.  An operator with few tiles is split along K
+  // into parts of whole weight pages so that it has about two tasks per CTA;
+  // the part that completes a tile sums the parts in a fixed order.  The O
+  // projection is split into one part per KV group, each waiting only for the
+  // attention of its group.  The down projection's parts are whole gate/up
+  // tiles' rows, as on the other path.
+  int tc_bpad = 0, tc_kx = 0, tc_kc = 0;
+  int split[5] = {1, 1, 1, 1, 1};      // QKV, O, gate/up, down, LM head
+  int kt[5] = {0, 0, 0, 0, 0};          // columns per part (0: unsplit)
+  if (tc) {
+    tc_bpad = align_up_i(maxB, 8);
+    tc_kx = kTcXBytes / (2 * tc_bpad * 2);   // bf16 hi + lo rows of tc_bpad sequences
+    tc_kc = 128;                             // 32 KB pages (128 rows x 128 columns)
+    R_qkv = R_o = R_gu = R_d = R_lm = kTcRows;
+    auto parts_for = [&](int tiles, int K, int i) {
+      int n = std::max(1, std::min(cdiv(2 * grid, tiles), K / tc_kc));
+      int w = align_up_i(cdiv(K, n), tc_kc);
+      n = cdiv(K, w);
+      split[i] = n;
+      kt[i] = n > 1 ? w : 0;
+    };
+    parts_for(NQKV / kTcRows, H, 0);
+    parts_for(cdiv(F, kTcRows), H, 2);
+    parts_for(cdiv(H, kTcRows), F, 3);
+    o_groups = 1;
+    n_o_parts = Hkv;
+    split[1] = n_o_parts;
+    kt[1] = n_o_parts > 1 ? G * d : 0;
+    n_ksplit = split[3];
+    kchunk_ffn = kt[3] > 0 ? kt[3] : F;
+    if (n_ksplit > 255 || split[0] > 255 || split[2] > 255)
+      return lfail(err, MK_ERR_UNSUPPORTED, "too many split-K parts");
+  } else {
+    split[1] = n_o_parts;
+    split[3] = n_ksplit;
+  }
 
   // ---- shared memory: activation staging and the weight-page ring ------------------
   // Activation staging holds fp32 rows of every sequence: a whole input when
@@ -148,14 +276,17 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   // chunk (<= 64 KB).
   const int max_chunks = cdiv(c.max_seq_len, P);
   const int x_whole = maxB * x_row_bytes(kx_limit);
-  const int red_bytes = kComputeWarps * 16 * 8 * n_tiles_for(maxB) * 4;
-  const int out_stride = 16 * mt_cap;
+  // (the tensor-core path reduces in tensor memory: no cross-warp scratch;
+  // its output buffers hold two 128-row tiles, two of them in flight)
+  const int red_bytes = tc ? 0 : kComputeWarps * 16 * 8 * n_tiles_for(maxB) * 4;
+  const int out_stride = tc ? 2 * kTcRows : 16 * mt_cap;
   const int out_bytes = align_up_i(maxB * out_stride * 4, 128);
+  const int n_out = tc ? 2 : kOutSlots;
   const int off_look = 1024;   // loader lookahead
   const int off_slots = off_look + kLookBytes;
   const int off_red = align_up_i(off_slots + kTaskSlots * kSlotBytes, 128);
   const int off_out = align_up_i(off_red + red_bytes, 128);
-  const int off_x = align_up_i(off_out + kOutSlots * out_bytes, 128);
+  const int off_x = align_up_i(off_out + n_out * out_bytes, tc ? 1024 : 128);
 
   struct Geom {
     int kp[4], page_bytes, tpp, x_cap, off_pages, n_pages, ring;
@@ -198,9 +329,24 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   // largest ring any width gives with at least 3 pages; wider pages mean
   // fewer hand-offs per byte.  Failing 3 pages, the most pages.
   std::vector<Geom> cands;
-  for (int cand = colcap; cand >= 32; cand -= (cand > 256 ? 256 : 32)) {
+  for (int cand = colcap; cand >= 32 && !tc; cand -= (cand > 256 ? 256 : 32)) {
     Geom g{};
     if (geometry(cand, g)) cands.push_back(g);
+  }
+  if (tc) {
+    // two activation chunk buffers (also the attention scratch), then the
+    // ring of 128-row weight pages
+    Geom g{};
+    for (int i = 0; i < 4; ++i) g.kp[i] = tc_kc;
+    g.page_bytes = kTcRows * tc_kc * 2;
+    g.tpp = std::min((g.page_bytes / (4 * d)) / P * P, 16 * P);
+    const int att_need = G * d * 4 + std::max((G * g.tpp + 3 * kMaxGroup) * 4 + 2 * d * 2,
+                                              (2 * max_chunks * G + 2 * G) * 4);
+    g.x_cap = std::max(2 * kTcXBytes, align_up_i(att_need, 1024));
+    g.off_pages = align_up_i(off_x + g.x_cap, 1024);
+    g.n_pages = std::min(kMaxPages, (smem_max - g.off_pages) / g.page_bytes);
+    g.ring = g.n_pages * g.page_bytes;
+    if (g.tpp >= P) cands.push_back(g);
   }
   int best_ring = 0;
   for (const Geom &g : cands)
@@ -257,6 +403,18 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   p.kchunk[K_ATT] = n_o_parts > 1 ? o_groups * G * d : 0;
   p.wait_limit_ns = o.wait_limit_ns;
   p.n_ffn_parts = n_ksplit;
+  p.n_out = n_out;
+  p.tile_rows = tc ? kTcRows : 16;
+  p.tc = tc ? 1 : 0;
+  p.tc_bpad = tc_bpad;
+  p.tc_n = 2 * tc_bpad;
+  p.tc_kc = tc_kc;
+  p.tc_kx = tc_kx;
+  p.tc_kt[T_QKV] = kt[0];
+  p.tc_kt[T_OPROJ] = kt[1];
+  p.tc_kt[T_GATEUP] = kt[2];
+  p.tc_kt[T_DOWN] = kt[3];
+  p.tc_kt[T_LMHEAD] = kt[4];
   p.ev_embed = 0;
   p.ev_layer0 = 1;
   // attn_ready[Hkv], o_ready[O parts], oproj, gateup[down parts], down
@@ -281,6 +439,9 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     return t;
   };
   const int n_o = cdiv(H, R_o), n_down = cdiv(H, R_d), n_lm = cdiv(V, R_lm);
+  // row tiles of `nr` rows: 16-row mma tiles, or 128-row tensor-core tiles
+  auto mtiles = [&](int nr) { return tc ? cdiv(nr, kTcRows) : cdiv(nr, 16); };
+  // (with split-K parts, only the part that completes a tile signals)
   p.qkv_tasks_per_group = (G + 2) * (d / R_qkv);
   // gate/up tasks per split-K part of the down projection
   std::vector<uint32_t> gu_per_part(n_ksplit, 0);
@@ -305,12 +466,16 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
         const int mat = j < G ? 0 : j - G + 1;          // 0 q, 1 k, 2 v
         const int hh = mat == 0 ? kvg * G + j : kvg;     // head within its matrix
         const int head = mat == 0 ? hh : (mat == 1 ? Hq + hh : Hq + Hkv + hh);
-        for (int r0 = 0; r0 < d; r0 += R_qkv) {
-          Task t = gemv(T_QKV, l, hh * d + r0, R_qkv, R_qkv / 16, dep, cnt, kNoEvent);
-          t.aux = mat;
-          t.aux2 = static_cast<uint32_t>(head);
-          T.push_back(t);
-        }
+        for (int r0 = 0; r0 < d; r0 += R_qkv)
+          for (int ks = 0; ks < split[0]; ++ks) {
+            Task t = gemv(T_QKV, l, hh * d + r0, R_qkv, mtiles(R_qkv), dep, cnt, kNoEvent);
+            t.aux = mat;
+            t.aux2 = static_cast<uint32_t>(head);
+            t.ksplit = static_cast<uint8_t>(ks);
+            t.nsplit = static_cast<uint8_t>(split[0]);
+            t.map0 = static_cast<uint32_t>(tc_map_index(l, mat));
+            T.push_back(t);
+          }
       }
     out.ops.push_back({b0, static_cast<int>(T.size())});
     b0 = static_cast<int>(T.size());
@@ -329,10 +494,11 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
       const int groups = std::min(o_groups, Hkv - k * o_groups);
       for (int r0 = 0; r0 < H; r0 += R_o) {
         const int nr = std::min(R_o, H - r0);
-        Task t = gemv(T_OPROJ, l, r0, nr, cdiv(nr, 16), ev_o_ready(p, l, k),
+        Task t = gemv(T_OPROJ, l, r0, nr, mtiles(nr), ev_o_ready(p, l, k),
                       static_cast<uint32_t>(groups * p.attn_spg), ev_oproj(p, l));
         t.ksplit = static_cast<uint8_t>(k);
         t.nsplit = static_cast<uint8_t>(n_o_parts);
+        t.map0 = static_cast<uint32_t>(tc_map_index(l, 3));
         T.push_back(t);
       }
     }
@@ -341,16 +507,26 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     for (int r0 = 0; r0 < F; r0 += R_gu) {
       const int nr = std::min(R_gu, F - r0);
       const int part = n_ksplit > 1 ? r0 / kchunk_ffn : 0;
-      T.push_back(gemv(T_GATEUP, l, r0, nr, 2 * cdiv(nr, 16), ev_oproj(p, l), n_o, ev_gateup(p, l, part)));
+      for (int ks = 0; ks < split[2]; ++ks) {
+        Task t = gemv(T_GATEUP, l, r0, nr, 2 * mtiles(nr), ev_oproj(p, l), n_o,
+                      ev_gateup(p, l, part));
+        t.ksplit = static_cast<uint8_t>(ks);
+        t.nsplit = static_cast<uint8_t>(split[2]);
+        t.map0 = static_cast<uint32_t>(tc_map_index(l, 4));
+        t.map1 = static_cast<uint32_t>(tc_map_index(l, 5));
+        T.push_back(t);
+      }
     }
     out.ops.push_back({b0, static_cast<int>(T.size())});
     b0 = static_cast<int>(T.size());
     for (int ks = 0; ks < n_ksplit; ++ks)
       for (int r0 = 0; r0 < H; r0 += R_d) {
         const int nr = std::min(R_d, H - r0);
-        Task t = gemv(T_DOWN, l, r0, nr, cdiv(nr, 16), ev_gateup(p, l, ks), gu_per_part[ks], ev_down(p, l));
+        Task t = gemv(T_DOWN, l, r0, nr, mtiles(nr), ev_gateup(p, l, ks), gu_per_part[ks],
+                      ev_down(p, l));
         t.ksplit = static_cast<uint8_t>(ks);
         t.nsplit = static_cast<uint8_t>(n_ksplit);
+        t.map0 = static_cast<uint32_t>(tc_map_index(l, 6));
         T.push_back(t);
       }
     out.ops.push_back({b0, static_cast<int>(T.size())});
@@ -359,12 +535,17 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     const int b0 = static_cast<int>(T.size());
     for (int r0 = 0; r0 < V; r0 += R_lm) {
       const int nr = std::min(R_lm, V - r0);
-      T.push_back(gemv(T_LMHEAD, L - 1, r0, nr, cdiv(nr, 16), ev_down(p, L - 1), n_down, kNoEvent));
+      Task t = gemv(T_LMHEAD, L - 1, r0, nr, mtiles(nr), ev_down(p, L - 1), n_down, kNoEvent);
+      t.map0 = static_cast<uint32_t>(tc_map_index(L, 0));
+      T.push_back(t);
     }
     out.ops.push_back({b0, static_cast<int>(T.size())});
   }
   p.n_lm_tasks = n_lm;
   p.n_tasks = static_cast<int>(T.size());
+  if (o.schedule < 0 || o.schedule > 1)
+    return lfail(err, MK_ERR_INVALID_ARG, "schedule %d: 0 dynamic queue, 1 solidified", o.schedule);
+  if (o.schedule == 1) solidify_schedule(p, T, grid, out.sched, out.sched_off);
   if (o.debug_unsatisfiable_dep) T[1].dep_count += 1;  // first QKV task
 
   // ---- RoPE: pair i at position t turns by t * theta^(-2i/d), in double ----------------
@@ -390,13 +571,32 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   out.o_o = carve(sizeof(float) * maxB * Hq * d);
   out.o_u = carve(sizeof(float) * maxB * F);
   out.o_arg = carve(sizeof(unsigned long long) * maxB);
-  const int kparts = std::max(n_ksplit > 1 ? n_ksplit : 0, n_o_parts > 1 ? n_o_parts : 0);
-  out.o_kpart = carve(sizeof(float) * static_cast<size_t>(kparts) * maxB * H);
+  // split-K partials: QKV and down share one area (a layer's QKV starts only
+  // after the previous layer's down projection is complete, and the down
+  // projection only after every QKV tile); the O projection (whose first
+  // part may start while later QKV tiles are still summed) and gate/up
+  // (which overlaps the down projection) have their own
+  size_t kpart_floats = 0;
+  if (split[0] > 1) kpart_floats = std::max(kpart_floats, static_cast<size_t>(split[0]) * NQKV);
+  if (split[3] > 1) kpart_floats = std::max(kpart_floats, static_cast<size_t>(split[3]) * H);
+  out.o_kpart = carve(sizeof(float) * kpart_floats * maxB);
+  out.o_kpart_o = carve(sizeof(float) * (split[1] > 1 ? static_cast<size_t>(split[1]) * H : 0) * maxB);
+  out.o_kpart2 = carve(sizeof(float) * (split[2] > 1 ? static_cast<size_t>(split[2]) * 2 * F : 0) *
+                       maxB);
+  // per-16-row sums of h^2, written by the producers of h (tensor-core path)
+  const size_t ssq_floats = tc ? static_cast<size_t>(H / 16) * maxB : 0;
+  out.o_ssq_attn = carve(sizeof(float) * ssq_floats);
+  out.o_ssq_mlp = carve(sizeof(float) * ssq_floats);
   out.ws_bytes = off;
   out.n_events = n_events;
   out.comb_words = static_cast<size_t>(maxB) * Hkv;
-  out.tile_words = static_cast<size_t>(H) / 16 + 1;
-  out.sync_words = S_EVENTS + n_events + out.comb_words + out.tile_words;
+  out.tile_words = static_cast<size_t>(std::max(H, tc ? NQKV : 0)) / 16 + 1;
+  out.tile2_words = static_cast<size_t>(F) / 16 + 1;
+  out.tile_o_words = static_cast<size_t>(H) / 16 + 1;
+  out.sync_words = S_EVENTS + n_events + out.comb_words + out.tile_words + out.tile2_words +
+                   out.tile_o_words;
+  out.n_maps = tc ? L * kTcMatsPerLayer + 1 : 0;
+  for (int i = 0; i < 5; ++i) out.splits[i] = split[i];
 
   out.grid = grid;
   out.smem = smem;
@@ -416,9 +616,15 @@ void bind_workspace(const Layout &lay, char *ws, uint32_t *sync, Params &p) {
   p.u = reinterpret_cast<float *>(ws + lay.o_u);
   p.argmax = reinterpret_cast<unsigned long long *>(ws + lay.o_arg);
   p.kpart = reinterpret_cast<float *>(ws + lay.o_kpart);
+  p.kpart2 = reinterpret_cast<float *>(ws + lay.o_kpart2);
+  p.ssq_attn = reinterpret_cast<float *>(ws + lay.o_ssq_attn);
+  p.ssq_mlp = reinterpret_cast<float *>(ws + lay.o_ssq_mlp);
   p.sync = sync;
   p.comb_ctr = sync + S_EVENTS + lay.n_events;
   p.tile_ctr = p.comb_ctr + lay.comb_words;
+  p.tile_ctr2 = p.tile_ctr + lay.tile_words;
+  p.kpart_o = reinterpret_cast<float *>(ws + lay.o_kpart_o);
+  p.tile_ctr_o = p.tile_ctr2 + lay.tile2_words;
 }
 
 void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vector<Task> &tasks) {
@@ -451,6 +657,66 @@ void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vect
       default: break;
     }
   }
+}
+
+}  // namespace mk
+
+// ---- tensor maps of the weight matrices (tensor-core path) -------------------------
+// One 2-D map per matrix [rows][K] (bf16, row-major): a box is 64 columns
+// (128 bytes, one swizzle atom) by 128 rows, copied with the 128-byte swizzle
+// that the tensor core's K-major operand layout expects.  Rows past the end
+// of a matrix (a ragged last tile) arrive as zeros.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+namespace mk {
+
+int encode_weight_maps(const mk_model_config &c, const mk_weights &w, const Layout &lay,
+                       std::vector<unsigned char> &out, std::string &err) {
+  out.clear();
+  if (lay.n_maps == 0) return MK_OK;
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (encode == nullptr) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return lfail(err, MK_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const int L = c.n_layers, H = c.hidden, F = c.ffn, d = c.head_dim;
+  const int Hq = c.n_q_heads, Hkv = c.n_kv_heads;
+  out.assign(static_cast<size_t>(lay.n_maps) * sizeof(CUtensorMap), 0);
+  auto one = [&](int idx, const void *ptr, int rows, int K) {
+    CUtensorMap m;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcAtomCols), static_cast<cuuint32_t>(kTcRows)};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return lfail(err, MK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", r);
+    std::memcpy(out.data() + static_cast<size_t>(idx) * sizeof(CUtensorMap), &m, sizeof(m));
+    return MK_OK;
+  };
+  int rc = MK_OK;
+  for (int l = 0; l < L && rc == MK_OK; ++l) {
+    const mk_layer_weights &s = w.layers[l];
+    if ((rc = one(tc_map_index(l, 0), s.wq, Hq * d, H)) ||
+        (rc = one(tc_map_index(l, 1), s.wk, Hkv * d, H)) ||
+        (rc = one(tc_map_index(l, 2), s.wv, Hkv * d, H)) ||
+        (rc = one(tc_map_index(l, 3), s.wo, H, Hq * d)) ||
+        (rc = one(tc_map_index(l, 4), s.w_gate, F, H)) ||
+        (rc = one(tc_map_index(l, 5), s.w_up, F, H)) ||
+        (rc = one(tc_map_index(l, 6), s.w_down, H, F)))
+      break;
+  }
+  if (rc == MK_OK) rc = one(tc_map_index(L, 0), w.lm_head, c.vocab, H);
+  return rc;
 }
 
 }  // namespace mk

@@ -50,7 +50,7 @@ struct Uploaded {
   int page = 0, batch = 0, nsm = 0, smem_optin = 0;
   std::vector<const void *> ptrs;   // every weight pointer, in a fixed order
   mk::Layout lay;
-  size_t o_tasks = 0, o_rope = 0, o_ws = 0, o_sync = 0;
+  size_t o_tasks = 0, o_rope = 0, o_ws = 0, o_sync = 0, o_maps = 0;
 };
 Uploaded g_up[kMaxDevices];
 
@@ -166,6 +166,13 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
     up.o_rope = carve(up.lay.rope.size() * sizeof(float2));
     up.o_ws = carve(up.lay.ws_bytes);
     up.o_sync = carve(up.lay.sync_words * sizeof(uint32_t));
+    std::vector<unsigned char> maps;   // tensor maps of the tensor-core path (or none)
+    {
+      std::string merr;
+      const int mrc = mk::encode_weight_maps(c, *w, up.lay, maps, merr);
+      if (mrc) return nfail(mrc, merr.c_str());
+    }
+    up.o_maps = carve(maps.size());
     if (off > MK_NOALLOC_SCRATCH_BYTES) {
       char msg[256];
       snprintf(msg, sizeof(msg),
@@ -177,7 +184,9 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
     if (cudaMemcpyAsync(base + up.o_tasks, up.lay.tasks.data(), up.lay.tasks.size() * sizeof(Task),
                         cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(base + up.o_rope, up.lay.rope.data(), up.lay.rope.size() * sizeof(float2),
-                        cudaMemcpyHostToDevice, s) != cudaSuccess)
+                        cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        (!maps.empty() && cudaMemcpyAsync(base + up.o_maps, maps.data(), maps.size(),
+                                          cudaMemcpyHostToDevice, s) != cudaSuccess))
       return nfail(MK_ERR_CUDA, "uploading the step's tables into the scratch array failed");
     up.cfg = c;
     up.page = P;
@@ -200,6 +209,7 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
 
   p.tasks = reinterpret_cast<const Task *>(base + o_tasks);
   p.rope_cs = reinterpret_cast<const float2 *>(base + o_rope);
+  p.tmaps = base + up.o_maps;
   mk::bind_workspace(lay, base + o_ws, reinterpret_cast<uint32_t *>(base + o_sync), p);
   p.embed = static_cast<const __nv_bfloat16 *>(w->embed);
 

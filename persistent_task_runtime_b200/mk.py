@@ -38,7 +38,7 @@ ERROR_NAMES = {MK_OK: "MK_OK", MK_ERR_INVALID_ARG: "MK_ERR_INVALID_ARG",
 EXPORTS = ["mk_plan_create", "mk_plan_create_ex", "mk_decode_step", "mk_decode_step_ex",
            "mk_decode_step_host", "mk_plan_status", "mk_plan_error_info", "mk_plan_reset",
            "mk_plan_info", "mk_last_error", "mk_plan_destroy", "mk_decode_step_noalloc",
-           "mk_plan_describe"]
+           "mk_plan_describe", "mk_plan_describe_schedule"]
 
 #: bytes of the library's static scratch array used by mk_decode_step_noalloc
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -71,7 +71,7 @@ class mk_plan_options(C.Structure):
     _fields_ = [("max_batch", C.c_int), ("kv_page_size", C.c_int), ("num_ctas", C.c_int),
                 ("wait_limit_ns", C.c_int64), ("rows_per_task", C.c_int * 5),
                 ("debug_unsatisfiable_dep", C.c_int), ("max_page_cols", C.c_int),
-                ("o_split", C.c_int)]
+                ("o_split", C.c_int), ("gemv_path", C.c_int), ("schedule", C.c_int)]
 
 
 class mk_step_args(C.Structure):
@@ -89,7 +89,9 @@ class mk_plan_info_t(C.Structure):
                 ("page_cols", C.c_int * 4), ("weight_bytes", C.c_int64),
                 ("events_per_layer", C.c_int), ("attn_slots_per_group", C.c_int),
                 ("qkv_tasks_per_group", C.c_int), ("ffn_parts", C.c_int),
-                ("ffn_part_cols", C.c_int), ("o_parts", C.c_int), ("o_part_cols", C.c_int)]
+                ("ffn_part_cols", C.c_int), ("o_parts", C.c_int), ("o_part_cols", C.c_int),
+                ("gemv_path", C.c_int), ("schedule", C.c_int), ("qkv_parts", C.c_int),
+                ("gateup_parts", C.c_int)]
 
 
 _lib = None
@@ -118,6 +120,10 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
     lib.mk_plan_info.argtypes = [P, C.POINTER(mk_plan_info_t)]
     lib.mk_plan_describe.argtypes = [C.POINTER(mk_model_config), C.POINTER(mk_plan_options),
                                      C.c_int, C.c_int, C.POINTER(mk_plan_info_t), P, C.c_int64]
+    lib.mk_plan_describe_schedule.argtypes = [C.POINTER(mk_model_config),
+                                              C.POINTER(mk_plan_options), C.c_int, C.c_int, P,
+                                              C.c_int64]
+    lib.mk_plan_describe_schedule.restype = C.c_int
     lib.mk_last_error.restype = C.c_char_p
     lib.mk_last_error.argtypes = []
     lib.mk_plan_destroy.argtypes = [P]
@@ -173,7 +179,7 @@ class KVCacheView:
 TASK_RECORD_DTYPE = [("type", "u1"), ("n_m", "u1"), ("layer", "<u2"), ("row0", "<u4"),
                      ("nrows", "<u2"), ("ksplit", "u1"), ("nsplit", "u1"), ("dep_event", "<u4"),
                      ("dep_count", "<u4"), ("out_event", "<u4"), ("aux", "<u4"), ("aux2", "<u4"),
-                     ("operands", "<u8", (4,))]
+                     ("operands", "<u8", (3,)), ("map0", "<u4"), ("map1", "<u4")]
 TASK_TYPES = {1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead"}
 NO_EVENT = 0xFFFFFFFF
 
@@ -194,7 +200,8 @@ def _config(cfg: Dict, max_seq_len: int) -> mk_model_config:
 
 def describe(cfg: Dict, max_batch: int = 1, page_size: int = 16, max_seq_len: int = 4096,
              num_sms: int = 148, smem_optin: int = 232448, rows_per_task=(0, 0, 0, 0, 0),
-             max_page_cols: int = 0, o_split: bool = False):
+             max_page_cols: int = 0, o_split: bool = False, gemv_path: int = 0,
+             schedule: int = 0):
     """The plan mk_plan_create_ex would build, without a GPU: (info, task records).
 
     The task records are a numpy structured array (TASK_RECORD_DTYPE)."""
@@ -202,7 +209,7 @@ def describe(cfg: Dict, max_batch: int = 1, page_size: int = 16, max_seq_len: in
     lib = load_library()
     c = _config(cfg, max_seq_len)
     opts = mk_plan_options(max_batch, page_size, 0, 0, (C.c_int * 5)(*rows_per_task), 0,
-                           max_page_cols, 1 if o_split else 0)
+                           max_page_cols, 1 if o_split else 0, gemv_path, schedule)
     info = mk_plan_info_t()
     _check(lib.mk_plan_describe(C.byref(c), C.byref(opts), num_sms, smem_optin, C.byref(info),
                                 None, 0))
@@ -213,13 +220,29 @@ def describe(cfg: Dict, max_batch: int = 1, page_size: int = 16, max_seq_len: in
     return _info_dict(info), tasks
 
 
+def describe_schedule(cfg: Dict, n_tasks: int, max_batch: int = 1, page_size: int = 16,
+                      max_seq_len: int = 4096, num_sms: int = 148, smem_optin: int = 232448,
+                      gemv_path: int = 0, schedule: int = 1):
+    """CTA of every task under the plan's solidified schedule (-1: dynamic queue)."""
+    import numpy as np
+    lib = load_library()
+    c = _config(cfg, max_seq_len)
+    opts = mk_plan_options(max_batch, page_size, 0, 0, (C.c_int * 5)(0, 0, 0, 0, 0), 0, 0, 0,
+                           gemv_path, schedule)
+    out = np.zeros(n_tasks, dtype=np.int32)
+    _check(lib.mk_plan_describe_schedule(C.byref(c), C.byref(opts), num_sms, smem_optin,
+                                         out.ctypes.data, n_tasks))
+    return out
+
+
 class Plan:
     """A decode plan over caller-owned bf16 weights (see include/mk.h)."""
 
     def __init__(self, cfg: Dict, weights: Dict, max_batch: int = 1, page_size: int = 16,
                  max_seq_len: int = 4096, num_ctas: int = 0, wait_limit_ns: int = 0,
                  rows_per_task: Sequence[int] = (0, 0, 0, 0, 0), debug_unsatisfiable_dep=False,
-                 max_page_cols: int = 0, o_split: bool = False):
+                 max_page_cols: int = 0, o_split: bool = False, gemv_path: int = 0,
+                 schedule: int = 0):
         lib = load_library()
         self.cfg = dict(cfg)
         self.max_batch = max_batch
@@ -236,7 +259,7 @@ class Plan:
                              _ptr(weights["lm_head"]))
         opts = mk_plan_options(max_batch, page_size, num_ctas, wait_limit_ns,
                                (C.c_int * 5)(*rows_per_task), 1 if debug_unsatisfiable_dep else 0,
-                               max_page_cols, 1 if o_split else 0)
+                               max_page_cols, 1 if o_split else 0, gemv_path, schedule)
         h = C.c_void_p()
         _check(lib.mk_plan_create_ex(C.byref(self._c), C.byref(self._w), C.byref(opts),
                                      C.byref(h)))

@@ -101,14 +101,18 @@ def test_long_context_many_attention_chunks(cuda_device):
     assert_report(rep)
 
 
-def test_large_batch_chunked_activations(cuda_device):
-    """B = 16 (two mma n-tiles) with activations too wide for one staging
-    buffer, so every projection stages its input in column chunks."""
+@pytest.mark.parametrize("path", [1, 2])
+def test_large_batch_chunked_activations(cuda_device, path):
+    """B = 16 with activations too wide for one staging buffer: on the
+    mma.sync path (four mma n-tiles) every projection stages its input in
+    column chunks; on the tensor-core path chunks stream through two
+    buffers."""
     cfg = dict(n_layers=2, hidden=1024, n_q_heads=8, n_kv_heads=2, head_dim=128, ffn=4096,
                vocab=8192, rms_eps=1e-6, rope_theta=1e6, qk_norm=True)
     B = 16
     lengths = [int(x) for x in np.linspace(1, 200, B)]
-    pair = Pair(cfg, _weights(cfg, seed=8, gain="random"), B, [n + 8 for n in lengths])
+    pair = Pair(cfg, _weights(cfg, seed=8, gain="random"), B, [n + 8 for n in lengths],
+                gemv_path=path)
     pair.load_history(synth.make_kv_history(cfg, lengths, seed=9), lengths)
     ids = synth.make_ids(cfg["vocab"], (3, B), seed=10)
     rep = StepReport()

@@ -69,7 +69,9 @@ def check_plan(cfg, info, t, max_batch):
     assert info["smem_bytes"] <= SMEM
     assert info["n_pages"] >= 2
     assert info["n_pages"] * info["page_bytes"] < info["smem_bytes"]
-    max_mt = 8 // n_tiles_for(max_batch)
+    tc = info["gemv_path"] == 2
+    tile = 128 if tc else 16                     # rows per row tile
+    max_mt = 2 if tc else 8 // n_tiles_for(max_batch)
 
     # ---- who signals what, per step ----------------------------------------------------
     signals = Counter()
@@ -82,7 +84,13 @@ def check_plan(cfg, info, t, max_batch):
             g = head // G if mat == 0 else (head - Hq if mat == 1 else head - Hq - Hkv)
             assert 0 <= g < Hkv
             ev = ev_attn_ready(int(r["layer"]), g)
-        elif ty in (T_OPROJ, T_DOWN) and r["nsplit"] > 1:
+            if r["nsplit"] > 1:
+                key = (ty, int(r["layer"]), mat, int(r["row0"]))
+                if key in split_tiles:
+                    producers[ev].append(i)
+                    continue
+                split_tiles.add(key)
+        elif ty in (T_OPROJ, T_DOWN, T_GATEUP) and r["nsplit"] > 1:
             # the part that completes a row tile signals once for the tile
             key = (ty, int(r["layer"]), int(r["row0"]))
             if key in split_tiles:
@@ -119,12 +127,14 @@ def check_plan(cfg, info, t, max_batch):
         qkv = lay[lay["type"] == T_QKV]
         for mat, rows in ((0, Hq * d), (1, Hkv * d), (2, Hkv * d)):
             m = qkv[qkv["aux"] == mat]
-            cover = np.zeros(rows, dtype=int)
-            for r in m:
-                r0, n = int(r["row0"]), int(r["nrows"])
-                assert r0 // d == (r0 + n - 1) // d          # never straddles heads
-                cover[r0:r0 + n] += 1
-            assert (cover == 1).all()
+            for ks in range(info["qkv_parts"]):
+                cover = np.zeros(rows, dtype=int)
+                for r in m[m["ksplit"] == ks]:
+                    r0, n = int(r["row0"]), int(r["nrows"])
+                    assert r0 // d == (r0 + n - 1) // d          # never straddles heads
+                    assert int(r["nsplit"]) == max(info["qkv_parts"], 1) or info["qkv_parts"] == 1
+                    cover[r0:r0 + n] += 1
+                assert (cover == 1).all()
         for ty, rows, parts in ((T_OPROJ, H, max(o_parts, 1)), (T_DOWN, H, max(ffn_parts, 1))):
             m = lay[lay["type"] == ty]
             for ks in range(parts):
@@ -133,16 +143,17 @@ def check_plan(cfg, info, t, max_batch):
                     cover[int(r["row0"]):int(r["row0"]) + int(r["nrows"])] += 1
                 assert (cover == 1).all(), (l, ty, ks)
         gu = lay[lay["type"] == T_GATEUP]
-        cover = np.zeros(F, dtype=int)
         cols = info["ffn_part_cols"]
-        for r in gu:
-            r0, n = int(r["row0"]), int(r["nrows"])
-            cover[r0:r0 + n] += 1
-            part = r0 // cols if ffn_parts > 1 else 0
-            assert (r0 + n - 1) // cols == r0 // cols or ffn_parts == 1
-            assert int(r["out_event"]) == ev_gateup(l, part)
-            assert int(r["n_m"]) % 2 == 0 and 16 * (int(r["n_m"]) // 2) >= n
-        assert (cover == 1).all()
+        for ks in range(info["gateup_parts"]):
+            cover = np.zeros(F, dtype=int)
+            for r in gu[gu["ksplit"] == ks]:
+                r0, n = int(r["row0"]), int(r["nrows"])
+                cover[r0:r0 + n] += 1
+                part = r0 // cols if ffn_parts > 1 else 0
+                assert (r0 + n - 1) // cols == r0 // cols or ffn_parts == 1
+                assert int(r["out_event"]) == ev_gateup(l, part)
+                assert int(r["n_m"]) % 2 == 0 and tile * (int(r["n_m"]) // 2) >= n
+            assert (cover == 1).all()
     assert ffn_parts * info["ffn_part_cols"] >= F > (ffn_parts - 1) * info["ffn_part_cols"]
     assert o_parts * info["o_part_cols"] >= Hq * d > (o_parts - 1) * info["o_part_cols"]
     lm = t[t["type"] == T_LMHEAD]
@@ -155,7 +166,26 @@ def check_plan(cfg, info, t, max_batch):
     gemv = t[np.isin(t["type"], [T_QKV, T_OPROJ, T_GATEUP, T_DOWN, T_LMHEAD])]
     assert int(gemv["n_m"].max()) <= max_mt
     ng = gemv[gemv["type"] != T_GATEUP]
-    assert (16 * ng["n_m"].astype(int) >= ng["nrows"].astype(int)).all()
+    assert (tile * ng["n_m"].astype(int) >= ng["nrows"].astype(int)).all()
+    if tc:
+        # every tile names its tensor maps: wq/wk/wv 0-2, wo 3, gate 4 / up 5, down 6, LM head
+        want = {T_OPROJ: 3, T_DOWN: 6}
+        for r in gemv:
+            ty, l = int(r["type"]), int(r["layer"])
+            if ty == T_QKV:
+                assert int(r["map0"]) == 7 * l + int(r["aux"])
+            elif ty == T_GATEUP:
+                assert (int(r["map0"]), int(r["map1"])) == (7 * l + 4, 7 * l + 5)
+            elif ty == T_LMHEAD:
+                assert int(r["map0"]) == 7 * L
+            else:
+                assert int(r["map0"]) == 7 * l + want[ty]
+        # split-K parts are whole weight pages and about two tasks per CTA
+        assert info["page_cols"] == [128] * 4
+        for ty, parts in ((T_QKV, info["qkv_parts"]), (T_GATEUP, info["gateup_parts"]),
+                          (T_OPROJ, o_parts), (T_DOWN, ffn_parts)):
+            assert (t[t["type"] == ty]["nsplit"].astype(int) == (parts if parts > 1 else 0)).all() \
+                or parts == 1
 
     # ---- attention slots: one block per KV group ------------------------------------------
     att = t[t["type"] == T_ATTN]

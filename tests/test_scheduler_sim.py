@@ -20,10 +20,11 @@ constraints.
 import random
 from collections import deque
 
+import numpy as np
 import pytest
 
 from persistent_task_runtime_b200 import build, mk
-from tests.test_plan_layout import SHAPES, T_ATTN, T_DOWN, T_EMBED, T_OPROJ, T_QKV
+from tests.test_plan_layout import SHAPES, T_ATTN, T_DOWN, T_EMBED, T_GATEUP, T_OPROJ, T_QKV
 
 GEMV = {2, 4, 5, 6, 7}
 
@@ -55,18 +56,21 @@ def compile_tasks(cfg, info, t):
         else:
             sig = int(r["out_event"])
             sig = -1 if sig == mk.NO_EVENT else sig
-        split = ty in (T_OPROJ, T_DOWN) and int(r["nsplit"]) > 1
-        out.append((ty, wait, need, sig, (ty, layer, int(r["row0"])) if split else None,
-                    int(r["nsplit"])))
+        split = ty in (T_QKV, T_OPROJ, T_GATEUP, T_DOWN) and int(r["nsplit"]) > 1
+        key = (ty, layer, int(r["aux"]) if ty == T_QKV else 0, int(r["row0"]))
+        out.append((ty, wait, need, sig, key if split else None, int(r["nsplit"])))
     return out
 
 
-def simulate(tasks, n_events, workers, seed):
+def simulate(tasks, n_events, workers, seed, lists=None):
+    """``lists`` (a solidified schedule): worker w pops only the tasks of
+    lists[w], in that order, instead of the next global ticket."""
     rng = random.Random(seed)
     n = len(tasks)
     ctr = [0] * n_events
     tile = {}
     nxt = 0
+    pos = [0] * workers
     done = [0] * n
     held = [deque() for _ in range(workers)]
     store = [deque() for _ in range(workers)]
@@ -82,7 +86,8 @@ def simulate(tasks, n_events, workers, seed):
         for w in range(workers):
             if gate[w] is not None and satisfied(*gate[w]):
                 gate[w] = None
-            if nxt < n and len(held[w]) < cap[w] and gate[w] is None:
+            more = pos[w] < len(lists[w]) if lists is not None else nxt < n
+            if more and len(held[w]) < cap[w] and gate[w] is None:
                 enabled.append((w, 0))
             if held[w]:
                 _, wait, need, *_ = tasks[held[w][0]]
@@ -93,8 +98,12 @@ def simulate(tasks, n_events, workers, seed):
         assert enabled, f"deadlock: {finished} of {n} tasks finished, next ticket {nxt}"
         w, act = rng.choice(enabled)
         if act == 0:                          # pop the next ticket
-            i = nxt
-            nxt += 1
+            if lists is not None:
+                i = lists[w][pos[w]]
+                pos[w] += 1
+            else:
+                i = nxt
+                nxt += 1
             held[w].append(i)
             ty, wait, need, *_ = tasks[i]
             if ty == T_ATTN or (ty in GEMV and not satisfied(wait, need)):
@@ -119,15 +128,20 @@ def simulate(tasks, n_events, workers, seed):
     return ctr
 
 
-CASES = [("tiny", 1, 1), ("tiny", 1, 5), ("tiny", 3, 148), ("tiny", 16, 37),
-         ("ragged", 1, 7), ("ragged", 4, 148), ("3groups", 2, 20), ("d32", 1, 148),
-         ("1.5b", 1, 8), ("8b", 1, 16)]
+# (shape, max_batch, workers, GEMV path: 0 automatic, 2 tensor cores with
+# split-K QKV / O / gate/up / down)
+CASES = [("tiny", 1, 1, 0), ("tiny", 1, 5, 0), ("tiny", 3, 148, 0), ("tiny", 16, 37, 0),
+         ("ragged", 1, 7, 0), ("ragged", 4, 148, 0), ("3groups", 2, 20, 0), ("d32", 1, 148, 0),
+         ("1.5b", 1, 8, 0), ("8b", 1, 16, 0),
+         ("3groups", 8, 20, 0), ("3groups", 1, 3, 2), ("3groups", 16, 148, 2), ("8b", 16, 16, 0)]
 
 
-@pytest.mark.parametrize("name,batch,workers", CASES)
-def test_no_deadlock_every_task_once(name, batch, workers):
+@pytest.mark.parametrize("name,batch,workers,path", CASES)
+def test_no_deadlock_every_task_once(name, batch, workers, path):
     cfg = SHAPES[name]
-    info, t = mk.describe(cfg, max_batch=batch, max_seq_len=600)
+    info, t = mk.describe(cfg, max_batch=batch, max_seq_len=600, gemv_path=path)
+    if path == 2 or (batch >= 5 and cfg["head_dim"] == 128):
+        assert info["gemv_path"] == 2
     tasks = compile_tasks(cfg, info, t)
     seeds = (1,) if name in ("1.5b", "8b") else (1, 2, 3)
     for seed in seeds:
@@ -160,3 +174,31 @@ def test_simulator_detects_a_consumer_before_its_producer():
     tasks = [tasks[1], tasks[0]] + tasks[2:]
     with pytest.raises(AssertionError, match="deadlock"):
         simulate(tasks, info["n_events"], 1, seed=1)
+
+
+@pytest.mark.parametrize("name,batch,workers,path", [("tiny", 1, 5, 0), ("3groups", 2, 20, 0),
+                                                     ("3groups", 16, 148, 2), ("1.5b", 1, 148, 0),
+                                                     ("8b", 1, 148, 0)])
+def test_solidified_schedule_no_deadlock(name, batch, workers, path):
+    """Each CTA runs the plan's offline task list in order: every task is on
+    exactly one list, lists ascend, and any interleaving finishes the step."""
+    cfg = SHAPES[name]
+    info, t = mk.describe(cfg, max_batch=batch, max_seq_len=600, gemv_path=path, schedule=1,
+                          num_sms=workers)
+    assert info["schedule"] == 1 and info["num_ctas"] == workers
+    owner = mk.describe_schedule(cfg, info["n_tasks"], max_batch=batch, max_seq_len=600,
+                                 gemv_path=path, num_sms=workers)
+    assert owner.min() >= 0 and owner.max() < workers
+    lists = [[int(i) for i in np.flatnonzero(owner == w)] for w in range(workers)]
+    assert sum(len(x) for x in lists) == len(t)
+    # the cost model spreads every operator's work over many CTAs
+    used = len({int(owner[i]) for i in range(len(t)) if int(t["type"][i]) == 6})
+    assert used >= min(workers, int((t["type"] == 6).sum())) // 2
+    tasks = compile_tasks(cfg, info, t)
+    ctr = simulate(tasks, info["n_events"], workers, seed=1, lists=lists)
+    for ty, wait, need, *_ in tasks:
+        if wait >= 0:
+            assert ctr[wait] == need
+    # the dynamic plan describes no schedule
+    assert (mk.describe_schedule(cfg, info["n_tasks"], max_batch=batch, max_seq_len=600,
+                                 gemv_path=path, num_sms=workers, schedule=0) == -1).all()
