@@ -227,7 +227,34 @@ def run_mk(args, rank: int, world: int, local_rank: int) -> dict:
         torch.cuda.set_stream(torch.cuda.Stream(dev))   # graph capture needs a created stream
     stream = torch.cuda.current_stream(dev)
 
-    if wl["prefill"] == "decode":
+    prefill_info = None
+    if wl["prefill"] == "decode" and args.prompt_path == "chunks":
+        # the prompt through prompt chunks of up to 16 tokens on a plan of its
+        # own (multi-token tasks; the LM head runs on the last chunk only)
+        pplan = mk.Plan(cfg, weights, max_batch=16, page_size=16, max_seq_len=max(cap) + 16,
+                        prefill=True)
+        prompt = synth.make_ids(cfg["vocab"], (B, lengths[0]), seed=1).to(dev).to(torch.int32)
+        first = torch.zeros(1, dtype=torch.int32, device=dev)
+        for b in range(B):   # warm the plan (and the cache pages) once
+            pplan.prefill(prompt[b], b, kv.view, first)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for b in range(B):
+            pplan.prefill(prompt[b], b, kv.view, nids[b:b + 1])
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        st = pplan.status()
+        if st != mk.MK_OK:
+            raise RuntimeError(f"prefill failed: {mk.ERROR_NAMES.get(st, st)}")
+        ms = e0.elapsed_time(e1)
+        prefill_info = {"tokens": B * lengths[0], "ms": round(ms, 3),
+                        "tokens_per_s": round(B * lengths[0] / (ms / 1e3), 1),
+                        "chunk": 16, "launches": B * ((lengths[0] + 15) // 16)}
+        pplan.close()
+        ids.copy_(nids)
+        pos.fill_(lengths[0])
+    elif wl["prefill"] == "decode":
         # teacher-forced prompt through the same decode step
         prompt = synth.make_ids(cfg["vocab"], (lengths[0], B), seed=1).to(dev)
         for t in range(lengths[0]):
@@ -322,6 +349,7 @@ def run_mk(args, rank: int, world: int, local_rank: int) -> dict:
                 launch_ms=launch_ms,
                 kv_bytes=kvb, weight_bytes=info["weight_bytes"], info=info, clocks=clk.summary(),
                 e2e=e2e, cfg=cfg, B=B, lengths=lengths, mode=args.mode, start_pos=start_pos,
+                prefill=prefill_info,
                 launches_per_step=(1 if mode == mk.MODE_MEGAKERNEL else
                                    2 + 5 * cfg["n_layers"]))
 
@@ -417,6 +445,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=32)
     ap.add_argument("--gemv-path", type=int, default=0, choices=[0, 1, 2],
                     help="projections: 0 automatic, 1 mma.sync pages, 2 tcgen05 tiles")
+    ap.add_argument("--prompt-path", choices=["chunks", "decode"], default="chunks",
+                    help="how a workload's prompt fills the cache: prompt chunks of 16 tokens "
+                         "(mk_prefill_chunk) or one decode step per token")
     ap.add_argument("--schedule", type=int, default=0, choices=[0, 1],
                     help="0 dynamic ticket queue, 1 solidified per-CTA task lists")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -433,7 +464,8 @@ def main():
     config = {"workload": args.workload, "model_shape": wl["model"], "batch": wl["batch"],
               "context": wl["lengths"] if len(set(wl["lengths"])) > 1 else wl["lengths"][0],
               "kv_page": 16, "weights": "random N(0,0.02) bf16", "ids": "uniform random",
-              "prefill": ("teacher-forced decode steps" if wl["prefill"] == "decode"
+              "prefill": (("prompt chunks of 16 tokens" if args.prompt_path == "chunks"
+                           else "teacher-forced decode steps") if wl["prefill"] == "decode"
                           else "synthetic KV history"),
               "l2": "inputs larger than L2 (every step streams all weights)",
               "parallelism": f"replicas{world}"}
@@ -492,6 +524,7 @@ def main():
                         "std": round(1e3 * (statistics.pstdev(r["launch_ms"])
                                             if len(r["launch_ms"]) > 1 else 0.0), 2)},
             "roofline": roofline, "clocks": r["clocks"], "e2e": r["e2e"],
+            "prompt": r["prefill"],
             "gpu_launches": K * r["launches_per_step"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         w = cpu_weights_sample(cfg)

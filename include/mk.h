@@ -157,6 +157,13 @@ typedef struct {
                              offline path solidification) and each CTA runs
                              its list in order.  Per-operator modes always
                              use the queue                                  */
+  int prefill;            /* nonzero: the plan can also run prompt chunks
+                             (mk_prefill_chunk).  Each layer then appends
+                             the step's K/V in tasks of their own, one per
+                             KV group, and the group's attention waits for
+                             them, so a row may attend to positions that
+                             other rows of the same launch write.  Decode
+                             steps on such a plan give the same results    */
 } mk_plan_options;
 
 typedef struct mk_plan mk_plan;
@@ -208,6 +215,38 @@ typedef struct {
                              times in ns of the GPU global timer           */
 } mk_step_args;
 
+/* A chunk of one sequence's prompt: n_tokens consecutive tokens at positions
+ * pos0 .. pos0 + n_tokens - 1, run as one launch in which row j is the
+ * token at pos0 + j.  The multi-token form of the decode step: every
+ * projection streams its weights once for the whole chunk, each row's K/V is
+ * appended to the cache, and row j attends causally to positions
+ * 0 .. pos0 + j (the MPK write-up, "2.2 混合任务启动机制", on running the
+ * same task graph for other input shapes; the Ada-MK summary, "Methodik",
+ * on prefill beside decode). */
+typedef struct {
+  const int32_t *d_ids;   /* [n_tokens] the chunk's token ids               */
+  int n_tokens;           /* 1 .. max_batch                                 */
+  int pos0;               /* position of the chunk's first token            */
+  int seq;                /* the sequence: block-table row (0 .. max_batch-1)*/
+  const mk_kv_cache *kv;
+  int32_t *d_out_ids;     /* [n_tokens] argmax after each token (the last one
+                             is the first generated token); may be NULL
+                             without the LM head                            */
+  float *d_out_logits;    /* [n_tokens, V] or NULL (needs with_lm_head)     */
+  float *d_hidden;        /* [n_layers, n_tokens, H] residual stream after
+                             each layer, or NULL                            */
+  int with_lm_head;       /* 0: stop after the last layer (a chunk whose
+                             logits nobody reads); 1: final norm, LM head and
+                             argmax for every row                           */
+} mk_prefill_args;
+
+/* Enqueue one prompt chunk on `stream` (asynchronous, like mk_decode_step).
+ * The plan must have been created with opts->prefill != 0 (else
+ * MK_ERR_INVALID_ARG); other argument errors are MK_ERR_INVALID_ARG, found
+ * before the launch.  Device errors go to mk_plan_status().  Chunks of one
+ * prompt must run in order (pos0 = 0, T, 2T, ...). */
+MK_API int mk_prefill_chunk(mk_plan *plan, const mk_prefill_args *args, void *stream);
+
 /* Enqueue one decode step on `stream` (a cudaStream_t; NULL = legacy default
  * stream).  Asynchronous: device-side errors (MK_ERR_RANGE, MK_ERR_TIMEOUT)
  * are reported by mk_plan_status().  A step enqueued while the plan holds a
@@ -256,6 +295,7 @@ typedef struct {
   int o_parts, o_part_cols; /* the same for the O projection               */
   int gemv_path;          /* the path the plan uses: 1 mma.sync, 2 tcgen05  */
   int schedule;           /* 0 dynamic queue, 1 solidified per-CTA lists    */
+  int prefill;            /* 1: created with the prefill option             */
   int qkv_parts, gateup_parts; /* split-K parts of the QKV and gate/up
                              projections (tensor-core path; 1 otherwise)   */
 } mk_plan_info_t;

@@ -116,6 +116,7 @@ int layout_options(const mk_plan_options *opts, mk::LayoutOptions &lo) {
   lo.o_split = o.o_split != 0;
   lo.gemv_path = o.gemv_path;
   lo.schedule = o.schedule;
+  lo.prefill = o.prefill != 0;
   for (int i = 0; i < 5; ++i) lo.rows_per_task[i] = o.rows_per_task[i];
   lo.wait_limit_ns = o.wait_limit_ns == 0 ? 2000000000LL : o.wait_limit_ns;
   lo.debug_unsatisfiable_dep = o.debug_unsatisfiable_dep != 0;
@@ -154,6 +155,7 @@ void fill_info(const mk::Layout &lay, const mk_model_config &c, mk_plan_info_t &
   }
   I.gemv_path = p.tc ? 2 : 1;
   I.schedule = lay.sched.empty() ? 0 : 1;
+  I.prefill = lay.p.kv_tasks;
   I.qkv_parts = lay.splits[0];
   I.gateup_parts = lay.splits[2];
 }
@@ -381,6 +383,7 @@ int mk_decode_step_ex(mk_plan *plan, const mk_step_args *a, void *stream) {
   plan->epoch += 1;
   p.epoch = plan->epoch;
   p.batch = a->batch;
+  p.chunk_seq = -1;
   p.mode = a->mode;
   p.ids = a->d_ids;
   p.pos = a->d_pos;
@@ -426,6 +429,65 @@ int mk_decode_step_ex(mk_plan *plan, const mk_step_args *a, void *stream) {
       cudaError_t e = mk::launch_step(p, grid, plan->smem, false, s);
       if (e != cudaSuccess) return fail(MK_ERR_CUDA, "per-op launch: %s", cudaGetErrorString(e));
     }
+  }
+  return MK_OK;
+}
+
+int mk_prefill_chunk(mk_plan *plan, const mk_prefill_args *a, void *stream) {
+  g_err.clear();
+  if (plan == nullptr || a == nullptr) return fail(MK_ERR_INVALID_ARG, "plan or args is NULL");
+  if (!plan->base.kv_tasks)
+    return fail(MK_ERR_INVALID_ARG, "the plan was not created with the prefill option");
+  if (a->n_tokens < 1 || a->n_tokens > plan->max_batch)
+    return fail(MK_ERR_INVALID_ARG, "n_tokens %d outside 1..max_batch %d", a->n_tokens,
+                plan->max_batch);
+  if (a->seq < 0 || a->seq >= plan->max_batch)
+    return fail(MK_ERR_INVALID_ARG, "seq %d outside 0..max_batch-1", a->seq);
+  if (a->pos0 < 0 || a->pos0 + a->n_tokens > plan->cfg.max_seq_len)
+    return fail(MK_ERR_INVALID_ARG, "positions %d..%d outside 0..max_seq_len-1", a->pos0,
+                a->pos0 + a->n_tokens - 1);
+  if (a->d_ids == nullptr || (a->with_lm_head && a->d_out_ids == nullptr))
+    return fail(MK_ERR_INVALID_ARG, "d_ids (and, with the LM head, d_out_ids) must not be NULL");
+  if (!a->with_lm_head && a->d_out_logits != nullptr)
+    return fail(MK_ERR_INVALID_ARG, "d_out_logits needs with_lm_head");
+  int rc = validate_kv(plan, a->kv);
+  if (rc) return rc;
+  Params p = plan->base;
+  plan->epoch += 1;
+  p.epoch = plan->epoch;
+  p.batch = a->n_tokens;
+  p.chunk_seq = a->seq;
+  p.chunk_pos0 = a->pos0;
+  p.mode = MK_MODE_MEGAKERNEL;
+  p.ids = a->d_ids;
+  p.pos = nullptr;
+  p.out_ids = a->d_out_ids;
+  p.out_pos = nullptr;
+  p.out_logits = a->d_out_logits;
+  p.hidden_dump = a->d_hidden;
+  p.trace = nullptr;
+  p.block_table = a->kv->block_table;
+  p.num_kv_pages = a->kv->num_pages;
+  p.max_pages_per_seq = a->kv->max_pages_per_seq;
+  const long long cap = static_cast<long long>(a->kv->max_pages_per_seq) * p.page_size;
+  p.max_pos = static_cast<int>(std::min<long long>(plan->cfg.max_seq_len, cap));
+  for (int l = 0; l < plan->cfg.n_layers; ++l) {
+    p.k_pages[l] = static_cast<__nv_bfloat16 *>(a->kv->k_pages[l]);
+    p.v_pages[l] = static_cast<__nv_bfloat16 *>(a->kv->v_pages[l]);
+  }
+  p.task_begin = 0;
+  // without the LM head the launch ends with the last layer (the queue and a
+  // solidified schedule both skip the LM-head tasks)
+  p.task_end = a->with_lm_head ? p.n_tasks : plan->lay.first_lm_task;
+  if (!a->with_lm_head && p.sched != nullptr) {
+    p.sched = nullptr;   // the per-CTA lists include LM-head tasks: use the queue
+    p.sched_off = nullptr;
+  }
+  const cudaError_t e = mk::launch_step(p, plan->grid, plan->smem, true,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    plan->epoch -= 1;
+    return fail(MK_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
   }
   return MK_OK;
 }

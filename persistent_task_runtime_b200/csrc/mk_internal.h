@@ -55,6 +55,7 @@ enum TaskType : uint8_t {
   T_GATEUP = 5,
   T_DOWN = 6,
   T_LMHEAD = 7,
+  T_KVAPP = 8,     // prefill plans: QK-norm + RoPE + KV append of one KV group, every row
   T_END = 255,
 };
 
@@ -130,6 +131,8 @@ struct Params {
   int n_lm_tasks;
   long long wait_limit_ns;
   int n_out;                          // compute -> storer output buffers in use (<= kOutSlots)
+  int kv_tasks;                       // 1: K/V of the step are appended by T_KVAPP tasks
+                                      //    before any attention reads the cache (prefill plans)
   int tile_rows;                      // rows per row tile: 16 (mma.sync) or kTcRows (tcgen05)
 
   // tensor-core GEMV path (tc = 1): every GEMV task runs on tcgen05 tiles
@@ -154,6 +157,9 @@ struct Params {
   // per step
   uint32_t epoch;
   int batch;
+  int chunk_seq;              // >= 0: a prompt chunk of one sequence: row b is that sequence's
+                              //       token at position chunk_pos0 + b (block-table row chunk_seq)
+  int chunk_pos0;
   int task_begin, task_end;   // launch covers tickets mapped onto [begin, end)
   int mode;
   const int32_t *ids, *pos;
@@ -182,6 +188,17 @@ __host__ __device__ inline int ev_gateup(const Params &p, int l, int part) {
 }
 __host__ __device__ inline int ev_down(const Params &p, int l) {
   return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + p.n_o_parts + 1 + p.n_ffn_parts;
+}
+// prefill plans: the K/V of KV group g of every row are in the cache
+__host__ __device__ inline int ev_kv_ready(const Params &p, int l, int g) {
+  return p.ev_layer0 + l * p.ev_per_layer + p.Hkv + p.n_o_parts + 2 + p.n_ffn_parts + g;
+}
+// what an attention chunk of KV group g waits for, and how many completions
+__host__ __device__ inline int ev_attn_input(const Params &p, int l, int g) {
+  return p.kv_tasks ? ev_kv_ready(p, l, g) : ev_attn_ready(p, l, g);
+}
+__host__ __device__ inline int attn_input_count(const Params &p) {
+  return p.kv_tasks ? 1 : p.qkv_tasks_per_group;
 }
 
 // Tensor map of weight matrix j (0 wq, 1 wk, 2 wv, 3 wo, 4 w_gate, 5 w_up,
@@ -215,6 +232,7 @@ struct LayoutOptions {
   bool o_split = false;         // O projection in two K parts of whole KV groups
   int gemv_path = 0;            // 0 automatic, 1 mma.sync pages, 2 tcgen05 tiles
   int schedule = 0;             // 0 dynamic ticket queue, 1 solidified per-CTA task lists
+  bool prefill = false;         // K/V appended by their own tasks (prompt chunks of one sequence)
   int rows_per_task[5] = {0, 0, 0, 0, 0};
   long long wait_limit_ns = 2000000000LL;
   bool debug_unsatisfiable_dep = false;
@@ -235,6 +253,7 @@ struct Layout {
   size_t ws_bytes = 0;
   size_t comb_words = 0, tile_words = 0, tile2_words = 0, tile_o_words = 0, sync_words = 0;
   int n_maps = 0;                      // tensor maps the tensor-core path needs (0: none)
+  int first_lm_task = 0;               // task index of the first LM-head task
   // solidified schedule (empty: dynamic queue): task indices per CTA, and
   // the CTA's first entry (grid + 1 offsets)
   std::vector<int> sched, sched_off;

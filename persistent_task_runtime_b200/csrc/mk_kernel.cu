@@ -480,11 +480,21 @@ __device__ __forceinline__ void gemv_tile(const Params &p, const Task &t, int m,
   rows_valid = left < 16 ? (left > 0 ? left : 0) : 16;
 }
 
+// Position of row b this step: its own, or (a prompt chunk of one sequence)
+// the chunk's first position + b.
+__device__ __forceinline__ int row_pos(const Params &p, int b) {
+  return p.chunk_seq >= 0 ? p.chunk_pos0 + b : p.pos[b];
+}
+// Block-table row of row b: its own, or the chunk's sequence.
+__device__ __forceinline__ int row_seq(const Params &p, int b) {
+  return p.chunk_seq >= 0 ? p.chunk_seq : b;
+}
+
 // Tokens attended by sequence b this step (positions 0..pos), clamped to
 // [1, max_pos] so a bad position cannot blow up the attention split (bad
 // positions are reported by the embedding task).
 __device__ __forceinline__ int seq_len(const Params &p, int b) {
-  int n = p.pos[b] + 1;
+  int n = row_pos(p, b) + 1;
   return n < 1 ? 1 : (n > p.max_pos ? p.max_pos : n);
 }
 
@@ -528,7 +538,7 @@ __device__ bool attn_resolve(const Params &p, int B, int s, Slot &o) {
 
 __device__ __forceinline__ int kv_phys_page(const Params &p, int b, int logical) {
   int lp = logical < p.max_pages_per_seq ? logical : p.max_pages_per_seq - 1;
-  int ph = p.block_table[b * p.max_pages_per_seq + lp];
+  int ph = p.block_table[row_seq(p, b) * p.max_pages_per_seq + lp];
   return (ph >= 0 && ph < p.num_kv_pages) ? ph : -1;
 }
 
@@ -689,8 +699,8 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
         // an attention chunk waits for its KV group's projections: one such
         // chunk per CTA, so a group's chunks run on as many SMs as it has
         blocked = true;
-        blk_ev = static_cast<uint32_t>(ev_attn_ready(p, t.layer, info.g));
-        blk_cnt = static_cast<uint32_t>(p.qkv_tasks_per_group);
+        blk_ev = static_cast<uint32_t>(ev_attn_input(p, t.layer, info.g));
+        blk_cnt = static_cast<uint32_t>(attn_input_count(p));
         blk_tix = tix;
       }
     }
@@ -763,6 +773,18 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       }
     } else if (t.type == T_ATTN && info.b >= 0) {
       const int l = t.layer;
+      if (p.kv_tasks) {
+        // the chunk's pages may hold K/V that this step's K/V tasks write:
+        // copy them only once those are complete, and order the copies
+        // (async proxy) after the acquired writes
+        if (lane == 0)
+          okl = wait_event(p, ctl, static_cast<uint32_t>(ev_attn_input(p, l, info.g)),
+                           static_cast<uint32_t>(attn_input_count(p)), static_cast<uint32_t>(tix));
+        ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+        if (!ok) break;
+        __syncwarp();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
       const int P = p.page_size, d = p.d;
       const size_t kvpage_elems = static_cast<size_t>(P) * d;
       const uint32_t kvpage_bytes = static_cast<uint32_t>(kvpage_elems * 2);
@@ -1554,9 +1576,9 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   st.xkey = 0xffffffffu;                                    // staging area reused
 
   {
-    const uint32_t ev = static_cast<uint32_t>(ev_attn_ready(p, l, g));
+    const uint32_t ev = static_cast<uint32_t>(ev_attn_input(p, l, g));
     bool okl = true;
-    if (ctid == 0) okl = wait_event(p, ctl, ev, static_cast<uint32_t>(p.qkv_tasks_per_group), S.idx);
+    if (ctid == 0) okl = wait_event(p, ctl, ev, static_cast<uint32_t>(attn_input_count(p)), S.idx);
     if (!st.gs.share(ctl, ctid, okl)) return false;
     if (ctid == 0) trace_mark(p, S.idx, 4);
   }
@@ -1565,8 +1587,10 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   // in the chunk that holds the current position, K (QK-norm, RoPE) and V of
   // the current token, rounded to bf16 and appended to the cache.
   const int P = p.page_size;
-  const int cur = p.pos[b];
-  const bool own_cur = cur >= S.t0 && cur < S.t1;
+  const int cur = row_pos(p, b);
+  // (in a plan whose K/V tasks append every row's K/V first, the cache
+  // already holds the current token's)
+  const bool own_cur = !p.kv_tasks && cur >= S.t0 && cur < S.t1;
   {
     const float qscale = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;
     // a position outside 0..max_pos-1 is reported by the embedding task; the
@@ -1622,7 +1646,7 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     uint8_t *vpg = kpg + static_cast<size_t>(p.tpp) * D * 2;
     // The page was copied from the cache before this step's K/V of the
     // current token were formed: put them into its slot.
-    const bool has_cur = cur >= tok0 && cur < tok0 + ntok;
+    const bool has_cur = own_cur && cur >= tok0 && cur < tok0 + ntok;
     if (has_cur) {
       const int j = cur - tok0;
       if (ctid < 2 * NB) {
@@ -1766,6 +1790,48 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
 }
 
 // ============================================================================
+// compute warps: K/V append of one KV group for every row (prefill plans)
+// ============================================================================
+
+// From this step's raw projections: K (QK-norm, RoPE at the row's position)
+// and V of KV group t.aux for every row, rounded to bf16 and written to the
+// cache, one warp per (row, K or V).  Attention chunks of the group wait for
+// this task, so a row may attend to positions that other rows of the same
+// step (earlier tokens of the same prompt chunk) write.
+template <int D>
+__device__ bool kv_append_task(const Params &p, Ctl *ctl, const Slot &S, ComputeState &st,
+                               int ctid) {
+  const Task &t = S.t;
+  const int warp = ctid >> 5, lane = ctid & 31;
+  const int g = static_cast<int>(t.aux), l = t.layer, P = p.page_size;
+  {
+    bool okl = true;
+    if (ctid == 0) okl = wait_event(p, ctl, t.dep_event, t.dep_count, S.idx);
+    if (!st.gs.share(ctl, ctid, okl)) return false;
+    if (ctid == 0) trace_mark(p, S.idx, 4);
+  }
+  for (int w = warp; w < 2 * p.batch; w += kComputeWarps) {
+    const int b = w >> 1, mat = 1 + (w & 1);   // 1 k, 2 v
+    const int cur = row_pos(p, b);
+    const int cpos = cur < 0 ? 0 : (cur >= p.max_pos ? p.max_pos - 1 : cur);
+    const float2 *cs = p.rope_cs + static_cast<size_t>(cpos) * (D / 2);
+    const float *raw = p.qkv + static_cast<size_t>(b) * p.NQKV +
+                       (mat == 1 ? (p.Hq + g) * D : (p.Hq + p.Hkv + g) * D);
+    float v[4];
+    head_norm_rope<D>(raw, t.w1, p.qk_norm != 0 && mat == 1, mat == 1, cs, p.eps, lane, v);
+    const int ph = kv_phys_page(p, b, cur / P);
+    if (lane < D / 4 && ph >= 0) {
+      const uint2 pk = make_uint2(pack2(__float2bfloat16_rn(v[0]), __float2bfloat16_rn(v[1])),
+                                  pack2(__float2bfloat16_rn(v[2]), __float2bfloat16_rn(v[3])));
+      __nv_bfloat16 *dst = (mat == 1 ? p.k_pages[l] : p.v_pages[l]) +
+                           ((static_cast<size_t>(ph) * p.Hkv + g) * P + cur % P) * D + lane * 4;
+      *reinterpret_cast<uint2 *>(dst) = pk;
+    }
+  }
+  return true;
+}
+
+// ============================================================================
 // compute warps: embedding gather
 // ============================================================================
 
@@ -1773,7 +1839,7 @@ __device__ void embed_task(const Params &p, const Slot &S, int ctid) {
   const int B = p.batch, H = p.H;
   for (int b = 0; b < B; ++b) {
     const int id = p.ids[b];
-    const int pos = p.pos[b];
+    const int pos = row_pos(p, b);
     const bool ok = id >= 0 && id < p.V && pos >= 0 && pos < p.max_pos &&
                     kv_phys_page(p, b, pos / p.page_size) >= 0;
     if (!ok) {
@@ -1841,6 +1907,13 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     switch (S.t.type) {
       case T_END: break;
       case T_EMBED: embed_task(p, S, ctid); break;
+      case T_KVAPP:
+        switch (p.d >> 5) {
+          case 1: tok = kv_append_task<32>(p, ctl, S, st, ctid); break;
+          case 2: tok = kv_append_task<64>(p, ctl, S, st, ctid); break;
+          default: tok = kv_append_task<128>(p, ctl, S, st, ctid); break;
+        }
+        break;
       case T_ATTN:
         if (S.b >= 0) {
           switch (p.d >> 5) {
@@ -2013,9 +2086,11 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
       }
       break;
     }
-    case T_ATTN: {
+    case T_ATTN:
+    case T_KVAPP: {
       // the compute warps wrote the chunk partial (and, for the chunk that
-      // completed its (sequence, KV head), the merged o) before handing over
+      // completed its (sequence, KV head), the merged o), or the K/V rows,
+      // before handing over
       if (lane == 0) signal(p, t.out_event);
       break;
     }
@@ -2052,7 +2127,7 @@ __device__ bool storer_epilogue(const Params &p, Ctl *ctl, const Slot &S, const 
         if (lane < B) {
           const unsigned long long k = ld_relaxed_u64(p.argmax + lane);
           p.out_ids[lane] = static_cast<int32_t>(~static_cast<uint32_t>(k & 0xffffffffull));
-          if (p.out_pos != nullptr) p.out_pos[lane] = p.pos[lane] + 1;
+          if (p.out_pos != nullptr) p.out_pos[lane] = row_pos(p, lane) + 1;
           p.argmax[lane] = 0ull;
         }
         __syncwarp();

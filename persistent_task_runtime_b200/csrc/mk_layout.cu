@@ -69,11 +69,11 @@ void solidify_schedule(const Params &p, const std::vector<Task> &T, int grid,
     uint32_t sig = t.out_event;
     if (t.type == T_ATTN) {
       const int g = static_cast<int>(t.aux) / p.attn_spg;
-      ready = ev_ready[static_cast<size_t>(ev_attn_ready(p, t.layer, g))];
+      ready = ev_ready[static_cast<size_t>(ev_attn_input(p, t.layer, g))];
     } else if (t.dep_event != kNoEvent) {
       ready = ev_ready[t.dep_event];
     }
-    if (t.type != T_ATTN && t.type != T_EMBED) {
+    if (t.type != T_ATTN && t.type != T_EMBED && t.type != T_KVAPP) {
       int K = t.type == T_OPROJ ? p.Hq * p.d : (t.type == T_DOWN ? p.F : p.H);
       const int kt = p.tc ? p.tc_kt[t.type] : (t.type == T_DOWN ? p.kchunk[K_FFN]
                                                 : (t.type == T_OPROJ ? p.kchunk[K_ATT] : 0));
@@ -418,7 +418,9 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   p.ev_embed = 0;
   p.ev_layer0 = 1;
   // attn_ready[Hkv], o_ready[O parts], oproj, gateup[down parts], down
-  p.ev_per_layer = Hkv + n_o_parts + 2 + n_ksplit;
+  // (prefill plans: then kv_ready[Hkv])
+  p.kv_tasks = o.prefill ? 1 : 0;
+  p.ev_per_layer = Hkv + n_o_parts + 2 + n_ksplit + (o.prefill ? Hkv : 0);
   const int n_events = 1 + L * p.ev_per_layer;
 
   // ---- task graph -----------------------------------------------------------------------
@@ -479,6 +481,19 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
       }
     out.ops.push_back({b0, static_cast<int>(T.size())});
     b0 = static_cast<int>(T.size());
+    if (o.prefill)
+      // one task per KV group appends every row's K/V before the group's
+      // attention reads the cache
+      for (int kvg = 0; kvg < Hkv; ++kvg) {
+        Task t{};
+        t.type = T_KVAPP;
+        t.layer = static_cast<uint16_t>(l);
+        t.dep_event = static_cast<uint32_t>(ev_attn_ready(p, l, kvg));
+        t.dep_count = static_cast<uint32_t>(p.qkv_tasks_per_group);
+        t.out_event = static_cast<uint32_t>(ev_kv_ready(p, l, kvg));
+        t.aux = static_cast<uint32_t>(kvg);
+        T.push_back(t);
+      }
     for (int s = 0; s < p.attn_slots; ++s) {
       Task t{};
       t.type = T_ATTN;
@@ -533,6 +548,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   }
   {
     const int b0 = static_cast<int>(T.size());
+    out.first_lm_task = b0;
     for (int r0 = 0; r0 < V; r0 += R_lm) {
       const int nr = std::min(R_lm, V - r0);
       Task t = gemv(T_LMHEAD, L - 1, r0, nr, mtiles(nr), ev_down(p, L - 1), n_down, kNoEvent);
@@ -644,6 +660,7 @@ void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vect
         t.gain = bf(lw.attn_norm);
         break;
       case T_ATTN:
+      case T_KVAPP:
         t.w0 = bf(lw.q_norm);
         t.w1 = bf(lw.k_norm);
         break;

@@ -38,7 +38,7 @@ ERROR_NAMES = {MK_OK: "MK_OK", MK_ERR_INVALID_ARG: "MK_ERR_INVALID_ARG",
 EXPORTS = ["mk_plan_create", "mk_plan_create_ex", "mk_decode_step", "mk_decode_step_ex",
            "mk_decode_step_host", "mk_plan_status", "mk_plan_error_info", "mk_plan_reset",
            "mk_plan_info", "mk_last_error", "mk_plan_destroy", "mk_decode_step_noalloc",
-           "mk_plan_describe", "mk_plan_describe_schedule"]
+           "mk_plan_describe", "mk_plan_describe_schedule", "mk_prefill_chunk"]
 
 #: bytes of the library's static scratch array used by mk_decode_step_noalloc
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -71,7 +71,8 @@ class mk_plan_options(C.Structure):
     _fields_ = [("max_batch", C.c_int), ("kv_page_size", C.c_int), ("num_ctas", C.c_int),
                 ("wait_limit_ns", C.c_int64), ("rows_per_task", C.c_int * 5),
                 ("debug_unsatisfiable_dep", C.c_int), ("max_page_cols", C.c_int),
-                ("o_split", C.c_int), ("gemv_path", C.c_int), ("schedule", C.c_int)]
+                ("o_split", C.c_int), ("gemv_path", C.c_int), ("schedule", C.c_int),
+                ("prefill", C.c_int)]
 
 
 class mk_step_args(C.Structure):
@@ -79,6 +80,12 @@ class mk_step_args(C.Structure):
                 ("batch", C.c_int), ("d_out_ids", C.c_void_p), ("d_out_logits", C.c_void_p),
                 ("d_out_pos", C.c_void_p), ("d_hidden", C.c_void_p), ("mode", C.c_int),
                 ("d_trace", C.c_void_p)]
+
+
+class mk_prefill_args(C.Structure):
+    _fields_ = [("d_ids", C.c_void_p), ("n_tokens", C.c_int), ("pos0", C.c_int), ("seq", C.c_int),
+                ("kv", C.POINTER(mk_kv_cache)), ("d_out_ids", C.c_void_p),
+                ("d_out_logits", C.c_void_p), ("d_hidden", C.c_void_p), ("with_lm_head", C.c_int)]
 
 
 class mk_plan_info_t(C.Structure):
@@ -90,7 +97,8 @@ class mk_plan_info_t(C.Structure):
                 ("events_per_layer", C.c_int), ("attn_slots_per_group", C.c_int),
                 ("qkv_tasks_per_group", C.c_int), ("ffn_parts", C.c_int),
                 ("ffn_part_cols", C.c_int), ("o_parts", C.c_int), ("o_part_cols", C.c_int),
-                ("gemv_path", C.c_int), ("schedule", C.c_int), ("qkv_parts", C.c_int),
+                ("gemv_path", C.c_int), ("schedule", C.c_int), ("prefill", C.c_int),
+                ("qkv_parts", C.c_int),
                 ("gateup_parts", C.c_int)]
 
 
@@ -124,6 +132,8 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
                                               C.POINTER(mk_plan_options), C.c_int, C.c_int, P,
                                               C.c_int64]
     lib.mk_plan_describe_schedule.restype = C.c_int
+    lib.mk_prefill_chunk.argtypes = [P, C.POINTER(mk_prefill_args), P]
+    lib.mk_prefill_chunk.restype = C.c_int
     lib.mk_last_error.restype = C.c_char_p
     lib.mk_last_error.argtypes = []
     lib.mk_plan_destroy.argtypes = [P]
@@ -201,7 +211,7 @@ def _config(cfg: Dict, max_seq_len: int) -> mk_model_config:
 def describe(cfg: Dict, max_batch: int = 1, page_size: int = 16, max_seq_len: int = 4096,
              num_sms: int = 148, smem_optin: int = 232448, rows_per_task=(0, 0, 0, 0, 0),
              max_page_cols: int = 0, o_split: bool = False, gemv_path: int = 0,
-             schedule: int = 0):
+             schedule: int = 0, prefill: bool = False):
     """The plan mk_plan_create_ex would build, without a GPU: (info, task records).
 
     The task records are a numpy structured array (TASK_RECORD_DTYPE)."""
@@ -209,7 +219,8 @@ def describe(cfg: Dict, max_batch: int = 1, page_size: int = 16, max_seq_len: in
     lib = load_library()
     c = _config(cfg, max_seq_len)
     opts = mk_plan_options(max_batch, page_size, 0, 0, (C.c_int * 5)(*rows_per_task), 0,
-                           max_page_cols, 1 if o_split else 0, gemv_path, schedule)
+                           max_page_cols, 1 if o_split else 0, gemv_path, schedule,
+                           1 if prefill else 0)
     info = mk_plan_info_t()
     _check(lib.mk_plan_describe(C.byref(c), C.byref(opts), num_sms, smem_optin, C.byref(info),
                                 None, 0))
@@ -242,7 +253,7 @@ class Plan:
                  max_seq_len: int = 4096, num_ctas: int = 0, wait_limit_ns: int = 0,
                  rows_per_task: Sequence[int] = (0, 0, 0, 0, 0), debug_unsatisfiable_dep=False,
                  max_page_cols: int = 0, o_split: bool = False, gemv_path: int = 0,
-                 schedule: int = 0):
+                 schedule: int = 0, prefill: bool = False):
         lib = load_library()
         self.cfg = dict(cfg)
         self.max_batch = max_batch
@@ -259,7 +270,8 @@ class Plan:
                              _ptr(weights["lm_head"]))
         opts = mk_plan_options(max_batch, page_size, num_ctas, wait_limit_ns,
                                (C.c_int * 5)(*rows_per_task), 1 if debug_unsatisfiable_dep else 0,
-                               max_page_cols, 1 if o_split else 0, gemv_path, schedule)
+                               max_page_cols, 1 if o_split else 0, gemv_path, schedule,
+                               1 if prefill else 0)
         h = C.c_void_p()
         _check(lib.mk_plan_create_ex(C.byref(self._c), C.byref(self._w), C.byref(opts),
                                      C.byref(h)))
@@ -281,6 +293,39 @@ class Plan:
         a = mk_step_args(_ptr(ids), _ptr(pos), C.pointer(kv.struct), b, _ptr(out_ids),
                          _ptr(out_logits), _ptr(out_pos), _ptr(hidden), mode, _ptr(trace))
         _check(self._lib.mk_decode_step_ex(self._h, C.byref(a), _stream_handle(stream)))
+
+    def prefill_chunk(self, ids: torch.Tensor, pos0: int, seq: int, kv: KVCacheView,
+                      out_ids: Optional[torch.Tensor] = None,
+                      out_logits: Optional[torch.Tensor] = None,
+                      hidden: Optional[torch.Tensor] = None, with_lm_head: bool = True,
+                      stream=None) -> None:
+        """mk_prefill_chunk: tokens ids[0..n) of sequence `seq` at positions
+        pos0.. as one launch (asynchronous; see status())."""
+        a = mk_prefill_args(_ptr(ids), ids.shape[0], pos0, seq, C.pointer(kv.struct),
+                            _ptr(out_ids), _ptr(out_logits), _ptr(hidden),
+                            1 if with_lm_head else 0)
+        _check(self._lib.mk_prefill_chunk(self._h, C.byref(a), _stream_handle(stream)))
+
+    def prefill(self, prompt: torch.Tensor, seq: int, kv: KVCacheView, out_ids: torch.Tensor,
+                chunk: Optional[int] = None, stream=None) -> None:
+        """A whole prompt (device int32 ids) of sequence `seq` from position 0,
+        in chunks of `chunk` tokens (default: max_batch); the LM head runs on
+        the last chunk only.  out_ids[0] receives the first generated token."""
+        n = prompt.shape[0]
+        T = chunk or self.max_batch
+        for p0 in range(0, n, T):
+            m = min(T, n - p0)
+            last = p0 + m == n
+            self.prefill_chunk(prompt[p0:p0 + m], p0, seq, kv,
+                               out_ids=self._chunk_out(m) if last else None,
+                               with_lm_head=last, stream=stream)
+            if last:
+                out_ids.copy_(self._chunk_ids[m - 1:m])
+
+    def _chunk_out(self, m):
+        if getattr(self, "_chunk_ids", None) is None:
+            self._chunk_ids = torch.zeros(self.max_batch, dtype=torch.int32, device="cuda")
+        return self._chunk_ids[:m]
 
     def step_plain(self, ids, pos, kv: KVCacheView, batch, out_ids, out_logits=None,
                    stream=None) -> None:

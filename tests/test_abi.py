@@ -50,6 +50,7 @@ STRUCTS = {
     "mk_plan_options": mk.mk_plan_options,
     "mk_step_args": mk.mk_step_args,
     "mk_plan_info_t": mk.mk_plan_info_t,
+    "mk_prefill_args": mk.mk_prefill_args,
 }
 
 

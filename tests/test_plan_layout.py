@@ -37,7 +37,7 @@ SHAPES = {
                 vocab=512, rms_eps=1e-6, rope_theta=1e6, qk_norm=True),
 }
 SMEM = 232448
-T_EMBED, T_QKV, T_ATTN, T_OPROJ, T_GATEUP, T_DOWN, T_LMHEAD = 1, 2, 3, 4, 5, 6, 7
+T_EMBED, T_QKV, T_ATTN, T_OPROJ, T_GATEUP, T_DOWN, T_LMHEAD, T_KVAPP = 1, 2, 3, 4, 5, 6, 7, 8
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -56,8 +56,12 @@ def check_plan(cfg, info, t, max_batch):
     epl, spg = info["events_per_layer"], info["attn_slots_per_group"]
     o_parts, ffn_parts = info["o_parts"], info["ffn_parts"]
     n_events = info["n_events"]
+    kvt = info["prefill"] == 1            # K/V appended by tasks of their own
     assert n_events == 1 + L * epl
-    assert epl == Hkv + o_parts + 2 + ffn_parts
+    assert epl == Hkv + o_parts + 2 + ffn_parts + (Hkv if kvt else 0)
+
+    def ev_kv_ready(l, g):
+        return 1 + l * epl + Hkv + o_parts + 2 + ffn_parts + g
 
     def ev_attn_ready(l, g):
         return 1 + l * epl + g
@@ -111,8 +115,10 @@ def check_plan(cfg, info, t, max_batch):
         ty = int(r["type"])
         if ty == T_ATTN:
             g = int(r["aux"]) // spg
-            ev = ev_attn_ready(int(r["layer"]), g)
-            need = info["qkv_tasks_per_group"]
+            if kvt:
+                ev, need = ev_kv_ready(int(r["layer"]), g), 1
+            else:
+                ev, need = ev_attn_ready(int(r["layer"]), g), info["qkv_tasks_per_group"]
         else:
             ev, need = int(r["dep_event"]), int(r["dep_count"])
             if ev == mk.NO_EVENT:
@@ -190,6 +196,17 @@ def check_plan(cfg, info, t, max_batch):
     # ---- attention slots: one block per KV group ------------------------------------------
     att = t[t["type"] == T_ATTN]
     assert len(att) == L * Hkv * spg == L * info["attn_slots"]
+    kva = t[t["type"] == T_KVAPP]
+    if kvt:
+        # one K/V task per (layer, KV group), waiting for the group's QKV tiles
+        assert len(kva) == L * Hkv
+        for r in kva:
+            l, g = int(r["layer"]), int(r["aux"])
+            assert int(r["dep_event"]) == ev_attn_ready(l, g)
+            assert int(r["dep_count"]) == info["qkv_tasks_per_group"]
+            assert int(r["out_event"]) == ev_kv_ready(l, g)
+    else:
+        assert len(kva) == 0
 
 
 CASES = [(name, b, split) for name in SHAPES for b in (1, 3, 4, 8, 16) for split in (False, True)]
@@ -200,6 +217,19 @@ def test_task_graph_invariants(name, batch, o_split):
     cfg = SHAPES[name]
     info, t = mk.describe(cfg, max_batch=batch, max_seq_len=2048 if name == "8b" else 600,
                           o_split=o_split)
+    check_plan(cfg, info, t, batch)
+
+
+PREFILL_CASES = [(name, b, path) for name in ("tiny", "3groups", "8b", "ragged")
+                 for b in (1, 4, 16) for path in (0, 1)]
+
+
+@pytest.mark.parametrize("name,batch,path", PREFILL_CASES)
+def test_prefill_plan_graph_invariants(name, batch, path):
+    cfg = SHAPES[name]
+    info, t = mk.describe(cfg, max_batch=batch, max_seq_len=2048 if name == "8b" else 600,
+                          prefill=True, gemv_path=path)
+    assert info["prefill"] == 1
     check_plan(cfg, info, t, batch)
 
 

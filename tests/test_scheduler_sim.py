@@ -45,8 +45,13 @@ def compile_tasks(cfg, info, t):
         ty, layer = int(r["type"]), int(r["layer"])
         wait, need = int(r["dep_event"]), int(r["dep_count"])
         if ty == T_ATTN:
-            wait = 1 + layer * epl + int(r["aux"]) // spg
-            need = info["qkv_tasks_per_group"]
+            g = int(r["aux"]) // spg
+            if info["prefill"]:
+                wait = 1 + layer * epl + Hkv + info["o_parts"] + 2 + info["ffn_parts"] + g
+                need = 1
+            else:
+                wait = 1 + layer * epl + g
+                need = info["qkv_tasks_per_group"]
         elif wait == mk.NO_EVENT:
             wait, need = -1, 0
         if ty == T_QKV:
@@ -202,3 +207,16 @@ def test_solidified_schedule_no_deadlock(name, batch, workers, path):
     # the dynamic plan describes no schedule
     assert (mk.describe_schedule(cfg, info["n_tasks"], max_batch=batch, max_seq_len=600,
                                  gemv_path=path, num_sms=workers, schedule=0) == -1).all()
+
+
+@pytest.mark.parametrize("name,batch,workers,path", [("tiny", 16, 9, 0), ("3groups", 16, 148, 2),
+                                                     ("8b", 16, 148, 0)])
+def test_prefill_plan_no_deadlock(name, batch, workers, path):
+    cfg = SHAPES[name]
+    info, t = mk.describe(cfg, max_batch=batch, max_seq_len=600, gemv_path=path, prefill=True)
+    tasks = compile_tasks(cfg, info, t)
+    for seed in (1, 2):
+        ctr = simulate(tasks, info["n_events"], workers, seed)
+        for ty, wait, need, *_ in tasks:
+            if wait >= 0:
+                assert ctr[wait] == need
