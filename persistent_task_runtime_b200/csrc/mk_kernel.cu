@@ -560,6 +560,7 @@ struct Look {
 constexpr int kLook = kLookBytes / static_cast<int>(sizeof(Look));
 static_assert(sizeof(Look) == 80 && kLook >= 2, "lookahead entry size");
 
+template <bool TC>
 __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol = l2_evict_first_policy();
@@ -710,7 +711,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     }
 
     // ---- stream the task's operands into the page ring ----
-    if (is_gemv(t.type) && p.tc) {
+    if (TC && is_gemv(t.type)) {
       // tensor-core path: per activation chunk, per 128-row tile, pages of
       // tc_kc columns, each one TMA box per 64-column swizzle atom
       const TcGeo g = tc_geo(p, t);
@@ -740,7 +741,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
           }
         }
       }
-    } else if (is_gemv(t.type)) {
+    } else if (!TC && is_gemv(t.type)) {
       const Geo geo = gemv_geo(p, t, B);
       const int pitch = row_pitch_bytes(geo.kp);
       for (int xc0 = geo.k0; xc0 < geo.k0 + geo.Kt && ok; xc0 += geo.kx) {
@@ -1258,36 +1259,109 @@ __device__ __forceinline__ void split8(const float4 &x0, const float4 &x1, bool 
 // (160 threads, sid 0..159) in the K-major 128-byte-swizzled layout: per
 // 64-column atom, rows of 128 bytes (hi rows 0..bpad-1, lo rows
 // bpad..2*bpad-1), the 16-byte chunk c of a row stored at chunk c XOR
-// (row address bits 7..9).  Sequences >= B are zeros.
+// (row address bits 7..9).  Sequences >= B are zeros.  Each thread first
+// issues the global loads of all of its 8-column blocks (up to kStageUnits),
+// then converts and stores them: one L2 round trip per batch.
+constexpr int kStagers = kComputeThreads - 32;
+constexpr int kStageUnits = 7;   // 7 x 160 >= 1024, the blocks of a full 32 KB chunk
 __device__ void stage_chunk_tc(const Params &p, const float *src, int stride,
                                const __nv_bfloat16 *gain, int xc0, int xlen, uint8_t *xbuf, int B,
                                int sid) {
   const int bpad = p.tc_bpad;
   const int nblk = xlen / 8;
+  const int units = bpad * nblk;
   const uint32_t xs = smem_u32(xbuf);
   const uint32_t atom_bytes = static_cast<uint32_t>(p.tc_n) * 128u;
-  for (int u = sid; u < bpad * nblk; u += kComputeThreads - 32) {
-    const int b = u / nblk, j = u - b * nblk;
-    uint4 hw = make_uint4(0, 0, 0, 0), lw = make_uint4(0, 0, 0, 0);
-    if (b < B) {
-      const float4 *sp = reinterpret_cast<const float4 *>(src + static_cast<size_t>(b) * stride + xc0 + j * 8);
-      const float4 x0 = __ldcg(sp), x1 = __ldcg(sp + 1);
-      const uint4 gw = gain != nullptr ? __ldg(reinterpret_cast<const uint4 *>(gain + xc0 + j * 8))
-                                       : make_uint4(0, 0, 0, 0);
-      split8(x0, x1, gain != nullptr, gw, hw, lw);
+  for (int u0 = sid; u0 < units; u0 += kStageUnits * kStagers) {
+    float4 x0[kStageUnits], x1[kStageUnits];
+    uint4 gw[kStageUnits];
+#pragma unroll
+    for (int k = 0; k < kStageUnits; ++k) {
+      const int u = u0 + k * kStagers;
+      const int b = u / nblk, j = u - b * nblk;
+      x0[k] = x1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      gw[k] = make_uint4(0, 0, 0, 0);
+      if (u < units && b < B) {
+        const float4 *sp =
+            reinterpret_cast<const float4 *>(src + static_cast<size_t>(b) * stride + xc0 + j * 8);
+        x0[k] = __ldcg(sp);
+        x1[k] = __ldcg(sp + 1);
+        if (gain != nullptr) gw[k] = __ldg(reinterpret_cast<const uint4 *>(gain + xc0 + j * 8));
+      }
     }
-    const uint32_t atom = xs + static_cast<uint32_t>(j >> 3) * atom_bytes;
-    const uint32_t ch = static_cast<uint32_t>(j & 7);
-    const uint32_t rh = atom + static_cast<uint32_t>(b) * 128u;
-    const uint32_t rl = atom + static_cast<uint32_t>(bpad + b) * 128u;
-    sts128(rh + ((ch ^ ((rh >> 7) & 7u)) << 4), hw);
-    sts128(rl + ((ch ^ ((rl >> 7) & 7u)) << 4), lw);
+#pragma unroll
+    for (int k = 0; k < kStageUnits; ++k) {
+      const int u = u0 + k * kStagers;
+      if (u >= units) break;
+      const int b = u / nblk, j = u - b * nblk;
+      uint4 hw, lw;
+      split8(x0[k], x1[k], gain != nullptr, gw[k], hw, lw);
+      const uint32_t atom = xs + static_cast<uint32_t>(j >> 3) * atom_bytes;
+      const uint32_t ch = static_cast<uint32_t>(j & 7);
+      const uint32_t rh = atom + static_cast<uint32_t>(b) * 128u;
+      const uint32_t rl = atom + static_cast<uint32_t>(bpad + b) * 128u;
+      sts128(rh + ((ch ^ ((rh >> 7) & 7u)) << 4), hw);
+      sts128(rl + ((ch ^ ((rl >> 7) & 7u)) << 4), lw);
+    }
   }
+}
+
+// Tensor-core path, normed inputs: the sums of h^2 per 128 rows that the
+// producers of h wrote -> each sequence's RMSNorm scale in ctl->rs.  One
+// warp; every load is issued before the first sum (fixed order: per lane
+// over its tiles, then a warp tree).
+template <int BP>
+__device__ void tc_norm_scales(const Params &p, Ctl *ctl, const float *ssq, int B, int lane) {
+  const int n = (p.H + kTcRows - 1) / kTcRows;
+  float v[BP];
+#pragma unroll
+  for (int b = 0; b < BP; ++b) v[b] = 0.f;
+  for (int i = lane; i < n; i += 32)
+#pragma unroll
+    for (int b = 0; b < BP; ++b)
+      if (b < B) v[b] += __ldcg(ssq + static_cast<size_t>(i) * p.max_batch + b);
+#pragma unroll
+  for (int b = 0; b < BP; ++b) {
+    const float s = warp_sum(v[b]);
+    if (lane == 0 && b < B) ctl->rs[b] = 1.0f / sqrtf(s / static_cast<float>(p.H) + p.eps);
+  }
+}
+
+// Split-K partials and tile counters of a tensor-core task (QKV and down
+// share one area; O and gate/up have their own).
+struct TcSplit {
+  float *kp;
+  int rstride;          // floats per sequence row of the partial area
+  size_t pstride;       // floats per part
+  uint32_t *ctr;
+  int grow0;            // the task's first row in its operator's row space
+};
+__device__ __forceinline__ TcSplit tc_split(const Params &p, const Task &t) {
+  TcSplit s;
+  const int qbase = t.aux == 0 ? 0 : (t.aux == 1 ? p.Hq * p.d : (p.Hq + p.Hkv) * p.d);
+  s.grow0 = static_cast<int>(t.row0) + (t.type == T_QKV ? qbase : 0);
+  s.kp = p.kpart;
+  s.rstride = p.H;
+  s.ctr = p.tile_ctr;
+  if (t.type == T_QKV) {
+    s.rstride = p.NQKV;
+  } else if (t.type == T_OPROJ) {
+    s.kp = p.kpart_o;
+    s.ctr = p.tile_ctr_o;
+  } else if (t.type == T_GATEUP) {
+    s.kp = p.kpart2;
+    s.rstride = 2 * p.F;
+    s.ctr = p.tile_ctr2;
+  }
+  s.pstride = static_cast<size_t>(p.max_batch) * s.rstride;
+  s.ctr += s.grow0 / 16;
+  return s;
 }
 
 template <int NT>   // accumulator columns / 16: 1 (N = 16, batch <= 8) or 2 (N = 32)
 __device__ bool gemv_task_tc(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
                              ComputeState &st, float *out, int ctid) {
+  constexpr int BP = 8 * NT;   // tc_bpad of a plan with this NT
   const Task &t = S.t;
   const int B = p.batch;
   const int warp = ctid >> 5, lane = ctid & 31;
@@ -1306,19 +1380,6 @@ __device__ bool gemv_task_tc(const Params &p, Ctl *ctl, uint8_t *smem, const Slo
   st.sat_ev = t.dep_event;
   st.sat_cnt = t.dep_count;
   if (ctid == 0) trace_mark(p, S.idx, 4);
-
-  // RMSNorm scale of each sequence from the per-16-row sums of h^2 that the
-  // producers of h wrote (fixed order: strided per lane, then a warp tree)
-  if (normed) {
-    const float *ssq = t.type == T_GATEUP ? p.ssq_mlp : p.ssq_attn;
-    const int n16 = p.H / 16;
-    for (int b = warp; b < B; b += kComputeWarps) {
-      float s = 0.f;
-      for (int i = lane; i < n16; i += 32) s += __ldcg(ssq + static_cast<size_t>(i) * p.max_batch + b);
-      s = warp_sum(s);
-      if (lane == 0) ctl->rs[b] = 1.0f / sqrtf(s / static_cast<float>(p.H) + p.eps);
-    }
-  }
 
   const int nchunks = (g.Kt + p.tc_kx - 1) / p.tc_kx;
   uint8_t *xbase = smem + p.off_x;
@@ -1348,71 +1409,63 @@ __device__ bool gemv_task_tc(const Params &p, Ctl *ctl, uint8_t *smem, const Slo
       compute_stage_bar();
       if (ctid == 32) mbar_arrive(&ctl->x_full[buf]);
     }
-  } else if (ctid == 0) {
-    // ---- MMA issuer ----
-    const uint32_t idesc = mma_idesc_bf16(kTcRows, p.tc_n);
-    const uint32_t tmem = ctl->tmem;
-    const uint32_t pages = smem_u32(smem + p.off_pages);
-    const uint32_t xs0 = smem_u32(xbase);
-    const uint32_t xatom = static_cast<uint32_t>(p.tc_n) * 128u;
-    bool bad = false;
-    bool started0 = false, started1 = false;   // tile 0 / 1 has its first MMA
-    for (int c = 0; c < nchunks; ++c) {
-      const uint32_t u = st.xuse + c;
-      const int buf = static_cast<int>(u & 1u);
-      const int xc0 = g.k0 + c * p.tc_kx;
-      const int xlen = min(p.tc_kx, g.k0 + g.Kt - xc0);
-      if (!bad && !wait_mbar(p, ctl, &ctl->x_full[buf], (u >> 1) & 1u, 0xfffa0000u, 2)) bad = true;
-      tc_fence_after();
-      const uint32_t xb = xs0 + static_cast<uint32_t>(buf) * kTcXBytes;
-      for (int m = 0; m < t.n_m; ++m) {
-        for (int c0 = xc0; c0 < xc0 + xlen; c0 += p.tc_kc) {
-          const int nc = min(p.tc_kc, xc0 + xlen - c0);
-          if (!bad && !wait_mbar(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff30000u, 2)) bad = true;
-          if (!bad) {
-            tc_fence_after();
-            const uint32_t pg = pages + static_cast<uint32_t>(st.pi) * p.page_bytes;
-            const uint32_t xa0 = xb + static_cast<uint32_t>((c0 - xc0) / kTcAtomCols) * xatom;
-            for (int a = 0; a < nc / kTcAtomCols; ++a)
+  } else {
+    // ---- warp 1: the RMSNorm scales, then lane 0 issues the MMAs ----
+    if (normed) tc_norm_scales<BP>(p, ctl, t.type == T_GATEUP ? p.ssq_mlp : p.ssq_attn, B, lane);
+    if (ctid == 0) {
+      const uint32_t idesc = mma_idesc_bf16(kTcRows, p.tc_n);
+      const uint32_t tmem = ctl->tmem;
+      const uint32_t pages = smem_u32(smem + p.off_pages);
+      const uint32_t xs0 = smem_u32(xbase);
+      const uint32_t xatom = static_cast<uint32_t>(p.tc_n) * 128u;
+      bool bad = false;
+      bool started0 = false, started1 = false;   // tile 0 / 1 has its first MMA
+      for (int c = 0; c < nchunks; ++c) {
+        const uint32_t u = st.xuse + c;
+        const int buf = static_cast<int>(u & 1u);
+        const int xc0 = g.k0 + c * p.tc_kx;
+        const int xlen = min(p.tc_kx, g.k0 + g.Kt - xc0);
+        if (!bad && !wait_mbar(p, ctl, &ctl->x_full[buf], (u >> 1) & 1u, 0xfffa0000u, 2)) bad = true;
+        tc_fence_after();
+        const uint32_t xb = xs0 + static_cast<uint32_t>(buf) * kTcXBytes;
+        for (int m = 0; m < t.n_m; ++m) {
+          for (int c0 = xc0; c0 < xc0 + xlen; c0 += p.tc_kc) {
+            const int nc = min(p.tc_kc, xc0 + xlen - c0);
+            if (!bad && !wait_mbar(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff30000u, 2)) bad = true;
+            if (!bad) {
+              tc_fence_after();
+              const uint32_t pg = pages + static_cast<uint32_t>(st.pi) * p.page_bytes;
+              const uint32_t xa0 = xb + static_cast<uint32_t>((c0 - xc0) / kTcAtomCols) * xatom;
+              for (int a = 0; a < nc / kTcAtomCols; ++a)
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint64_t ad = sw128_desc(pg + a * kTcAtomBytes + j * 32);
-                const uint64_t bd = sw128_desc(xa0 + a * xatom + j * 32);
-                tc_mma(tmem + m * p.tc_n, ad, bd, idesc, m == 0 ? started0 : started1);
-                if (m == 0) started0 = true; else started1 = true;
-              }
-            tc_commit(&ctl->empty[st.pi]);   // the page is free once these MMAs complete
-          }
-          if (++st.pi == p.n_pages) {
-            st.pi = 0;
-            st.pg_par ^= 1u;
+                for (int j = 0; j < 4; ++j) {
+                  const uint64_t ad = sw128_desc(pg + a * kTcAtomBytes + j * 32);
+                  const uint64_t bd = sw128_desc(xa0 + a * xatom + j * 32);
+                  tc_mma(tmem + m * p.tc_n, ad, bd, idesc, m == 0 ? started0 : started1);
+                  if (m == 0) started0 = true; else started1 = true;
+                }
+              tc_commit(&ctl->empty[st.pi]);   // the page is free once these MMAs complete
+            }
+            if (++st.pi == p.n_pages) {
+              st.pi = 0;
+              st.pg_par ^= 1u;
+            }
           }
         }
+        tc_commit(&ctl->x_free[buf]);
       }
-      tc_commit(&ctl->x_free[buf]);
-    }
-    tc_commit(&ctl->acc_bar);
-    // wait for the accumulators (also after a failed wait: no MMA may still
-    // be running when the task returns)
-    if (!wait_mbar(p, ctl, &ctl->acc_bar, st.accuse & 1u, 0xfffb0000u, 4)) bad = true;
-    if (bad) {
-      ctl->cbad = 1;
-      ctl->cta_abort = 1;
+      tc_commit(&ctl->acc_bar);
+      // wait for the accumulators (also after a failed wait: no MMA may still
+      // be running when the task returns)
+      if (!wait_mbar(p, ctl, &ctl->acc_bar, st.accuse & 1u, 0xfffb0000u, 4)) bad = true;
+      if (bad) {
+        ctl->cbad = 1;
+        ctl->cta_abort = 1;
+      }
     }
   }
-  if (ctid < 32 && ctid != 0) {
-    // the rest of the MMA warp: keep the page-ring position in step with thread 0
-    for (int c = 0; c < nchunks; ++c) {
-      const int xc0 = g.k0 + c * p.tc_kx;
-      const int xlen = min(p.tc_kx, g.k0 + g.Kt - xc0);
-      const int np = t.n_m * ((xlen + p.tc_kc - 1) / p.tc_kc);
-      for (int k = 0; k < np; ++k)
-        if (++st.pi == p.n_pages) {
-          st.pi = 0;
-          st.pg_par ^= 1u;
-        }
-    }
-  } else if (ctid >= 32) {
+  if (ctid != 0) {
+    // everyone but the MMA issuer: keep the page-ring position in step with it
     for (int c = 0; c < nchunks; ++c) {
       const int xc0 = g.k0 + c * p.tc_kx;
       const int xlen = min(p.tc_kx, g.k0 + g.Kt - xc0);
@@ -1431,36 +1484,153 @@ __device__ bool gemv_task_tc(const Params &p, Ctl *ctl, uint8_t *smem, const Slo
   if (ctl->cbad != 0) return false;
   if (ctid == 0) trace_mark(p, S.idx, 5);
   tc_fence_after();
+  ++st.accuse;
 
-  // ---- epilogue: accumulators -> the output buffer ----
-  if (ctid < 128) {
-    const int q = (warp + 1) & 3;            // CTA warp warp+1 reads lanes 32q..32q+31
-    const int row = q * 32 + lane;
-    constexpr int BP = 8 * NT;               // tc_bpad of a plan with this NT
-    for (int m = 0; m < t.n_m; ++m) {
+  // ---- epilogue: warps 1-4 read tensor-memory lane quarters 1, 2, 3, 0 ----
+  // thread (warp, lane) holds row 32 q + lane of the tile(s): the sum of the
+  // hi and lo columns of each sequence, times the RMSNorm scale
+  const bool epi = ctid < 128;
+  const int q = (warp + 1) & 3;
+  const int row = q * 32 + lane;
+  const bool vrow = epi && row < static_cast<int>(t.nrows);
+  float acc[2][BP];
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int b = 0; b < BP; ++b) acc[m][b] = 0.f;
+  if (epi) {
+    for (int m = 0; m < t.n_m && m < 2; ++m) {
       const uint32_t ta = ctl->tmem + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(m * p.tc_n);
       float v[NT][16];
       tmem_ld16(ta, v[0]);
       if (NT > 1) tmem_ld16(ta + 16, v[NT - 1]);
-      if (row < static_cast<int>(t.nrows)) {
 #pragma unroll
-        for (int b = 0; b < 8 * NT; ++b) {
-          if (b < B) {
-            // hi column b, lo column BP + b
-            const float hi = v[b / 16][b % 16];
-            const float lo = v[(BP + b) / 16][(BP + b) % 16];
-            float r = hi + lo;
-            if (normed) r *= ctl->rs[b];
-            out[b * p.out_stride + m * kTcRows + row] = r;
-          }
-        }
+      for (int b = 0; b < BP; ++b) {
+        float r = v[b / 16][b % 16] + v[(BP + b) / 16][(BP + b) % 16];
+        if (normed && b < B) r *= ctl->rs[b];
+        if (m == 0) acc[0][b] = r; else acc[1][b] = r;
       }
     }
   }
   tc_fence_before();
+
+  if (t.type == T_LMHEAD) {
+    // logits and argmax: the storer, from the output buffer
+    if (vrow)
+#pragma unroll
+      for (int b = 0; b < BP; ++b)
+        if (b < B) out[b * p.out_stride + row] = acc[0][b];
+    compute_bar();
+    return true;
+  }
+
+  // ---- split-K: publish this part; the part that completes the tile sums ----
+  const bool split = t.nsplit > 1;
+  TcSplit sp{};
+  if (split) {
+    sp = tc_split(p, t);
+    if (vrow)
+#pragma unroll
+      for (int b = 0; b < BP; ++b)
+        if (b < B) {
+          float *dst = sp.kp + t.ksplit * sp.pstride + static_cast<size_t>(b) * sp.rstride + sp.grow0 + row;
+          __stcg(dst, acc[0][b]);
+          if (t.type == T_GATEUP) __stcg(dst + p.F, acc[1][b]);
+        }
+    compute_bar();
+    bool last = false;
+    if (ctid == 0) last = atom_add_acq_rel(sp.ctr, 1u) + 1u == static_cast<uint32_t>(t.nsplit);
+    if (!st.gs.share(ctl, ctid, last)) return true;   // not the last part: nothing to release
+    if (vrow) {
+      // the parts in a fixed order (0, 1, ...); this part's own from registers
+      float sum[2][BP];
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int b = 0; b < BP; ++b) sum[m][b] = 0.f;
+      for (int k = 0; k < t.nsplit; ++k) {
+        const float *srck = sp.kp + k * sp.pstride + sp.grow0 + row;
+        float v0[BP], v1[BP];
+#pragma unroll
+        for (int b = 0; b < BP; ++b) {
+          v0[b] = v1[b] = 0.f;
+          if (b < B && k != t.ksplit) {
+            v0[b] = __ldcg(srck + static_cast<size_t>(b) * sp.rstride);
+            if (t.type == T_GATEUP) v1[b] = __ldcg(srck + static_cast<size_t>(b) * sp.rstride + p.F);
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < BP; ++b) {
+          sum[0][b] += k == t.ksplit ? acc[0][b] : v0[b];
+          sum[1][b] += k == t.ksplit ? acc[1][b] : v1[b];
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int b = 0; b < BP; ++b) acc[m][b] = sum[m][b];
+    }
+  }
+
+  // ---- the operator's epilogue, one row per thread ----
+  float *red = reinterpret_cast<float *>(out);   // [4 warps][BP] per-warp sums of h^2
+  if (t.type == T_QKV) {
+    // raw q/k/v rows: QK-norm, RoPE and the KV append happen in the attention
+    // (or K/V) tasks of the head's KV group
+    const int qbase = t.aux == 0 ? 0 : (t.aux == 1 ? p.Hq * p.d : (p.Hq + p.Hkv) * p.d);
+    if (vrow)
+#pragma unroll
+      for (int b = 0; b < BP; ++b)
+        if (b < B)
+          __stcg(p.qkv + static_cast<size_t>(b) * p.NQKV + qbase + t.row0 + row, acc[0][b]);
+  } else if (t.type == T_GATEUP) {
+    if (vrow)
+#pragma unroll
+      for (int b = 0; b < BP; ++b)
+        if (b < B) {
+          const float gt = acc[0][b];
+          __stcg(p.u + static_cast<size_t>(b) * p.F + t.row0 + row,
+                 gt / (1.0f + __expf(-gt)) * acc[1][b]);
+        }
+  } else {
+    // O / down: residual add, per-layer dump, sums of h^2 for the next RMSNorm
+    float hv[BP];
+#pragma unroll
+    for (int b = 0; b < BP; ++b)
+      hv[b] = (vrow && b < B) ? __ldcg(p.h + static_cast<size_t>(b) * p.H + t.row0 + row) : 0.f;
+#pragma unroll
+    for (int b = 0; b < BP; ++b) {
+      float v = 0.f;
+      if (vrow && b < B) {
+        v = hv[b] + acc[0][b];
+        __stcg(p.h + static_cast<size_t>(b) * p.H + t.row0 + row, v);
+        if (t.type == T_DOWN && p.hidden_dump != nullptr)
+          p.hidden_dump[(static_cast<size_t>(t.layer) * B + b) * p.H + t.row0 + row] = v;
+      }
+      const float s = warp_sum(v * v);
+      if (epi && lane == 0) red[q * BP + b] = s;
+    }
+    compute_bar();
+    if (ctid < B) {
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) s += red[w * BP + ctid];   // rows 0-31, 32-63, ...
+      float *ssq = t.type == T_OPROJ ? p.ssq_mlp : p.ssq_attn;
+      __stcg(ssq + static_cast<size_t>(t.row0 / kTcRows) * p.max_batch + ctid, s);
+    }
+  }
   compute_bar();
-  ++st.accuse;
+  if (ctid == 0) {
+    if (split) *sp.ctr = 0u;   // rearm for the next layer / step
+    if (t.type == T_QKV) {
+      const int head = static_cast<int>(t.aux2);
+      const int gq = t.aux == 0 ? head / p.G : (t.aux == 1 ? head - p.Hq : head - p.Hq - p.Hkv);
+      red_add_release(p.sync + S_EVENTS + ev_attn_ready(p, t.layer, gq), 1u);
+    } else {
+      red_add_release(p.sync + S_EVENTS + t.out_event, 1u);
+    }
+  }
   return true;
 }
 
@@ -1858,18 +2028,21 @@ __device__ void embed_task(const Params &p, const Slot &S, int ctid) {
     }
   }
   if (p.tc) {
-    // sums of h^2 per 16 rows for the first QKV tasks' RMSNorm (tensor-core path)
-    const int n16 = H / 16;
-    for (int u = ctid; u < B * n16; u += kComputeThreads) {
-      const int b = u / n16, i = u - b * n16;
+    // sums of h^2 per 128 rows for the first QKV tasks' RMSNorm (tensor-core path)
+    const int nt = (H + kTcRows - 1) / kTcRows;
+    for (int u = ctid; u < B * nt; u += kComputeThreads) {
+      const int b = u / nt, i = u - b * nt;
       const int id = p.ids[b];
       if (id < 0 || id >= p.V) continue;   // reported above
-      const uint4 *e = reinterpret_cast<const uint4 *>(p.embed + static_cast<size_t>(id) * H + i * 16);
-      const uint4 w0 = __ldg(e), w1 = __ldg(e + 1);
-      const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const __nv_bfloat16 *e = p.embed + static_cast<size_t>(id) * H + i * kTcRows;
+      const int n = min(kTcRows, H - i * kTcRows);
       float sq = 0.f;
+      for (int k = 0; k < n; k += 8) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(e + k));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int k = 0; k < 8; ++k) sq += bf_lo(ww[k]) * bf_lo(ww[k]) + bf_hi(ww[k]) * bf_hi(ww[k]);
+        for (int j = 0; j < 4; ++j) sq += bf_lo(ww[j]) * bf_lo(ww[j]) + bf_hi(ww[j]) * bf_hi(ww[j]);
+      }
       __stcg(p.ssq_attn + static_cast<size_t>(i) * p.max_batch + b, sq);
     }
   }
@@ -1880,6 +2053,7 @@ __device__ void embed_task(const Params &p, const Slot &S, int ctid) {
 // compute warps: main loop
 // ============================================================================
 
+template <bool TC>
 __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   const int ctid = threadIdx.x - 32;
   Slot *slots = reinterpret_cast<Slot *>(smem + p.off_slots);
@@ -1924,7 +2098,7 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
         }
         break;
       default:
-        if (p.tc)
+        if constexpr (TC)
           tok = p.tc_n > 16 ? gemv_task_tc<2>(p, ctl, smem, S, st, out, ctid)
                             : gemv_task_tc<1>(p, ctl, smem, S, st, out, ctid);
         else
@@ -2156,7 +2330,9 @@ __device__ void storer_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     const Slot S = slots[ts];
     if (S.t.type == T_END) break;
     const float *out = reinterpret_cast<const float *>(smem + p.off_out + os * p.out_bytes);
-    storer_epilogue(p, ctl, S, out, lane);
+    // (tensor-core plans: the compute warps ran the projections' epilogues
+    // and released their events; only the LM head's argmax is left here)
+    if (!(p.tc && is_gemv(S.t.type) && S.t.type != T_LMHEAD)) storer_epilogue(p, ctl, S, out, lane);
     __syncwarp();
     if (lane == 0) trace_mark(p, S.idx, 7);
     if (lane == 0) {
@@ -2180,6 +2356,9 @@ __device__ void storer_main(const Params &p, Ctl *ctl, uint8_t *smem) {
 // kernel
 // ============================================================================
 
+// One instantiation per GEMV path (TC: tcgen05 tiles; else mma.sync pages),
+// so neither carries the other's code.
+template <bool TC>
 __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Ctl *ctl = reinterpret_cast<Ctl *>(smem);
@@ -2225,11 +2404,11 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   if (!ctl->skip) {
     const int warp = threadIdx.x >> 5;
     if (warp == kLoaderWarp) {
-      loader_main(p, ctl, smem);
+      loader_main<TC>(p, ctl, smem);
     } else if (warp == kStorerWarp) {
       storer_main(p, ctl, smem);
     } else {
-      compute_main(p, ctl, smem);
+      compute_main<TC>(p, ctl, smem);
     }
   }
   if (p.tc) tc_fence_before();
@@ -2254,16 +2433,25 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
 // later, smaller setting would fail the launches of an earlier, larger one.
 cudaError_t configure_kernel(int smem_optin) {
   const int lim = smem_optin < kMaxSmem ? smem_optin : kMaxSmem;
-  return cudaFuncSetAttribute(mk_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+  cudaError_t e = cudaFuncSetAttribute(mk_step_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(mk_step_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+  return e;
 }
 
 cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative, cudaStream_t stream) {
   if (cooperative) {
     void *args[] = {const_cast<Params *>(&p)};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(mk_step_kernel), dim3(grid),
+    const void *fn = p.tc ? reinterpret_cast<const void *>(mk_step_kernel<true>)
+                          : reinterpret_cast<const void *>(mk_step_kernel<false>);
+    return cudaLaunchCooperativeKernel(fn, dim3(grid),
                                        dim3(kThreads), args, static_cast<size_t>(smem), stream);
   }
-  mk_step_kernel<<<grid, kThreads, smem, stream>>>(p);
+  if (p.tc)
+    mk_step_kernel<true><<<grid, kThreads, smem, stream>>>(p);
+  else
+    mk_step_kernel<false><<<grid, kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

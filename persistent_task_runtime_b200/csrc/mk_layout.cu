@@ -233,7 +233,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   // ---- tensor-core path: 128-row tiles, split along K for load balance ----------------
   // A task is one 128-row tile (gate/up: the gate tile and the up tile of the
   // same rows) over a K range.  An operator with few tiles is split along K
-  // into parts of whole weight pages so that it has about two tasks per CTA;
+  // into parts of whole weight pages so that it has enough tasks to spread;
   // the part that completes a tile sums the parts in a fixed order.  The O
   // projection is split into one part per KV group, each waiting only for the
   // attention of its group.  The down projection's parts are whole gate/up
@@ -247,7 +247,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     tc_kc = 128;                             // 32 KB pages (128 rows x 128 columns)
     R_qkv = R_o = R_gu = R_d = R_lm = kTcRows;
     auto parts_for = [&](int tiles, int K, int i) {
-      int n = std::max(1, std::min(cdiv(2 * grid, tiles), K / tc_kc));
+      int n = std::max(1, std::min(cdiv(3 * grid, 2 * tiles), K / tc_kc));
       int w = align_up_i(cdiv(K, n), tc_kc);
       n = cdiv(K, w);
       split[i] = n;
