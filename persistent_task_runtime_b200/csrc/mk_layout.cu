@@ -403,6 +403,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   p.kchunk[K_ATT] = n_o_parts > 1 ? o_groups * G * d : 0;
   p.wait_limit_ns = o.wait_limit_ns;
   p.n_ffn_parts = n_ksplit;
+  p.chunk_seq = -1;   // decode steps (a prompt chunk sets its sequence)
   p.n_out = n_out;
   p.tile_rows = tc ? kTcRows : 16;
   p.tc = tc ? 1 : 0;

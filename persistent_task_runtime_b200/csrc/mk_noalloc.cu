@@ -215,6 +215,7 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
 
   p.epoch = 1;  // counters were just zeroed
   p.batch = B;
+  p.chunk_seq = -1;
   p.mode = MK_MODE_MEGAKERNEL;
   p.ids = a->d_ids;
   p.pos = a->d_pos;

@@ -20,7 +20,8 @@ from typing import Dict, Optional
 
 import numpy as np
 
-TYPE_NAMES = {1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead"}
+TYPE_NAMES = {1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead",
+              8: "kvapp"}
 
 
 def decode(raw: np.ndarray) -> Dict[str, np.ndarray]:
@@ -62,7 +63,7 @@ def summarize(raw: np.ndarray) -> str:
     for i in np.nonzero(valid)[0]:
         win[(int(d["layer"][i]), int(ty[i]))].append((t[i, 2], t[i, 6]))
     lines.append("layer op windows (us): first start, last release")
-    for l in sorted({k[0] for k in win})[:3]:
+    for l in sorted({k[0] for k in win})[:4]:
         parts = []
         for code, name in TYPE_NAMES.items():
             if (l, code) in win:
