@@ -231,12 +231,6 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
     if ((rc = upload(&plan->d_sched, both.data(), both.size() * sizeof(int), "schedule")))
       return cleanup_fail(rc);
   }
-  if (lay.n_maps > 0) {
-    std::vector<unsigned char> maps;
-    rc = mk::encode_weight_maps(*cfg, *w, lay, maps, g_err);
-    if (rc) return cleanup_fail(rc);
-    if ((rc = upload(&plan->d_maps, maps.data(), maps.size(), "tensor maps"))) return cleanup_fail(rc);
-  }
   cudaError_t e = cudaMalloc(&plan->d_ws, lay.ws_bytes);
   if (e == cudaSuccess) e = cudaMemset(plan->d_ws, 0, lay.ws_bytes);
   if (e != cudaSuccess) return cleanup_fail(fail(MK_ERR_CUDA, "workspace: %s", cudaGetErrorString(e)));
@@ -244,6 +238,12 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   if (e == cudaSuccess) e = cudaMemset(plan->d_sync, 0, lay.sync_words * sizeof(uint32_t));
   if (e != cudaSuccess) return cleanup_fail(fail(MK_ERR_CUDA, "counters: %s", cudaGetErrorString(e)));
   plan->sync_words = lay.sync_words;
+  if (lay.n_maps > 0) {   // (the staged-input maps point into the workspace)
+    std::vector<unsigned char> maps;
+    rc = mk::encode_weight_maps(*cfg, *w, lay, static_cast<const char *>(plan->d_ws), maps, g_err);
+    if (rc) return cleanup_fail(rc);
+    if ((rc = upload(&plan->d_maps, maps.data(), maps.size(), "tensor maps"))) return cleanup_fail(rc);
+  }
   mk::bind_workspace(lay, static_cast<char *>(plan->d_ws), plan->d_sync, p);
   p.tasks = static_cast<const Task *>(plan->d_tasks);
   p.embed = static_cast<const __nv_bfloat16 *>(w->embed);

@@ -143,8 +143,13 @@ struct Params {
   int tc_kx;                          // staged activation chunk columns (a multiple of tc_kc)
   int tc_kt[8];                       // split-K part columns per task type (0: unsplit)
   const void *tmaps;                  // CUtensorMap[L * 7 + 1], 128 B each (LM head last)
-  float *ssq_attn;                    // [H/16][maxB] sums of h^2 per 16 rows: QKV / LM head input
-  float *ssq_mlp;                     // [H/16][maxB] the same for the gate/up input
+  float *ssq_attn;                    // [H/128][maxB] sums of h^2 per 128 rows: QKV / LM head input
+  float *ssq_mlp;                     // [H/128][maxB] the same for the gate/up input
+  // the GEMV inputs as the tensor cores read them, written once by their
+  // producers: bf16 [2 * tc_bpad][K] (rows 0..bpad-1: high halves of x * g,
+  // rows bpad..: low halves), copied per chunk by a TMA tensor copy
+  __nv_bfloat16 *xs[4];               // XS_ATTN (h * g_attn / g_final), XS_MLP (h * g_mlp), XS_O, XS_U
+  int xs_map0;                        // tensor map of xs[0]; xs[i] uses xs_map0 + i
   float *kpart2;                      // [parts][maxB][2F] split-K partials of gate/up
   uint32_t *tile_ctr2;                // [F/16 + 1] split-K parts done per gate/up row tile
   // solidified schedule (NULL: the global ticket queue): CTA c runs tasks
@@ -201,6 +206,9 @@ __host__ __device__ inline int attn_input_count(const Params &p) {
   return p.kv_tasks ? 1 : p.qkv_tasks_per_group;
 }
 
+// Tensor-core path: the staged-input buffers (Params::xs)
+enum XsKind : int { XS_ATTN = 0, XS_MLP = 1, XS_O = 2, XS_U = 3 };
+
 // Tensor map of weight matrix j (0 wq, 1 wk, 2 wv, 3 wo, 4 w_gate, 5 w_up,
 // 6 w_down) of layer l; the LM head's is the last.
 __host__ __device__ inline int tc_map_index(int l, int j) { return l * kTcMatsPerLayer + j; }
@@ -250,6 +258,7 @@ struct Layout {
   // workspace byte offsets and size; counter words
   size_t o_h = 0, o_qkv = 0, o_part = 0, o_o = 0, o_u = 0, o_arg = 0, o_kpart = 0;
   size_t o_kpart2 = 0, o_kpart_o = 0, o_ssq_attn = 0, o_ssq_mlp = 0;
+  size_t o_xs[4] = {0, 0, 0, 0};
   size_t ws_bytes = 0;
   size_t comb_words = 0, tile_words = 0, tile2_words = 0, tile_o_words = 0, sync_words = 0;
   int n_maps = 0;                      // tensor maps the tensor-core path needs (0: none)
@@ -265,10 +274,12 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
 void bind_workspace(const Layout &lay, char *ws, uint32_t *sync, Params &p);
 // Fill every task's operand pointers (weights, norm gains) from `w`.
 void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vector<Task> &tasks);
-// Encode the tensor maps of every weight matrix (lay.n_maps of them, 128
-// bytes each) into `out` for the tensor-core path.  Needs the CUDA driver.
+// Encode the tensor maps of every weight matrix and of the staged-input
+// buffers (lay.n_maps of them, 128 bytes each) into `out` for the
+// tensor-core path; `ws` is the workspace the plan binds.  Needs the CUDA
+// driver.
 int encode_weight_maps(const mk_model_config &c, const mk_weights &w, const Layout &lay,
-                       std::vector<unsigned char> &out, std::string &err);
+                       const char *ws, std::vector<unsigned char> &out, std::string &err);
 
 cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative,
                         cudaStream_t stream);

@@ -72,6 +72,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -1226,84 +1232,15 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
 // quarters 1, 2, 3, 0) read the accumulators and hand the task's rows to the
 // storer, scaled by the RMSNorm factor for normed inputs.
 
-__device__ __forceinline__ void compute_stage_bar() {
-  asm volatile("bar.sync 2, %0;" ::"n"(kComputeThreads - 32) : "memory");
-}
-
-// 8 fp32 values times their gains -> 8 bf16 high parts and 8 low parts.
-__device__ __forceinline__ void split8(const float4 &x0, const float4 &x1, bool has_gain, uint4 gw,
-                                      uint4 &hw, uint4 &lw) {
-  float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-  if (has_gain) {
-    const uint32_t gg[4] = {gw.x, gw.y, gw.z, gw.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      v[2 * e] *= bf_lo(gg[e]);
-      v[2 * e + 1] *= bf_hi(gg[e]);
-    }
-  }
-  uint32_t h[4], l[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    __nv_bfloat16 h0, l0, h1, l1;
-    split_bf16(v[2 * e], h0, l0);
-    split_bf16(v[2 * e + 1], h1, l1);
-    h[e] = pack2(h0, h1);
-    l[e] = pack2(l0, l1);
-  }
-  hw = make_uint4(h[0], h[1], h[2], h[3]);
-  lw = make_uint4(l[0], l[1], l[2], l[3]);
-}
-
-// Stage activation columns [xc0, xc0 + xlen) of every sequence into `xbuf`
-// (160 threads, sid 0..159) in the K-major 128-byte-swizzled layout: per
-// 64-column atom, rows of 128 bytes (hi rows 0..bpad-1, lo rows
-// bpad..2*bpad-1), the 16-byte chunk c of a row stored at chunk c XOR
-// (row address bits 7..9).  Sequences >= B are zeros.  Each thread first
-// issues the global loads of all of its 8-column blocks (up to kStageUnits),
-// then converts and stores them: one L2 round trip per batch.
-constexpr int kStagers = kComputeThreads - 32;
-constexpr int kStageUnits = 7;   // 7 x 160 >= 1024, the blocks of a full 32 KB chunk
-__device__ void stage_chunk_tc(const Params &p, const float *src, int stride,
-                               const __nv_bfloat16 *gain, int xc0, int xlen, uint8_t *xbuf, int B,
-                               int sid) {
-  const int bpad = p.tc_bpad;
-  const int nblk = xlen / 8;
-  const int units = bpad * nblk;
-  const uint32_t xs = smem_u32(xbuf);
-  const uint32_t atom_bytes = static_cast<uint32_t>(p.tc_n) * 128u;
-  for (int u0 = sid; u0 < units; u0 += kStageUnits * kStagers) {
-    float4 x0[kStageUnits], x1[kStageUnits];
-    uint4 gw[kStageUnits];
-#pragma unroll
-    for (int k = 0; k < kStageUnits; ++k) {
-      const int u = u0 + k * kStagers;
-      const int b = u / nblk, j = u - b * nblk;
-      x0[k] = x1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-      gw[k] = make_uint4(0, 0, 0, 0);
-      if (u < units && b < B) {
-        const float4 *sp =
-            reinterpret_cast<const float4 *>(src + static_cast<size_t>(b) * stride + xc0 + j * 8);
-        x0[k] = __ldcg(sp);
-        x1[k] = __ldcg(sp + 1);
-        if (gain != nullptr) gw[k] = __ldg(reinterpret_cast<const uint4 *>(gain + xc0 + j * 8));
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < kStageUnits; ++k) {
-      const int u = u0 + k * kStagers;
-      if (u >= units) break;
-      const int b = u / nblk, j = u - b * nblk;
-      uint4 hw, lw;
-      split8(x0[k], x1[k], gain != nullptr, gw[k], hw, lw);
-      const uint32_t atom = xs + static_cast<uint32_t>(j >> 3) * atom_bytes;
-      const uint32_t ch = static_cast<uint32_t>(j & 7);
-      const uint32_t rh = atom + static_cast<uint32_t>(b) * 128u;
-      const uint32_t rl = atom + static_cast<uint32_t>(bpad + b) * 128u;
-      sts128(rh + ((ch ^ ((rh >> 7) & 7u)) << 4), hw);
-      sts128(rl + ((ch ^ ((rl >> 7) & 7u)) << 4), lw);
-    }
-  }
+// Tensor-core path: store v (already times the consumer's gain) as column
+// `col` of sequence b in a staged-input buffer [2 * bpad][K]: its bf16 high
+// half in row b, the low half (v - high, rounded) in row bpad + b.
+__device__ __forceinline__ void put_staged(__nv_bfloat16 *xs, int bpad, int K, int b, int col,
+                                           float v) {
+  __nv_bfloat16 hi, lo;
+  split_bf16(v, hi, lo);
+  xs[static_cast<size_t>(b) * K + col] = hi;
+  xs[static_cast<size_t>(bpad + b) * K + col] = lo;
 }
 
 // Tensor-core path, normed inputs: the sums of h^2 per 128 rows that the
@@ -1383,84 +1320,91 @@ __device__ bool gemv_task_tc(const Params &p, Ctl *ctl, uint8_t *smem, const Slo
 
   const int nchunks = (g.Kt + p.tc_kx - 1) / p.tc_kx;
   uint8_t *xbase = smem + p.off_x;
-  if (ctid >= 32) {
-    // ---- stagers: one chunk ahead of the MMAs, in two buffers ----
+  if (ctid >= 32 && ctid < 64) {
+    // ---- warp 2: the RMSNorm scales (read by the epilogue) ----
+    if (normed) tc_norm_scales<BP>(p, ctl, t.type == T_GATEUP ? p.ssq_mlp : p.ssq_attn, B, lane);
+  } else if (ctid == 0) {
+    // ---- thread 0: the activation chunks (TMA copies of the staged input,
+    // one chunk ahead, two buffers) and the MMAs ----
+    const int kind = t.type == T_QKV || t.type == T_LMHEAD ? XS_ATTN
+                     : t.type == T_GATEUP                  ? XS_MLP
+                     : t.type == T_OPROJ                   ? XS_O
+                                                           : XS_U;
+    const void *xmap = static_cast<const uint8_t *>(p.tmaps) + static_cast<size_t>(p.xs_map0 + kind) * 128;
+    const uint64_t xpol = l2_evict_last_policy();
+    const uint32_t idesc = mma_idesc_bf16(kTcRows, p.tc_n);
+    const uint32_t tmem = ctl->tmem;
+    const uint32_t pages = smem_u32(smem + p.off_pages);
+    const uint32_t xs0 = smem_u32(xbase);
+    const uint32_t xatom = static_cast<uint32_t>(p.tc_n) * 128u;
     bool bad = false;
-    for (int c = 0; c < nchunks; ++c) {
+    // the producers' writes were acquired (input event) by the generic proxy;
+    // the tensor copies read through the async proxy
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    auto issue_x = [&](int c) {
       const uint32_t u = st.xuse + c;
       const int buf = static_cast<int>(u & 1u);
       const uint32_t use = u >> 1;
+      // the buffer's previous chunk: its MMAs must be complete
+      if (!bad && use > 0 && !wait_mbar(p, ctl, &ctl->x_free[buf], (use - 1u) & 1u, 0xfff90000u, 2))
+        bad = true;
+      if (bad) return;
+      const int xc0 = g.k0 + c * p.tc_kx;
+      const int nbox = min(p.tc_kx, g.k0 + g.Kt - xc0) / kTcAtomCols;
+      mbar_arrive_expect_tx(&ctl->x_full[buf], static_cast<uint32_t>(nbox) * xatom);
+      for (int a = 0; a < nbox; ++a)
+        tma_load_2d(xbase + buf * kTcXBytes + a * xatom, xmap, xc0 + a * kTcAtomCols, 0,
+                    &ctl->x_full[buf], xpol);
+    };
+    issue_x(0);
+    bool started0 = false, started1 = false;   // tile 0 / 1 has its first MMA
+    for (int c = 0; c < nchunks; ++c) {
+      const uint32_t u = st.xuse + c;
+      const int buf = static_cast<int>(u & 1u);
       const int xc0 = g.k0 + c * p.tc_kx;
       const int xlen = min(p.tc_kx, g.k0 + g.Kt - xc0);
-      if (use > 0 && !bad &&
-          !warp_wait_page(p, ctl, &ctl->x_free[buf], (use - 1u) & 1u, 0xfff90000u)) {
-        bad = true;
-        if (lane == 0) {
-          ctl->cbad = 1;
-          ctl->cta_abort = 1;
-        }
-      }
-      // (the MMAs that last read this buffer did so through the async proxy)
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      if (!bad)
-        stage_chunk_tc(p, src, stride, gain, xc0, xlen, xbase + buf * kTcXBytes, B, ctid - 32);
-      // the tensor core reads the buffer through the async proxy
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      compute_stage_bar();
-      if (ctid == 32) mbar_arrive(&ctl->x_full[buf]);
-    }
-  } else {
-    // ---- warp 1: the RMSNorm scales, then lane 0 issues the MMAs ----
-    if (normed) tc_norm_scales<BP>(p, ctl, t.type == T_GATEUP ? p.ssq_mlp : p.ssq_attn, B, lane);
-    if (ctid == 0) {
-      const uint32_t idesc = mma_idesc_bf16(kTcRows, p.tc_n);
-      const uint32_t tmem = ctl->tmem;
-      const uint32_t pages = smem_u32(smem + p.off_pages);
-      const uint32_t xs0 = smem_u32(xbase);
-      const uint32_t xatom = static_cast<uint32_t>(p.tc_n) * 128u;
-      bool bad = false;
-      bool started0 = false, started1 = false;   // tile 0 / 1 has its first MMA
-      for (int c = 0; c < nchunks; ++c) {
-        const uint32_t u = st.xuse + c;
-        const int buf = static_cast<int>(u & 1u);
-        const int xc0 = g.k0 + c * p.tc_kx;
-        const int xlen = min(p.tc_kx, g.k0 + g.Kt - xc0);
-        if (!bad && !wait_mbar(p, ctl, &ctl->x_full[buf], (u >> 1) & 1u, 0xfffa0000u, 2)) bad = true;
-        tc_fence_after();
-        const uint32_t xb = xs0 + static_cast<uint32_t>(buf) * kTcXBytes;
-        for (int m = 0; m < t.n_m; ++m) {
-          for (int c0 = xc0; c0 < xc0 + xlen; c0 += p.tc_kc) {
-            const int nc = min(p.tc_kc, xc0 + xlen - c0);
-            if (!bad && !wait_mbar(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff30000u, 2)) bad = true;
-            if (!bad) {
-              tc_fence_after();
-              const uint32_t pg = pages + static_cast<uint32_t>(st.pi) * p.page_bytes;
-              const uint32_t xa0 = xb + static_cast<uint32_t>((c0 - xc0) / kTcAtomCols) * xatom;
-              for (int a = 0; a < nc / kTcAtomCols; ++a)
+      if (c + 1 < nchunks) issue_x(c + 1);
+      if (!bad && !wait_mbar(p, ctl, &ctl->x_full[buf], (u >> 1) & 1u, 0xfffa0000u, 2)) bad = true;
+      tc_fence_after();
+      const uint32_t xb = xs0 + static_cast<uint32_t>(buf) * kTcXBytes;
+      for (int m = 0; m < t.n_m; ++m) {
+        for (int c0 = xc0; c0 < xc0 + xlen; c0 += p.tc_kc) {
+          const int nc = min(p.tc_kc, xc0 + xlen - c0);
+          if (!bad && !wait_mbar(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff30000u, 2)) bad = true;
+          if (!bad) {
+            tc_fence_after();
+            const uint32_t pg = pages + static_cast<uint32_t>(st.pi) * p.page_bytes;
+            const uint32_t xa0 = xb + static_cast<uint32_t>((c0 - xc0) / kTcAtomCols) * xatom;
+            for (int a = 0; a < nc / kTcAtomCols; ++a)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const uint64_t ad = sw128_desc(pg + a * kTcAtomBytes + j * 32);
-                  const uint64_t bd = sw128_desc(xa0 + a * xatom + j * 32);
-                  tc_mma(tmem + m * p.tc_n, ad, bd, idesc, m == 0 ? started0 : started1);
-                  if (m == 0) started0 = true; else started1 = true;
-                }
-              tc_commit(&ctl->empty[st.pi]);   // the page is free once these MMAs complete
-            }
-            if (++st.pi == p.n_pages) {
-              st.pi = 0;
-              st.pg_par ^= 1u;
-            }
+              for (int j = 0; j < 4; ++j) {
+                const uint64_t ad = sw128_desc(pg + a * kTcAtomBytes + j * 32);
+                const uint64_t bd = sw128_desc(xa0 + a * xatom + j * 32);
+                tc_mma(tmem + m * p.tc_n, ad, bd, idesc, m == 0 ? started0 : started1);
+                if (m == 0) started0 = true; else started1 = true;
+              }
+            tc_commit(&ctl->empty[st.pi]);   // the page is free once these MMAs complete
+          }
+          if (++st.pi == p.n_pages) {
+            st.pi = 0;
+            st.pg_par ^= 1u;
           }
         }
-        tc_commit(&ctl->x_free[buf]);
       }
-      tc_commit(&ctl->acc_bar);
-      // wait for the accumulators (also after a failed wait: no MMA may still
-      // be running when the task returns)
-      if (!wait_mbar(p, ctl, &ctl->acc_bar, st.accuse & 1u, 0xfffb0000u, 4)) bad = true;
-      if (bad) {
-        ctl->cbad = 1;
-        ctl->cta_abort = 1;
+      tc_commit(&ctl->x_free[buf]);
+    }
+    tc_commit(&ctl->acc_bar);
+    // wait for the accumulators (also after a failed wait: no MMA may still
+    // be running when the task returns) and for any activation copy in flight
+    if (!wait_mbar(p, ctl, &ctl->acc_bar, st.accuse & 1u, 0xfffb0000u, 4)) bad = true;
+    if (bad) {
+      ctl->cbad = 1;
+      ctl->cta_abort = 1;
+      for (int c = 0; c < 2; ++c) {   // copies issued but never waited for
+        const uint32_t u = st.xuse + nchunks - 1 + c;
+        const uint64_t t0 = gtimer();
+        while (!mbar_try_wait(&ctl->x_full[u & 1u], (u >> 1) & 1u))
+          if (gtimer() - t0 > static_cast<uint64_t>(p.wait_limit_ns)) break;
       }
     }
   }
@@ -1590,11 +1534,15 @@ __device__ bool gemv_task_tc(const Params &p, Ctl *ctl, uint8_t *smem, const Slo
       for (int b = 0; b < BP; ++b)
         if (b < B) {
           const float gt = acc[0][b];
-          __stcg(p.u + static_cast<size_t>(b) * p.F + t.row0 + row,
-                 gt / (1.0f + __expf(-gt)) * acc[1][b]);
+          const float uv = gt / (1.0f + __expf(-gt)) * acc[1][b];
+          __stcg(p.u + static_cast<size_t>(b) * p.F + t.row0 + row, uv);
+          put_staged(p.xs[XS_U], BP, p.F, b, t.row0 + row, uv);   // the down projection's input
         }
   } else {
-    // O / down: residual add, per-layer dump, sums of h^2 for the next RMSNorm
+    // O / down: residual add, per-layer dump, the next normed input (x * its
+    // gain, staged) and its sums of h^2
+    __nv_bfloat16 *xs_next = p.xs[t.type == T_OPROJ ? XS_MLP : XS_ATTN];
+    const float gnext = vrow ? __bfloat162float(t.w1[t.row0 + row]) : 0.f;
     float hv[BP];
 #pragma unroll
     for (int b = 0; b < BP; ++b)
@@ -1605,6 +1553,7 @@ __device__ bool gemv_task_tc(const Params &p, Ctl *ctl, uint8_t *smem, const Slo
       if (vrow && b < B) {
         v = hv[b] + acc[0][b];
         __stcg(p.h + static_cast<size_t>(b) * p.H + t.row0 + row, v);
+        put_staged(xs_next, BP, p.H, b, t.row0 + row, v * gnext);
         if (t.type == T_DOWN && p.hidden_dump != nullptr)
           p.hidden_dump[(static_cast<size_t>(t.layer) * B + b) * p.H + t.row0 + row] = v;
       }
@@ -1950,8 +1899,17 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     for (int c0 = kCombRegs; c0 < nch; c0 += kCombRegs)
       comb_batch<D>(p0 + c0 * cstride + h * rw, cstride, i, nch - c0, M, den, num);
     const float r = 1.0f / den;
-    __stcg(reinterpret_cast<float4 *>(p.o + static_cast<size_t>(b) * p.Hq * d + (g * G + h) * d + i),
-           make_float4(num.x * r, num.y * r, num.z * r, num.w * r));
+    const float4 ov = make_float4(num.x * r, num.y * r, num.z * r, num.w * r);
+    const int col = (g * G + h) * d + i;
+    __stcg(reinterpret_cast<float4 *>(p.o + static_cast<size_t>(b) * p.Hq * d + col), ov);
+    if (p.tc) {
+      // the O projection's input, staged for the tensor cores
+      const int K = p.Hq * d;
+      put_staged(p.xs[XS_O], p.tc_bpad, K, b, col, ov.x);
+      put_staged(p.xs[XS_O], p.tc_bpad, K, b, col + 1, ov.y);
+      put_staged(p.xs[XS_O], p.tc_bpad, K, b, col + 2, ov.z);
+      put_staged(p.xs[XS_O], p.tc_bpad, K, b, col + 3, ov.w);
+    }
   }
   compute_bar();
   if (ctid == 0) *ctr = 0u;   // rearm for the next layer / step
@@ -2025,6 +1983,15 @@ __device__ void embed_task(const Params &p, const Slot &S, int ctid) {
       float4 c = make_float4(bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
       __stcg(reinterpret_cast<float4 *>(p.h + b * H + i), a);
       __stcg(reinterpret_cast<float4 *>(p.h + b * H + i + 4), c);
+      if (p.tc) {
+        // the first QKV input, times its gain, staged for the tensor cores
+        const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(S.t.w1 + i));
+        const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+        const float gg[8] = {bf_lo(gw.x), bf_hi(gw.x), bf_lo(gw.y), bf_hi(gw.y),
+                             bf_lo(gw.z), bf_hi(gw.z), bf_lo(gw.w), bf_hi(gw.w)};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) put_staged(p.xs[XS_ATTN], p.tc_bpad, H, b, i + k, v[k] * gg[k]);
+      }
     }
   }
   if (p.tc) {

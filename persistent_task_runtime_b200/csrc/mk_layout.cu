@@ -600,10 +600,16 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   out.o_kpart_o = carve(sizeof(float) * (split[1] > 1 ? static_cast<size_t>(split[1]) * H : 0) * maxB);
   out.o_kpart2 = carve(sizeof(float) * (split[2] > 1 ? static_cast<size_t>(split[2]) * 2 * F : 0) *
                        maxB);
-  // per-16-row sums of h^2, written by the producers of h (tensor-core path)
-  const size_t ssq_floats = tc ? static_cast<size_t>(H / 16) * maxB : 0;
+  // per-128-row sums of h^2, written by the producers of h (tensor-core path)
+  const size_t ssq_floats = tc ? static_cast<size_t>(cdiv(H, kTcRows)) * maxB : 0;
   out.o_ssq_attn = carve(sizeof(float) * ssq_floats);
   out.o_ssq_mlp = carve(sizeof(float) * ssq_floats);
+  // the staged GEMV inputs, bf16 [2 * bpad][K] (tensor-core path)
+  {
+    const int xk[4] = {H, H, Hq * d, F};
+    for (int i = 0; i < 4; ++i)
+      out.o_xs[i] = carve(tc ? sizeof(__nv_bfloat16) * 2 * tc_bpad * static_cast<size_t>(xk[i]) : 0);
+  }
   out.ws_bytes = off;
   out.n_events = n_events;
   out.comb_words = static_cast<size_t>(maxB) * Hkv;
@@ -612,7 +618,8 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   out.tile_o_words = static_cast<size_t>(H) / 16 + 1;
   out.sync_words = S_EVENTS + n_events + out.comb_words + out.tile_words + out.tile2_words +
                    out.tile_o_words;
-  out.n_maps = tc ? L * kTcMatsPerLayer + 1 : 0;
+  out.n_maps = tc ? L * kTcMatsPerLayer + 1 + 4 : 0;
+  p.xs_map0 = L * kTcMatsPerLayer + 1;
   for (int i = 0; i < 5; ++i) out.splits[i] = split[i];
 
   out.grid = grid;
@@ -636,6 +643,7 @@ void bind_workspace(const Layout &lay, char *ws, uint32_t *sync, Params &p) {
   p.kpart2 = reinterpret_cast<float *>(ws + lay.o_kpart2);
   p.ssq_attn = reinterpret_cast<float *>(ws + lay.o_ssq_attn);
   p.ssq_mlp = reinterpret_cast<float *>(ws + lay.o_ssq_mlp);
+  for (int i = 0; i < 4; ++i) p.xs[i] = reinterpret_cast<__nv_bfloat16 *>(ws + lay.o_xs[i]);
   p.sync = sync;
   p.comb_ctr = sync + S_EVENTS + lay.n_events;
   p.tile_ctr = p.comb_ctr + lay.comb_words;
@@ -648,7 +656,11 @@ void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vect
   auto bf = [](const void *q) { return static_cast<const __nv_bfloat16 *>(q); };
   for (Task &t : tasks) {
     t.w0 = t.w1 = t.gain = nullptr;
-    if (t.type == T_EMBED || t.type == T_END) continue;
+    if (t.type == T_END) continue;
+    if (t.type == T_EMBED) {
+      t.w1 = bf(w.layers[0].attn_norm);   // the first QKV input's gain (staged input)
+      continue;
+    }
     if (t.type == T_LMHEAD) {
       t.w0 = bf(w.lm_head);
       t.gain = bf(w.final_norm);
@@ -665,13 +677,20 @@ void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vect
         t.w0 = bf(lw.q_norm);
         t.w1 = bf(lw.k_norm);
         break;
-      case T_OPROJ: t.w0 = bf(lw.wo); break;
+      case T_OPROJ:
+        t.w0 = bf(lw.wo);
+        t.w1 = bf(lw.mlp_norm);   // the gain of the input it produces (gate/up's)
+        break;
       case T_GATEUP:
         t.w0 = bf(lw.w_gate);
         t.w1 = bf(lw.w_up);
         t.gain = bf(lw.mlp_norm);
         break;
-      case T_DOWN: t.w0 = bf(lw.w_down); break;
+      case T_DOWN:
+        t.w0 = bf(lw.w_down);
+        // the gain of the input it produces: the next layer's QKV, or the LM head
+        t.w1 = bf(t.layer + 1 < c.n_layers ? w.layers[t.layer + 1].attn_norm : w.final_norm);
+        break;
       default: break;
     }
   }
@@ -691,7 +710,7 @@ void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vect
 namespace mk {
 
 int encode_weight_maps(const mk_model_config &c, const mk_weights &w, const Layout &lay,
-                       std::vector<unsigned char> &out, std::string &err) {
+                       const char *ws, std::vector<unsigned char> &out, std::string &err) {
   out.clear();
   if (lay.n_maps == 0) return MK_OK;
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
@@ -707,11 +726,11 @@ int encode_weight_maps(const mk_model_config &c, const mk_weights &w, const Layo
   const int L = c.n_layers, H = c.hidden, F = c.ffn, d = c.head_dim;
   const int Hq = c.n_q_heads, Hkv = c.n_kv_heads;
   out.assign(static_cast<size_t>(lay.n_maps) * sizeof(CUtensorMap), 0);
-  auto one = [&](int idx, const void *ptr, int rows, int K) {
+  auto one = [&](int idx, const void *ptr, int rows, int K, int box_rows = kTcRows) {
     CUtensorMap m;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcAtomCols), static_cast<cuuint32_t>(kTcRows)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcAtomCols), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     const CUresult r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
                               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -734,6 +753,10 @@ int encode_weight_maps(const mk_model_config &c, const mk_weights &w, const Layo
       break;
   }
   if (rc == MK_OK) rc = one(tc_map_index(L, 0), w.lm_head, c.vocab, H);
+  // the staged inputs: one box is every row (2 * bpad) of 64 columns
+  const int xk[4] = {H, H, c.n_q_heads * d, F};
+  for (int i = 0; i < 4 && rc == MK_OK; ++i)
+    rc = one(lay.p.xs_map0 + i, ws + lay.o_xs[i], lay.p.tc_n, xk[i], lay.p.tc_n);
   return rc;
 }
 

@@ -169,7 +169,7 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
     std::vector<unsigned char> maps;   // tensor maps of the tensor-core path (or none)
     {
       std::string merr;
-      const int mrc = mk::encode_weight_maps(c, *w, up.lay, maps, merr);
+      const int mrc = mk::encode_weight_maps(c, *w, up.lay, base + up.o_ws, maps, merr);
       if (mrc) return nfail(mrc, merr.c_str());
     }
     up.o_maps = carve(maps.size());
