@@ -395,8 +395,11 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   p.off_pages = geo.off_pages;
   // attention slots: a fixed block per KV group (so each group's completion
   // is a static count), enough for about one chunk per CTA in all plus one
-  // partial chunk per sequence
-  p.attn_spg = cdiv(grid, Hkv) + maxB;
+  // partial chunk per sequence -- at larger batches about maxB / 4 chunks per
+  // CTA, so that many sequences' long contexts split into chunks small enough
+  // to spread evenly over the CTAs (16 sequences at context 1024: chunks of
+  // 224 tokens instead of 864)
+  p.attn_spg = cdiv(grid * std::max(1, maxB / 4), Hkv) + maxB;
   p.attn_slots = Hkv * p.attn_spg;
   p.n_o_parts = n_o_parts;
   p.o_groups = o_groups;
