@@ -15,8 +15,10 @@ invariants, brute force on tiny inputs and independent library routines.
 from .decoder import (  # noqa: F401
     DecoderConfig,
     KVCache,
+    W4Weights,
     Weights,
     apply_rope,
+    dequantize_w4,
     attend,
     decode_step,
     forward_full,

@@ -125,6 +125,58 @@ class Weights:
 
 
 # --------------------------------------------------------------------------
+# 4-bit weights (W4A16)
+# --------------------------------------------------------------------------
+
+W4_GROUP = 128     # columns that share one scale
+W4_ZERO = 8        # the code that stands for 0
+W4_MATRICES = ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down")
+
+
+def dequantize_w4(codes, scales) -> np.ndarray:
+    """The bf16 weight matrix a 4-bit matrix stands for.
+
+    ``codes`` [rows, cols] hold integers 0..15, ``scales`` [rows, cols/128]
+    bf16 values; element (r, c) is  bf16( scales[r, c // 128] * (codes[r, c] - 8) ).
+    READING (the Ada-MK summary, "Quantisierungs-bewusste Optimierung", names
+    GPTQ-style W4A16 without fixing its details): symmetric codes with zero
+    point 8, one bf16 scale per row and group of 128 input columns, and the
+    dequantized weight rounded once (to nearest, ties to even) to bf16, the
+    precision the bf16 activations meet it in.  The product scale * (code - 8)
+    is exact in float64; round_bf16 is the only rounding.
+    """
+    q = np.asarray(as_f64(codes), dtype=np.float64)
+    s = as_f64(scales)
+    rows, cols = q.shape
+    assert s.shape == (rows, cols // W4_GROUP) and cols % W4_GROUP == 0
+    return round_bf16(np.repeat(s, W4_GROUP, axis=1) * (q - W4_ZERO))
+
+
+class W4Weights(Weights):
+    """A decoder whose seven projection matrices per layer are 4-bit: layer
+    ``l`` of ``tensors`` holds ``w4[name] = (codes, scales)`` for each name in
+    W4_MATRICES (and the norms as bf16); embedding, final norm and LM head are
+    bf16.  Each matrix is dequantized (dequantize_w4) when the layer is used."""
+
+    def layer(self, l: int) -> Dict[str, np.ndarray]:
+        src = self.t["layers"][l]
+        out = {}
+        for k in self.LAYER_KEYS:
+            if k in W4_MATRICES:
+                codes, scales = src["w4"][k]
+                if self.keep:
+                    key = (l, k, "w4")
+                    if key not in self._cache:
+                        self._cache[key] = dequantize_w4(codes, scales)
+                    out[k] = self._cache[key]
+                else:
+                    out[k] = dequantize_w4(codes, scales)
+            else:
+                out[k] = self._get((l, k), src[k])
+        return out
+
+
+# --------------------------------------------------------------------------
 # elementwise pieces
 # --------------------------------------------------------------------------
 

@@ -97,10 +97,45 @@ def make_weights(cfg: dict, seed: int = 0, device="cpu", gain: str = "ones",
     return w
 
 
+W4_MATRIX_NAMES = ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down")
+W4_GROUP = 128
+
+
+def make_w4_weights(cfg: dict, seed: int = 0, device="cpu", gain: str = "ones",
+                    layers: Optional[int] = None) -> dict:
+    """Random-init 4-bit weights: the seven projection matrices of every layer
+    as (codes, scales) pairs, everything else bf16 as in make_weights.
+
+    codes: uint8 [out, in], uniform in 0..15; scales: bf16 [out, in / 128],
+    uniform in [0.003, 0.006) (with codes centred on 8 that gives weights of
+    about the 0.02 standard deviation of the bf16 initialisation).  Layer l
+    holds ``w4[name] = (codes, scales)``.  Only random numbers are drawn here;
+    what a code and a scale stand for is the decoder's business."""
+    base = make_weights(cfg, seed=seed, device=device, gain=gain, layers=layers)
+    g = _gen(seed + 1000, device)
+    for lw in base["layers"]:
+        q = {}
+        for name in W4_MATRIX_NAMES:
+            rows, cols = lw[name].shape
+            codes = torch.randint(0, 16, (rows, cols), generator=g, device=device,
+                                  dtype=torch.int64).to(torch.uint8)
+            scales = (0.003 + 0.003 * torch.rand(rows, cols // W4_GROUP, generator=g,
+                                                 device=device)).to(torch.bfloat16)
+            q[name] = (codes, scales)
+            del lw[name]
+        lw["w4"] = q
+    return base
+
+
 def weights_to(w: dict, device) -> dict:
     """Copy a weight dict to another device (same values)."""
     out = {k: v.to(device) for k, v in w.items() if k != "layers"}
-    out["layers"] = [{k: v.to(device) for k, v in lw.items()} for lw in w["layers"]]
+    out["layers"] = []
+    for lw in w["layers"]:
+        d = {k: v.to(device) for k, v in lw.items() if k != "w4"}
+        if "w4" in lw:
+            d["w4"] = {k: (c.to(device), sc.to(device)) for k, (c, sc) in lw["w4"].items()}
+        out["layers"].append(d)
     return out
 
 

@@ -404,6 +404,50 @@ def pin_prefill_equals_incremental(O):
         np.testing.assert_allclose(nxt_a["logits"], nxt_b["logits"], rtol=1e-10, atol=1e-11)
 
 
+def pin_dequantize_w4(O):
+    """4-bit weights: hand-worked codes and scales, the bf16 rounding of an
+    inexact product, the group boundary at column 128, and torch's own
+    float32 product and bf16 conversion (exact product, one rounding)."""
+    codes = np.full((2, 256), 8, dtype=np.uint8)
+    codes[0, :16] = np.arange(16)
+    scales = np.array([[0.5, 2.0], [1.0078125, 0.25]])
+    codes[1, 0] = 15            # 1.0078125 * 7 = 7.0546875 -> bf16 7.0625 (ties/nearest)
+    codes[1, 127] = 0           # last column of group 0: scale 1.0078125
+    codes[1, 128] = 0           # first column of group 1: scale 0.25
+    got = O.dequantize_w4(codes, scales)
+    np.testing.assert_array_equal(got[0, :16], 0.5 * (np.arange(16) - 8))
+    assert got[0, 16] == 0.0 and got[0, 130] == 0.0
+    assert got[1, 0] == 7.0625
+    assert got[1, 127] == -8.0625         # 1.0078125 * -8 = -8.0625, exact in bf16
+    assert got[1, 128] == -2.0
+    # library: torch float32 product (exact: 8 + 4 significant bits) rounded to bf16
+    rng = np.random.default_rng(17)
+    c = torch.from_numpy(rng.integers(0, 16, (8, 384)).astype(np.uint8))
+    sc = (0.003 + 0.003 * torch.rand(8, 3, generator=torch.Generator().manual_seed(5))).to(
+        torch.bfloat16)
+    ref = (sc.float().repeat_interleave(128, dim=1) * (c.float() - 8)).to(torch.bfloat16)
+    np.testing.assert_array_equal(O.dequantize_w4(c, sc), ref.double().numpy())
+
+
+def pin_w4_decoder_is_the_dequantized_decoder(O):
+    """A 4-bit decoder computes what the bf16 decoder computes on its
+    dequantized (torch-built) matrices."""
+    d = dict(MICRO, hidden=128, ffn=256, n_q_heads=4, n_kv_heads=2, head_dim=32)
+    cfg = _cfg(O, d)
+    w4 = synth.make_w4_weights(d, seed=41, gain="random")
+    wb = {k: v for k, v in w4.items() if k != "layers"}
+    wb["layers"] = []
+    for lw in w4["layers"]:
+        e = {k: v for k, v in lw.items() if k != "w4"}
+        for name, (c, sc) in lw["w4"].items():
+            e[name] = (sc.float().repeat_interleave(128, dim=1) * (c.float() - 8)).to(torch.bfloat16)
+        wb["layers"].append(e)
+    ids = [1, 7, 3, 12]
+    a = O.forward_full(cfg, O.W4Weights(w4), ids)["logits"]
+    b = O.forward_full(cfg, O.Weights(wb), ids)["logits"]
+    np.testing.assert_array_equal(a, b)
+
+
 # ------------------------------------------ torch library composition ------
 
 
@@ -469,6 +513,7 @@ ALL_PINS = [
     pin_incremental_equals_full, pin_causality, pin_batch_rows_independent,
     pin_gqa_head_mapping, pin_mha_equals_expanded_gqa, pin_brute_force_micro,
     pin_torch_composition_tiny, pin_greedy_decode_hand_loop, pin_prefill_equals_incremental,
+    pin_dequantize_w4, pin_w4_decoder_is_the_dequantized_decoder,
 ]
 
 

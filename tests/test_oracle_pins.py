@@ -45,6 +45,11 @@ MUTATIONS = {
     "greedy_position_off_by_one": ("[n + s - 1] * len(prompts)", "[n + s] * len(prompts)"),
     "greedy_first_token_wrong_row": ('last.append(out["logits"][-1])',
                                      'last.append(out["logits"][-2])'),
+    "w4_zero_point": ("(q - W4_ZERO)", "(q - W4_ZERO + 1)"),
+    "w4_no_rounding": ("return round_bf16(np.repeat(s, W4_GROUP, axis=1) * (q - W4_ZERO))",
+                       "return np.repeat(s, W4_GROUP, axis=1) * (q - W4_ZERO)"),
+    "w4_scale_groups_transposed": ("np.repeat(s, W4_GROUP, axis=1)",
+                                   "np.tile(s, (1, W4_GROUP))"),
     "prefill_drops_last_position": ("cache.load_history(l, b, out[\"k\"][l], out[\"v\"][l])",
                                     "cache.load_history(l, b, out[\"k\"][l][:, :-1], "
                                     "out[\"v\"][l][:, :-1])"),
