@@ -58,6 +58,9 @@ def parse_workload(name: str) -> dict:
         return dict(model="1.5b", batch=1, lengths=[256], prefill="decode")
     if name == "8b_b1_ctx512":
         return dict(model="8b", batch=1, lengths=[512], prefill="decode")
+    if name == "8b_w4_b1_ctx512":
+        # the 8B shape with 4-bit (W4A16) projections, batch 1, context 512
+        return dict(model="8b", batch=1, lengths=[512], prefill="decode", w4=True)
     if name == "8b4l_b1_ctx512":
         # profiling case: 8B-shaped layers, 4 of them, same kernel (not a bench line)
         return dict(model="8b", layers=4, batch=1, lengths=[512], prefill="synthetic")
@@ -212,7 +215,8 @@ def run_mk(args, rank: int, world: int, local_rank: int) -> dict:
     B, lengths = wl["batch"], list(wl["lengths"])
     W, K = args.warmup, args.steps
     horizon = W + K + max(args.e2e_steps, 0) + 8
-    weights = synth.make_weights(cfg, seed=0, device=dev)
+    weights = (synth.make_w4_weights(cfg, seed=0, device=dev) if wl.get("w4")
+               else synth.make_weights(cfg, seed=0, device=dev))
     cap = [n + horizon for n in lengths]
     kv = PagedKVCache(cfg, B, cap, page=16, device=dev)
     plan = mk.Plan(cfg, weights, max_batch=B, page_size=16, max_seq_len=max(cap) + 16,
@@ -370,7 +374,8 @@ def oracle_layer_timing(cfg: dict, B: int, lengths, weights_cpu, reps: int = 1):
     ocfg1 = oracle.DecoderConfig(**{k: one[k] for k in (
         "n_layers", "hidden", "n_q_heads", "n_kv_heads", "head_dim", "ffn", "vocab",
         "rms_eps", "rope_theta", "qk_norm")})
-    W = oracle.Weights(weights_cpu, keep_f64=False)
+    wcls = oracle.W4Weights if "w4" in weights_cpu["layers"][0] else oracle.Weights
+    W = wcls(weights_cpu, keep_f64=False)
     hist = synth.make_kv_history(one, lengths, seed=3)
     cache = oracle.KVCache(ocfg1, B, max(lengths) + 2)
     for b, n in enumerate(lengths):
@@ -391,9 +396,11 @@ def oracle_layer_timing(cfg: dict, B: int, lengths, weights_cpu, reps: int = 1):
     return head_s, max(1e-9, statistics.median(layer_s)), ocfg.n_layers
 
 
-def cpu_weights_sample(cfg: dict) -> dict:
+def cpu_weights_sample(cfg: dict, w4: bool = False) -> dict:
     """CPU copy of the weights the oracle sample touches (first layer + head),
-    drawn by the same generator on the CPU."""
+    drawn by the same generator on the CPU (4-bit layers for a 4-bit workload)."""
+    if w4:
+        return synth.make_w4_weights(cfg, seed=0, device="cpu", layers=1)
     return synth.make_weights(cfg, seed=0, device="cpu", layers=1)
 
 
@@ -420,7 +427,7 @@ def run_reference(args) -> dict:
     wl = parse_workload(args.workload)
     cfg = model_config(wl)
     B, lengths = wl["batch"], list(wl["lengths"])
-    w = cpu_weights_sample(cfg)
+    w = cpu_weights_sample(cfg, bool(wl.get("w4")))
     head_s, _, L = oracle_layer_timing(cfg, B, lengths, w)
     per_step = []
     for i in range(args.warmup + args.steps):
@@ -462,6 +469,8 @@ def main():
     wl = parse_workload(args.workload)
     cfg = model_config(wl)
     config = {"workload": args.workload, "model_shape": wl["model"], "batch": wl["batch"],
+              "weights_format": "4-bit codes + bf16 scale per 128 columns (W4A16)"
+              if wl.get("w4") else "bf16",
               "context": wl["lengths"] if len(set(wl["lengths"])) > 1 else wl["lengths"][0],
               "kv_page": 16, "weights": "random N(0,0.02) bf16", "ids": "uniform random",
               "prefill": (("prompt chunks of 16 tokens" if args.prompt_path == "chunks"
@@ -527,7 +536,7 @@ def main():
             "prompt": r["prefill"],
             "gpu_launches": K * r["launches_per_step"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        w = cpu_weights_sample(cfg)
+        w = cpu_weights_sample(cfg, bool(wl.get("w4")))
         ctx, cores = oracle_threads(args.oracle_threads)
         with ctx:
             head_s, layer_s, L = oracle_layer_timing(cfg, r["B"], r["lengths"], w)

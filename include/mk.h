@@ -91,16 +91,50 @@ typedef struct {
       *w_gate, *w_up, *w_down;
 } mk_layer_weights;
 
+/* 4-bit weights (W4A16; the Ada-MK summary's GPTQ-W4A16, "Quantisierungs-
+ * bewusste Optimierung").  A matrix W [rows, cols] is given as codes
+ * c[r][k] in 0..15 and bf16 scales s[r][k / 128]; it stands for the bf16
+ * matrix bf16_rn(s[r][k / 128] * (c[r][k] - 8)).  cols must be a multiple of
+ * MK_W4_BLOCK_COLS.  The kernel reads it in the layout mk_w4_pack writes:
+ * per 16 rows (a row tile; missing rows are code 8, scale 0) and 1024
+ * columns, one MK_W4_BLOCK_BYTES block = 8 x 16 scales (group-major) then
+ * 32 sub-blocks of 32 columns; a sub-block holds, for each lane (g, q) of an
+ * mma.sync warp (lane = 4 g + q), the 8 codes of row g and then of row g + 8
+ * at columns 8 q .. 8 q + 7, two codes per 16-bit half so that shifting a
+ * word by 4 k and masking 0x000F000F leaves the codes of columns 2 k and
+ * 2 k + 1 -- the order in which the tensor-core fragments consume them. */
+#define MK_W4_GROUP 128
+#define MK_W4_BLOCK_COLS 1024
+#define MK_W4_BLOCK_BYTES 8448
+typedef struct {
+  const void *q[7];       /* packed wq, wk, wv, wo, w_gate, w_up, w_down    */
+} mk_w4_layer_weights;
+
 /* embed [V, H], final_norm [H], lm_head [V, H] (bf16 device pointers; embed
  * and lm_head may be the same pointer).  `layers` is a HOST array of
  * n_layers entries.  The plan copies the pointers, not the weights: the
- * weights must stay allocated and unchanged for the plan's lifetime. */
+ * weights must stay allocated and unchanged for the plan's lifetime.
+ * w4_layers: NULL for bf16 projections; else a HOST array of n_layers
+ * packed 4-bit layers, whose matrices replace the bf16 ones of `layers`
+ * (which may then be NULL; the norms still come from `layers`). */
 typedef struct {
   const void *embed;
   const mk_layer_weights *layers;
   const void *final_norm;
   const void *lm_head;
+  const mk_w4_layer_weights *w4_layers;
 } mk_weights;
+
+/* Bytes of a packed 4-bit matrix of rows x cols (cols a multiple of 1024),
+ * or -1 for an unsupported size. */
+MK_API int64_t mk_w4_packed_bytes(int rows, int cols);
+/* Pack a 4-bit matrix (HOST memory, no GPU): codes uint8 [rows][cols]
+ * (0..15), scales bf16 [rows][cols / 128] -> `packed`
+ * (mk_w4_packed_bytes(rows, cols) bytes; copy it to the device yourself).
+ * MK_ERR_INVALID_ARG for NULL pointers, a code above 15 or a size
+ * mk_w4_packed_bytes rejects. */
+MK_API int mk_w4_pack(const uint8_t *codes, const void *scales, int rows, int cols,
+                      void *packed);
 
 /* Paged KV cache.  For layer l, k_pages[l] and v_pages[l] point to bf16
  * arrays [num_pages, n_kv_heads, page_size, head_dim] (head-major inside a
@@ -157,6 +191,12 @@ typedef struct {
                              offline path solidification) and each CTA runs
                              its list in order.  Per-operator modes always
                              use the queue                                  */
+  int weight_bits;        /* 0: as the weights are given (mk_plan_describe:
+                             bf16); 16: bf16 projections; 4: 4-bit (the
+                             weights must carry w4_layers).  4-bit plans run
+                             the mma.sync path (gemv_path 0 or 1); hidden,
+                             ffn and n_q_heads*head_dim must be multiples
+                             of 1024                                        */
   int prefill;            /* nonzero: the plan can also run prompt chunks
                              (mk_prefill_chunk).  Each layer then appends
                              the step's K/V in tasks of their own, one per
@@ -296,6 +336,7 @@ typedef struct {
   int gemv_path;          /* the path the plan uses: 1 mma.sync, 2 tcgen05  */
   int schedule;           /* 0 dynamic queue, 1 solidified per-CTA lists    */
   int prefill;            /* 1: created with the prefill option             */
+  int weight_bits;        /* 16 bf16 or 4 (W4A16) projections              */
   int qkv_parts, gateup_parts; /* split-K parts of the QKV and gate/up
                              projections (tensor-core path; 1 otherwise)   */
 } mk_plan_info_t;

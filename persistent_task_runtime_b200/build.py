@@ -16,7 +16,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SOURCES = [os.path.join(HERE, "csrc", f) for f in ("mk_kernel.cu", "mk_api.cu", "mk_layout.cu",
-                                                          "mk_noalloc.cu")]
+                                                          "mk_noalloc.cu", "mk_w4.cu")]
 HEADERS = [os.path.join(HERE, "csrc", "mk_internal.h"), os.path.join(ROOT, "include", "mk.h")]
 OUT_DIR = os.path.join(HERE, "_lib")
 LIB = os.path.join(OUT_DIR, "libmk.so")

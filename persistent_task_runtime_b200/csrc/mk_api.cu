@@ -93,21 +93,38 @@ int validate_weights(const mk_model_config *c, const mk_weights *w) {
   }
   for (int l = 0; l < c->n_layers; ++l) {
     const mk_layer_weights &L = w->layers[l];
-    const void *ps[] = {L.attn_norm, L.wq, L.wk, L.wv, L.wo, L.mlp_norm, L.w_gate, L.w_up, L.w_down};
-    for (const void *p : ps) {
+    const void *ps[] = {L.attn_norm, L.mlp_norm, L.wq, L.wk, L.wv, L.wo, L.w_gate, L.w_up, L.w_down};
+    // (4-bit plans take the projections from w4_layers: only the norms here)
+    const int np = w->w4_layers != nullptr ? 2 : 9;
+    for (int i = 0; i < np; ++i) {
+      const void *p = ps[i];
       if (p == nullptr) return fail(MK_ERR_INVALID_ARG, "layer %d: a weight pointer is NULL", l);
       if (!aligned16(p)) return fail(MK_ERR_INVALID_ARG, "layer %d: weight not 16-byte aligned", l);
     }
+    if (w->w4_layers != nullptr)
+      for (int j = 0; j < 7; ++j) {
+        const void *p = w->w4_layers[l].q[j];
+        if (p == nullptr || !aligned16(p))
+          return fail(MK_ERR_INVALID_ARG, "layer %d: a 4-bit matrix is NULL or not 16-byte aligned", l);
+      }
     if (c->qk_norm && (L.q_norm == nullptr || L.k_norm == nullptr))
       return fail(MK_ERR_INVALID_ARG, "layer %d: q_norm/k_norm NULL with qk_norm on", l);
   }
   return MK_OK;
 }
 
-// Plan options -> layout options (defaults filled in).
-int layout_options(const mk_plan_options *opts, mk::LayoutOptions &lo) {
+// Plan options -> layout options (defaults filled in).  `w` (NULL when
+// describing a plan) says whether the weights are 4-bit.
+int layout_options(const mk_plan_options *opts, mk::LayoutOptions &lo, const mk_weights *w = nullptr) {
   mk_plan_options o{};
   if (opts) o = *opts;
+  if (o.weight_bits != 0 && o.weight_bits != 4 && o.weight_bits != 16)
+    return fail(MK_ERR_INVALID_ARG, "weight_bits %d: 0, 4 or 16", o.weight_bits);
+  const bool have4 = w != nullptr && w->w4_layers != nullptr;
+  if (w != nullptr && o.weight_bits != 0 && (o.weight_bits == 4) != have4)
+    return fail(MK_ERR_INVALID_ARG, "weight_bits %d does not match the weights (w4_layers %s)",
+                o.weight_bits, have4 ? "set" : "NULL");
+  lo.w4 = have4 || (w == nullptr && o.weight_bits == 4);
   if (o.wait_limit_ns < 0) return fail(MK_ERR_INVALID_ARG, "wait_limit_ns < 0");
   lo.max_batch = o.max_batch == 0 ? 1 : o.max_batch;
   lo.page_size = o.kv_page_size == 0 ? 16 : o.kv_page_size;
@@ -142,6 +159,14 @@ void fill_info(const mk::Layout &lay, const mk_model_config &c, mk_plan_info_t &
                        (static_cast<long long>(p.NQKV) * H + static_cast<long long>(H) * c.n_q_heads * d +
                         3LL * F * H) +
                    2LL * V * H;
+  if (p.w4) {   // packed 4-bit projections (codes and scales) + the bf16 LM head
+    const long long per_layer = mk_w4_packed_bytes(p.NQKV - 2 * c.n_kv_heads * d, H) +
+                                2 * mk_w4_packed_bytes(c.n_kv_heads * d, H) +
+                                mk_w4_packed_bytes(H, c.n_q_heads * d) +
+                                2 * mk_w4_packed_bytes(F, H) + mk_w4_packed_bytes(H, F);
+    I.weight_bytes = L * per_layer + 2LL * V * H;
+  }
+  I.weight_bits = p.w4 ? 4 : 16;
   I.events_per_layer = p.ev_per_layer;
   I.attn_slots_per_group = p.attn_spg;
   I.qkv_tasks_per_group = p.qkv_tasks_per_group;
@@ -185,7 +210,7 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   rc = validate_weights(cfg, w);
   if (rc) return rc;
   mk::LayoutOptions lo;
-  rc = layout_options(opts, lo);
+  rc = layout_options(opts, lo, w);
   if (rc) return rc;
 
   int dev = 0, nsm = 0, smem_optin = 0, coop = 0;

@@ -131,6 +131,7 @@ struct Params {
   int n_lm_tasks;
   long long wait_limit_ns;
   int n_out;                          // compute -> storer output buffers in use (<= kOutSlots)
+  int w4;                             // 1: the projections (not the LM head) are packed 4-bit
   int kv_tasks;                       // 1: K/V of the step are appended by T_KVAPP tasks
                                       //    before any attention reads the cache (prefill plans)
   int tile_rows;                      // rows per row tile: 16 (mma.sync) or kTcRows (tcgen05)
@@ -227,6 +228,11 @@ __host__ __device__ inline int row_pitch_bytes(int cols) {
   return ((cols * 2 + 127) / 128) * 128 + 64;
 }
 
+// 4-bit pages: one packed block per 16 rows x 1024 columns
+constexpr int kW4PageBlocks = 4;                   // a page: up to 4096 columns of one row tile
+constexpr int kW4PageBytes = kW4PageBlocks * MK_W4_BLOCK_BYTES;
+__host__ __device__ inline bool is_w4_task(int w4, uint8_t type) { return w4 && type != T_LMHEAD; }
+
 // Staged activation: fp32 rows, pitch rounded to 128 B and offset by 16 B so
 // the fragments of consecutive sequences fall on complementary banks.
 __host__ __device__ inline int x_row_bytes(int cols) { return ((cols * 4 + 127) / 128) * 128 + 16; }
@@ -241,6 +247,7 @@ struct LayoutOptions {
   int gemv_path = 0;            // 0 automatic, 1 mma.sync pages, 2 tcgen05 tiles
   int schedule = 0;             // 0 dynamic ticket queue, 1 solidified per-CTA task lists
   bool prefill = false;         // K/V appended by their own tasks (prompt chunks of one sequence)
+  bool w4 = false;              // 4-bit projections (packed, MK_W4_BLOCK_BYTES blocks)
   int rows_per_task[5] = {0, 0, 0, 0, 0};
   long long wait_limit_ns = 2000000000LL;
   bool debug_unsatisfiable_dep = false;

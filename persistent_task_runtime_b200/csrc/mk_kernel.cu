@@ -762,11 +762,25 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
             ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
             if (!ok) break;
             uint8_t *pg = pages + static_cast<size_t>(pi) * p.page_bytes;
-            if (lane == 0) mbar_arrive_expect_tx(&ctl->full[pi], static_cast<uint32_t>(rv * nc * 2));
-            __syncwarp();
-            if (lane < rv) {
-              const __nv_bfloat16 *src = W + (static_cast<size_t>(row + lane) * geo.K + c0);
-              bulk_load(pg + lane * pitch, src, static_cast<uint32_t>(nc * 2), &ctl->full[pi], pol);
+            if (is_w4_task(p.w4, t.type)) {
+              // 4-bit: the row tile's packed blocks of these columns are
+              // contiguous -- one bulk copy
+              const uint32_t bytes = static_cast<uint32_t>(nc / MK_W4_BLOCK_COLS) * MK_W4_BLOCK_BYTES;
+              const uint8_t *src = reinterpret_cast<const uint8_t *>(W) +
+                                   (static_cast<size_t>(row / 16) * (geo.K / MK_W4_BLOCK_COLS) +
+                                    c0 / MK_W4_BLOCK_COLS) * MK_W4_BLOCK_BYTES;
+              if (lane == 0) {
+                mbar_arrive_expect_tx(&ctl->full[pi], bytes);
+                bulk_load(pg, src, bytes, &ctl->full[pi], pol);
+              }
+              __syncwarp();
+            } else {
+              if (lane == 0) mbar_arrive_expect_tx(&ctl->full[pi], static_cast<uint32_t>(rv * nc * 2));
+              __syncwarp();
+              if (lane < rv) {
+                const __nv_bfloat16 *src = W + (static_cast<size_t>(row + lane) * geo.K + c0);
+                bulk_load(pg + lane * pitch, src, static_cast<uint32_t>(nc * 2), &ctl->full[pi], pol);
+              }
             }
             issued |= 1u << pi;
             last_par = (last_par & ~(1u << pi)) | (pe_par << pi);
@@ -895,6 +909,61 @@ __device__ __forceinline__ void page_mma(float (&acc)[NN][4], const uint8_t *pg,
         xv = *reinterpret_cast<const uint4 *>(xs + b * xpitch + (xcol0 + c) * 4 + xhalf);
       mma_bf16(acc[nt], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
       mma_bf16(c1[nt], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NN; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] += c1[nt][e];
+}
+
+// One 4-bit page (a 16-row tile over nc columns, nc / 1024 packed blocks)
+// against the staged activation.  The lane (g, q) reads, per 32-column
+// group, 8 bytes: the codes of row g and of row g + 8 at columns 8 q .. 8 q + 7
+// (the packed order), and the two rows' scales of the group's 128 columns.
+// A code pair becomes a bf16 pair exactly: OR-ing the nibble into the bits of
+// 128.0 gives 128 + code, minus 136 gives code - 8 (small integers are exact
+// in bf16), and one bf16 multiply by the scale rounds the product once, as
+// the 4-bit format defines the weight.  Then the same mma as a bf16 page.
+template <int NN>
+__device__ __forceinline__ void page_mma_w4(float (&acc)[NN][4], const uint8_t *pg, int nc,
+                                            const uint8_t *xs, int xpitch, int xcol0, int B,
+                                            int warp, int lane) {
+  const int g = lane >> 2, q = lane & 3;
+  const int groups = nc >> 5;
+  const int xhalf = (g >> 2) * 16;   // 0: hi block, 16: lo block
+  const __nv_bfloat162 k136 = __floats2bfloat162_rn(136.f, 136.f);
+  float c1[NN][4];
+#pragma unroll
+  for (int nt = 0; nt < NN; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c1[nt][e] = 0.f;
+#pragma unroll 2
+  for (int grp = warp; grp < groups; grp += kComputeWarps) {
+    const int blk = grp >> 5, sub = grp & 31;
+    const uint8_t *bp = pg + blk * MK_W4_BLOCK_BYTES;
+    const uint2 cw = *reinterpret_cast<const uint2 *>(bp + 256 + sub * 256 + lane * 8);
+    const __nv_bfloat16 *scl = reinterpret_cast<const __nv_bfloat16 *>(bp) + (sub >> 2) * 16;
+    const __nv_bfloat162 s0 = __bfloat162bfloat162(scl[g]);
+    const __nv_bfloat162 s1 = __bfloat162bfloat162(scl[g + 8]);
+    uint32_t wa[4], wb[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t na = ((cw.x >> (4 * k)) & 0x000F000Fu) | 0x43004300u;
+      const uint32_t nb = ((cw.y >> (4 * k)) & 0x000F000Fu) | 0x43004300u;
+      const __nv_bfloat162 va = __hmul2(__hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&na), k136), s0);
+      const __nv_bfloat162 vb = __hmul2(__hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&nb), k136), s1);
+      wa[k] = *reinterpret_cast<const uint32_t *>(&va);
+      wb[k] = *reinterpret_cast<const uint32_t *>(&vb);
+    }
+    const int c = grp * 32 + q * 8;
+#pragma unroll
+    for (int nt = 0; nt < NN; ++nt) {
+      const int b = nt * 4 + (g & 3);
+      uint4 xv = make_uint4(0, 0, 0, 0);
+      if (b < B) xv = *reinterpret_cast<const uint4 *>(xs + b * xpitch + (xcol0 + c) * 4 + xhalf);
+      mma_bf16(acc[nt], wa[0], wb[0], wa[1], wb[1], xv.x, xv.y);
+      mma_bf16(c1[nt], wa[2], wb[2], wa[3], wb[3], xv.z, xv.w);
     }
   }
 #pragma unroll
@@ -1148,12 +1217,17 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
           continue;
         }
         const uint8_t *pg = pages + static_cast<size_t>(st.pi) * p.page_bytes;
+        const bool w4 = is_w4_task(p.w4, t.type);
         switch (m) {
-#define MK_PAGE_CASE(M)                                                                      \
-  case M:                                                                                    \
-    if (M < MT)                                                                              \
-      page_mma<NN>(acc[M < MT ? M : 0], pg, pitch, nc, xs, xstride * 4, c0 - xc0, B, warp, \
-                   lane);                                                                    \
+#define MK_PAGE_CASE(M)                                                                        \
+  case M:                                                                                      \
+    if (M < MT) {                                                                              \
+      if (w4)                                                                                  \
+        page_mma_w4<NN>(acc[M < MT ? M : 0], pg, nc, xs, xstride * 4, c0 - xc0, B, warp, lane); \
+      else                                                                                     \
+        page_mma<NN>(acc[M < MT ? M : 0], pg, pitch, nc, xs, xstride * 4, c0 - xc0, B, warp,   \
+                     lane);                                                                    \
+    }                                                                                          \
     break;
           MK_PAGE_CASE(0)
           MK_PAGE_CASE(1)

@@ -164,8 +164,17 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
                  "n_q_heads*head_dim multiples of 64");
   if (o.gemv_path == 2 && o.o_split)
     return lfail(err, MK_ERR_INVALID_ARG, "o_split is an option of the mma.sync path");
-  const bool tc = o.gemv_path == 2 || (o.gemv_path == 0 && tc_ok && !o.o_split &&
-                                       maxB >= kTcAutoBatch);
+  if (o.w4) {
+    if (H % MK_W4_BLOCK_COLS || F % MK_W4_BLOCK_COLS || (Hq * d) % MK_W4_BLOCK_COLS)
+      return lfail(err, MK_ERR_UNSUPPORTED,
+                   "4-bit weights need hidden, ffn and n_q_heads*head_dim multiples of %d",
+                   MK_W4_BLOCK_COLS);
+    if (o.gemv_path == 2)
+      return lfail(err, MK_ERR_UNSUPPORTED, "4-bit weights run on the mma.sync GEMV path");
+    if (o.o_split) return lfail(err, MK_ERR_INVALID_ARG, "o_split is not available with 4-bit weights");
+  }
+  const bool tc = !o.w4 && (o.gemv_path == 2 || (o.gemv_path == 0 && tc_ok && !o.o_split &&
+                                                  maxB >= kTcAutoBatch));
   if (tc) {
     for (int i = 0; i < 5; ++i)
       if (o.rows_per_task[i] != 0)
@@ -209,7 +218,8 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   int n_ksplit = F > kx_limit ? cdiv(F, kx_limit) : 1;
   int kchunk_ffn = F;
   if (n_ksplit > 1) {
-    const int unit = (R_gu % 32 == 0) ? R_gu : 2 * R_gu;   // multiple of 32 and of R_gu
+    // multiple of 32 and of R_gu (4-bit: of the 1024-column packed blocks)
+    const int unit = o.w4 ? MK_W4_BLOCK_COLS : ((R_gu % 32 == 0) ? R_gu : 2 * R_gu);
     kchunk_ffn = align_up_i(cdiv(F, n_ksplit), unit);
     n_ksplit = cdiv(F, kchunk_ffn);
     if (n_ksplit < 2) {
@@ -329,9 +339,37 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   // largest ring any width gives with at least 3 pages; wider pages mean
   // fewer hand-offs per byte.  Failing 3 pages, the most pages.
   std::vector<Geom> cands;
-  for (int cand = colcap; cand >= 32 && !tc; cand -= (cand > 256 ? 256 : 32)) {
+  for (int cand = colcap; cand >= 32 && !tc && !o.w4; cand -= (cand > 256 ? 256 : 32)) {
     Geom g{};
     if (geometry(cand, g)) cands.push_back(g);
+  }
+  // 4-bit projections: a page is one packed row tile over up to 4096 columns
+  // (4 blocks, 33 KB; fewer blocks when a page-wide activation chunk of every
+  // sequence would not fit the staging area); the bf16 LM head streams in
+  // pages of 16 rows that fit the same size
+  for (int nb = kW4PageBlocks; nb >= 1 && o.w4 && cands.empty(); nb /= 2) {
+    Geom g{};
+    const int kw = nb * MK_W4_BLOCK_COLS;
+    g.kp[K_HID] = std::min(H, kw);
+    g.kp[K_ATT] = std::min(Hq * d, kw);
+    g.kp[K_FFN] = std::min(kchunk_ffn, kw);
+    g.page_bytes = nb * MK_W4_BLOCK_BYTES;
+    g.kp[K_LM] = 32;
+    while (16 * row_pitch_bytes(g.kp[K_LM] + 32) <= g.page_bytes && g.kp[K_LM] + 32 <= kMaxPageCols)
+      g.kp[K_LM] += 32;
+    const int kp_big = std::max(std::max(g.kp[0], g.kp[1]), g.kp[2]);
+    const int x_chunk = maxB * x_row_bytes(kp_big);
+    if (x_chunk <= kXWholeMax) {
+      const int x_cap = x_whole <= kXWholeMax ? std::max(x_whole, x_chunk) : x_chunk;
+      g.tpp = std::min((g.page_bytes / (4 * d)) / P * P, 16 * P);
+      const int att_need = G * d * 4 + std::max((G * g.tpp + 3 * kMaxGroup) * 4 + 2 * d * 2,
+                                                (2 * max_chunks * G + 2 * G) * 4);
+      g.x_cap = std::max(x_cap, att_need);
+      g.off_pages = align_up_i(off_x + g.x_cap, 1024);
+      g.n_pages = std::min(kMaxPages, (smem_max - g.off_pages) / g.page_bytes);
+      g.ring = g.n_pages * g.page_bytes;
+      if (g.tpp >= P && g.n_pages >= 2) cands.push_back(g);
+    }
   }
   if (tc) {
     // two activation chunk buffers (also the attention scratch), then the
@@ -407,6 +445,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   p.wait_limit_ns = o.wait_limit_ns;
   p.n_ffn_parts = n_ksplit;
   p.chunk_seq = -1;   // decode steps (a prompt chunk sets its sequence)
+  p.w4 = o.w4 ? 1 : 0;
   p.n_out = n_out;
   p.tile_rows = tc ? kTcRows : 16;
   p.tc = tc ? 1 : 0;
@@ -669,10 +708,14 @@ void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vect
       t.gain = bf(w.final_norm);
       continue;
     }
-    const mk_layer_weights &lw = w.layers[t.layer < c.n_layers ? t.layer : 0];
+    const int li = t.layer < c.n_layers ? t.layer : 0;
+    const mk_layer_weights &lw = w.layers[li];
+    // 4-bit plans: the projections' packed matrices instead of the bf16 ones
+    const mk_w4_layer_weights *q4 = w.w4_layers != nullptr ? &w.w4_layers[li] : nullptr;
+    auto mat = [&](int j, const void *bf16_ptr) { return bf(q4 != nullptr ? q4->q[j] : bf16_ptr); };
     switch (t.type) {
       case T_QKV:
-        t.w0 = bf(t.aux == 0 ? lw.wq : (t.aux == 1 ? lw.wk : lw.wv));
+        t.w0 = t.aux == 0 ? mat(0, lw.wq) : (t.aux == 1 ? mat(1, lw.wk) : mat(2, lw.wv));
         t.gain = bf(lw.attn_norm);
         break;
       case T_ATTN:
@@ -681,16 +724,16 @@ void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vect
         t.w1 = bf(lw.k_norm);
         break;
       case T_OPROJ:
-        t.w0 = bf(lw.wo);
+        t.w0 = mat(3, lw.wo);
         t.w1 = bf(lw.mlp_norm);   // the gain of the input it produces (gate/up's)
         break;
       case T_GATEUP:
-        t.w0 = bf(lw.w_gate);
-        t.w1 = bf(lw.w_up);
+        t.w0 = mat(4, lw.w_gate);
+        t.w1 = mat(5, lw.w_up);
         t.gain = bf(lw.mlp_norm);
         break;
       case T_DOWN:
-        t.w0 = bf(lw.w_down);
+        t.w0 = mat(6, lw.w_down);
         // the gain of the input it produces: the next layer's QKV, or the LM head
         t.w1 = bf(t.layer + 1 < c.n_layers ? w.layers[t.layer + 1].attn_norm : w.final_norm);
         break;

@@ -60,7 +60,10 @@ std::vector<const void *> weight_ptrs(const mk_model_config &c, const mk_weights
     const mk_layer_weights &s = w.layers[l];
     v.insert(v.end(), {s.attn_norm, s.wq, s.wk, s.wv, s.q_norm, s.k_norm, s.wo, s.mlp_norm,
                        s.w_gate, s.w_up, s.w_down});
+    if (w.w4_layers != nullptr)
+      for (int j = 0; j < 7; ++j) v.push_back(w.w4_layers[l].q[j]);
   }
+  v.push_back(w.w4_layers != nullptr ? w.w4_layers : nullptr);
   return v;
 }
 
@@ -105,11 +108,17 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
     if (q == nullptr || !aligned16(q)) return nfail(MK_ERR_INVALID_ARG, "NULL or unaligned pointer");
   for (int l = 0; l < L; ++l) {
     const mk_layer_weights &s = w->layers[l];
-    const void *ps[] = {s.attn_norm, s.wq, s.wk, s.wv, s.wo, s.mlp_norm, s.w_gate, s.w_up,
-                        s.w_down, a->kv->k_pages[l], a->kv->v_pages[l]};
-    for (const void *q : ps)
-      if (q == nullptr || !aligned16(q))
+    const void *ps[] = {s.attn_norm, s.mlp_norm, a->kv->k_pages[l], a->kv->v_pages[l], s.wq,
+                        s.wk, s.wv, s.wo, s.w_gate, s.w_up, s.w_down};
+    // (4-bit weights: the projections come from w4_layers)
+    const int np = w->w4_layers != nullptr ? 4 : 11;
+    for (int i = 0; i < np; ++i)
+      if (ps[i] == nullptr || !aligned16(ps[i]))
         return nfail(MK_ERR_INVALID_ARG, "NULL or unaligned weight / KV pointer");
+    if (w->w4_layers != nullptr)
+      for (int j = 0; j < 7; ++j)
+        if (w->w4_layers[l].q[j] == nullptr || !aligned16(w->w4_layers[l].q[j]))
+          return nfail(MK_ERR_INVALID_ARG, "NULL or unaligned 4-bit matrix");
     if (c.qk_norm && (s.q_norm == nullptr || s.k_norm == nullptr))
       return nfail(MK_ERR_INVALID_ARG, "q_norm/k_norm NULL with qk_norm on");
   }
@@ -151,6 +160,7 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
     mk::LayoutOptions lo;
     lo.max_batch = B;
     lo.page_size = P;
+    lo.w4 = w->w4_layers != nullptr;
     std::string err;
     const int rc = mk::build_layout(c, lo, nsm, smem_optin, up.lay, err);
     if (rc) return nfail(rc, err.c_str());

@@ -38,7 +38,8 @@ ERROR_NAMES = {MK_OK: "MK_OK", MK_ERR_INVALID_ARG: "MK_ERR_INVALID_ARG",
 EXPORTS = ["mk_plan_create", "mk_plan_create_ex", "mk_decode_step", "mk_decode_step_ex",
            "mk_decode_step_host", "mk_plan_status", "mk_plan_error_info", "mk_plan_reset",
            "mk_plan_info", "mk_last_error", "mk_plan_destroy", "mk_decode_step_noalloc",
-           "mk_plan_describe", "mk_plan_describe_schedule", "mk_prefill_chunk"]
+           "mk_plan_describe", "mk_plan_describe_schedule", "mk_prefill_chunk",
+           "mk_w4_packed_bytes", "mk_w4_pack"]
 
 #: bytes of the library's static scratch array used by mk_decode_step_noalloc
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -56,9 +57,14 @@ class mk_layer_weights(C.Structure):
                                            "wo", "mlp_norm", "w_gate", "w_up", "w_down")]
 
 
+class mk_w4_layer_weights(C.Structure):
+    _fields_ = [("q", C.c_void_p * 7)]
+
+
 class mk_weights(C.Structure):
     _fields_ = [("embed", C.c_void_p), ("layers", C.POINTER(mk_layer_weights)),
-                ("final_norm", C.c_void_p), ("lm_head", C.c_void_p)]
+                ("final_norm", C.c_void_p), ("lm_head", C.c_void_p),
+                ("w4_layers", C.POINTER(mk_w4_layer_weights))]
 
 
 class mk_kv_cache(C.Structure):
@@ -72,7 +78,7 @@ class mk_plan_options(C.Structure):
                 ("wait_limit_ns", C.c_int64), ("rows_per_task", C.c_int * 5),
                 ("debug_unsatisfiable_dep", C.c_int), ("max_page_cols", C.c_int),
                 ("o_split", C.c_int), ("gemv_path", C.c_int), ("schedule", C.c_int),
-                ("prefill", C.c_int)]
+                ("weight_bits", C.c_int), ("prefill", C.c_int)]
 
 
 class mk_step_args(C.Structure):
@@ -98,7 +104,7 @@ class mk_plan_info_t(C.Structure):
                 ("qkv_tasks_per_group", C.c_int), ("ffn_parts", C.c_int),
                 ("ffn_part_cols", C.c_int), ("o_parts", C.c_int), ("o_part_cols", C.c_int),
                 ("gemv_path", C.c_int), ("schedule", C.c_int), ("prefill", C.c_int),
-                ("qkv_parts", C.c_int),
+                ("weight_bits", C.c_int), ("qkv_parts", C.c_int),
                 ("gateup_parts", C.c_int)]
 
 
@@ -134,6 +140,10 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
     lib.mk_plan_describe_schedule.restype = C.c_int
     lib.mk_prefill_chunk.argtypes = [P, C.POINTER(mk_prefill_args), P]
     lib.mk_prefill_chunk.restype = C.c_int
+    lib.mk_w4_packed_bytes.argtypes = [C.c_int, C.c_int]
+    lib.mk_w4_packed_bytes.restype = C.c_int64
+    lib.mk_w4_pack.argtypes = [P, P, C.c_int, C.c_int, P]
+    lib.mk_w4_pack.restype = C.c_int
     lib.mk_last_error.restype = C.c_char_p
     lib.mk_last_error.argtypes = []
     lib.mk_plan_destroy.argtypes = [P]
@@ -211,7 +221,7 @@ def _config(cfg: Dict, max_seq_len: int) -> mk_model_config:
 def describe(cfg: Dict, max_batch: int = 1, page_size: int = 16, max_seq_len: int = 4096,
              num_sms: int = 148, smem_optin: int = 232448, rows_per_task=(0, 0, 0, 0, 0),
              max_page_cols: int = 0, o_split: bool = False, gemv_path: int = 0,
-             schedule: int = 0, prefill: bool = False):
+             schedule: int = 0, prefill: bool = False, weight_bits: int = 0):
     """The plan mk_plan_create_ex would build, without a GPU: (info, task records).
 
     The task records are a numpy structured array (TASK_RECORD_DTYPE)."""
@@ -219,7 +229,7 @@ def describe(cfg: Dict, max_batch: int = 1, page_size: int = 16, max_seq_len: in
     lib = load_library()
     c = _config(cfg, max_seq_len)
     opts = mk_plan_options(max_batch, page_size, 0, 0, (C.c_int * 5)(*rows_per_task), 0,
-                           max_page_cols, 1 if o_split else 0, gemv_path, schedule,
+                           max_page_cols, 1 if o_split else 0, gemv_path, schedule, weight_bits,
                            1 if prefill else 0)
     info = mk_plan_info_t()
     _check(lib.mk_plan_describe(C.byref(c), C.byref(opts), num_sms, smem_optin, C.byref(info),
@@ -246,6 +256,53 @@ def describe_schedule(cfg: Dict, n_tasks: int, max_batch: int = 1, page_size: in
     return out
 
 
+W4_MATRIX_NAMES = ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down")
+
+
+def w4_pack(codes: torch.Tensor, scales: torch.Tensor) -> torch.Tensor:
+    """mk_w4_pack on the host: codes uint8 [rows, cols] (0..15), scales bf16
+    [rows, cols/128] -> the packed uint8 buffer the kernel streams (CPU)."""
+    lib = load_library()
+    rows, cols = codes.shape
+    n = lib.mk_w4_packed_bytes(rows, cols)
+    if n < 0:
+        raise MkError(MK_ERR_INVALID_ARG, f"unsupported 4-bit matrix {rows} x {cols}")
+    c = codes.detach().to("cpu", torch.uint8).contiguous()
+    sc = scales.detach().to("cpu", torch.bfloat16).contiguous()
+    out = torch.empty(n, dtype=torch.uint8)
+    _check(lib.mk_w4_pack(c.data_ptr(), sc.data_ptr(), rows, cols, out.data_ptr()))
+    return out
+
+
+def _weight_structs(weights: Dict, L: int, device=None):
+    """(mk_weights, keep-alive list): bf16 layers, plus packed 4-bit matrices
+    on `device` when the layers carry ``w4`` (synth.make_w4_weights)."""
+    keep = []
+    lw = (mk_layer_weights * L)()
+    w4 = "w4" in weights["layers"][0]
+    for l, w in enumerate(weights["layers"]):
+        lw[l] = mk_layer_weights(*[_ptr(w.get(k)) for k in (
+            "attn_norm", "wq", "wk", "wv", "q_norm", "k_norm", "wo", "mlp_norm",
+            "w_gate", "w_up", "w_down")])
+    keep.append(lw)
+    w4l = None
+    if w4:
+        dev = device or weights["embed"].device
+        w4l = (mk_w4_layer_weights * L)()
+        for l, w in enumerate(weights["layers"]):
+            ptrs = []
+            for name in W4_MATRIX_NAMES:
+                codes, scales = w["w4"][name]
+                packed = w4_pack(codes, scales).to(dev)
+                keep.append(packed)
+                ptrs.append(packed.data_ptr())
+            w4l[l] = mk_w4_layer_weights((C.c_void_p * 7)(*ptrs))
+        keep.append(w4l)
+    mw = mk_weights(_ptr(weights["embed"]), lw, _ptr(weights["final_norm"]),
+                    _ptr(weights["lm_head"]), w4l)
+    return mw, keep
+
+
 class Plan:
     """A decode plan over caller-owned bf16 weights (see include/mk.h)."""
 
@@ -260,17 +317,10 @@ class Plan:
         self._c = _config(cfg, max_seq_len)
         L = cfg["n_layers"]
         self._weights = weights  # keep the tensors alive
-        lw = (mk_layer_weights * L)()
-        for l, w in enumerate(weights["layers"]):
-            lw[l] = mk_layer_weights(*[_ptr(w[k]) for k in (
-                "attn_norm", "wq", "wk", "wv", "q_norm", "k_norm", "wo", "mlp_norm",
-                "w_gate", "w_up", "w_down")])
-        self._lw = lw
-        self._w = mk_weights(_ptr(weights["embed"]), lw, _ptr(weights["final_norm"]),
-                             _ptr(weights["lm_head"]))
+        self._w, self._keep = _weight_structs(weights, L)
         opts = mk_plan_options(max_batch, page_size, num_ctas, wait_limit_ns,
                                (C.c_int * 5)(*rows_per_task), 1 if debug_unsatisfiable_dep else 0,
-                               max_page_cols, 1 if o_split else 0, gemv_path, schedule,
+                               max_page_cols, 1 if o_split else 0, gemv_path, schedule, 0,
                                1 if prefill else 0)
         h = C.c_void_p()
         _check(lib.mk_plan_create_ex(C.byref(self._c), C.byref(self._w), C.byref(opts),
@@ -395,11 +445,4 @@ class ModelRef:
         self._c = _config(cfg, max_seq_len)
         L = cfg["n_layers"]
         self._weights = weights
-        lw = (mk_layer_weights * L)()
-        for l, w in enumerate(weights["layers"]):
-            lw[l] = mk_layer_weights(*[_ptr(w[k]) for k in (
-                "attn_norm", "wq", "wk", "wv", "q_norm", "k_norm", "wo", "mlp_norm",
-                "w_gate", "w_up", "w_down")])
-        self._lw = lw
-        self._w = mk_weights(_ptr(weights["embed"]), lw, _ptr(weights["final_norm"]),
-                             _ptr(weights["lm_head"]))
+        self._w, self._keep = _weight_structs(weights, L)

@@ -77,7 +77,9 @@ class Pair:
         self.cfg = cfg
         self.B = max_batch
         self.ocfg = oracle_cfg(cfg)
-        self.W = oracle.Weights(weights, keep_f64=keep_f64)
+        # (4-bit layers: the oracle dequantizes them by the format's definition)
+        wcls = oracle.W4Weights if "w4" in weights["layers"][0] else oracle.Weights
+        self.W = wcls(weights, keep_f64=keep_f64)
         msl = max_seq_len or max(capacity)
         self.plan = mk.Plan(cfg, weights, max_batch=max_batch, page_size=page,
                             max_seq_len=msl, **plan_kw)

@@ -24,7 +24,7 @@ def lib():
 
 def header_functions():
     src = open(HEADER).read()
-    return sorted(set(re.findall(r"\b(mk_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(mk_[a-z_0-9]+)\s*\(", src)))
 
 
 def test_header_functions_are_the_binding_exports():
