@@ -72,6 +72,9 @@ struct mk_plan {
   mk::Layout lay;           // tasks, per-operator ranges, workspace layout
   void *d_tasks = nullptr, *d_rope = nullptr, *d_ws = nullptr, *d_maps = nullptr;
   void *d_sched = nullptr;   // solidified schedule: offsets [grid + 1], then task indices
+  void *d_kvmaps = nullptr;  // tensor maps of the KV cache (2 per layer) for the attention
+  std::vector<const void *> kv_key;        // the KV cache those maps describe
+  std::vector<unsigned char> kv_maps_host;
   uint32_t *d_sync = nullptr;
   size_t sync_words = 0;
   int32_t *d_host_ids = nullptr, *d_host_pos = nullptr, *d_host_out = nullptr;
@@ -274,6 +277,11 @@ int mk_plan_create_ex(const mk_model_config *cfg, const mk_weights *w, const mk_
   p.embed = static_cast<const __nv_bfloat16 *>(w->embed);
   p.rope_cs = static_cast<const float2 *>(plan->d_rope);
   p.tmaps = plan->d_maps;
+  if (p.attn_mma) {
+    e = cudaMalloc(&plan->d_kvmaps, static_cast<size_t>(2 * cfg->n_layers) * 128);
+    if (e != cudaSuccess) return cleanup_fail(fail(MK_ERR_CUDA, "KV maps: %s", cudaGetErrorString(e)));
+    p.kvmaps = plan->d_kvmaps;
+  }
   if (plan->d_sched != nullptr) {
     p.sched_off = static_cast<const int *>(plan->d_sched);
     p.sched = p.sched_off + lay.sched_off.size();
@@ -309,6 +317,29 @@ static int validate_kv(const mk_plan *plan, const mk_kv_cache *kv) {
 }
 
 namespace {
+
+// The attention copies K/V pages with TMA tensor copies: the tensor maps of
+// the step's KV cache, encoded when the cache (its pointers or page count)
+// differs from the previous step's and copied to the device on the step's
+// stream ahead of the launch.
+int ensure_kv_maps(mk_plan *plan, const mk_kv_cache *kv, cudaStream_t s) {
+  if (!plan->base.attn_mma) return MK_OK;
+  std::vector<const void *> key;
+  key.reserve(2 * plan->cfg.n_layers + 1);
+  key.push_back(reinterpret_cast<const void *>(static_cast<intptr_t>(kv->num_pages)));
+  for (int l = 0; l < plan->cfg.n_layers; ++l) {
+    key.push_back(kv->k_pages[l]);
+    key.push_back(kv->v_pages[l]);
+  }
+  if (key == plan->kv_key) return MK_OK;
+  std::string err;
+  const int rc = mk::encode_kv_maps(plan->cfg, *kv, plan->base.page_size, plan->kv_maps_host, err);
+  if (rc) return fail(rc, "%s", err.c_str());
+  MK_CUDA(cudaMemcpyAsync(plan->d_kvmaps, plan->kv_maps_host.data(), plan->kv_maps_host.size(),
+                          cudaMemcpyHostToDevice, s));
+  plan->kv_key = std::move(key);
+  return MK_OK;
+}
 
 void release_graph(OpGraph &g) {
   if (g.exec != nullptr) cudaGraphExecDestroy(g.exec);
@@ -403,6 +434,8 @@ int mk_decode_step_ex(mk_plan *plan, const mk_step_args *a, void *stream) {
     return fail(MK_ERR_INVALID_ARG, "graph mode needs a created stream, not the legacy default stream");
   int rc = validate_kv(plan, a->kv);
   if (rc) return rc;
+  rc = ensure_kv_maps(plan, a->kv, static_cast<cudaStream_t>(stream));
+  if (rc) return rc;
 
   Params p = plan->base;
   plan->epoch += 1;
@@ -476,6 +509,8 @@ int mk_prefill_chunk(mk_plan *plan, const mk_prefill_args *a, void *stream) {
   if (!a->with_lm_head && a->d_out_logits != nullptr)
     return fail(MK_ERR_INVALID_ARG, "d_out_logits needs with_lm_head");
   int rc = validate_kv(plan, a->kv);
+  if (rc) return rc;
+  rc = ensure_kv_maps(plan, a->kv, static_cast<cudaStream_t>(stream));
   if (rc) return rc;
   Params p = plan->base;
   plan->epoch += 1;
@@ -656,6 +691,7 @@ void mk_plan_destroy(mk_plan *plan) {
   cudaFree(plan->d_rope);
   cudaFree(plan->d_maps);
   cudaFree(plan->d_sched);
+  cudaFree(plan->d_kvmaps);
   cudaFree(plan->d_ws);
   cudaFree(plan->d_sync);
   cudaFree(plan->d_host_ids);

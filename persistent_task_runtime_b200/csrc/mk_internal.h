@@ -131,6 +131,9 @@ struct Params {
   int n_lm_tasks;
   long long wait_limit_ns;
   int n_out;                          // compute -> storer output buffers in use (<= kOutSlots)
+  int attn_mma;                       // 1: attention on mma.sync tiles over swizzled K/V pages
+                                      //    copied by TMA tensor copies (head_dim 64 or 128)
+  const void *kvmaps;                 // CUtensorMap[2 L]: K then V of each layer (attn_mma)
   int w4;                             // 1: the projections (not the LM head) are packed 4-bit
   int kv_tasks;                       // 1: K/V of the step are appended by T_KVAPP tasks
                                       //    before any attention reads the cache (prefill plans)
@@ -293,5 +296,11 @@ cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative,
 // Allow the kernel the device's opt-in shared memory (capped at kMaxSmem).
 cudaError_t configure_kernel(int smem_optin);
 void set_last_error(const char *msg);  // message returned by mk_last_error()
+
+// Tensor maps of a KV cache for the mma.sync attention: per layer, K then V,
+// each a 2-D map over [num_pages * n_kv_heads * page, head_dim] bf16 with
+// boxes of 64 dims x page rows, 128-byte swizzle.  Needs the CUDA driver.
+int encode_kv_maps(const mk_model_config &c, const mk_kv_cache &kv, int page_size,
+                   std::vector<unsigned char> &out, std::string &err);
 
 }  // namespace mk

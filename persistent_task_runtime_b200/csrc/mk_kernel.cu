@@ -819,7 +819,26 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
         if (lane == 0) mbar_arrive_expect_tx(&ctl->full[pi], 2u * nkv * kvpage_bytes);
         __syncwarp();
         const int j = lane & 15;
-        if (j < nkv) {
+        if (p.attn_mma) {
+          // TMA tensor copies, 64 dims x P tokens per box, 128-byte swizzle:
+          // the layout the attention's ldmatrix fragment loads read without
+          // bank conflicts
+          const int na = d / 64;
+          const uint8_t *maps = static_cast<const uint8_t *>(p.kvmaps);
+          for (int idx = lane; idx < nkv * 2 * na; idx += 32) {
+            const int jj = idx / (2 * na), kvi = (idx / na) & 1, a = idx % na;
+            int ph = kv_phys_page(p, info.b, tok0 / P + jj);
+            if (ph < 0) {
+              raise_error(p, MK_ERR_RANGE, static_cast<uint32_t>(tix), 0xfffffffdu,
+                          static_cast<uint32_t>(info.b));
+              ph = 0;  // keep the copy in bounds; the step is being abandoned
+            }
+            uint8_t *dst = pg + (kvi ? static_cast<size_t>(p.tpp) * d * 2 : 0) +
+                           static_cast<size_t>(jj) * kvpage_bytes + a * (P * 128);
+            tma_load_2d(dst, maps + static_cast<size_t>(2 * l + kvi) * 128, a * 64,
+                        (ph * p.Hkv + info.g) * P, &ctl->full[pi], pol);
+          }
+        } else if (j < nkv) {
           int ph = kv_phys_page(p, info.b, tok0 / P + j);
           if (ph < 0) {
             raise_error(p, MK_ERR_RANGE, static_cast<uint32_t>(tix), 0xfffffffdu,
@@ -1741,90 +1760,27 @@ __device__ __forceinline__ void comb_batch(const float *ph, size_t cstride, int 
   M = Mb;
 }
 
-// Attention for one chunk of one (sequence, KV head): scores for the G query
-// heads over the chunk's tokens, softmax statistics, and the unnormalised
-// P.V, all in three parallel phases per shared-memory page:
-//   1. thread <- (token, head): full dot product q.k over d, reading the
-//      8-element column blocks in a rotated order (block (c + t) mod d/8) so
-//      the 32 lanes of a warp hit distinct banks;
-//   2. warp <- head: running max m, rescale factor, p = 2^(s - m), running sum;
-//   3. thread <- (head, 4 columns of d): acc = acc * rescale + sum_t p v.
-// Scores are in log2 units (q is pre-scaled by log2(e)/sqrt(d)).
+// The attention scratch in the staging area (see attn_task).
+struct AttnSmem {
+  float *qs, *sc, *mst, *lst, *cor;
+  __nv_bfloat16 *kvcur;
+};
+
+// The chunk's pages on the CUDA cores (head_dim 32, or a plan without the
+// tensor-map copies): three parallel phases per page, see attn_task; writes
+// the chunk's unnormalised partial sums to `part` ([G][D + 4]).
 template <int D>
-__device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
-                          ComputeState &st, float *out, int ctid) {
-  const Task &t = S.t;
+__device__ bool attn_pages_cuda(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
+                                ComputeState &st, const AttnSmem &A, bool own_cur, int cur,
+                                float *part, int ctid) {
   const int warp = ctid >> 5, lane = ctid & 31;
-  const int G = p.G, l = t.layer;
-  const int b = S.b, g = S.g;
-  constexpr int NB = D / 8;                 // 8-element column blocks per row
-  constexpr int Q4 = D / 4;                 // 4-column slices per head
+  const int G = p.G;
+  constexpr int NB = D / 8;
+  constexpr int Q4 = D / 4;
   constexpr int MAXP = (kMaxGroup * Q4 + kComputeThreads - 1) / kComputeThreads;
-  float *qs = reinterpret_cast<float *>(smem + p.off_x);   // [G][D]
-  float *sc = qs + G * D;                                   // [G][tpp] scores, then p
-  float *mst = sc + G * p.tpp;                              // [G] running max
-  float *lst = mst + kMaxGroup;                             // [G] running sum
-  float *cor = lst + kMaxGroup;                             // [G] rescale of this page
-  __nv_bfloat16 *kvcur = reinterpret_cast<__nv_bfloat16 *>(cor + kMaxGroup);  // [2][D] K, V at pos
-  st.xkey = 0xffffffffu;                                    // staging area reused
-
-  {
-    const uint32_t ev = static_cast<uint32_t>(ev_attn_input(p, l, g));
-    bool okl = true;
-    if (ctid == 0) okl = wait_event(p, ctl, ev, static_cast<uint32_t>(attn_input_count(p)), S.idx);
-    if (!st.gs.share(ctl, ctid, okl)) return false;
-    if (ctid == 0) trace_mark(p, S.idx, 4);
-  }
-  // From this step's raw projections, one warp per head: the G query heads
-  // (QK-norm, RoPE, pre-scaled by log2(e)/sqrt(d) for the exp2 softmax) and,
-  // in the chunk that holds the current position, K (QK-norm, RoPE) and V of
-  // the current token, rounded to bf16 and appended to the cache.
-  const int P = p.page_size;
-  const int cur = row_pos(p, b);
-  // (in a plan whose K/V tasks append every row's K/V first, the cache
-  // already holds the current token's)
-  const bool own_cur = !p.kv_tasks && cur >= S.t0 && cur < S.t1;
-  {
-    const float qscale = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;
-    // a position outside 0..max_pos-1 is reported by the embedding task; the
-    // table row stays in range regardless
-    const int cpos = cur < 0 ? 0 : (cur >= p.max_pos ? p.max_pos - 1 : cur);
-    const float2 *cs = p.rope_cs + static_cast<size_t>(cpos) * (D / 2);
-    const float *raw = p.qkv + static_cast<size_t>(b) * p.NQKV;
-    const int nh = G + (own_cur ? 2 : 0);
-    for (int h = warp; h < nh; h += kComputeWarps) {
-      const int mat = h < G ? 0 : h - G + 1;   // 0 q, 1 k, 2 v
-      const int col = mat == 0 ? (g * G + h) * D
-                               : (mat == 1 ? (p.Hq + g) * D : (p.Hq + p.Hkv + g) * D);
-      float v[4];
-      head_norm_rope<D>(raw + col, mat == 0 ? t.w0 : t.w1, p.qk_norm != 0 && mat != 2,
-                        mat != 2, cs, p.eps, lane, v);
-      if (lane < D / 4) {
-        const int e0 = lane * 4;
-        if (mat == 0) {
-          *reinterpret_cast<float4 *>(qs + h * D + e0) =
-              make_float4(v[0] * qscale, v[1] * qscale, v[2] * qscale, v[3] * qscale);
-        } else {
-          const uint2 pk = make_uint2(pack2(__float2bfloat16_rn(v[0]), __float2bfloat16_rn(v[1])),
-                                      pack2(__float2bfloat16_rn(v[2]), __float2bfloat16_rn(v[3])));
-          *reinterpret_cast<uint2 *>(kvcur + (mat - 1) * D + e0) = pk;
-          const int ph = kv_phys_page(p, b, cur / P);
-          if (ph >= 0) {
-            __nv_bfloat16 *dst = (mat == 1 ? p.k_pages[l] : p.v_pages[l]) +
-                                 ((static_cast<size_t>(ph) * p.Hkv + g) * P + cur % P) * D + e0;
-            *reinterpret_cast<uint2 *>(dst) = pk;
-          }
-        }
-      }
-    }
-  }
-  if (ctid < G) {
-    mst[ctid] = -INFINITY;
-    lst[ctid] = 0.f;
-  }
-  compute_bar();
-  if (ctid == 0) trace_mark(p, S.idx, 5);
-
+  float *qs = A.qs, *sc = A.sc, *mst = A.mst, *lst = A.lst, *cor = A.cor;
+  const __nv_bfloat16 *kvcur = A.kvcur;
+  const int rw = D + 4;
   float acc[MAXP][4];
 #pragma unroll
   for (int k = 0; k < MAXP; ++k) acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
@@ -1928,8 +1884,6 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   }
 
   // the chunk's partial goes straight to global memory: row h = (acc, m, l, pad)
-  const int rw = D + 4;
-  float *part = p.attn_part + static_cast<size_t>(t.aux) * G * rw;
 #pragma unroll
   for (int k = 0; k < MAXP; ++k) {
     const int pq = ctid + k * kComputeThreads;
@@ -1939,6 +1893,303 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
              make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]));
     }
   }
+  return true;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t &r0, uint32_t &r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+
+// Shared-memory address of dims k..k+7 (k a multiple of 8) of token t of a
+// K or V area holding P-token KV pages as the TMA copies laid them out: per
+// KV page, 64-dim atoms of P rows x 128 bytes, the 16-byte chunk c of a row
+// at chunk c XOR (row address bits 7..9) (128-byte swizzle).
+template <int D>
+__device__ __forceinline__ uint32_t kv_addr(uint32_t base, int t, int k, int P) {
+  const int j = t / P, r = t - j * P;
+  const uint32_t row = base + static_cast<uint32_t>(j * (P * D * 2) + (k >> 6) * (P * 128) + r * 128);
+  return row + (((static_cast<uint32_t>((k & 63) >> 3)) ^ ((row >> 7) & 7u)) << 4);
+}
+
+// fp32 pair -> (hi, lo) bf16x2 pairs, hi + lo == x to ~2^-16.
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+  __nv_bfloat16 h0, l0, h1, l1;
+  split_bf16(x0, h0, l0);
+  split_bf16(x1, h1, l1);
+  hi = pack2(h0, h1);
+  lo = pack2(l0, l1);
+}
+
+// The chunk's pages on the tensor cores (mma.sync m16n8k16, bf16 -> fp32),
+// K and V pages copied by TMA in the 128-byte-swizzled layout (kv_addr), so
+// every ldmatrix reads conflict-free.  Per page:
+//   1. S = Q K^T: A = the G query heads as rows, bf16 high halves in rows
+//      0..7 and low halves in rows 8..15 (registers, built once per chunk);
+//      B = 8 tokens x 16 dims from ldmatrix; score(head g, token) = row g +
+//      row g + 8 of the result;
+//   2. softmax statistics, one warp per head, as on the CUDA cores;
+//   3. O += P V: A = p of the G heads (high/low rows), 16 tokens per step;
+//      B = V tokens x 8 dims from ldmatrix.trans; each warp owns a few 8-dim
+//      tiles of O, rescaled by the page's correction before it adds.
+// Tokens past the chunk's end in the page's last 16: p = 0 and their V rows
+// zeroed (the cache may hold anything there).
+template <int D>
+__device__ bool attn_pages_mma(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
+                               ComputeState &st, const AttnSmem &A, bool own_cur, int cur,
+                               float *part, int ctid) {
+  const int warp = ctid >> 5, lane = ctid & 31;
+  const int G = p.G, P = p.page_size, tpp = p.tpp;
+  const int g = lane >> 2, q = lane & 3;
+  constexpr int NB = D / 8;
+  constexpr int KS = D / 16;                 // k-steps of the scores
+  constexpr int NT = (D / 8 + kComputeWarps - 1) / kComputeWarps;   // O tiles per warp
+  float *sc = A.sc, *mst = A.mst, *lst = A.lst, *cor = A.cor;
+  const int rw = D + 4;
+
+  // the query fragments (rows g: high halves of head g, g + 8: low halves)
+  uint32_t qa[KS][4];
+#pragma unroll
+  for (int s = 0; s < KS; ++s) {
+    float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+    if (g < G) {
+      const float *qh = A.qs + g * D + 16 * s + 2 * q;
+      x0 = qh[0]; x1 = qh[1]; x2 = qh[8]; x3 = qh[9];
+    }
+    split_pair(x0, x1, qa[s][0], qa[s][1]);
+    split_pair(x2, x3, qa[s][2], qa[s][3]);
+  }
+  float acc[NT][4];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+  for (int tok0 = S.t0; tok0 < S.t1; tok0 += tpp) {
+    const int ntok = min(tpp, S.t1 - tok0);
+    bool okl = true;
+    if (ctid == 0) okl = wait_mbar(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff40000u, 2);
+    if (!st.gs.share(ctl, ctid, okl)) return false;
+    mbar_try_wait(&ctl->full[st.pi], st.pg_par);
+    uint8_t *kpg = smem + p.off_pages + static_cast<size_t>(st.pi) * p.page_bytes;
+    uint8_t *vpg = kpg + static_cast<size_t>(tpp) * D * 2;
+    const uint32_t ks = smem_u32(kpg), vs = smem_u32(vpg);
+    // the current token's K/V into its slot (the page was copied before they
+    // were formed), and zero V rows past the chunk's end up to a multiple of 16
+    const bool has_cur = own_cur && cur >= tok0 && cur < tok0 + ntok;
+    const int nz = ((ntok + 15) & ~15) - ntok;
+    if (has_cur && ctid < 2 * NB) {
+      const bool isv = ctid >= NB;
+      const int e = (isv ? ctid - NB : ctid) * 8;
+      sts128(kv_addr<D>(isv ? vs : ks, cur - tok0, e, P),
+             *reinterpret_cast<const uint4 *>(A.kvcur + (isv ? D : 0) + e));
+    }
+    for (int u = ctid; u < nz * NB; u += kComputeThreads)
+      sts128(kv_addr<D>(vs, ntok + u / NB, (u % NB) * 8, P), make_uint4(0, 0, 0, 0));
+    if (has_cur || nz > 0) compute_bar();
+
+    // phase 1: scores, 8 tokens per mma tile
+    const int ntl = (ntok + 7) >> 3;
+    for (int j = warp; j < ntl; j += kComputeWarps) {
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s2 = 0; s2 < KS / 2; ++s2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kv_addr<D>(ks, 8 * j + (lane & 7), 32 * s2 + 8 * (lane >> 3), P), b0, b1, b2, b3);
+        mma_bf16(c, qa[2 * s2][0], qa[2 * s2][1], qa[2 * s2][2], qa[2 * s2][3], b0, b1);
+        mma_bf16(c, qa[2 * s2 + 1][0], qa[2 * s2 + 1][1], qa[2 * s2 + 1][2], qa[2 * s2 + 1][3],
+                 b2, b3);
+      }
+      const int t0 = 8 * j + 2 * q;
+      if (g < G) {
+        if (t0 < ntok) sc[g * tpp + t0] = c[0] + c[2];
+        if (t0 + 1 < ntok) sc[g * tpp + t0 + 1] = c[1] + c[3];
+      }
+    }
+    compute_bar();
+    // phase 2: softmax statistics, one warp per head
+    for (int h = warp; h < G; h += kComputeWarps) {
+      float *row = sc + h * tpp;
+      float mx = -INFINITY;
+      for (int tk = lane; tk < ntok; tk += 32) mx = fmaxf(mx, row[tk]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float mold = mst[h];
+      const float mnew = fmaxf(mold, mx);
+      float sum = 0.f;
+      for (int tk = lane; tk < ntok; tk += 32) {
+        const float pr = exp2f(row[tk] - mnew);
+        row[tk] = pr;
+        sum += pr;
+      }
+      sum = warp_sum(sum);
+      __syncwarp();
+      if (lane == 0) {
+        const float cc = exp2f(mold - mnew);   // 0 on the first page (mold = -inf)
+        cor[h] = cc;
+        lst[h] = lst[h] * cc + sum;
+        mst[h] = mnew;
+      }
+    }
+    compute_bar();
+    // phase 3: O = O * correction + P V over 16-token steps
+    {
+      const float cg = g < G ? cor[g] : 0.f;
+#pragma unroll
+      for (int i = 0; i < NT; ++i) {
+        acc[i][0] *= cg; acc[i][1] *= cg; acc[i][2] *= cg; acc[i][3] *= cg;
+      }
+      const int nks = (ntok + 15) >> 4;
+      for (int u = 0; u < nks; ++u) {
+        const int t = 16 * u + 2 * q;
+        float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+        if (g < G) {
+          const float *prow = sc + g * tpp;
+          if (t < ntok) p0 = prow[t];
+          if (t + 1 < ntok) p1 = prow[t + 1];
+          if (t + 8 < ntok) p2 = prow[t + 8];
+          if (t + 9 < ntok) p3 = prow[t + 9];
+        }
+        uint32_t a0, a1, a2, a3;
+        split_pair(p0, p1, a0, a1);
+        split_pair(p2, p3, a2, a3);
+#pragma unroll
+        for (int i = 0; i < NT; ++i) {
+          const int dt = warp + i * kComputeWarps;   // this warp's 8-dim tile
+          if (dt < D / 8) {
+            uint32_t b0, b1;
+            ldsm_x2_trans(kv_addr<D>(vs, 16 * u + (lane & 15), 8 * dt, P), b0, b1);
+            mma_bf16(acc[i], a0, a1, a2, a3, b0, b1);
+          }
+        }
+      }
+    }
+    if (has_cur || nz > 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (!p.tc && lane == 0) mbar_arrive(&ctl->empty[st.pi]);
+    compute_bar();   // sc is rewritten by the next page
+    // (tensor-core plans release a page once, after every warp is done with it)
+    if (p.tc && ctid == 0) mbar_arrive(&ctl->empty[st.pi]);
+    if (++st.pi == p.n_pages) {
+      st.pi = 0;
+      st.pg_par ^= 1u;
+    }
+  }
+  // the chunk's partial: row h = (sum, m, l, pad); head g's sums are the
+  // high row g plus the low row g + 8
+  if (g < G) {
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      const int dt = warp + i * kComputeWarps;
+      if (dt < D / 8) {
+        const int d0 = 8 * dt + 2 * q;
+        __stcg(reinterpret_cast<float2 *>(part + g * rw + d0),
+               make_float2(acc[i][0] + acc[i][2], acc[i][1] + acc[i][3]));
+      }
+    }
+  }
+  return true;
+}
+
+// Attention for one chunk of one (sequence, KV head): scores for the G query
+// heads over the chunk's tokens, softmax statistics, and the unnormalised
+// P.V, all in three parallel phases per shared-memory page:
+//   1. thread <- (token, head): full dot product q.k over d, reading the
+//      8-element column blocks in a rotated order (block (c + t) mod d/8) so
+//      the 32 lanes of a warp hit distinct banks;
+//   2. warp <- head: running max m, rescale factor, p = 2^(s - m), running sum;
+//   3. thread <- (head, 4 columns of d): acc = acc * rescale + sum_t p v.
+// Scores are in log2 units (q is pre-scaled by log2(e)/sqrt(d)).
+template <int D>
+__device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
+                          ComputeState &st, float *out, int ctid) {
+  const Task &t = S.t;
+  const int warp = ctid >> 5, lane = ctid & 31;
+  const int G = p.G, l = t.layer;
+  const int b = S.b, g = S.g;
+  constexpr int NB = D / 8;                 // 8-element column blocks per row
+  constexpr int Q4 = D / 4;                 // 4-column slices per head
+  constexpr int MAXP = (kMaxGroup * Q4 + kComputeThreads - 1) / kComputeThreads;
+  float *qs = reinterpret_cast<float *>(smem + p.off_x);   // [G][D]
+  float *sc = qs + G * D;                                   // [G][tpp] scores, then p
+  float *mst = sc + G * p.tpp;                              // [G] running max
+  float *lst = mst + kMaxGroup;                             // [G] running sum
+  float *cor = lst + kMaxGroup;                             // [G] rescale of this page
+  __nv_bfloat16 *kvcur = reinterpret_cast<__nv_bfloat16 *>(cor + kMaxGroup);  // [2][D] K, V at pos
+  st.xkey = 0xffffffffu;                                    // staging area reused
+
+  {
+    const uint32_t ev = static_cast<uint32_t>(ev_attn_input(p, l, g));
+    bool okl = true;
+    if (ctid == 0) okl = wait_event(p, ctl, ev, static_cast<uint32_t>(attn_input_count(p)), S.idx);
+    if (!st.gs.share(ctl, ctid, okl)) return false;
+    if (ctid == 0) trace_mark(p, S.idx, 4);
+  }
+  // From this step's raw projections, one warp per head: the G query heads
+  // (QK-norm, RoPE, pre-scaled by log2(e)/sqrt(d) for the exp2 softmax) and,
+  // in the chunk that holds the current position, K (QK-norm, RoPE) and V of
+  // the current token, rounded to bf16 and appended to the cache.
+  const int P = p.page_size;
+  const int cur = row_pos(p, b);
+  // (in a plan whose K/V tasks append every row's K/V first, the cache
+  // already holds the current token's)
+  const bool own_cur = !p.kv_tasks && cur >= S.t0 && cur < S.t1;
+  {
+    const float qscale = rsqrtf(static_cast<float>(D)) * 1.4426950408889634f;
+    // a position outside 0..max_pos-1 is reported by the embedding task; the
+    // table row stays in range regardless
+    const int cpos = cur < 0 ? 0 : (cur >= p.max_pos ? p.max_pos - 1 : cur);
+    const float2 *cs = p.rope_cs + static_cast<size_t>(cpos) * (D / 2);
+    const float *raw = p.qkv + static_cast<size_t>(b) * p.NQKV;
+    const int nh = G + (own_cur ? 2 : 0);
+    for (int h = warp; h < nh; h += kComputeWarps) {
+      const int mat = h < G ? 0 : h - G + 1;   // 0 q, 1 k, 2 v
+      const int col = mat == 0 ? (g * G + h) * D
+                               : (mat == 1 ? (p.Hq + g) * D : (p.Hq + p.Hkv + g) * D);
+      float v[4];
+      head_norm_rope<D>(raw + col, mat == 0 ? t.w0 : t.w1, p.qk_norm != 0 && mat != 2,
+                        mat != 2, cs, p.eps, lane, v);
+      if (lane < D / 4) {
+        const int e0 = lane * 4;
+        if (mat == 0) {
+          *reinterpret_cast<float4 *>(qs + h * D + e0) =
+              make_float4(v[0] * qscale, v[1] * qscale, v[2] * qscale, v[3] * qscale);
+        } else {
+          const uint2 pk = make_uint2(pack2(__float2bfloat16_rn(v[0]), __float2bfloat16_rn(v[1])),
+                                      pack2(__float2bfloat16_rn(v[2]), __float2bfloat16_rn(v[3])));
+          *reinterpret_cast<uint2 *>(kvcur + (mat - 1) * D + e0) = pk;
+          const int ph = kv_phys_page(p, b, cur / P);
+          if (ph >= 0) {
+            __nv_bfloat16 *dst = (mat == 1 ? p.k_pages[l] : p.v_pages[l]) +
+                                 ((static_cast<size_t>(ph) * p.Hkv + g) * P + cur % P) * D + e0;
+            *reinterpret_cast<uint2 *>(dst) = pk;
+          }
+        }
+      }
+    }
+  }
+  if (ctid < G) {
+    mst[ctid] = -INFINITY;
+    lst[ctid] = 0.f;
+  }
+  compute_bar();
+  if (ctid == 0) trace_mark(p, S.idx, 5);
+
+  const int rw = D + 4;
+  float *part = p.attn_part + static_cast<size_t>(t.aux) * G * rw;
+  AttnSmem A{qs, sc, mst, lst, cor, kvcur};
+  bool pages_ok;
+  if constexpr (D >= 64)
+    pages_ok = p.attn_mma ? attn_pages_mma<D>(p, ctl, smem, S, st, A, own_cur, cur, part, ctid)
+                          : attn_pages_cuda<D>(p, ctl, smem, S, st, A, own_cur, cur, part, ctid);
+  else
+    pages_ok = attn_pages_cuda<D>(p, ctl, smem, S, st, A, own_cur, cur, part, ctid);
+  if (!pages_ok) return false;
   if (ctid < G) {
     __stcg(part + ctid * rw + D, mst[ctid]);
     __stcg(part + ctid * rw + D + 1, lst[ctid]);

@@ -353,7 +353,8 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     g.kp[K_HID] = std::min(H, kw);
     g.kp[K_ATT] = std::min(Hq * d, kw);
     g.kp[K_FFN] = std::min(kchunk_ffn, kw);
-    g.page_bytes = nb * MK_W4_BLOCK_BYTES;
+    // (pages start on 1024-byte boundaries: the attention's swizzled K/V copies)
+    g.page_bytes = align_up_i(nb * MK_W4_BLOCK_BYTES, 1024);
     g.kp[K_LM] = 32;
     while (16 * row_pitch_bytes(g.kp[K_LM] + 32) <= g.page_bytes && g.kp[K_LM] + 32 <= kMaxPageCols)
       g.kp[K_LM] += 32;
@@ -445,6 +446,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   p.wait_limit_ns = o.wait_limit_ns;
   p.n_ffn_parts = n_ksplit;
   p.chunk_seq = -1;   // decode steps (a prompt chunk sets its sequence)
+  p.attn_mma = (d == 64 || d == 128) ? 1 : 0;
   p.w4 = o.w4 ? 1 : 0;
   p.n_out = n_out;
   p.tile_rows = tc ? kTcRows : 16;
@@ -755,20 +757,54 @@ void bind_task_operands(const mk_model_config &c, const mk_weights &w, std::vect
 
 namespace mk {
 
-int encode_weight_maps(const mk_model_config &c, const mk_weights &w, const Layout &lay,
-                       const char *ws, std::vector<unsigned char> &out, std::string &err) {
-  out.clear();
-  if (lay.n_maps == 0) return MK_OK;
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder(std::string &err) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (encode == nullptr) {
     void *fn = nullptr;
     cudaDriverEntryPointQueryResult q{};
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
             cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || fn == nullptr)
-      return lfail(err, MK_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+        q != cudaDriverEntryPointSuccess || fn == nullptr) {
+      lfail(err, MK_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+      return nullptr;
+    }
     encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
+  return encode;
+}
+}  // namespace
+
+int encode_kv_maps(const mk_model_config &c, const mk_kv_cache &kv, int page_size,
+                   std::vector<unsigned char> &out, std::string &err) {
+  auto encode = tensor_map_encoder(err);
+  if (encode == nullptr) return MK_ERR_CUDA;
+  const int L = c.n_layers, d = c.head_dim;
+  out.assign(static_cast<size_t>(2 * L) * sizeof(CUtensorMap), 0);
+  const cuuint64_t rows = static_cast<cuuint64_t>(kv.num_pages) * c.n_kv_heads * page_size;
+  for (int l = 0; l < L; ++l)
+    for (int kvi = 0; kvi < 2; ++kvi) {
+      CUtensorMap m;
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), rows};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+      cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(page_size)};
+      cuuint32_t estr[2] = {1, 1};
+      void *base = kvi == 0 ? kv.k_pages[l] : kv.v_pages[l];
+      const CUresult r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return lfail(err, MK_ERR_CUDA, "KV tensor map: cuTensorMapEncodeTiled failed (%d)", r);
+      std::memcpy(out.data() + static_cast<size_t>(2 * l + kvi) * sizeof(CUtensorMap), &m, sizeof(m));
+    }
+  return MK_OK;
+}
+
+int encode_weight_maps(const mk_model_config &c, const mk_weights &w, const Layout &lay,
+                       const char *ws, std::vector<unsigned char> &out, std::string &err) {
+  out.clear();
+  if (lay.n_maps == 0) return MK_OK;
+  auto encode = tensor_map_encoder(err);
+  if (encode == nullptr) return MK_ERR_CUDA;
   const int L = c.n_layers, H = c.hidden, F = c.ffn, d = c.head_dim;
   const int Hq = c.n_q_heads, Hkv = c.n_kv_heads;
   out.assign(static_cast<size_t>(lay.n_maps) * sizeof(CUtensorMap), 0);

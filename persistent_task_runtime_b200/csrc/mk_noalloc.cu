@@ -50,7 +50,9 @@ struct Uploaded {
   int page = 0, batch = 0, nsm = 0, smem_optin = 0;
   std::vector<const void *> ptrs;   // every weight pointer, in a fixed order
   mk::Layout lay;
-  size_t o_tasks = 0, o_rope = 0, o_ws = 0, o_sync = 0, o_maps = 0;
+  size_t o_tasks = 0, o_rope = 0, o_ws = 0, o_sync = 0, o_maps = 0, o_kvmaps = 0;
+  std::vector<const void *> kv_key;         // the KV cache whose tensor maps the array holds
+  std::vector<unsigned char> kv_maps_host;
 };
 Uploaded g_up[kMaxDevices];
 
@@ -183,6 +185,8 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
       if (mrc) return nfail(mrc, merr.c_str());
     }
     up.o_maps = carve(maps.size());
+    up.o_kvmaps = carve(up.lay.p.attn_mma ? static_cast<size_t>(2 * c.n_layers) * 128 : 0);
+    up.kv_key.clear();
     if (off > MK_NOALLOC_SCRATCH_BYTES) {
       char msg[256];
       snprintf(msg, sizeof(msg),
@@ -206,6 +210,27 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
     up.ptrs = std::move(ptrs);
     up.valid = true;
   }
+  // the attention's tensor maps of this call's KV cache (re-encoded when the
+  // cache differs from the previous call's)
+  if (up.lay.p.attn_mma) {
+    std::vector<const void *> key;
+    key.push_back(reinterpret_cast<const void *>(static_cast<intptr_t>(a->kv->num_pages)));
+    for (int l = 0; l < L; ++l) {
+      key.push_back(a->kv->k_pages[l]);
+      key.push_back(a->kv->v_pages[l]);
+    }
+    if (key != up.kv_key) {
+      std::string kerr;
+      const int krc = mk::encode_kv_maps(c, *a->kv, P, up.kv_maps_host, kerr);
+      if (krc) return nfail(krc, kerr.c_str());
+      if (cudaMemcpyAsync(base + up.o_kvmaps, up.kv_maps_host.data(), up.kv_maps_host.size(),
+                          cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        up.valid = false;
+        return nfail(MK_ERR_CUDA, "uploading the KV tensor maps into the scratch array failed");
+      }
+      up.kv_key = std::move(key);
+    }
+  }
   const mk::Layout &lay = up.lay;
   Params p = lay.p;
   const int grid = lay.grid, smem = lay.smem;
@@ -220,6 +245,7 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
   p.tasks = reinterpret_cast<const Task *>(base + o_tasks);
   p.rope_cs = reinterpret_cast<const float2 *>(base + o_rope);
   p.tmaps = base + up.o_maps;
+  p.kvmaps = up.lay.p.attn_mma ? base + up.o_kvmaps : nullptr;
   mk::bind_workspace(lay, base + o_ws, reinterpret_cast<uint32_t *>(base + o_sync), p);
   p.embed = static_cast<const __nv_bfloat16 *>(w->embed);
 

@@ -73,6 +73,7 @@ def check_plan(cfg, info, t, max_batch):
     assert info["smem_bytes"] <= SMEM
     assert info["n_pages"] >= 2
     assert info["n_pages"] * info["page_bytes"] < info["smem_bytes"]
+    assert info["page_bytes"] % 1024 == 0     # swizzled TMA copies land on 1024-byte boundaries
     tc = info["gemv_path"] == 2
     tile = 128 if tc else 16                     # rows per row tile
     max_mt = 2 if tc else 8 // n_tiles_for(max_batch)
