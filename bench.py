@@ -220,7 +220,7 @@ def run_mk(args, rank: int, world: int, local_rank: int) -> dict:
     cap = [n + horizon for n in lengths]
     kv = PagedKVCache(cfg, B, cap, page=16, device=dev)
     plan = mk.Plan(cfg, weights, max_batch=B, page_size=16, max_seq_len=max(cap) + 16,
-                   gemv_path=args.gemv_path, schedule=args.schedule)
+                   gemv_path=args.gemv_path, schedule=args.schedule, attn_path=args.attn_path)
     info = plan.info()
     ids = torch.zeros(B, dtype=torch.int32, device=dev)
     pos = torch.zeros(B, dtype=torch.int32, device=dev)
@@ -236,7 +236,7 @@ def run_mk(args, rank: int, world: int, local_rank: int) -> dict:
         # the prompt through prompt chunks of up to 16 tokens on a plan of its
         # own (multi-token tasks; the LM head runs on the last chunk only)
         pplan = mk.Plan(cfg, weights, max_batch=16, page_size=16, max_seq_len=max(cap) + 16,
-                        prefill=True)
+                        prefill=True, attn_path=args.attn_path)
         prompt = synth.make_ids(cfg["vocab"], (B, lengths[0]), seed=1).to(dev).to(torch.int32)
         first = torch.zeros(1, dtype=torch.int32, device=dev)
         for b in range(B):   # warm the plan (and the cache pages) once
@@ -452,6 +452,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=32)
     ap.add_argument("--gemv-path", type=int, default=0, choices=[0, 1, 2],
                     help="projections: 0 automatic, 1 mma.sync pages, 2 tcgen05 tiles")
+    ap.add_argument("--attn-path", type=int, default=0, choices=[0, 1, 2],
+                    help="attention: 0 automatic, 1 CUDA-core FMA, 2 mma.sync tiles")
     ap.add_argument("--prompt-path", choices=["chunks", "decode"], default="chunks",
                     help="how a workload's prompt fills the cache: prompt chunks of 16 tokens "
                          "(mk_prefill_chunk) or one decode step per token")
@@ -525,7 +527,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": config, "mode": r["mode"],
             "plan": {"gemv_path": r["info"]["gemv_path"], "schedule": r["info"]["schedule"],
-                     "n_tasks": r["info"]["n_tasks"]},
+                     "attn_path": r["info"]["attn_path"], "n_tasks": r["info"]["n_tasks"]},
             "step_us": {"mean": round(1e3 * statistics.mean(r["launch_ms"]), 1),
                         "p50": round(1e3 * statistics.median(r["launch_ms"]), 1),
                         "min": round(1e3 * min(r["launch_ms"]), 1),

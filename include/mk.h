@@ -204,6 +204,13 @@ typedef struct {
                              them, so a row may attend to positions that
                              other rows of the same launch write.  Decode
                              steps on such a plan give the same results    */
+  int attn_path;          /* how attention runs: 0 = automatic (1), 1 = CUDA
+                             cores: fp32 FMA over K/V pages bulk-copied into
+                             shared memory; 2 = mma.sync tensor-core tiles:
+                             K/V pages copied by TMA tensor copies with the
+                             128-byte swizzle, q.K and P.V as m16n8k16 MMAs
+                             fed by ldmatrix (head_dim 64 or 128, else
+                             MK_ERR_UNSUPPORTED)                            */
 } mk_plan_options;
 
 typedef struct mk_plan mk_plan;
@@ -339,6 +346,7 @@ typedef struct {
   int weight_bits;        /* 16 bf16 or 4 (W4A16) projections              */
   int qkv_parts, gateup_parts; /* split-K parts of the QKV and gate/up
                              projections (tensor-core path; 1 otherwise)   */
+  int attn_path;          /* 1 CUDA-core attention, 2 mma.sync tiles        */
 } mk_plan_info_t;
 MK_API int mk_plan_info(const mk_plan *plan, mk_plan_info_t *info);
 

@@ -137,6 +137,7 @@ int layout_options(const mk_plan_options *opts, mk::LayoutOptions &lo, const mk_
   lo.gemv_path = o.gemv_path;
   lo.schedule = o.schedule;
   lo.prefill = o.prefill != 0;
+  lo.attn_path = o.attn_path;
   for (int i = 0; i < 5; ++i) lo.rows_per_task[i] = o.rows_per_task[i];
   lo.wait_limit_ns = o.wait_limit_ns == 0 ? 2000000000LL : o.wait_limit_ns;
   lo.debug_unsatisfiable_dep = o.debug_unsatisfiable_dep != 0;
@@ -186,6 +187,7 @@ void fill_info(const mk::Layout &lay, const mk_model_config &c, mk_plan_info_t &
   I.prefill = lay.p.kv_tasks;
   I.qkv_parts = lay.splits[0];
   I.gateup_parts = lay.splits[2];
+  I.attn_path = p.attn_mma ? 2 : 1;
 }
 
 }  // namespace

@@ -46,6 +46,11 @@ constexpr int kTcTmemCols = 128;                  // tensor-memory columns alloc
 constexpr int kTcAutoBatch = 5;                   // smallest max_batch that takes it by default
 constexpr int kTcMatsPerLayer = 7;                // tensor maps: wq wk wv wo w_gate w_up w_down
 
+// ---- kernel variants (template argument of the step kernel) -------------------
+constexpr int kVarTc = 1;        // projections on tcgen05 tiles (else mma.sync pages)
+constexpr int kVarW4 = 2;        // 4-bit weight consumer
+constexpr int kVarAttnMma = 4;   // attention on mma.sync tiles over swizzled K/V pages
+
 // ---- task descriptor (64 bytes, four 16-byte loads) ---------------------------
 enum TaskType : uint8_t {
   T_EMBED = 1,
@@ -251,6 +256,7 @@ struct LayoutOptions {
   int schedule = 0;             // 0 dynamic ticket queue, 1 solidified per-CTA task lists
   bool prefill = false;         // K/V appended by their own tasks (prompt chunks of one sequence)
   bool w4 = false;              // 4-bit projections (packed, MK_W4_BLOCK_BYTES blocks)
+  int attn_path = 0;            // 0 automatic / 1 CUDA-core FMA, 2 mma.sync tiles (d 64, 128)
   int rows_per_task[5] = {0, 0, 0, 0, 0};
   long long wait_limit_ns = 2000000000LL;
   bool debug_unsatisfiable_dep = false;
@@ -295,6 +301,8 @@ cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative,
                         cudaStream_t stream);
 // Allow the kernel the device's opt-in shared memory (capped at kMaxSmem).
 cudaError_t configure_kernel(int smem_optin);
+// The kernel variant (kVar* bits) a plan's parameters select.
+int kernel_variant(const Params &p);
 void set_last_error(const char *msg);  // message returned by mk_last_error()
 
 // Tensor maps of a KV cache for the mma.sync attention: per layer, K then V,

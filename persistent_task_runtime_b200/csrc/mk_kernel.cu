@@ -504,42 +504,57 @@ __device__ __forceinline__ int seq_len(const Params &p, int b) {
   return n < 1 ? 1 : (n > p.max_pos ? p.max_pos : n);
 }
 
-// Tokens per attention chunk: a whole number of KV pages, sized so each KV
-// group's chunks over all sequences fit its block of slots (one partial
-// chunk per sequence is allowed for).
-__device__ int attn_span(const Params &p, int B) {
+// The loader's view of the batch for one launch: lane b (< B) holds the
+// number of tokens sequence b attends (positions 0..pos, clamped to
+// [1, max_pos]); every lane holds the attention chunk span: a whole number
+// of KV pages, sized so each KV group's chunks over all sequences fit its
+// block of slots (one partial chunk per sequence is allowed for).  Read once
+// per launch, one position per lane, so resolving a slot later costs no
+// global round trip.
+struct SeqView {
+  int len, span;
+};
+__device__ SeqView seq_view(const Params &p, int B, int lane) {
+  SeqView v;
   const int P = p.page_size;
-  int units = 0;
-  for (int b = 0; b < B; ++b) units += (seq_len(p, b) + P - 1) / P;
+  v.len = lane < B ? seq_len(p, lane) : 0;
+  const int units = __reduce_add_sync(0xffffffffu, (v.len + P - 1) / P);
   const int target = p.attn_spg - B;
   const int c = (units + target - 1) / target;
-  return (c < 1 ? 1 : c) * P;
+  v.span = (c < 1 ? 1 : c) * P;
+  return v;
 }
 
-// Slot s of a layer -> (sequence, KV head, token range).  Slots come in one
-// block per KV group; inside a block, the chunks of sequence 0, then 1, ...
-__device__ bool attn_resolve(const Params &p, int B, int s, Slot &o) {
-  const int span = attn_span(p, B);
+// Slot s of a layer -> (sequence, KV head, token range) (warp-uniform, all
+// lanes).  Slots come in one block per KV group; inside a block, the chunks
+// of sequence 0, then 1, ...
+__device__ bool attn_resolve(const Params &p, int B, int s, const SeqView &v, int lane, Slot &o) {
   const int g = s / p.attn_spg;
   const int r = s - g * p.attn_spg;
-  int base = 0;
-  for (int b = 0; b < B; ++b) {
-    const int len = seq_len(p, b);
-    const int nb = (len + span - 1) / span;
-    if (r < base + nb) {
-      const int c = r - base;
-      o.b = b;
-      o.g = g;
-      o.t0 = c * span;
-      o.t1 = min(len, o.t0 + span);
-      o.first_slot = g * p.attn_spg + base;
-      o.n_chunks = nb;
-      return true;
-    }
-    base += nb;
+  const int nb = lane < B ? (v.len + v.span - 1) / v.span : 0;
+  int incl = nb;   // inclusive prefix sum of chunks over sequences 0..lane
+#pragma unroll
+  for (int k = 1; k < 32; k <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, k);
+    if (lane >= k) incl += y;
   }
-  o.b = -1;
-  return false;
+  const int excl = incl - nb;
+  const unsigned hit = __ballot_sync(0xffffffffu, lane < B && r >= excl && r < incl);
+  if (hit == 0u) {
+    o.b = -1;
+    return false;
+  }
+  const int b = __ffs(hit) - 1;
+  const int base = __shfl_sync(0xffffffffu, excl, b);
+  const int nbb = __shfl_sync(0xffffffffu, nb, b);
+  const int len = __shfl_sync(0xffffffffu, v.len, b);
+  o.b = b;
+  o.g = g;
+  o.t0 = (r - base) * v.span;
+  o.t1 = min(len, o.t0 + v.span);
+  o.first_slot = g * p.attn_spg + base;
+  o.n_chunks = nbb;
+  return true;
 }
 
 __device__ __forceinline__ int kv_phys_page(const Params &p, int b, int logical) {
@@ -566,8 +581,9 @@ struct Look {
 constexpr int kLook = kLookBytes / static_cast<int>(sizeof(Look));
 static_assert(sizeof(Look) == 80 && kLook >= 2, "lookahead entry size");
 
-template <bool TC>
+template <int V>
 __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
+  constexpr bool TC = (V & kVarTc) != 0, W4 = (V & kVarW4) != 0, AMMA = (V & kVarAttnMma) != 0;
   const int lane = threadIdx.x & 31;
   const uint64_t pol = l2_evict_first_policy();
   Slot *slots = reinterpret_cast<Slot *>(smem + p.off_slots);
@@ -592,6 +608,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   int la_head = 0, la_count = 0;
   bool exhausted = false;
   uint32_t la_ev = 0;   // lane 0: input-event counter read when the task was popped
+  const SeqView sv = seq_view(p, B, lane);
 
   // Pop one task into the lookahead (warp-uniform).  The next ticket is
   // always requested one pop ahead, so a pop waits only for the descriptor.
@@ -674,7 +691,13 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     info.idx = tix;
     info.b = -1;
     info.dep_ok = 0;
-    if (t.type == T_ATTN) attn_resolve(p, B, static_cast<int>(t.aux), info);
+    // attention: the chunk's KV pages from the block table, one per lane,
+    // read now so the lookups overlap the wait for free ring pages
+    int ph_pre = -1;
+    if (t.type == T_ATTN && attn_resolve(p, B, static_cast<int>(t.aux), sv, lane, info)) {
+      const int npg = (info.t1 - info.t0 + p.page_size - 1) / p.page_size;
+      if (lane < npg) ph_pre = kv_phys_page(p, info.b, info.t0 / p.page_size + lane);
+    }
     __syncwarp();
     if (lane == 0) {
       // an input event already complete when the task was popped: acquire
@@ -762,7 +785,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
             ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
             if (!ok) break;
             uint8_t *pg = pages + static_cast<size_t>(pi) * p.page_bytes;
-            if (is_w4_task(p.w4, t.type)) {
+            if (W4 && is_w4_task(p.w4, t.type)) {
               // 4-bit: the row tile's packed blocks of these columns are
               // contiguous -- one bulk copy
               const uint32_t bytes = static_cast<uint32_t>(nc / MK_W4_BLOCK_COLS) * MK_W4_BLOCK_BYTES;
@@ -819,15 +842,22 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
         if (lane == 0) mbar_arrive_expect_tx(&ctl->full[pi], 2u * nkv * kvpage_bytes);
         __syncwarp();
         const int j = lane & 15;
-        if (p.attn_mma) {
+        const int lp0 = info.t0 / P, jbase = (tok0 - info.t0) / P;
+        if (AMMA) {
           // TMA tensor copies, 64 dims x P tokens per box, 128-byte swizzle:
           // the layout the attention's ldmatrix fragment loads read without
           // bank conflicts
           const int na = d / 64;
           const uint8_t *maps = static_cast<const uint8_t *>(p.kvmaps);
-          for (int idx = lane; idx < nkv * 2 * na; idx += 32) {
-            const int jj = idx / (2 * na), kvi = (idx / na) & 1, a = idx % na;
-            int ph = kv_phys_page(p, info.b, tok0 / P + jj);
+          const int n_copies = nkv * 2 * na;
+          for (int i0 = 0; i0 < n_copies; i0 += 32) {
+            const int idx = i0 + lane;
+            const bool act = idx < n_copies;
+            const int jj = act ? idx / (2 * na) : 0, kvi = (idx / na) & 1, a = idx % na;
+            const int jg = jbase + jj;   // page of the chunk
+            int ph = __shfl_sync(0xffffffffu, ph_pre, jg & 31);
+            if (!act) continue;
+            if (jg >= 32) ph = kv_phys_page(p, info.b, lp0 + jg);
             if (ph < 0) {
               raise_error(p, MK_ERR_RANGE, static_cast<uint32_t>(tix), 0xfffffffdu,
                           static_cast<uint32_t>(info.b));
@@ -838,19 +868,24 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
             tma_load_2d(dst, maps + static_cast<size_t>(2 * l + kvi) * 128, a * 64,
                         (ph * p.Hkv + info.g) * P, &ctl->full[pi], pol);
           }
-        } else if (j < nkv) {
-          int ph = kv_phys_page(p, info.b, tok0 / P + j);
-          if (ph < 0) {
-            raise_error(p, MK_ERR_RANGE, static_cast<uint32_t>(tix), 0xfffffffdu,
-                        static_cast<uint32_t>(info.b));
-            ph = 0;  // keep the copy in bounds; the step is being abandoned
-          }
-          const size_t off = (static_cast<size_t>(ph) * p.Hkv + info.g) * kvpage_elems;
-          if (lane < 16) {
-            bulk_load(pg + j * kvpage_bytes, p.k_pages[l] + off, kvpage_bytes, &ctl->full[pi], pol);
-          } else {
-            bulk_load(pg + static_cast<size_t>(p.tpp) * d * 2 + j * kvpage_bytes,
-                      p.v_pages[l] + off, kvpage_bytes, &ctl->full[pi], pol);
+        } else {
+          const int jg = jbase + j;   // page of the chunk
+          int ph = __shfl_sync(0xffffffffu, ph_pre, jg & 31);
+          if (j < nkv) {
+            if (jg >= 32) ph = kv_phys_page(p, info.b, lp0 + jg);
+            if (ph < 0) {
+              raise_error(p, MK_ERR_RANGE, static_cast<uint32_t>(tix), 0xfffffffdu,
+                          static_cast<uint32_t>(info.b));
+              ph = 0;  // keep the copy in bounds; the step is being abandoned
+            }
+            const size_t off = (static_cast<size_t>(ph) * p.Hkv + info.g) * kvpage_elems;
+            if (lane < 16) {
+              bulk_load(pg + j * kvpage_bytes, p.k_pages[l] + off, kvpage_bytes, &ctl->full[pi],
+                        pol);
+            } else {
+              bulk_load(pg + static_cast<size_t>(p.tpp) * d * 2 + j * kvpage_bytes,
+                        p.v_pages[l] + off, kvpage_bytes, &ctl->full[pi], pol);
+            }
           }
         }
         issued |= 1u << pi;
@@ -1162,7 +1197,7 @@ __device__ bool stage_x(const Params &p, Ctl *ctl, uint8_t *smem, const Task &t,
 // NN = batch n-tiles (1: B <= 4, 2: B <= 8, 4: B <= 16).  A task holds at
 // most kMaxMTiles / NN row tiles (the plan caps rows per task) so that the
 // accumulators stay in registers.
-template <int NN, int MT = kMaxMTiles / NN>
+template <int NN, bool W4, int MT = kMaxMTiles / NN>
 __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
                           ComputeState &st, float *out, int ctid) {
   const Task &t = S.t;
@@ -1236,7 +1271,7 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
           continue;
         }
         const uint8_t *pg = pages + static_cast<size_t>(st.pi) * p.page_bytes;
-        const bool w4 = is_w4_task(p.w4, t.type);
+        const bool w4 = W4 && is_w4_task(p.w4, t.type);
         switch (m) {
 #define MK_PAGE_CASE(M)                                                                        \
   case M:                                                                                      \
@@ -2105,16 +2140,13 @@ __device__ bool attn_pages_mma(const Params &p, Ctl *ctl, uint8_t *smem, const S
 //   2. warp <- head: running max m, rescale factor, p = 2^(s - m), running sum;
 //   3. thread <- (head, 4 columns of d): acc = acc * rescale + sum_t p v.
 // Scores are in log2 units (q is pre-scaled by log2(e)/sqrt(d)).
-template <int D>
+template <int D, bool AMMA>
 __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
                           ComputeState &st, float *out, int ctid) {
   const Task &t = S.t;
   const int warp = ctid >> 5, lane = ctid & 31;
   const int G = p.G, l = t.layer;
   const int b = S.b, g = S.g;
-  constexpr int NB = D / 8;                 // 8-element column blocks per row
-  constexpr int Q4 = D / 4;                 // 4-column slices per head
-  constexpr int MAXP = (kMaxGroup * Q4 + kComputeThreads - 1) / kComputeThreads;
   float *qs = reinterpret_cast<float *>(smem + p.off_x);   // [G][D]
   float *sc = qs + G * D;                                   // [G][tpp] scores, then p
   float *mst = sc + G * p.tpp;                              // [G] running max
@@ -2184,9 +2216,8 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   float *part = p.attn_part + static_cast<size_t>(t.aux) * G * rw;
   AttnSmem A{qs, sc, mst, lst, cor, kvcur};
   bool pages_ok;
-  if constexpr (D >= 64)
-    pages_ok = p.attn_mma ? attn_pages_mma<D>(p, ctl, smem, S, st, A, own_cur, cur, part, ctid)
-                          : attn_pages_cuda<D>(p, ctl, smem, S, st, A, own_cur, cur, part, ctid);
+  if constexpr (AMMA && D >= 64)
+    pages_ok = attn_pages_mma<D>(p, ctl, smem, S, st, A, own_cur, cur, part, ctid);
   else
     pages_ok = attn_pages_cuda<D>(p, ctl, smem, S, st, A, own_cur, cur, part, ctid);
   if (!pages_ok) return false;
@@ -2345,8 +2376,9 @@ __device__ void embed_task(const Params &p, const Slot &S, int ctid) {
 // compute warps: main loop
 // ============================================================================
 
-template <bool TC>
+template <int V>
 __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
+  constexpr bool TC = (V & kVarTc) != 0, W4 = (V & kVarW4) != 0, AMMA = (V & kVarAttnMma) != 0;
   const int ctid = threadIdx.x - 32;
   Slot *slots = reinterpret_cast<Slot *>(smem + p.off_slots);
   ComputeState st;
@@ -2383,9 +2415,9 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       case T_ATTN:
         if (S.b >= 0) {
           switch (p.d >> 5) {
-            case 1: tok = attn_task<32>(p, ctl, smem, S, st, out, ctid); break;
-            case 2: tok = attn_task<64>(p, ctl, smem, S, st, out, ctid); break;
-            default: tok = attn_task<128>(p, ctl, smem, S, st, out, ctid); break;
+            case 1: tok = attn_task<32, AMMA>(p, ctl, smem, S, st, out, ctid); break;
+            case 2: tok = attn_task<64, AMMA>(p, ctl, smem, S, st, out, ctid); break;
+            default: tok = attn_task<128, AMMA>(p, ctl, smem, S, st, out, ctid); break;
           }
         }
         break;
@@ -2394,9 +2426,9 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
           tok = p.tc_n > 16 ? gemv_task_tc<2>(p, ctl, smem, S, st, out, ctid)
                             : gemv_task_tc<1>(p, ctl, smem, S, st, out, ctid);
         else
-          tok = p.batch > 8   ? gemv_task<4>(p, ctl, smem, S, st, out, ctid)
-                : p.batch > 4 ? gemv_task<2>(p, ctl, smem, S, st, out, ctid)
-                              : gemv_task<1>(p, ctl, smem, S, st, out, ctid);
+          tok = p.batch > 8   ? gemv_task<4, W4>(p, ctl, smem, S, st, out, ctid)
+                : p.batch > 4 ? gemv_task<2, W4>(p, ctl, smem, S, st, out, ctid)
+                              : gemv_task<1, W4>(p, ctl, smem, S, st, out, ctid);
         break;
     }
     if (!tok) {
@@ -2648,9 +2680,11 @@ __device__ void storer_main(const Params &p, Ctl *ctl, uint8_t *smem) {
 // kernel
 // ============================================================================
 
-// One instantiation per GEMV path (TC: tcgen05 tiles; else mma.sync pages),
-// so neither carries the other's code.
-template <bool TC>
+// One instantiation per variant V (kVarTc: tcgen05 tiles, else mma.sync
+// pages; kVarW4: the 4-bit weight consumer; kVarAttnMma: attention on
+// mma.sync tiles over swizzled K/V pages), so no plan carries code (and
+// register pressure) of a path it does not run.
+template <int V>
 __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Ctl *ctl = reinterpret_cast<Ctl *>(smem);
@@ -2696,11 +2730,11 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   if (!ctl->skip) {
     const int warp = threadIdx.x >> 5;
     if (warp == kLoaderWarp) {
-      loader_main<TC>(p, ctl, smem);
+      loader_main<V>(p, ctl, smem);
     } else if (warp == kStorerWarp) {
       storer_main(p, ctl, smem);
     } else {
-      compute_main<TC>(p, ctl, smem);
+      compute_main<V>(p, ctl, smem);
     }
   }
   if (p.tc) tc_fence_before();
@@ -2723,28 +2757,50 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
 // min(device opt-in, kMaxSmem)), never to one plan's own size: plans of
 // different shapes and the no-allocation entry point share the kernel, and a
 // later, smaller setting would fail the launches of an earlier, larger one.
+namespace {
+// the variants plans use: mma.sync or tcgen05 projections, 4-bit weights
+// only on mma.sync, each with either attention path
+constexpr int kVariants[] = {0, kVarTc, kVarW4, kVarAttnMma, kVarTc | kVarAttnMma,
+                             kVarW4 | kVarAttnMma};
+
+const void *kernel_for(int v) {
+  switch (v) {
+    case 0: return reinterpret_cast<const void *>(mk_step_kernel<0>);
+    case kVarTc: return reinterpret_cast<const void *>(mk_step_kernel<kVarTc>);
+    case kVarW4: return reinterpret_cast<const void *>(mk_step_kernel<kVarW4>);
+    case kVarAttnMma: return reinterpret_cast<const void *>(mk_step_kernel<kVarAttnMma>);
+    case kVarTc | kVarAttnMma:
+      return reinterpret_cast<const void *>(mk_step_kernel<kVarTc | kVarAttnMma>);
+    case kVarW4 | kVarAttnMma:
+      return reinterpret_cast<const void *>(mk_step_kernel<kVarW4 | kVarAttnMma>);
+    default: return nullptr;
+  }
+}
+}  // namespace
+
+int kernel_variant(const Params &p) {
+  return (p.tc ? kVarTc : 0) | (p.w4 ? kVarW4 : 0) | (p.attn_mma ? kVarAttnMma : 0);
+}
+
 cudaError_t configure_kernel(int smem_optin) {
   const int lim = smem_optin < kMaxSmem ? smem_optin : kMaxSmem;
-  cudaError_t e = cudaFuncSetAttribute(mk_step_kernel<false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(mk_step_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-  return e;
+  for (int v : kVariants) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel_for(v), cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_step(const Params &p, int grid, int smem, bool cooperative, cudaStream_t stream) {
-  if (cooperative) {
-    void *args[] = {const_cast<Params *>(&p)};
-    const void *fn = p.tc ? reinterpret_cast<const void *>(mk_step_kernel<true>)
-                          : reinterpret_cast<const void *>(mk_step_kernel<false>);
-    return cudaLaunchCooperativeKernel(fn, dim3(grid),
-                                       dim3(kThreads), args, static_cast<size_t>(smem), stream);
-  }
-  if (p.tc)
-    mk_step_kernel<true><<<grid, kThreads, smem, stream>>>(p);
-  else
-    mk_step_kernel<false><<<grid, kThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  const void *fn = kernel_for(kernel_variant(p));
+  if (fn == nullptr) return cudaErrorInvalidValue;
+  void *args[] = {const_cast<Params *>(&p)};
+  if (cooperative)
+    return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kThreads), args,
+                                       static_cast<size_t>(smem), stream);
+  return cudaLaunchKernel(fn, dim3(grid), dim3(kThreads), args, static_cast<size_t>(smem),
+                          stream);
 }
 
 }  // namespace mk

@@ -148,6 +148,11 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     return lfail(err, MK_ERR_INVALID_ARG, "max_page_cols %d: 32..%d, a multiple of 32", colcap,
                  kMaxPageCols);
   const int grid = o.num_ctas > 0 ? std::min(o.num_ctas, nsm) : nsm;
+  if (o.attn_path < 0 || o.attn_path > 2)
+    return lfail(err, MK_ERR_INVALID_ARG, "attn_path %d: 0 automatic, 1 CUDA cores, 2 mma.sync",
+                 o.attn_path);
+  if (o.attn_path == 2 && d != 64 && d != 128)
+    return lfail(err, MK_ERR_UNSUPPORTED, "the mma.sync attention path needs head_dim 64 or 128");
   const int smem_max = std::min(smem_optin, kMaxSmem);
   const int mt_cap = max_mtiles_for(maxB);
 
@@ -446,7 +451,9 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   p.wait_limit_ns = o.wait_limit_ns;
   p.n_ffn_parts = n_ksplit;
   p.chunk_seq = -1;   // decode steps (a prompt chunk sets its sequence)
-  p.attn_mma = (d == 64 || d == 128) ? 1 : 0;
+  // the CUDA-core attention is the default: it measured faster at every
+  // batch size of the 8B decode workloads
+  p.attn_mma = o.attn_path == 2 ? 1 : 0;
   p.w4 = o.w4 ? 1 : 0;
   p.n_out = n_out;
   p.tile_rows = tc ? kTcRows : 16;

@@ -78,7 +78,7 @@ class mk_plan_options(C.Structure):
                 ("wait_limit_ns", C.c_int64), ("rows_per_task", C.c_int * 5),
                 ("debug_unsatisfiable_dep", C.c_int), ("max_page_cols", C.c_int),
                 ("o_split", C.c_int), ("gemv_path", C.c_int), ("schedule", C.c_int),
-                ("weight_bits", C.c_int), ("prefill", C.c_int)]
+                ("weight_bits", C.c_int), ("prefill", C.c_int), ("attn_path", C.c_int)]
 
 
 class mk_step_args(C.Structure):
@@ -105,7 +105,7 @@ class mk_plan_info_t(C.Structure):
                 ("ffn_part_cols", C.c_int), ("o_parts", C.c_int), ("o_part_cols", C.c_int),
                 ("gemv_path", C.c_int), ("schedule", C.c_int), ("prefill", C.c_int),
                 ("weight_bits", C.c_int), ("qkv_parts", C.c_int),
-                ("gateup_parts", C.c_int)]
+                ("gateup_parts", C.c_int), ("attn_path", C.c_int)]
 
 
 _lib = None
@@ -221,7 +221,8 @@ def _config(cfg: Dict, max_seq_len: int) -> mk_model_config:
 def describe(cfg: Dict, max_batch: int = 1, page_size: int = 16, max_seq_len: int = 4096,
              num_sms: int = 148, smem_optin: int = 232448, rows_per_task=(0, 0, 0, 0, 0),
              max_page_cols: int = 0, o_split: bool = False, gemv_path: int = 0,
-             schedule: int = 0, prefill: bool = False, weight_bits: int = 0):
+             schedule: int = 0, prefill: bool = False, weight_bits: int = 0,
+             attn_path: int = 0):
     """The plan mk_plan_create_ex would build, without a GPU: (info, task records).
 
     The task records are a numpy structured array (TASK_RECORD_DTYPE)."""
@@ -230,7 +231,7 @@ def describe(cfg: Dict, max_batch: int = 1, page_size: int = 16, max_seq_len: in
     c = _config(cfg, max_seq_len)
     opts = mk_plan_options(max_batch, page_size, 0, 0, (C.c_int * 5)(*rows_per_task), 0,
                            max_page_cols, 1 if o_split else 0, gemv_path, schedule, weight_bits,
-                           1 if prefill else 0)
+                           1 if prefill else 0, attn_path)
     info = mk_plan_info_t()
     _check(lib.mk_plan_describe(C.byref(c), C.byref(opts), num_sms, smem_optin, C.byref(info),
                                 None, 0))
@@ -310,7 +311,7 @@ class Plan:
                  max_seq_len: int = 4096, num_ctas: int = 0, wait_limit_ns: int = 0,
                  rows_per_task: Sequence[int] = (0, 0, 0, 0, 0), debug_unsatisfiable_dep=False,
                  max_page_cols: int = 0, o_split: bool = False, gemv_path: int = 0,
-                 schedule: int = 0, prefill: bool = False):
+                 schedule: int = 0, prefill: bool = False, attn_path: int = 0):
         lib = load_library()
         self.cfg = dict(cfg)
         self.max_batch = max_batch
@@ -321,7 +322,7 @@ class Plan:
         opts = mk_plan_options(max_batch, page_size, num_ctas, wait_limit_ns,
                                (C.c_int * 5)(*rows_per_task), 1 if debug_unsatisfiable_dep else 0,
                                max_page_cols, 1 if o_split else 0, gemv_path, schedule, 0,
-                               1 if prefill else 0)
+                               1 if prefill else 0, attn_path)
         h = C.c_void_p()
         _check(lib.mk_plan_create_ex(C.byref(self._c), C.byref(self._w), C.byref(opts),
                                      C.byref(h)))

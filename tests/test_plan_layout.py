@@ -251,6 +251,27 @@ def test_batch1_8b_plan_facts():
     assert info["o_parts"] == 1
 
 
+def test_attention_path_option():
+    """CUDA-core attention by default; the mma.sync attention on request for
+    head_dim 64 and 128 only; out-of-range values are argument errors.  The
+    task graph does not depend on the attention path."""
+    for name in ("tiny", "8b"):
+        i0, t0 = mk.describe(SHAPES[name], max_batch=4, max_seq_len=256)
+        i2, t2 = mk.describe(SHAPES[name], max_batch=4, max_seq_len=256, attn_path=2)
+        assert i0["attn_path"] == 1 and i2["attn_path"] == 2
+        assert (t0 == t2).all()
+        assert i0["smem_bytes"] == i2["smem_bytes"] and i0["page_bytes"] == i2["page_bytes"]
+    d32 = dict(SHAPES["tiny"], head_dim=32)
+    assert mk.describe(d32, attn_path=1)[0]["attn_path"] == 1
+    with pytest.raises(mk.MkError) as e:
+        mk.describe(d32, attn_path=2)
+    assert e.value.code == mk.MK_ERR_UNSUPPORTED
+    for bad in (-1, 3):
+        with pytest.raises(mk.MkError) as e:
+            mk.describe(SHAPES["tiny"], attn_path=bad)
+        assert e.value.code == mk.MK_ERR_INVALID_ARG
+
+
 def test_describe_rejects_what_create_rejects():
     cfg = dict(SHAPES["tiny"], head_dim=96)
     with pytest.raises(mk.MkError):
