@@ -204,13 +204,17 @@ typedef struct {
                              them, so a row may attend to positions that
                              other rows of the same launch write.  Decode
                              steps on such a plan give the same results    */
-  int attn_path;          /* how attention runs: 0 = automatic (1), 1 = CUDA
-                             cores: fp32 FMA over K/V pages bulk-copied into
-                             shared memory; 2 = mma.sync tensor-core tiles:
-                             K/V pages copied by TMA tensor copies with the
-                             128-byte swizzle, q.K and P.V as m16n8k16 MMAs
-                             fed by ldmatrix (head_dim 64 or 128, else
-                             MK_ERR_UNSUPPORTED)                            */
+  int attn_path;          /* how attention runs: 0 = automatic (2 when
+                             max_batch >= 2 and head_dim is 64 or 128, else
+                             1); 1 = CUDA cores: fp32 FMA over K/V pages
+                             bulk-copied into shared memory, three phases
+                             per page; 2 = mma.sync tensor-core tiles: K/V
+                             pages copied by TMA tensor copies with the
+                             128-byte swizzle, each warp an online softmax
+                             over its own 16-token slices (q.K and P.V as
+                             m16n8k16 MMAs fed by ldmatrix), the warps
+                             merged at the chunk's end (head_dim 64 or 128,
+                             else MK_ERR_UNSUPPORTED)                       */
 } mk_plan_options;
 
 typedef struct mk_plan mk_plan;

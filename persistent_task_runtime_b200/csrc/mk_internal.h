@@ -44,6 +44,7 @@ constexpr int kTcAtomBytes = kTcRows * 128;       // one weight atom: 128 rows x
 constexpr int kTcXBytes = 32 * 1024;              // one staged activation chunk buffer
 constexpr int kTcTmemCols = 128;                  // tensor-memory columns allocated per CTA
 constexpr int kTcAutoBatch = 5;                   // smallest max_batch that takes it by default
+constexpr int kAttnMmaAutoBatch = 2;              // smallest max_batch that takes the mma.sync attention
 constexpr int kTcMatsPerLayer = 7;                // tensor maps: wq wk wv wo w_gate w_up w_down
 
 // ---- kernel variants (template argument of the step kernel) -------------------

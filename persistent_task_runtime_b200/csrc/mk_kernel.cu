@@ -1799,6 +1799,8 @@ __device__ __forceinline__ void comb_batch(const float *ph, size_t cstride, int 
 struct AttnSmem {
   float *qs, *sc, *mst, *lst, *cor;
   __nv_bfloat16 *kvcur;
+  float *wmerge;   // mma.sync path: the warps' (O, m, l) before their merge
+  int *pg_cnt;     // mma.sync path, tensor-core plans: warps done per ring page
 };
 
 // The chunk's pages on the CUDA cores (head_dim 32, or a plan without the
@@ -1937,45 +1939,45 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
 }
-__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t &r0, uint32_t &r1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
-               : "=r"(r0), "=r"(r1)
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1,
+                                              uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
 }
 
-// Shared-memory address of dims k..k+7 (k a multiple of 8) of token t of a
-// K or V area holding P-token KV pages as the TMA copies laid them out: per
-// KV page, 64-dim atoms of P rows x 128 bytes, the 16-byte chunk c of a row
-// at chunk c XOR (row address bits 7..9) (128-byte swizzle).
-template <int D>
-__device__ __forceinline__ uint32_t kv_addr(uint32_t base, int t, int k, int P) {
-  const int j = t / P, r = t - j * P;
-  const uint32_t row = base + static_cast<uint32_t>(j * (P * D * 2) + (k >> 6) * (P * 128) + r * 128);
-  return row + (((static_cast<uint32_t>((k & 63) >> 3)) ^ ((row >> 7) & 7u)) << 4);
+// 16-byte chunk `c` (0..7) of the 128-byte row at `row` in a 128-byte-swizzled
+// TMA box (box base 1024-byte aligned): the chunk sits at c XOR row bits 7..9.
+__device__ __forceinline__ uint32_t sw128(uint32_t row, int c) {
+  return row + ((static_cast<uint32_t>(c) ^ ((row >> 7) & 7u)) << 4);
 }
 
-// fp32 pair -> (hi, lo) bf16x2 pairs, hi + lo == x to ~2^-16.
+// fp32 pair -> (hi, lo) bf16x2 pairs (first value in the low half),
+// hi + lo == x to ~2^-16: two paired conversions.
 __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uint32_t &lo) {
-  __nv_bfloat16 h0, l0, h1, l1;
-  split_bf16(x0, h0, l0);
-  split_bf16(x1, h1, l1);
-  hi = pack2(h0, h1);
-  lo = pack2(l0, l1);
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __low2float(h), x1 - __high2float(h));
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
 // The chunk's pages on the tensor cores (mma.sync m16n8k16, bf16 -> fp32),
-// K and V pages copied by TMA in the 128-byte-swizzled layout (kv_addr), so
-// every ldmatrix reads conflict-free.  Per page:
-//   1. S = Q K^T: A = the G query heads as rows, bf16 high halves in rows
-//      0..7 and low halves in rows 8..15 (registers, built once per chunk);
-//      B = 8 tokens x 16 dims from ldmatrix; score(head g, token) = row g +
-//      row g + 8 of the result;
-//   2. softmax statistics, one warp per head, as on the CUDA cores;
-//   3. O += P V: A = p of the G heads (high/low rows), 16 tokens per step;
-//      B = V tokens x 8 dims from ldmatrix.trans; each warp owns a few 8-dim
-//      tiles of O, rescaled by the page's correction before it adds.
-// Tokens past the chunk's end in the page's last 16: p = 0 and their V rows
-// zeroed (the cache may hold anything there).
+// K and V pages copied by TMA in the 128-byte-swizzled layout (per KV page,
+// 64-dim boxes of P rows x 128 bytes), so every ldmatrix reads conflict-free.
+// Flash decoding inside the CTA: the chunk's tokens are cut into 16-token
+// slices dealt round-robin to the compute warps, and each warp keeps its own
+// online softmax (running max m, sum l) and unnormalised O in registers, so
+// warps never wait for one another inside the chunk.  Per slice:
+//   S = Q K^T: A = the G query heads as rows, bf16 high halves in rows
+//   0..7 and low halves in rows 8..15 (registers, built once per chunk); B =
+//   8 tokens x 16 dims by ldmatrix; the score of head g = row g + row g + 8;
+//   the slice's max (a quad shuffle), rescale, p = 2^(s - m);
+//   O += P V: A = p of the G heads as high/low rows, straight from the score
+//   registers; B = 16 tokens x 8 dims by ldmatrix.trans.
+// Tokens past the page's end: score -inf and their V rows zeroed (the cache
+// may hold anything there).  At the end the warps' (m, l, O) merge through
+// shared memory by log-sum-exp into the chunk's partial.  A page goes back
+// to the loader when its last warp is done with it.
 template <int D>
 __device__ bool attn_pages_mma(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
                                ComputeState &st, const AttnSmem &A, bool own_cur, int cur,
@@ -1983,151 +1985,193 @@ __device__ bool attn_pages_mma(const Params &p, Ctl *ctl, uint8_t *smem, const S
   const int warp = ctid >> 5, lane = ctid & 31;
   const int G = p.G, P = p.page_size, tpp = p.tpp;
   const int g = lane >> 2, q = lane & 3;
-  constexpr int NB = D / 8;
+  constexpr int NB = D / 8;                  // 16-byte chunks per row
   constexpr int KS = D / 16;                 // k-steps of the scores
-  constexpr int NT = (D / 8 + kComputeWarps - 1) / kComputeWarps;   // O tiles per warp
-  float *sc = A.sc, *mst = A.mst, *lst = A.lst, *cor = A.cor;
-  const int rw = D + 4;
+  constexpr int DT = D / 8;                  // 8-dim tiles of O
+  const bool hrow = g < G;                   // rows g / g + 8 carry head g
+  const uint32_t kvbytes = static_cast<uint32_t>(P * D * 2);   // one KV page of K (or V)
 
   // the query fragments (rows g: high halves of head g, g + 8: low halves)
   uint32_t qa[KS][4];
 #pragma unroll
   for (int s = 0; s < KS; ++s) {
     float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
-    if (g < G) {
+    if (hrow) {
       const float *qh = A.qs + g * D + 16 * s + 2 * q;
       x0 = qh[0]; x1 = qh[1]; x2 = qh[8]; x3 = qh[9];
     }
     split_pair(x0, x1, qa[s][0], qa[s][1]);
     split_pair(x2, x3, qa[s][2], qa[s][3]);
   }
-  float acc[NT][4];
+  float m_run = -INFINITY, l_run = 0.f;   // head g; l_run: this lane's tokens only
+  float acc[DT][4];
 #pragma unroll
-  for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  for (int i = 0; i < DT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 
+  bool bad = false;
+  int slice0 = 0;   // chunk-relative index of the page's first slice
   for (int tok0 = S.t0; tok0 < S.t1; tok0 += tpp) {
     const int ntok = min(tpp, S.t1 - tok0);
-    bool okl = true;
-    if (ctid == 0) okl = wait_mbar(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff40000u, 2);
-    if (!st.gs.share(ctl, ctid, okl)) return false;
-    mbar_try_wait(&ctl->full[st.pi], st.pg_par);
-    uint8_t *kpg = smem + p.off_pages + static_cast<size_t>(st.pi) * p.page_bytes;
-    uint8_t *vpg = kpg + static_cast<size_t>(tpp) * D * 2;
-    const uint32_t ks = smem_u32(kpg), vs = smem_u32(vpg);
-    // the current token's K/V into its slot (the page was copied before they
-    // were formed), and zero V rows past the chunk's end up to a multiple of 16
-    const bool has_cur = own_cur && cur >= tok0 && cur < tok0 + ntok;
-    const int nz = ((ntok + 15) & ~15) - ntok;
-    if (has_cur && ctid < 2 * NB) {
-      const bool isv = ctid >= NB;
-      const int e = (isv ? ctid - NB : ctid) * 8;
-      sts128(kv_addr<D>(isv ? vs : ks, cur - tok0, e, P),
-             *reinterpret_cast<const uint4 *>(A.kvcur + (isv ? D : 0) + e));
-    }
-    for (int u = ctid; u < nz * NB; u += kComputeThreads)
-      sts128(kv_addr<D>(vs, ntok + u / NB, (u % NB) * 8, P), make_uint4(0, 0, 0, 0));
-    if (has_cur || nz > 0) compute_bar();
-
-    // phase 1: scores, 8 tokens per mma tile
-    const int ntl = (ntok + 7) >> 3;
-    for (int j = warp; j < ntl; j += kComputeWarps) {
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int s2 = 0; s2 < KS / 2; ++s2) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kv_addr<D>(ks, 8 * j + (lane & 7), 32 * s2 + 8 * (lane >> 3), P), b0, b1, b2, b3);
-        mma_bf16(c, qa[2 * s2][0], qa[2 * s2][1], qa[2 * s2][2], qa[2 * s2][3], b0, b1);
-        mma_bf16(c, qa[2 * s2 + 1][0], qa[2 * s2 + 1][1], qa[2 * s2 + 1][2], qa[2 * s2 + 1][3],
-                 b2, b3);
-      }
-      const int t0 = 8 * j + 2 * q;
-      if (g < G) {
-        if (t0 < ntok) sc[g * tpp + t0] = c[0] + c[2];
-        if (t0 + 1 < ntok) sc[g * tpp + t0 + 1] = c[1] + c[3];
-      }
-    }
-    compute_bar();
-    // phase 2: softmax statistics, one warp per head
-    for (int h = warp; h < G; h += kComputeWarps) {
-      float *row = sc + h * tpp;
-      float mx = -INFINITY;
-      for (int tk = lane; tk < ntok; tk += 32) mx = fmaxf(mx, row[tk]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float mold = mst[h];
-      const float mnew = fmaxf(mold, mx);
-      float sum = 0.f;
-      for (int tk = lane; tk < ntok; tk += 32) {
-        const float pr = exp2f(row[tk] - mnew);
-        row[tk] = pr;
-        sum += pr;
-      }
-      sum = warp_sum(sum);
-      __syncwarp();
+    const int nsl = (ntok + 15) >> 4;
+    if (!bad && !warp_wait_page(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff40000u)) {
+      bad = true;
       if (lane == 0) {
-        const float cc = exp2f(mold - mnew);   // 0 on the first page (mold = -inf)
-        cor[h] = cc;
-        lst[h] = lst[h] * cc + sum;
-        mst[h] = mnew;
+        ctl->cbad = 1;
+        ctl->cta_abort = 1;
       }
     }
-    compute_bar();
-    // phase 3: O = O * correction + P V over 16-token steps
-    {
-      const float cg = g < G ? cor[g] : 0.f;
+    if (!bad) {
+      const uint32_t ks = smem_u32(smem + p.off_pages + static_cast<size_t>(st.pi) * p.page_bytes);
+      const uint32_t vs = ks + static_cast<uint32_t>(tpp * D * 2);
+      bool wrote = false;
+      for (int sl = (warp + kComputeWarps - slice0 % kComputeWarps) % kComputeWarps; sl < nsl;
+           sl += kComputeWarps) {
+        const int tb = 16 * sl;                       // first token of the slice in the page
+        const int jp = tb / P;                        // its KV page
+        const uint32_t krow = ks + jp * kvbytes + static_cast<uint32_t>(tb - jp * P) * 128u;
+        const uint32_t vrow = vs + jp * kvbytes + static_cast<uint32_t>(tb - jp * P) * 128u;
+        const uint32_t atom = static_cast<uint32_t>(P * 128);   // one 64-dim box
+        // the current token's K/V into its row (the page was copied before
+        // they were formed), and V rows past the page's end zeroed
+        const int rc = cur - tok0 - tb;
+        if (own_cur && rc >= 0 && rc < 16 && tb + rc < ntok) {
+          if (lane < 2 * NB) {
+            const bool isv = lane >= NB;
+            const int c = isv ? lane - NB : lane;
+            sts128(sw128((isv ? vrow : krow) + (c >> 3) * atom + rc * 128u, c & 7),
+                   *reinterpret_cast<const uint4 *>(A.kvcur + (isv ? D : 0) + 8 * c));
+          }
+          wrote = true;
+        }
+        const int nvalid = min(16, ntok - tb);
+        if (nvalid < 16) {
+          for (int u = lane; u < (16 - nvalid) * NB; u += 32) {
+            const int r = nvalid + u / NB, c = u % NB;
+            sts128(sw128(vrow + (c >> 3) * atom + r * 128u, c & 7), make_uint4(0, 0, 0, 0));
+          }
+          wrote = true;
+        }
+        __syncwarp();
+        // scores: two 8-token tiles
+        float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        acc[i][0] *= cg; acc[i][1] *= cg; acc[i][2] *= cg; acc[i][3] *= cg;
-      }
-      const int nks = (ntok + 15) >> 4;
-      for (int u = 0; u < nks; ++u) {
-        const int t = 16 * u + 2 * q;
+        for (int s2 = 0; s2 < KS / 2; ++s2) {
+          const int dim = 32 * s2 + 8 * (lane >> 3);
+          const uint32_t rb = krow + (dim >> 6) * atom;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(sw128(rb + (lane & 7) * 128u, (dim & 63) >> 3), b0, b1, b2, b3);
+          mma_bf16(c0, qa[2 * s2][0], qa[2 * s2][1], qa[2 * s2][2], qa[2 * s2][3], b0, b1);
+          mma_bf16(c0, qa[2 * s2 + 1][0], qa[2 * s2 + 1][1], qa[2 * s2 + 1][2], qa[2 * s2 + 1][3],
+                   b2, b3);
+          ldsm_x4(sw128(rb + (8 + (lane & 7)) * 128u, (dim & 63) >> 3), b0, b1, b2, b3);
+          mma_bf16(c1, qa[2 * s2][0], qa[2 * s2][1], qa[2 * s2][2], qa[2 * s2][3], b0, b1);
+          mma_bf16(c1, qa[2 * s2 + 1][0], qa[2 * s2 + 1][1], qa[2 * s2 + 1][2], qa[2 * s2 + 1][3],
+                   b2, b3);
+        }
+        // this lane's tokens: 2q, 2q + 1, 8 + 2q, 9 + 2q of the slice
+        float s0 = c0[0] + c0[2], s1 = c0[1] + c0[3], s2v = c1[0] + c1[2], s3 = c1[1] + c1[3];
+        if (2 * q >= nvalid) s0 = -INFINITY;
+        if (2 * q + 1 >= nvalid) s1 = -INFINITY;
+        if (8 + 2 * q >= nvalid) s2v = -INFINITY;
+        if (9 + 2 * q >= nvalid) s3 = -INFINITY;
+        float mx = fmaxf(fmaxf(s0, s1), fmaxf(s2v, s3));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        // (token 0 of a slice is always valid: mx is finite for head rows)
         float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-        if (g < G) {
-          const float *prow = sc + g * tpp;
-          if (t < ntok) p0 = prow[t];
-          if (t + 1 < ntok) p1 = prow[t + 1];
-          if (t + 8 < ntok) p2 = prow[t + 8];
-          if (t + 9 < ntok) p3 = prow[t + 9];
+        if (hrow) {
+          const float mnew = fmaxf(m_run, mx);
+          const float sc = exp2f(m_run - mnew);   // 0 on the first slice (m_run = -inf)
+          p0 = exp2f(s0 - mnew);
+          p1 = exp2f(s1 - mnew);
+          p2 = exp2f(s2v - mnew);
+          p3 = exp2f(s3 - mnew);
+          l_run = l_run * sc + ((p0 + p1) + (p2 + p3));
+          m_run = mnew;
+#pragma unroll
+          for (int i = 0; i < DT; ++i) {
+            acc[i][0] *= sc; acc[i][1] *= sc; acc[i][2] *= sc; acc[i][3] *= sc;
+          }
         }
         uint32_t a0, a1, a2, a3;
         split_pair(p0, p1, a0, a1);
         split_pair(p2, p3, a2, a3);
+        // O += P V, two 8-dim tiles per ldmatrix
 #pragma unroll
-        for (int i = 0; i < NT; ++i) {
-          const int dt = warp + i * kComputeWarps;   // this warp's 8-dim tile
-          if (dt < D / 8) {
-            uint32_t b0, b1;
-            ldsm_x2_trans(kv_addr<D>(vs, 16 * u + (lane & 15), 8 * dt, P), b0, b1);
-            mma_bf16(acc[i], a0, a1, a2, a3, b0, b1);
-          }
+        for (int i = 0; i < DT; i += 2) {
+          const int dim = 8 * i + 8 * (lane >> 4);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_trans(sw128(vrow + (dim >> 6) * atom + (lane & 15) * 128u, (dim & 63) >> 3), b0,
+                        b1, b2, b3);
+          mma_bf16(acc[i], a0, a1, a2, a3, b0, b1);
+          mma_bf16(acc[i + 1], a0, a1, a2, a3, b2, b3);
         }
       }
+      if (wrote) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (has_cur || nz > 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    // the page goes back to the loader once every warp is done with it
     __syncwarp();
-    if (!p.tc && lane == 0) mbar_arrive(&ctl->empty[st.pi]);
-    compute_bar();   // sc is rewritten by the next page
-    // (tensor-core plans release a page once, after every warp is done with it)
-    if (p.tc && ctid == 0) mbar_arrive(&ctl->empty[st.pi]);
+    if (lane == 0) {
+      if (p.tc) {
+        __threadfence_block();
+        if (atomicAdd(&A.pg_cnt[st.pi], 1) == kComputeWarps - 1) {
+          A.pg_cnt[st.pi] = 0;
+          mbar_arrive(&ctl->empty[st.pi]);
+        }
+      } else {
+        mbar_arrive(&ctl->empty[st.pi]);
+      }
+    }
+    slice0 += nsl;
     if (++st.pi == p.n_pages) {
       st.pi = 0;
       st.pg_par ^= 1u;
     }
   }
-  // the chunk's partial: row h = (sum, m, l, pad); head g's sums are the
-  // high row g plus the low row g + 8
-  if (g < G) {
+
+  // merge the warps: (m, l) per head and O per (head, dim) through shared memory
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  float *wO = A.wmerge;                                   // [warp][G][D]
+  float *wM = wO + kComputeWarps * G * D;                 // [warp][G]
+  float *wL = wM + kComputeWarps * G;                     // [warp][G]
+  if (hrow) {
+    float *o = wO + (warp * G + g) * D;
 #pragma unroll
-    for (int i = 0; i < NT; ++i) {
-      const int dt = warp + i * kComputeWarps;
-      if (dt < D / 8) {
-        const int d0 = 8 * dt + 2 * q;
-        __stcg(reinterpret_cast<float2 *>(part + g * rw + d0),
-               make_float2(acc[i][0] + acc[i][2], acc[i][1] + acc[i][3]));
-      }
+    for (int i = 0; i < DT; ++i)
+      *reinterpret_cast<float2 *>(o + 8 * i + 2 * q) =
+          make_float2(acc[i][0] + acc[i][2], acc[i][1] + acc[i][3]);
+    if (q == 0) {
+      wM[warp * G + g] = m_run;
+      wL[warp * G + g] = l_run;
     }
   }
+  compute_bar();
+  if (ctl->cbad != 0) return false;
+  constexpr int Q4 = D / 4;
+  for (int e = ctid; e < G * Q4; e += kComputeThreads) {
+    const int h = e / Q4, i4 = (e % Q4) * 4;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, wM[w * G + h]);
+    float den = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kComputeWarps; ++w) {
+      const float mw = wM[w * G + h];
+      const float wt = mw == -INFINITY ? 0.f : exp2f(mw - M);   // a warp without tokens
+      den += wt * wL[w * G + h];
+      const float4 o = *reinterpret_cast<const float4 *>(wO + (w * G + h) * D + i4);
+      num.x += wt * o.x; num.y += wt * o.y; num.z += wt * o.z; num.w += wt * o.w;
+    }
+    const int rw = D + 4;
+    __stcg(reinterpret_cast<float4 *>(part + h * rw + i4), num);
+    if (i4 == 0) {
+      A.mst[h] = M;
+      A.lst[h] = den;
+    }
+  }
+  compute_bar();
   return true;
 }
 
@@ -2153,6 +2197,8 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
   float *lst = mst + kMaxGroup;                             // [G] running sum
   float *cor = lst + kMaxGroup;                             // [G] rescale of this page
   __nv_bfloat16 *kvcur = reinterpret_cast<__nv_bfloat16 *>(cor + kMaxGroup);  // [2][D] K, V at pos
+  int *pg_cnt = reinterpret_cast<int *>(kvcur + 2 * D);     // [kMaxPages]
+  float *wmerge = reinterpret_cast<float *>(pg_cnt + kMaxPages);   // [warps][G][D + 2]
   st.xkey = 0xffffffffu;                                    // staging area reused
 
   {
@@ -2209,12 +2255,13 @@ __device__ bool attn_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     mst[ctid] = -INFINITY;
     lst[ctid] = 0.f;
   }
+  if (AMMA && ctid < kMaxPages) pg_cnt[ctid] = 0;
   compute_bar();
   if (ctid == 0) trace_mark(p, S.idx, 5);
 
   const int rw = D + 4;
   float *part = p.attn_part + static_cast<size_t>(t.aux) * G * rw;
-  AttnSmem A{qs, sc, mst, lst, cor, kvcur};
+  AttnSmem A{qs, sc, mst, lst, cor, kvcur, wmerge, pg_cnt};
   bool pages_ok;
   if constexpr (AMMA && D >= 64)
     pages_ok = attn_pages_mma<D>(p, ctl, smem, S, st, A, own_cur, cur, part, ctid);

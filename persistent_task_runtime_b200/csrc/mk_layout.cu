@@ -153,6 +153,11 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
                  o.attn_path);
   if (o.attn_path == 2 && d != 64 && d != 128)
     return lfail(err, MK_ERR_UNSUPPORTED, "the mma.sync attention path needs head_dim 64 or 128");
+  // attention on mma.sync tiles on request, and by default from batch 2 up
+  // (measured on the 8B shape: as fast as the CUDA-core path at batch 1,
+  // 4-17% faster steps from batch 2 to 16)
+  const bool attn_mma = o.attn_path == 2 ||
+                        (o.attn_path == 0 && (d == 64 || d == 128) && maxB >= kAttnMmaAutoBatch);
   const int smem_max = std::min(smem_optin, kMaxSmem);
   const int mt_cap = max_mtiles_for(maxB);
 
@@ -261,16 +266,35 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     tc_kx = kTcXBytes / (2 * tc_bpad * 2);   // bf16 hi + lo rows of tc_bpad sequences
     tc_kc = 128;                             // 32 KB pages (128 rows x 128 columns)
     R_qkv = R_o = R_gu = R_d = R_lm = kTcRows;
-    auto parts_for = [&](int tiles, int K, int i) {
-      int n = std::max(1, std::min(cdiv(3 * grid, 2 * tiles), K / tc_kc));
-      int w = align_up_i(cdiv(K, n), tc_kc);
-      n = cdiv(K, w);
-      split[i] = n;
-      kt[i] = n > 1 ? w : 0;
+    // Split-K parts of an operator of `tiles` tasks' worth of n_m 128-row
+    // tiles over K columns: the count that minimises the operator's makespan
+    // on `grid` CTAs in a simple model, rounds of tasks (ceil(tasks / grid))
+    // times a task's weight columns (per tile) plus a fixed cost per task
+    // (epilogue, split-K sum and hand-offs, about 4 us: the time one SM's
+    // share of HBM streams 640 columns of a 128-row tile).  Ties go to fewer
+    // parts.
+    auto parts_for = [&](int tiles, int nm, int K, int i) {
+      constexpr long long kTaskCostCols = 640;
+      const int nmax = std::max(1, K / tc_kc);
+      long long best = -1;
+      int bn = 1, bw = K;
+      for (int n = 1; n <= nmax; ++n) {
+        const int w = align_up_i(cdiv(K, n), tc_kc);
+        if (cdiv(K, w) != n) continue;   // the same split as a smaller count
+        const long long rounds = cdiv(tiles * n, grid);
+        const long long cost = rounds * (static_cast<long long>(nm) * w + kTaskCostCols);
+        if (best < 0 || cost < best) {
+          best = cost;
+          bn = n;
+          bw = w;
+        }
+      }
+      split[i] = bn;
+      kt[i] = bn > 1 ? bw : 0;
     };
-    parts_for(NQKV / kTcRows, H, 0);
-    parts_for(cdiv(F, kTcRows), H, 2);
-    parts_for(cdiv(H, kTcRows), F, 3);
+    parts_for(NQKV / kTcRows, 1, H, 0);
+    parts_for(cdiv(F, kTcRows), 2, H, 2);
+    parts_for(cdiv(H, kTcRows), 1, F, 3);
     o_groups = 1;
     n_o_parts = Hkv;
     split[1] = n_o_parts;
@@ -306,6 +330,15 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   struct Geom {
     int kp[4], page_bytes, tpp, x_cap, off_pages, n_pages, ring;
   };
+  // attention scratch in the staging area: q [G][d] plus either the page's
+  // scores [G][tpp], per-head statistics, the current token's K and V (bf16)
+  // and (mma.sync attention) the per-page warp counters and the warps'
+  // (O, m, l) before their merge, or the combine's per-chunk (m, l) pairs
+  auto attn_need = [&](int tpp) {
+    const int pages = (G * tpp + 3 * kMaxGroup) * 4 + 2 * d * 2 +
+                      (attn_mma ? kMaxPages * 4 + kComputeWarps * G * (d + 2) * 4 : 0);
+    return G * d * 4 + std::max(pages, (2 * max_chunks * G + 2 * G) * 4);
+  };
   // Geometry for pages of at most `kpmax` columns; false if the staging
   // area cannot hold one page-wide chunk within 64 KB.
   auto geometry = [&](int kpmax, Geom &g) {
@@ -329,11 +362,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
       g.page_bytes = align_up_i(4 * d * P, 128);
     }
     g.tpp = std::min(tpp, 16 * P);
-    // attention scratch in the staging area: q [G][d] plus either the page's
-    // scores [G][tpp], per-head statistics and the current token's K and V
-    // (bf16), or the combine's per-chunk (m, l) pairs
-    const int att_need = G * d * 4 + std::max((G * g.tpp + 3 * kMaxGroup) * 4 + 2 * d * 2,
-                                              (2 * max_chunks * G + 2 * G) * 4);
+    const int att_need = attn_need(g.tpp);
     g.x_cap = std::max(x_cap, att_need);
     g.off_pages = align_up_i(off_x + g.x_cap, 1024);
     g.n_pages = std::min(kMaxPages, (smem_max - g.off_pages) / g.page_bytes);
@@ -368,8 +397,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     if (x_chunk <= kXWholeMax) {
       const int x_cap = x_whole <= kXWholeMax ? std::max(x_whole, x_chunk) : x_chunk;
       g.tpp = std::min((g.page_bytes / (4 * d)) / P * P, 16 * P);
-      const int att_need = G * d * 4 + std::max((G * g.tpp + 3 * kMaxGroup) * 4 + 2 * d * 2,
-                                                (2 * max_chunks * G + 2 * G) * 4);
+      const int att_need = attn_need(g.tpp);
       g.x_cap = std::max(x_cap, att_need);
       g.off_pages = align_up_i(off_x + g.x_cap, 1024);
       g.n_pages = std::min(kMaxPages, (smem_max - g.off_pages) / g.page_bytes);
@@ -384,8 +412,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     for (int i = 0; i < 4; ++i) g.kp[i] = tc_kc;
     g.page_bytes = kTcRows * tc_kc * 2;
     g.tpp = std::min((g.page_bytes / (4 * d)) / P * P, 16 * P);
-    const int att_need = G * d * 4 + std::max((G * g.tpp + 3 * kMaxGroup) * 4 + 2 * d * 2,
-                                              (2 * max_chunks * G + 2 * G) * 4);
+    const int att_need = attn_need(g.tpp);
     g.x_cap = std::max(2 * kTcXBytes, align_up_i(att_need, 1024));
     g.off_pages = align_up_i(off_x + g.x_cap, 1024);
     g.n_pages = std::min(kMaxPages, (smem_max - g.off_pages) / g.page_bytes);
@@ -451,9 +478,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   p.wait_limit_ns = o.wait_limit_ns;
   p.n_ffn_parts = n_ksplit;
   p.chunk_seq = -1;   // decode steps (a prompt chunk sets its sequence)
-  // the CUDA-core attention is the default: it measured faster at every
-  // batch size of the 8B decode workloads
-  p.attn_mma = o.attn_path == 2 ? 1 : 0;
+  p.attn_mma = attn_mma ? 1 : 0;
   p.w4 = o.w4 ? 1 : 0;
   p.n_out = n_out;
   p.tile_rows = tc ? kTcRows : 16;
