@@ -610,26 +610,43 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   uint32_t la_ev = 0;   // lane 0: input-event counter read when the task was popped
   const SeqView sv = seq_view(p, B, lane);
 
+  // The descriptor of the next ticket is read ahead: lanes 0..3 hold its
+  // 16-byte quarters (ticket pf_ticket, task pf_tix), requested at a top-up
+  // after the ticket arrived, so that a pop finds it in registers.
+  uint4 pf_q = make_uint4(0u, 0u, 0u, 0u);
+  int pf_tix = 0;
+  uint32_t pf_ticket = 0xffffffffu;   // warp-uniform; none in flight
+  auto prefetch_desc = [&]() {
+    const uint32_t ticket = __shfl_sync(0xffffffffu, next, 0);
+    if (ticket == pf_ticket || static_cast<int>(ticket) >= n_launch) return;
+    const int tix = fixed ? p.sched[s_begin + static_cast<int>(ticket)]
+                          : p.task_begin + static_cast<int>(ticket);
+    if (lane < 4) pf_q = reinterpret_cast<const uint4 *>(p.tasks + tix)[lane];
+    pf_tix = tix;
+    pf_ticket = ticket;
+  };
   // Pop one task into the lookahead (warp-uniform).  The next ticket is
-  // always requested one pop ahead, so a pop waits only for the descriptor.
-  // Lane 0 also starts reading the GEMV task's input-event counter; the
-  // value is looked at only when the task is handed over, a task later.
+  // always requested one pop ahead and its descriptor read ahead.  Lane 0
+  // also starts reading the GEMV task's input-event counter; the value is
+  // looked at only when the task is handed over, a task later.
   auto pop_one = [&]() {
     const uint32_t ticket = __shfl_sync(0xffffffffu, next, 0);
     if (static_cast<int>(ticket) >= n_launch) {
       exhausted = true;
       return;
     }
+    prefetch_desc();   // (a no-op when the descriptor is already in flight)
     if (lane == 0) next = fixed ? ticket + 1u : atomicAdd(p.sync + S_QUEUE, 1u);
-    const int tix = fixed ? p.sched[s_begin + static_cast<int>(ticket)]
-                          : p.task_begin + static_cast<int>(ticket);
-    const Task t = p.tasks[tix];
     const int e = (la_head + la_count) % kLook;
+    if (lane < 4) reinterpret_cast<uint4 *>(&la[e].t)[lane] = pf_q;
+    __syncwarp();
     if (lane == 0) {
-      la[e].t = t;
-      la[e].tix = tix;
-      if (is_gemv(t.type) && t.dep_event != kNoEvent) la_ev = ld_relaxed(p.sync + S_EVENTS + t.dep_event);
+      la[e].tix = pf_tix;
+      const uint8_t type = la[e].t.type;
+      const uint32_t dep = la[e].t.dep_event;
+      if (is_gemv(type) && dep != kNoEvent) la_ev = ld_relaxed(p.sync + S_EVENTS + dep);
     }
+    pf_ticket = 0xffffffffu;
     ++la_count;
   };
   // A handed-over GEMV task whose input was not yet complete, or an
@@ -639,15 +656,25 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   bool blocked = false;
   uint32_t blk_ev = kNoEvent, blk_cnt = 0;
   int blk_tix = 0;   // the blocked task (named in a timeout report)
+  // The blocking event is polled without waiting for the read: each call
+  // looks at the value the previous call requested and requests the next
+  // (lane 0), so a poll never stalls the loader for a round trip.
+  uint32_t poll_v = 0;
+  bool poll_out = false;   // lane 0: a read of the blocking event is in flight
   auto may_pop = [&]() {
     if (!blocked) return true;
     int ok = 0;
-    if (lane == 0) ok = static_cast<int32_t>(ld_relaxed(p.sync + S_EVENTS + blk_ev) - p.epoch * blk_cnt) >= 0;
+    if (lane == 0) {
+      if (poll_out) ok = static_cast<int32_t>(poll_v - p.epoch * blk_cnt) >= 0;
+      poll_v = ld_relaxed(p.sync + S_EVENTS + blk_ev);
+      poll_out = true;
+    }
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (ok) blocked = false;
     return ok != 0;
   };
   auto top_up = [&](int max_pops) {
+    if (!exhausted && la_count >= 1) prefetch_desc();
     for (int k = 0; k < max_pops; ++k) {
       // one task ahead: every popped task is reserved for this CTA, so
       // popping further ahead would delay the last tasks of an operator
@@ -722,6 +749,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       const int dok = __shfl_sync(0xffffffffu, info.dep_ok, 0);
       if (is_gemv(t.type) && t.dep_event != kNoEvent && !dok) {
         blocked = true;
+        poll_out = false;
         blk_ev = t.dep_event;
         blk_cnt = t.dep_count;
         blk_tix = tix;
@@ -729,6 +757,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
         // an attention chunk waits for its KV group's projections: one such
         // chunk per CTA, so a group's chunks run on as many SMs as it has
         blocked = true;
+        poll_out = false;
         blk_ev = static_cast<uint32_t>(ev_attn_input(p, t.layer, info.g));
         blk_cnt = static_cast<uint32_t>(attn_input_count(p));
         blk_tix = tix;
