@@ -450,8 +450,9 @@ def main():
     ap.add_argument("--mode", choices=["mega", "perop", "perop-graph"], default="mega")
     ap.add_argument("--impl", choices=["mk", "reference"], default="mk")
     ap.add_argument("--e2e-steps", type=int, default=32)
-    ap.add_argument("--gemv-path", type=int, default=0, choices=[0, 1, 2],
-                    help="projections: 0 automatic, 1 mma.sync pages, 2 tcgen05 tiles")
+    ap.add_argument("--gemv-path", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="projections: 0 automatic, 1 mma.sync pages, 2 tcgen05 tiles, "
+                         "3 mma.sync pages staged in tensor memory")
     ap.add_argument("--attn-path", type=int, default=0, choices=[0, 1, 2],
                     help="attention: 0 automatic, 1 CUDA-core FMA, 2 mma.sync tiles")
     ap.add_argument("--prompt-path", choices=["chunks", "decode"], default="chunks",

@@ -182,7 +182,16 @@ typedef struct {
                              in tensor memory.  2 needs head_dim 128 and
                              hidden, ffn and n_q_heads*head_dim multiples of
                              64 (else MK_ERR_UNSUPPORTED); rows_per_task,
-                             max_page_cols and o_split apply to path 1 only */
+                             max_page_cols and o_split apply to path 1 only.
+                             3 = path 1 with its weight pages staged in
+                             tensor memory: TMA copies 16-row pages in
+                             128-column boxes, the loader copies each landed
+                             page into tensor memory (tcgen05.cp) and frees
+                             its shared memory, the compute warps read mma
+                             A fragments back (tcgen05.ld), so more bytes
+                             stay in flight per SM.  3 needs hidden, ffn and
+                             n_q_heads*head_dim multiples of 128, no 4-bit
+                             weights and no o_split                         */
   int schedule;           /* 0 = dynamic: every CTA takes the next task from
                              one in-GPU ticket queue; 1 = solidified: the
                              plan assigns each CTA its task list offline (list
@@ -344,7 +353,8 @@ typedef struct {
   int ffn_parts, ffn_part_cols; /* split-K parts of the down projection and
                              columns per part (1 part: ffn_part_cols = ffn) */
   int o_parts, o_part_cols; /* the same for the O projection               */
-  int gemv_path;          /* the path the plan uses: 1 mma.sync, 2 tcgen05  */
+  int gemv_path;          /* the path the plan uses: 1 mma.sync, 2 tcgen05,
+                             3 mma.sync from tensor memory                  */
   int schedule;           /* 0 dynamic queue, 1 solidified per-CTA lists    */
   int prefill;            /* 1: created with the prefill option             */
   int weight_bits;        /* 16 bf16 or 4 (W4A16) projections              */

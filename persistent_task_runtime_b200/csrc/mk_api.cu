@@ -182,7 +182,7 @@ void fill_info(const mk::Layout &lay, const mk_model_config &c, mk_plan_info_t &
     I.o_part_cols = p.tc_kt[mk::T_OPROJ] > 0 ? p.tc_kt[mk::T_OPROJ] : c.n_q_heads * d;
     I.ffn_part_cols = p.tc_kt[mk::T_DOWN] > 0 ? p.tc_kt[mk::T_DOWN] : F;
   }
-  I.gemv_path = p.tc ? 2 : 1;
+  I.gemv_path = p.tc ? 2 : (p.tm ? 3 : 1);
   I.schedule = lay.sched.empty() ? 0 : 1;
   I.prefill = lay.p.kv_tasks;
   I.qkv_parts = lay.splits[0];

@@ -45,12 +45,24 @@ constexpr int kTcXBytes = 32 * 1024;              // one staged activation chunk
 constexpr int kTcTmemCols = 128;                  // tensor-memory columns allocated per CTA
 constexpr int kTcAutoBatch = 5;                   // smallest max_batch that takes it by default
 constexpr int kAttnMmaAutoBatch = 2;              // smallest max_batch that takes the mma.sync attention
+
+// ---- mma.sync GEMV over weights staged in tensor memory -------------------------
+// 16-row weight pages arrive by TMA in 128-column boxes (32-byte swizzle, as
+// 128 "virtual rows" of 16 columns: column block b of row r at row 16 b + r),
+// are copied into tensor memory (tcgen05.cp, one 128 x 256-bit copy per box)
+// and read back as mma.sync A fragments (tcgen05.ld.16x256b), so a page
+// leaves shared memory as soon as it is copied and tensor memory adds
+// kTmSlots pages of bytes in flight per SM.
+constexpr int kTmSlots = 4;                       // tensor-memory page slots
+constexpr int kTmSlotCols = 128;                  // columns per slot (a 2048-column page)
+constexpr int kTmBoxCols = 128;                   // weight columns per TMA box / tcgen05.cp
 constexpr int kTcMatsPerLayer = 7;                // tensor maps: wq wk wv wo w_gate w_up w_down
 
 // ---- kernel variants (template argument of the step kernel) -------------------
 constexpr int kVarTc = 1;        // projections on tcgen05 tiles (else mma.sync pages)
 constexpr int kVarW4 = 2;        // 4-bit weight consumer
 constexpr int kVarAttnMma = 4;   // attention on mma.sync tiles over swizzled K/V pages
+constexpr int kVarTm = 8;        // mma.sync GEMV reading its weight pages from tensor memory
 
 // ---- task descriptor (64 bytes, four 16-byte loads) ---------------------------
 enum TaskType : uint8_t {
@@ -146,6 +158,7 @@ struct Params {
   int tile_rows;                      // rows per row tile: 16 (mma.sync) or kTcRows (tcgen05)
 
   // tensor-core GEMV path (tc = 1): every GEMV task runs on tcgen05 tiles
+  int tm;                             // 1: mma.sync GEMV pages staged in tensor memory
   int tc;
   int tc_bpad;                        // sequences per half of the MMA's N (max_batch rounded to 8)
   int tc_n;                           // MMA N = 2 * tc_bpad: bf16 hi rows, then lo rows
@@ -253,7 +266,7 @@ struct LayoutOptions {
   int num_ctas = 0;             // 0: one per SM
   int max_page_cols = 0;        // 0: kMaxPageCols
   bool o_split = false;         // O projection in two K parts of whole KV groups
-  int gemv_path = 0;            // 0 automatic, 1 mma.sync pages, 2 tcgen05 tiles
+  int gemv_path = 0;            // 0 automatic, 1 mma.sync pages, 2 tcgen05 tiles, 3 mma.sync pages through tensor memory
   int schedule = 0;             // 0 dynamic ticket queue, 1 solidified per-CTA task lists
   bool prefill = false;         // K/V appended by their own tasks (prompt chunks of one sequence)
   bool w4 = false;              // 4-bit projections (packed, MK_W4_BLOCK_BYTES blocks)

@@ -118,6 +118,48 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, 
       : "memory");
 }
 
+// 3-D tensor copy (x innermost) into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, int x, int y, int z,
+                                            uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor of 128 rows of 32 bytes in the 32-byte
+// swizzled K-major layout that a TMA copy with 32-byte swizzle writes: rows
+// 32 bytes apart, 8-row groups 256 bytes apart; layout type 6 = 32-byte
+// swizzle (bits 61-63).  The source of one tcgen05.cp.128x256b.
+__device__ __forceinline__ uint64_t sw32_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (1ull << 16) |
+         (static_cast<uint64_t>(256 >> 4) << 32) | (1ull << 46) | (6ull << 61);
+}
+
+// Copy 128 rows x 256 bits from shared memory (descriptor) into tensor memory:
+// row i to lane i, its 32 bytes to 8 consecutive columns.  Issued by one
+// thread; completion is tracked by tcgen05.commit.
+__device__ __forceinline__ void tm_cp(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Warp-wide: 16 lanes x 256 bits of tensor memory starting at lane
+// (taddr >> 16) (a multiple of 16 inside this warp's lane quarter).  Thread
+// (g = lane / 4, q = lane % 4) receives, of rows g and g + 8, the 32-bit
+// words 2q and 2q + 1: r0 = (g, 2q), r1 = (g, 2q + 1), r2 = (g + 8, 2q),
+// r3 = (g + 8, 2q + 1).  (Completion: tcgen05.wait::ld.)
+__device__ __forceinline__ void tm_ld16x256(uint32_t taddr, uint32_t &r0, uint32_t &r1,
+                                            uint32_t &r2, uint32_t &r3) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(taddr)
+               : "memory");
+}
+__device__ __forceinline__ void tm_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte
 // swizzled layout: 8-row groups 1024 bytes apart, rows 128 bytes apart.
 // Fields: start address >> 4 (bits 0-13), leading-dimension offset (unused
@@ -578,12 +620,23 @@ struct Look {
   int tix;
   int pad[3];
 };
-constexpr int kLook = kLookBytes / static_cast<int>(sizeof(Look));
+// the end of the lookahead area holds the tensor-memory slot barriers
+constexpr int kTmBarBytes = 2 * kTmSlots * 8;
+constexpr int kLook = (kLookBytes - kTmBarBytes) / static_cast<int>(sizeof(Look));
+// Tensor-memory page slot i: filled by the mover's commit (tm_full), read by
+// every compute warp (tm_empty).
+__device__ __forceinline__ uint64_t *tm_full_bar(uint8_t *smem, const Params &p, int i) {
+  return reinterpret_cast<uint64_t *>(smem + p.off_look + kLookBytes - kTmBarBytes) + i;
+}
+__device__ __forceinline__ uint64_t *tm_empty_bar(uint8_t *smem, const Params &p, int i) {
+  return reinterpret_cast<uint64_t *>(smem + p.off_look + kLookBytes - kTmBarBytes) + kTmSlots + i;
+}
 static_assert(sizeof(Look) == 80 && kLook >= 2, "lookahead entry size");
 
 template <int V>
 __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   constexpr bool TC = (V & kVarTc) != 0, W4 = (V & kVarW4) != 0, AMMA = (V & kVarAttnMma) != 0;
+  constexpr bool TM = (V & kVarTm) != 0;
   const int lane = threadIdx.x & 31;
   const uint64_t pol = l2_evict_first_policy();
   Slot *slots = reinterpret_cast<Slot *>(smem + p.off_slots);
@@ -609,6 +662,103 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   bool exhausted = false;
   uint32_t la_ev = 0;   // lane 0: input-event counter read when the task was popped
   const SeqView sv = seq_view(p, B, lane);
+
+  // ---- tensor-memory staging (lane 0): the mover ----
+  // Pages are moved in ring order.  A GEMV page, once landed, is copied into
+  // the next free tensor-memory slot (one tcgen05.cp per 128-column box);
+  // the copies' completion frees the shared-memory page and fills the slot.
+  // An attention page is passed over (the compute warps read it from shared
+  // memory and free it).  service() never blocks: every wait of the loader
+  // calls it, so pages keep moving while the loader waits.
+  const uint32_t tmem = TM ? ctl->tmem : 0u;
+  int mv_pm = 0, mv_n = 0;          // next page to move; pages issued and not yet moved
+  uint32_t mv_ppar = 0;             // its ring round parity
+  uint32_t mv_kind = 0;             // per ring page: 1 = GEMV page for tensor memory
+  uint64_t mv_ng = 0;               // per ring page: boxes - 1 (4 bits)
+  int tslot = 0;                    // next tensor-memory slot and its round parity
+  uint32_t tpar = 0;
+  int last_slot = -1;               // the slot of the last commit (drained at exit)
+  uint32_t last_tpar = 0;
+  auto service = [&]() {
+    if constexpr (TM) {
+      while (mv_n > 0) {
+        const int pm = mv_pm;
+        if ((mv_kind >> pm) & 1u) {
+          if (!mbar_try_wait(&ctl->full[pm], mv_ppar)) return;
+          if (!mbar_try_wait(tm_empty_bar(smem, p, tslot), tpar ^ 1u)) return;
+          tc_fence_after();
+          const int nb = static_cast<int>((mv_ng >> (4 * pm)) & 15u) + 1;
+          const uint32_t src = smem_u32(pages + static_cast<size_t>(pm) * p.page_bytes);
+          const uint32_t dst = tmem + static_cast<uint32_t>(tslot * kTmSlotCols);
+          for (int b = 0; b < nb; ++b) tm_cp(dst + 8u * b, sw32_desc(src + 4096u * b));
+          tc_commit(&ctl->empty[pm]);      // the shared-memory page is free once copied
+          tc_commit(tm_full_bar(smem, p, tslot));
+          last_slot = tslot;
+          last_tpar = tpar;
+          if (++tslot == kTmSlots) {
+            tslot = 0;
+            tpar ^= 1u;
+          }
+        }
+        if (++mv_pm == p.n_pages) {
+          mv_pm = 0;
+          mv_ppar ^= 1u;
+        }
+        --mv_n;
+      }
+    }
+  };
+  // lane 0: wait for a barrier phase (bounded), moving pages meanwhile
+  auto lwait = [&](uint64_t *bar, uint32_t parity, uint32_t where) -> bool {
+    if constexpr (!TM) {
+      return wait_mbar(p, ctl, bar, parity, where, 2);
+    } else {
+      uint64_t t0 = 0;
+      for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        service();
+        if ((it & 7u) == 7u) {
+          if (ctl->cta_abort != 0) return false;
+          if ((it & 255u) == 255u && ld_relaxed(p.sync + S_ABORT) != 0u) return false;
+          const uint64_t now = gtimer();
+          if (t0 == 0) {
+            t0 = now;
+          } else if (now - t0 > static_cast<uint64_t>(p.wait_limit_ns) * 2) {
+            raise_error(p, MK_ERR_TIMEOUT, where, 0xfffffffeu, parity);
+            return false;
+          }
+        }
+      }
+    }
+  };
+  // lane 0: wait for an event (bounded, acquire), moving pages meanwhile
+  auto lwait_event = [&](uint32_t ev, uint32_t count, uint32_t task_idx) -> bool {
+    if constexpr (!TM) {
+      return wait_event(p, ctl, ev, count, task_idx);
+    } else {
+      const uint32_t target = p.epoch * count;
+      const uint32_t *ctr = p.sync + S_EVENTS + ev;
+      uint64_t t0 = 0;
+      for (uint32_t it = 0;; ++it) {
+        const uint32_t v = ld_relaxed(ctr);
+        if (static_cast<int32_t>(v - target) >= 0) {
+          (void)ld_acquire(ctr);
+          return true;
+        }
+        service();
+        if ((it & 3u) == 3u) {
+          if (aborted(p, ctl)) return false;
+          const uint64_t now = gtimer();
+          if (t0 == 0) {
+            t0 = now;
+          } else if (now - t0 > static_cast<uint64_t>(p.wait_limit_ns)) {
+            raise_error(p, MK_ERR_TIMEOUT, task_idx, ev, v);
+            return false;
+          }
+        }
+      }
+    }
+  };
 
   // The descriptor of the next ticket is read ahead: lanes 0..3 hold its
   // 16-byte quarters (ticket pf_ticket, task pf_tix), requested at a top-up
@@ -688,7 +838,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     top_up(kLook);
     if (la_count == 0 && !exhausted && blocked) {
       int okw = 1;
-      if (lane == 0) okw = wait_event(p, ctl, blk_ev, blk_cnt, static_cast<uint32_t>(blk_tix));
+      if (lane == 0) okw = lwait_event(blk_ev, blk_cnt, static_cast<uint32_t>(blk_tix));
       if (__shfl_sync(0xffffffffu, okw, 0) == 0) {
         ok = false;
         break;
@@ -697,7 +847,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       top_up(kLook);
     }
     int okl = 1;
-    if (lane == 0) okl = wait_mbar(p, ctl, &ctl->slot_empty[ts], ts_par ^ 1u, 0xfff00000u, 2);
+    if (lane == 0) okl = lwait(&ctl->slot_empty[ts], ts_par ^ 1u, 0xfff00000u);
     ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
     if (!ok) break;
 
@@ -810,11 +960,28 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
           gemv_tile(p, t, m, W, row, rv);
           for (int c0 = xc0; c0 < xend; c0 += geo.kp) {
             const int nc = min(geo.kp, xend - c0);
-            if (lane == 0) okl = wait_mbar(p, ctl, &ctl->empty[pi], pe_par ^ 1u, 0xfff10000u, 2);
+            if (lane == 0) okl = lwait(&ctl->empty[pi], pe_par ^ 1u, 0xfff10000u);
             ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
             if (!ok) break;
             uint8_t *pg = pages + static_cast<size_t>(pi) * p.page_bytes;
-            if (W4 && is_w4_task(p.w4, t.type)) {
+            if (TM) {
+              // 128-column boxes of 16 rows (rows past the matrix arrive as
+              // zeros), each landing as one tcgen05.cp source
+              const int nb = nc / kTmBoxCols;
+              const bool up = t.type == T_GATEUP && m >= (t.n_m >> 1);
+              const void *map = static_cast<const uint8_t *>(p.tmaps) +
+                                static_cast<size_t>(up ? t.map1 : t.map0) * 128;
+              if (lane == 0) {
+                mbar_arrive_expect_tx(&ctl->full[pi], static_cast<uint32_t>(nb) * 4096u);
+                mv_kind |= 1u << pi;
+                mv_ng = (mv_ng & ~(15ull << (4 * pi))) | (static_cast<uint64_t>(nb - 1) << (4 * pi));
+                ++mv_n;
+              }
+              __syncwarp();
+              if (lane < nb)
+                tma_load_3d(pg + lane * 4096, map, 0, row, (c0 + lane * kTmBoxCols) / 16,
+                            &ctl->full[pi], pol);
+            } else if (W4 && is_w4_task(p.w4, t.type)) {
               // 4-bit: the row tile's packed blocks of these columns are
               // contiguous -- one bulk copy
               const uint32_t bytes = static_cast<uint32_t>(nc / MK_W4_BLOCK_COLS) * MK_W4_BLOCK_BYTES;
@@ -851,8 +1018,8 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
         // copy them only once those are complete, and order the copies
         // (async proxy) after the acquired writes
         if (lane == 0)
-          okl = wait_event(p, ctl, static_cast<uint32_t>(ev_attn_input(p, l, info.g)),
-                           static_cast<uint32_t>(attn_input_count(p)), static_cast<uint32_t>(tix));
+          okl = lwait_event(static_cast<uint32_t>(ev_attn_input(p, l, info.g)),
+                            static_cast<uint32_t>(attn_input_count(p)), static_cast<uint32_t>(tix));
         ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
         if (!ok) break;
         __syncwarp();
@@ -864,7 +1031,11 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       for (int tok0 = info.t0; tok0 < info.t1 && ok; tok0 += p.tpp) {
         const int ntok = min(p.tpp, info.t1 - tok0);
         const int nkv = (ntok + P - 1) / P;
-        if (lane == 0) okl = wait_mbar(p, ctl, &ctl->empty[pi], pe_par ^ 1u, 0xfff20000u, 2);
+        if (lane == 0) okl = lwait(&ctl->empty[pi], pe_par ^ 1u, 0xfff20000u);
+        if (TM && lane == 0) {   // an attention page: the mover passes it over
+          mv_kind &= ~(1u << pi);
+          ++mv_n;
+        }
         ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
         if (!ok) break;
         uint8_t *pg = pages + static_cast<size_t>(pi) * p.page_bytes;
@@ -930,6 +1101,21 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     if (!ok) break;
   }
 
+  if constexpr (TM) {
+    // the compute warps still need every page issued: move the rest (bounded)
+    if (ok && lane == 0) {
+      const uint64_t t0 = gtimer();
+      while (mv_n > 0) {
+        service();
+        if (ctl->cta_abort != 0 || gtimer() - t0 > static_cast<uint64_t>(p.wait_limit_ns) * 2) {
+          if (ctl->cta_abort == 0) raise_error(p, MK_ERR_TIMEOUT, 0xfffffff1u, 0xfffffffeu, 0u);
+          ok = false;
+          break;
+        }
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  }
   if (!ok) {
     // Abandoning the step: no bulk copy may still be landing in shared
     // memory when this CTA exits.  Wait (bounded) for every page's last copy.
@@ -942,6 +1128,16 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
         while (!mbar_try_wait(&ctl->full[q], par)) {
           if (gtimer() - t0 > static_cast<uint64_t>(p.wait_limit_ns) * 4) break;
         }
+      }
+    }
+  }
+  if constexpr (TM) {
+    // no copy into tensor memory may still run when the CTA frees it: the
+    // last commit tracks every earlier copy (bounded wait)
+    if (lane == 0 && last_slot >= 0) {
+      const uint64_t t0 = gtimer();
+      while (!mbar_try_wait(tm_full_bar(smem, p, last_slot), last_tpar)) {
+        if (gtimer() - t0 > static_cast<uint64_t>(p.wait_limit_ns) * 4) break;
       }
     }
   }
@@ -1055,6 +1251,59 @@ __device__ __forceinline__ void page_mma_w4(float (&acc)[NN][4], const uint8_t *
     for (int e = 0; e < 4; ++e) acc[nt][e] += c1[nt][e];
 }
 
+// One 16-row weight page staged in tensor memory (slot columns at `slot`)
+// against the staged activation.  The page's 128-column boxes sit at slot
+// columns 8 box .. 8 box + 7, and column block b (16 columns) of the box in
+// lanes 16 b .. 16 b + 15: a 16x256b load there is the block's mma A
+// fragment for the k order (4q, 4q + 1 | 4q + 2, 4q + 3) of lane quarter q,
+// which the activation fragment follows (columns 4q .. 4q + 3 of the block,
+// 8 bytes of the staged hi or lo half).  A warp reads only its lane quarter
+// qq of tensor memory: column blocks 2 qq and 2 qq + 1 of every box; the two
+// warps of quarters 1 and 2 take alternate boxes.
+template <int NN>
+__device__ __forceinline__ void page_tm(float (&acc)[NN][4], uint32_t slot, int nc,
+                                        const uint8_t *xs, int xpitch, int xcol0, int B, int warp,
+                                        int lane) {
+  const int g = lane >> 2, q = lane & 3;
+  const int qq = (warp + 1) & 3;
+  const int bstep = (qq == 1 || qq == 2) ? 2 : 1;
+  const int b0 = (bstep == 2 && warp >= 4) ? 1 : 0;
+  const int nbox = nc / kTmBoxCols;
+  const int xq = (8 * (q >> 1)) * 4 + (q & 1) * 8 + (g >> 2) * 16;   // bytes, within a block
+  float c1[NN][4];
+#pragma unroll
+  for (int nt = 0; nt < NN; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c1[nt][e] = 0.f;
+#pragma unroll 2
+  for (int bx = b0; bx < nbox; bx += bstep) {
+    uint32_t a[2][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      tm_ld16x256(slot + (static_cast<uint32_t>(32 * qq + 16 * h) << 16) + 8u * bx, a[h][0],
+                  a[h][1], a[h][2], a[h][3]);
+    tm_wait_ld();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int xo = (xcol0 + 16 * (8 * bx + 2 * qq + h)) * 4 + xq;
+#pragma unroll
+      for (int nt = 0; nt < NN; ++nt) {
+        const int b = nt * 4 + (g & 3);
+        uint2 xv = make_uint2(0u, 0u);
+        if (b < B) xv = *reinterpret_cast<const uint2 *>(xs + b * xpitch + xo);
+        if (h == 0)
+          mma_bf16(acc[nt], a[h][0], a[h][2], a[h][1], a[h][3], xv.x, xv.y);
+        else
+          mma_bf16(c1[nt], a[h][0], a[h][2], a[h][1], a[h][3], xv.x, xv.y);
+      }
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NN; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] += c1[nt][e];
+}
+
 // All lanes of a compute warp wait (bounded) for a full ring page; the
 // result is warp-uniform.
 __device__ __forceinline__ bool warp_wait_page(const Params &p, Ctl *ctl, uint64_t *bar,
@@ -1069,6 +1318,8 @@ __device__ __forceinline__ bool warp_wait_page(const Params &p, Ctl *ctl, uint64
 struct ComputeState {
   int pi = 0;
   uint32_t pg_par = 0;
+  int tslot = 0;                 // tensor-memory staging: next page slot and its round parity
+  uint32_t tpar = 0;
   uint32_t xuse = 0;             // tensor-core path: staged chunks so far (buffer = xuse & 1)
   uint32_t accuse = 0;           // tensor-core path: tasks whose accumulators were read
   uint32_t x_par = 0;            // phase of the activation-copy barrier
@@ -1226,7 +1477,7 @@ __device__ bool stage_x(const Params &p, Ctl *ctl, uint8_t *smem, const Task &t,
 // NN = batch n-tiles (1: B <= 4, 2: B <= 8, 4: B <= 16).  A task holds at
 // most kMaxMTiles / NN row tiles (the plan caps rows per task) so that the
 // accumulators stay in registers.
-template <int NN, bool W4, int MT = kMaxMTiles / NN>
+template <int NN, bool W4, bool TM, int MT = kMaxMTiles / NN>
 __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &S,
                           ComputeState &st, float *out, int ctid) {
   const Task &t = S.t;
@@ -1285,6 +1536,49 @@ __device__ bool gemv_task(const Params &p, Ctl *ctl, uint8_t *smem, const Slot &
     for (int m = 0; m < t.n_m; ++m) {
       for (int c0 = xc0; c0 < xend; c0 += geo.kp) {
         const int nc = min(geo.kp, xend - c0);
+        if constexpr (TM) {
+          // the page waits in a tensor-memory slot (the loader freed its ring
+          // page once it was copied there)
+          if (!bad && !warp_wait_page(p, ctl, tm_full_bar(smem, p, st.tslot), st.tpar, 0xfff30000u)) {
+            bad = true;
+            if (lane == 0) {
+              ctl->cbad = 1;
+              ctl->cta_abort = 1;
+            }
+          }
+          if (!bad) {
+            tc_fence_after();
+            const uint32_t slot = ctl->tmem + static_cast<uint32_t>(st.tslot * kTmSlotCols);
+            switch (m) {
+#define MK_TM_CASE(M)                                                                          \
+  case M:                                                                                      \
+    if (M < MT) page_tm<NN>(acc[M < MT ? M : 0], slot, nc, xs, xstride * 4, c0 - xc0, B, warp, lane); \
+    break;
+              MK_TM_CASE(0)
+              MK_TM_CASE(1)
+              MK_TM_CASE(2)
+              MK_TM_CASE(3)
+              MK_TM_CASE(4)
+              MK_TM_CASE(5)
+              MK_TM_CASE(6)
+              MK_TM_CASE(7)
+#undef MK_TM_CASE
+              default: break;
+            }
+            tc_fence_before();
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tm_empty_bar(smem, p, st.tslot));
+          if (++st.tslot == kTmSlots) {
+            st.tslot = 0;
+            st.tpar ^= 1u;
+          }
+          if (++st.pi == p.n_pages) {
+            st.pi = 0;
+            st.pg_par ^= 1u;
+          }
+          continue;
+        }
         if (!bad && !warp_wait_page(p, ctl, &ctl->full[st.pi], st.pg_par, 0xfff30000u)) {
           bad = true;
           if (lane == 0) {
@@ -1939,10 +2233,10 @@ __device__ bool attn_pages_cuda(const Params &p, Ctl *ctl, uint8_t *smem, const 
     }
     if (has_cur) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
-    if (!p.tc && lane == 0) mbar_arrive(&ctl->empty[st.pi]);
+    if (!(p.tc || p.tm) && lane == 0) mbar_arrive(&ctl->empty[st.pi]);
     compute_bar();   // sc is rewritten by the next page
     // (tensor-core plans release a page once, after every warp is done with it)
-    if (p.tc && ctid == 0) mbar_arrive(&ctl->empty[st.pi]);
+    if ((p.tc || p.tm) && ctid == 0) mbar_arrive(&ctl->empty[st.pi]);
     if (++st.pi == p.n_pages) {
       st.pi = 0;
       st.pg_par ^= 1u;
@@ -2141,7 +2435,7 @@ __device__ bool attn_pages_mma(const Params &p, Ctl *ctl, uint8_t *smem, const S
     // the page goes back to the loader once every warp is done with it
     __syncwarp();
     if (lane == 0) {
-      if (p.tc) {
+      if (p.tc || p.tm) {
         __threadfence_block();
         if (atomicAdd(&A.pg_cnt[st.pi], 1) == kComputeWarps - 1) {
           A.pg_cnt[st.pi] = 0;
@@ -2455,6 +2749,7 @@ __device__ void embed_task(const Params &p, const Slot &S, int ctid) {
 template <int V>
 __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
   constexpr bool TC = (V & kVarTc) != 0, W4 = (V & kVarW4) != 0, AMMA = (V & kVarAttnMma) != 0;
+  constexpr bool TM = (V & kVarTm) != 0;
   const int ctid = threadIdx.x - 32;
   Slot *slots = reinterpret_cast<Slot *>(smem + p.off_slots);
   ComputeState st;
@@ -2502,9 +2797,9 @@ __device__ void compute_main(const Params &p, Ctl *ctl, uint8_t *smem) {
           tok = p.tc_n > 16 ? gemv_task_tc<2>(p, ctl, smem, S, st, out, ctid)
                             : gemv_task_tc<1>(p, ctl, smem, S, st, out, ctid);
         else
-          tok = p.batch > 8   ? gemv_task<4, W4>(p, ctl, smem, S, st, out, ctid)
-                : p.batch > 4 ? gemv_task<2, W4>(p, ctl, smem, S, st, out, ctid)
-                              : gemv_task<1, W4>(p, ctl, smem, S, st, out, ctid);
+          tok = p.batch > 8   ? gemv_task<4, W4, TM>(p, ctl, smem, S, st, out, ctid)
+                : p.batch > 4 ? gemv_task<2, W4, TM>(p, ctl, smem, S, st, out, ctid)
+                              : gemv_task<1, W4, TM>(p, ctl, smem, S, st, out, ctid);
         break;
     }
     if (!tok) {
@@ -2769,13 +3064,17 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       mbar_init(&ctl->full[i], 1);
       // a page is released by each compute warp, or (tensor-core path) once:
       // by the MMAs' commit, or by one thread after an attention page
-      mbar_init(&ctl->empty[i], p.tc ? 1 : kComputeWarps);
+      mbar_init(&ctl->empty[i], (p.tc || p.tm) ? 1 : kComputeWarps);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl->x_full[i], 1);
       mbar_init(&ctl->x_free[i], 1);
     }
     mbar_init(&ctl->acc_bar, 1);
+    for (int i = 0; i < kTmSlots; ++i) {
+      mbar_init(tm_full_bar(smem, p, i), 1);               // the mover's commit
+      mbar_init(tm_empty_bar(smem, p, i), kComputeWarps);  // every compute warp, after reading
+    }
     for (int i = 0; i < kTaskSlots; ++i) {
       mbar_init(&ctl->slot_full[i], 1);
       mbar_init(&ctl->slot_empty[i], 1);
@@ -2791,18 +3090,19 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     // a device error from an earlier step is sticky until the host resets
     ctl->skip = (ld_relaxed(p.sync + S_STATUS) != 0u || ld_relaxed(p.sync + S_ABORT) != 0u);
     // the swizzled operand layouts assume 1024-byte aligned shared memory
-    if (p.tc && (smem_u32(smem) & 1023u) != 0u) {
+    if ((p.tc || p.tm) && (smem_u32(smem) & 1023u) != 0u) {
       raise_error(p, MK_ERR_UNSUPPORTED, 0xfffffff0u, smem_u32(smem), 0u);
       ctl->skip = 1;
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  const bool tmem_owner = p.tc && !ctl->skip && (threadIdx.x >> 5) == 1;
-  if (tmem_owner) tmem_alloc(&ctl->tmem, kTcTmemCols);
-  if (p.tc) tc_fence_before();
+  const bool tmem_owner = (p.tc || p.tm) && !ctl->skip && (threadIdx.x >> 5) == 1;
+  const uint32_t tmem_cols = p.tm ? static_cast<uint32_t>(kTmSlots * kTmSlotCols) : kTcTmemCols;
+  if (tmem_owner) tmem_alloc(&ctl->tmem, tmem_cols);
+  if (p.tc || p.tm) tc_fence_before();
   __syncthreads();
-  if (p.tc) tc_fence_after();
+  if (p.tc || p.tm) tc_fence_after();
   if (!ctl->skip) {
     const int warp = threadIdx.x >> 5;
     if (warp == kLoaderWarp) {
@@ -2813,10 +3113,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       compute_main<V>(p, ctl, smem);
     }
   }
-  if (p.tc) tc_fence_before();
+  if (p.tc || p.tm) tc_fence_before();
   __syncthreads();
-  if (p.tc) tc_fence_after();
-  if (tmem_owner) tmem_dealloc(ctl->tmem, kTcTmemCols);
+  if (p.tc || p.tm) tc_fence_after();
+  if (tmem_owner) tmem_dealloc(ctl->tmem, tmem_cols);
   if (threadIdx.x == 0) {
     __threadfence();
     const uint32_t old = atomicAdd(p.sync + S_EXIT, 1u);
@@ -2836,8 +3136,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
 namespace {
 // the variants plans use: mma.sync or tcgen05 projections, 4-bit weights
 // only on mma.sync, each with either attention path
-constexpr int kVariants[] = {0, kVarTc, kVarW4, kVarAttnMma, kVarTc | kVarAttnMma,
-                             kVarW4 | kVarAttnMma};
+constexpr int kVariants[] = {0,           kVarTc,   kVarW4, kVarAttnMma, kVarTc | kVarAttnMma,
+                             kVarW4 | kVarAttnMma, kVarTm, kVarTm | kVarAttnMma};
 
 const void *kernel_for(int v) {
   switch (v) {
@@ -2849,13 +3149,17 @@ const void *kernel_for(int v) {
       return reinterpret_cast<const void *>(mk_step_kernel<kVarTc | kVarAttnMma>);
     case kVarW4 | kVarAttnMma:
       return reinterpret_cast<const void *>(mk_step_kernel<kVarW4 | kVarAttnMma>);
+    case kVarTm: return reinterpret_cast<const void *>(mk_step_kernel<kVarTm>);
+    case kVarTm | kVarAttnMma:
+      return reinterpret_cast<const void *>(mk_step_kernel<kVarTm | kVarAttnMma>);
     default: return nullptr;
   }
 }
 }  // namespace
 
 int kernel_variant(const Params &p) {
-  return (p.tc ? kVarTc : 0) | (p.w4 ? kVarW4 : 0) | (p.attn_mma ? kVarAttnMma : 0);
+  return (p.tc ? kVarTc : 0) | (p.w4 ? kVarW4 : 0) | (p.attn_mma ? kVarAttnMma : 0) |
+         (p.tm ? kVarTm : 0);
 }
 
 cudaError_t configure_kernel(int smem_optin) {

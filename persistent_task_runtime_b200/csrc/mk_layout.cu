@@ -165,9 +165,24 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   // The tensor-core path needs one 128-row tile per head (head_dim 128) and
   // inputs whose width is a whole number of 64-column swizzle atoms.
   const bool tc_ok = d == kTcRows && H % 64 == 0 && F % 64 == 0 && (Hq * d) % 64 == 0;
-  if (o.gemv_path < 0 || o.gemv_path > 2)
-    return lfail(err, MK_ERR_INVALID_ARG, "gemv_path %d: 0 automatic, 1 mma.sync, 2 tcgen05",
+  if (o.gemv_path < 0 || o.gemv_path > 3)
+    return lfail(err, MK_ERR_INVALID_ARG,
+                 "gemv_path %d: 0 automatic, 1 mma.sync, 2 tcgen05, 3 mma.sync from tensor memory",
                  o.gemv_path);
+  // mma.sync pages staged in tensor memory: weight pages arrive in boxes of
+  // kTmBoxCols columns, so every input width is a whole number of boxes
+  const bool tm = o.gemv_path == 3;
+  if (tm) {
+    if (o.w4) return lfail(err, MK_ERR_UNSUPPORTED, "4-bit weights run on the mma.sync GEMV path");
+    if (H % kTmBoxCols || F % kTmBoxCols || (Hq * d) % kTmBoxCols)
+      return lfail(err, MK_ERR_UNSUPPORTED,
+                   "the tensor-memory GEMV path needs hidden, ffn and n_q_heads*head_dim "
+                   "multiples of %d", kTmBoxCols);
+    if (o.max_page_cols % kTmBoxCols)
+      return lfail(err, MK_ERR_INVALID_ARG, "max_page_cols must be a multiple of %d on this path",
+                   kTmBoxCols);
+    if (o.o_split) return lfail(err, MK_ERR_INVALID_ARG, "o_split is not available on this path");
+  }
   if (o.gemv_path == 2 && !tc_ok)
     return lfail(err, MK_ERR_UNSUPPORTED,
                  "the tensor-core GEMV path needs head_dim 128 and hidden, ffn and "
@@ -183,8 +198,8 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
       return lfail(err, MK_ERR_UNSUPPORTED, "4-bit weights run on the mma.sync GEMV path");
     if (o.o_split) return lfail(err, MK_ERR_INVALID_ARG, "o_split is not available with 4-bit weights");
   }
-  const bool tc = !o.w4 && (o.gemv_path == 2 || (o.gemv_path == 0 && tc_ok && !o.o_split &&
-                                                  maxB >= kTcAutoBatch));
+  const bool tc = !o.w4 && !tm && (o.gemv_path == 2 || (o.gemv_path == 0 && tc_ok && !o.o_split &&
+                                                         maxB >= kTcAutoBatch));
   if (tc) {
     for (int i = 0; i < 5; ++i)
       if (o.rows_per_task[i] != 0)
@@ -229,7 +244,12 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   int kchunk_ffn = F;
   if (n_ksplit > 1) {
     // multiple of 32 and of R_gu (4-bit: of the 1024-column packed blocks)
-    const int unit = o.w4 ? MK_W4_BLOCK_COLS : ((R_gu % 32 == 0) ? R_gu : 2 * R_gu);
+    int unit = o.w4 ? MK_W4_BLOCK_COLS : ((R_gu % 32 == 0) ? R_gu : 2 * R_gu);
+    if (tm) {   // ... and of the tensor-memory boxes
+      int u = unit;
+      while (u % kTmBoxCols) u += unit;
+      unit = u;
+    }
     kchunk_ffn = align_up_i(cdiv(F, n_ksplit), unit);
     n_ksplit = cdiv(F, kchunk_ffn);
     if (n_ksplit < 2) {
@@ -342,9 +362,11 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   // Geometry for pages of at most `kpmax` columns; false if the staging
   // area cannot hold one page-wide chunk within 64 KB.
   auto geometry = [&](int kpmax, Geom &g) {
+    // (tensor-memory staging: whole boxes of kTmBoxCols columns)
+    const int pc_unit = tm ? kTmBoxCols : 32;
     auto page_cols = [&](int K) {
       if (K <= kpmax) return K;
-      return align_up_i(cdiv(K, cdiv(K, kpmax)), 32);
+      return align_up_i(cdiv(K, cdiv(K, kpmax)), pc_unit);
     };
     g.kp[K_HID] = page_cols(H);
     g.kp[K_ATT] = page_cols(n_o_parts > 1 ? o_groups * G * d : Hq * d);
@@ -373,7 +395,8 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   // largest ring any width gives with at least 3 pages; wider pages mean
   // fewer hand-offs per byte.  Failing 3 pages, the most pages.
   std::vector<Geom> cands;
-  for (int cand = colcap; cand >= 32 && !tc && !o.w4; cand -= (cand > 256 ? 256 : 32)) {
+  for (int cand = tm ? colcap / kTmBoxCols * kTmBoxCols : colcap; cand >= (tm ? kTmBoxCols : 32) && !tc && !o.w4;
+       cand -= (cand > 256 ? 256 : (tm ? kTmBoxCols : 32))) {
     Geom g{};
     if (geometry(cand, g)) cands.push_back(g);
   }
@@ -483,6 +506,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   p.n_out = n_out;
   p.tile_rows = tc ? kTcRows : 16;
   p.tc = tc ? 1 : 0;
+  p.tm = tm ? 1 : 0;
   p.tc_bpad = tc_bpad;
   p.tc_n = 2 * tc_bpad;
   p.tc_kc = tc_kc;
@@ -694,7 +718,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   out.tile_o_words = static_cast<size_t>(H) / 16 + 1;
   out.sync_words = S_EVENTS + n_events + out.comb_words + out.tile_words + out.tile2_words +
                    out.tile_o_words;
-  out.n_maps = tc ? L * kTcMatsPerLayer + 1 + 4 : 0;
+  out.n_maps = tc ? L * kTcMatsPerLayer + 1 + 4 : (tm ? L * kTcMatsPerLayer + 1 : 0);
   p.xs_map0 = L * kTcMatsPerLayer + 1;
   for (int i = 0; i < 5; ++i) out.splits[i] = split[i];
 
@@ -854,7 +878,40 @@ int encode_weight_maps(const mk_model_config &c, const mk_weights &w, const Layo
     std::memcpy(out.data() + static_cast<size_t>(idx) * sizeof(CUtensorMap), &m, sizeof(m));
     return MK_OK;
   };
+  // tensor-memory staging (mma.sync pages): a 3-D view of each matrix,
+  // x = 16 columns (32 bytes), y = rows, z = 16-column blocks, so that a box
+  // of 16 x 16 x 8 lands as 128 rows of 32 bytes (row 16 b + r = block b of
+  // weight row r), 32-byte swizzled: one tcgen05.cp source
+  auto one_tm = [&](int idx, const void *ptr, int rows, int K) {
+    CUtensorMap m;
+    cuuint64_t dims[3] = {16, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K / 16)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, 32};
+    cuuint32_t box[3] = {16, 16, static_cast<cuuint32_t>(kTmBoxCols / 16)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return lfail(err, MK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", r);
+    std::memcpy(out.data() + static_cast<size_t>(idx) * sizeof(CUtensorMap), &m, sizeof(m));
+    return MK_OK;
+  };
   int rc = MK_OK;
+  if (lay.p.tm) {
+    for (int l = 0; l < L && rc == MK_OK; ++l) {
+      const mk_layer_weights &s = w.layers[l];
+      if ((rc = one_tm(tc_map_index(l, 0), s.wq, Hq * d, H)) ||
+          (rc = one_tm(tc_map_index(l, 1), s.wk, Hkv * d, H)) ||
+          (rc = one_tm(tc_map_index(l, 2), s.wv, Hkv * d, H)) ||
+          (rc = one_tm(tc_map_index(l, 3), s.wo, H, Hq * d)) ||
+          (rc = one_tm(tc_map_index(l, 4), s.w_gate, F, H)) ||
+          (rc = one_tm(tc_map_index(l, 5), s.w_up, F, H)) ||
+          (rc = one_tm(tc_map_index(l, 6), s.w_down, H, F)))
+        break;
+    }
+    if (rc == MK_OK) rc = one_tm(tc_map_index(L, 0), w.lm_head, c.vocab, H);
+    return rc;
+  }
   for (int l = 0; l < L && rc == MK_OK; ++l) {
     const mk_layer_weights &s = w.layers[l];
     if ((rc = one(tc_map_index(l, 0), s.wq, Hq * d, H)) ||
