@@ -156,6 +156,17 @@ __device__ __forceinline__ void tm_ld16x256(uint32_t taddr, uint32_t &r0, uint32
                : "r"(taddr)
                : "memory");
 }
+// The same for 4 consecutive 8-column groups: r[4 i .. 4 i + 3] hold group i.
+__device__ __forceinline__ void tm_ld16x256_x4(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
 __device__ __forceinline__ void tm_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -708,14 +719,18 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       }
     }
   };
-  // lane 0: wait for a barrier phase (bounded), moving pages meanwhile
-  auto lwait = [&](uint64_t *bar, uint32_t parity, uint32_t where) -> bool {
+  // lane 0: wait for a barrier phase (bounded), moving pages meanwhile.
+  // For a ring page (`ring`), also until the mover has passed the page's
+  // previous occupant: an attention page is freed by the compute warps, and
+  // the mover, behind on a page waiting for a tensor-memory slot, must not
+  // read the new occupant's kind in its place.
+  auto lwait = [&](uint64_t *bar, uint32_t parity, uint32_t where, bool ring = false) -> bool {
     if constexpr (!TM) {
       return wait_mbar(p, ctl, bar, parity, where, 2);
     } else {
       uint64_t t0 = 0;
       for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if ((!ring || mv_n < p.n_pages) && mbar_try_wait(bar, parity)) return true;
         service();
         if ((it & 7u) == 7u) {
           if (ctl->cta_abort != 0) return false;
@@ -960,7 +975,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
           gemv_tile(p, t, m, W, row, rv);
           for (int c0 = xc0; c0 < xend; c0 += geo.kp) {
             const int nc = min(geo.kp, xend - c0);
-            if (lane == 0) okl = lwait(&ctl->empty[pi], pe_par ^ 1u, 0xfff10000u);
+            if (lane == 0) okl = lwait(&ctl->empty[pi], pe_par ^ 1u, 0xfff10000u, true);
             ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
             if (!ok) break;
             uint8_t *pg = pages + static_cast<size_t>(pi) * p.page_bytes;
@@ -1031,7 +1046,7 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       for (int tok0 = info.t0; tok0 < info.t1 && ok; tok0 += p.tpp) {
         const int ntok = min(p.tpp, info.t1 - tok0);
         const int nkv = (ntok + P - 1) / P;
-        if (lane == 0) okl = lwait(&ctl->empty[pi], pe_par ^ 1u, 0xfff20000u);
+        if (lane == 0) okl = lwait(&ctl->empty[pi], pe_par ^ 1u, 0xfff20000u, true);
         if (TM && lane == 0) {   // an attention page: the mover passes it over
           mv_kind &= ~(1u << pi);
           ++mv_n;
@@ -1258,16 +1273,18 @@ __device__ __forceinline__ void page_mma_w4(float (&acc)[NN][4], const uint8_t *
 // fragment for the k order (4q, 4q + 1 | 4q + 2, 4q + 3) of lane quarter q,
 // which the activation fragment follows (columns 4q .. 4q + 3 of the block,
 // 8 bytes of the staged hi or lo half).  A warp reads only its lane quarter
-// qq of tensor memory: column blocks 2 qq and 2 qq + 1 of every box; the two
-// warps of quarters 1 and 2 take alternate boxes.
+// qq of tensor memory: column blocks 2 qq and 2 qq + 1 of every box, four
+// boxes per load; the two warps of quarters 1 and 2 take alternate runs of
+// four boxes.
 template <int NN>
 __device__ __forceinline__ void page_tm(float (&acc)[NN][4], uint32_t slot, int nc,
                                         const uint8_t *xs, int xpitch, int xcol0, int B, int warp,
                                         int lane) {
   const int g = lane >> 2, q = lane & 3;
   const int qq = (warp + 1) & 3;
-  const int bstep = (qq == 1 || qq == 2) ? 2 : 1;
-  const int b0 = (bstep == 2 && warp >= 4) ? 1 : 0;
+  const bool pair = qq == 1 || qq == 2;   // two warps on this quarter: alternate 4-box runs
+  const int r0 = (pair && warp >= 4) ? 4 : 0;
+  const int rstep = pair ? 8 : 4;
   const int nbox = nc / kTmBoxCols;
   const int xq = (8 * (q >> 1)) * 4 + (q & 1) * 8 + (g >> 2) * 16;   // bytes, within a block
   float c1[NN][4];
@@ -1275,26 +1292,55 @@ __device__ __forceinline__ void page_tm(float (&acc)[NN][4], uint32_t slot, int 
   for (int nt = 0; nt < NN; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) c1[nt][e] = 0.f;
-#pragma unroll 2
-  for (int bx = b0; bx < nbox; bx += bstep) {
-    uint32_t a[2][4];
+  // the activation fragment of column block cb (16 columns) of box bx
+  auto xfrag = [&](int bx, int cb, int nt) {
+    const int b = nt * 4 + (g & 3);
+    uint2 xv = make_uint2(0u, 0u);
+    if (b < B)
+      xv = *reinterpret_cast<const uint2 *>(xs + b * xpitch + (xcol0 + 16 * (8 * bx + cb)) * 4 + xq);
+    return xv;
+  };
+  for (int bx0 = r0; bx0 < nbox; bx0 += rstep) {
+    const int nb = min(4, nbox - bx0);
+    if (nb == 4) {
+      // four boxes per load: one wait for 8 fragments
+      uint32_t a[2][16];
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
-      tm_ld16x256(slot + (static_cast<uint32_t>(32 * qq + 16 * h) << 16) + 8u * bx, a[h][0],
-                  a[h][1], a[h][2], a[h][3]);
-    tm_wait_ld();
+      for (int h = 0; h < 2; ++h)
+        tm_ld16x256_x4(slot + (static_cast<uint32_t>(32 * qq + 16 * h) << 16) + 8u * bx0, a[h]);
+      tm_wait_ld();
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int xo = (xcol0 + 16 * (8 * bx + 2 * qq + h)) * 4 + xq;
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int nt = 0; nt < NN; ++nt) {
-        const int b = nt * 4 + (g & 3);
-        uint2 xv = make_uint2(0u, 0u);
-        if (b < B) xv = *reinterpret_cast<const uint2 *>(xs + b * xpitch + xo);
-        if (h == 0)
-          mma_bf16(acc[nt], a[h][0], a[h][2], a[h][1], a[h][3], xv.x, xv.y);
-        else
-          mma_bf16(c1[nt], a[h][0], a[h][2], a[h][1], a[h][3], xv.x, xv.y);
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int nt = 0; nt < NN; ++nt) {
+            const uint2 xv = xfrag(bx0 + i, 2 * qq + h, nt);
+            if (h == 0)
+              mma_bf16(acc[nt], a[h][4 * i], a[h][4 * i + 2], a[h][4 * i + 1], a[h][4 * i + 3], xv.x,
+                       xv.y);
+            else
+              mma_bf16(c1[nt], a[h][4 * i], a[h][4 * i + 2], a[h][4 * i + 1], a[h][4 * i + 3], xv.x,
+                       xv.y);
+          }
+    } else {
+      for (int bx = bx0; bx < bx0 + nb; ++bx) {
+        uint32_t a[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          tm_ld16x256(slot + (static_cast<uint32_t>(32 * qq + 16 * h) << 16) + 8u * bx, a[h][0],
+                      a[h][1], a[h][2], a[h][3]);
+        tm_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int nt = 0; nt < NN; ++nt) {
+            const uint2 xv = xfrag(bx, 2 * qq + h, nt);
+            if (h == 0)
+              mma_bf16(acc[nt], a[h][0], a[h][2], a[h][1], a[h][3], xv.x, xv.y);
+            else
+              mma_bf16(c1[nt], a[h][0], a[h][2], a[h][1], a[h][3], xv.x, xv.y);
+          }
       }
     }
   }
