@@ -185,12 +185,12 @@ typedef struct {
                              max_page_cols and o_split apply to path 1 only.
                              3 = path 1 with its weight pages staged in
                              tensor memory: TMA copies 16-row pages in
-                             128-column boxes, the loader copies each landed
+                             512-column boxes, the loader copies each landed
                              page into tensor memory (tcgen05.cp) and frees
                              its shared memory, the compute warps read mma
                              A fragments back (tcgen05.ld), so more bytes
                              stay in flight per SM.  3 needs hidden, ffn and
-                             n_q_heads*head_dim multiples of 128, no 4-bit
+                             n_q_heads*head_dim multiples of 512, no 4-bit
                              weights and no o_split                         */
   int schedule;           /* 0 = dynamic: every CTA takes the next task from
                              one in-GPU ticket queue; 1 = solidified: the

@@ -47,15 +47,16 @@ constexpr int kTcAutoBatch = 5;                   // smallest max_batch that tak
 constexpr int kAttnMmaAutoBatch = 2;              // smallest max_batch that takes the mma.sync attention
 
 // ---- mma.sync GEMV over weights staged in tensor memory -------------------------
-// 16-row weight pages arrive by TMA in 128-column boxes (32-byte swizzle, as
-// 128 "virtual rows" of 16 columns: column block b of row r at row 16 b + r),
-// are copied into tensor memory (tcgen05.cp, one 128 x 256-bit copy per box)
-// and read back as mma.sync A fragments (tcgen05.ld.16x256b), so a page
-// leaves shared memory as soon as it is copied and tensor memory adds
-// kTmSlots pages of bytes in flight per SM.
+// 16-row weight pages arrive by TMA in 512-column boxes (128-byte swizzle, as
+// 128 "virtual rows" of 64 columns: 64-column block b of weight row r at row
+// 16 b + r), are copied into tensor memory (tcgen05.cp, four 128 x 256-bit
+// copies per box, one per 16 columns of the blocks) and read back as mma.sync
+// A fragments (tcgen05.ld.16x256b), so a page leaves shared memory as soon as
+// it is copied and tensor memory adds kTmSlots pages of bytes in flight per SM.
 constexpr int kTmSlots = 4;                       // tensor-memory page slots
 constexpr int kTmSlotCols = 128;                  // columns per slot (a 2048-column page)
-constexpr int kTmBoxCols = 128;                   // weight columns per TMA box / tcgen05.cp
+constexpr int kTmBoxCols = 512;                   // weight columns per TMA box (16 KB)
+constexpr int kTmBoxBytes = 16 * kTmBoxCols * 2;
 constexpr int kTcMatsPerLayer = 7;                // tensor maps: wq wk wv wo w_gate w_up w_down
 
 // ---- kernel variants (template argument of the step kernel) -------------------

@@ -72,6 +72,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of a phase (try_wait may suspend the thread for a while
+// before it reports an incomplete phase; test_wait returns at once).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, P1;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
@@ -128,15 +142,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, int x, 
       : "memory");
 }
 
-// Shared-memory matrix descriptor of 128 rows of 32 bytes in the 32-byte
-// swizzled K-major layout that a TMA copy with 32-byte swizzle writes: rows
-// 32 bytes apart, 8-row groups 256 bytes apart; layout type 6 = 32-byte
-// swizzle (bits 61-63).  The source of one tcgen05.cp.128x256b.
-__device__ __forceinline__ uint64_t sw32_desc(uint32_t saddr) {
-  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (1ull << 16) |
-         (static_cast<uint64_t>(256 >> 4) << 32) | (1ull << 46) | (6ull << 61);
-}
-
 // Copy 128 rows x 256 bits from shared memory (descriptor) into tensor memory:
 // row i to lane i, its 32 bytes to 8 consecutive columns.  Issued by one
 // thread; completion is tracked by tcgen05.commit.
@@ -144,19 +149,12 @@ __device__ __forceinline__ void tm_cp(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-// Warp-wide: 16 lanes x 256 bits of tensor memory starting at lane
-// (taddr >> 16) (a multiple of 16 inside this warp's lane quarter).  Thread
-// (g = lane / 4, q = lane % 4) receives, of rows g and g + 8, the 32-bit
-// words 2q and 2q + 1: r0 = (g, 2q), r1 = (g, 2q + 1), r2 = (g + 8, 2q),
-// r3 = (g + 8, 2q + 1).  (Completion: tcgen05.wait::ld.)
-__device__ __forceinline__ void tm_ld16x256(uint32_t taddr, uint32_t &r0, uint32_t &r1,
-                                            uint32_t &r2, uint32_t &r3) {
-  asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(taddr)
-               : "memory");
-}
-// The same for 4 consecutive 8-column groups: r[4 i .. 4 i + 3] hold group i.
+// Warp-wide: 16 lanes x 4 x 256 bits of tensor memory starting at lane
+// (taddr >> 16) (a multiple of 16 inside this warp's lane quarter): four
+// consecutive 8-column groups.  Of group i, thread (g = lane / 4, q = lane % 4)
+// receives the 32-bit words 2q and 2q + 1 of rows g and g + 8:
+// r[4i] = (g, 2q), r[4i + 1] = (g, 2q + 1), r[4i + 2] = (g + 8, 2q),
+// r[4i + 3] = (g + 8, 2q + 1).  (Completion: tcgen05.wait::ld.)
 __device__ __forceinline__ void tm_ld16x256_x4(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
@@ -695,13 +693,17 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
       while (mv_n > 0) {
         const int pm = mv_pm;
         if ((mv_kind >> pm) & 1u) {
-          if (!mbar_try_wait(&ctl->full[pm], mv_ppar)) return;
-          if (!mbar_try_wait(tm_empty_bar(smem, p, tslot), tpar ^ 1u)) return;
+          if (!mbar_test_wait(&ctl->full[pm], mv_ppar)) return;
+          if (!mbar_test_wait(tm_empty_bar(smem, p, tslot), tpar ^ 1u)) return;
           tc_fence_after();
           const int nb = static_cast<int>((mv_ng >> (4 * pm)) & 15u) + 1;
           const uint32_t src = smem_u32(pages + static_cast<size_t>(pm) * p.page_bytes);
           const uint32_t dst = tmem + static_cast<uint32_t>(tslot * kTmSlotCols);
-          for (int b = 0; b < nb; ++b) tm_cp(dst + 8u * b, sw32_desc(src + 4096u * b));
+          // box b, 16-column slice j of its 64-column blocks -> columns 32 b + 8 j
+          for (int b = 0; b < nb; ++b)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tm_cp(dst + 32u * b + 8u * j, sw128_desc(src + static_cast<uint32_t>(kTmBoxBytes) * b + 32u * j));
           tc_commit(&ctl->empty[pm]);      // the shared-memory page is free once copied
           tc_commit(tm_full_bar(smem, p, tslot));
           last_slot = tslot;
@@ -730,8 +732,8 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
     } else {
       uint64_t t0 = 0;
       for (uint32_t it = 0;; ++it) {
-        if ((!ring || mv_n < p.n_pages) && mbar_try_wait(bar, parity)) return true;
-        service();
+        service();   // (first: pages that landed meanwhile move without delay)
+        if ((!ring || mv_n < p.n_pages) && mbar_test_wait(bar, parity)) return true;
         if ((it & 7u) == 7u) {
           if (ctl->cta_abort != 0) return false;
           if ((it & 255u) == 255u && ld_relaxed(p.sync + S_ABORT) != 0u) return false;
@@ -980,21 +982,21 @@ __device__ void loader_main(const Params &p, Ctl *ctl, uint8_t *smem) {
             if (!ok) break;
             uint8_t *pg = pages + static_cast<size_t>(pi) * p.page_bytes;
             if (TM) {
-              // 128-column boxes of 16 rows (rows past the matrix arrive as
-              // zeros), each landing as one tcgen05.cp source
+              // 512-column boxes of 16 rows (rows past the matrix arrive as
+              // zeros), each landing as four tcgen05.cp sources
               const int nb = nc / kTmBoxCols;
               const bool up = t.type == T_GATEUP && m >= (t.n_m >> 1);
               const void *map = static_cast<const uint8_t *>(p.tmaps) +
                                 static_cast<size_t>(up ? t.map1 : t.map0) * 128;
               if (lane == 0) {
-                mbar_arrive_expect_tx(&ctl->full[pi], static_cast<uint32_t>(nb) * 4096u);
+                mbar_arrive_expect_tx(&ctl->full[pi], static_cast<uint32_t>(nb * kTmBoxBytes));
                 mv_kind |= 1u << pi;
                 mv_ng = (mv_ng & ~(15ull << (4 * pi))) | (static_cast<uint64_t>(nb - 1) << (4 * pi));
                 ++mv_n;
               }
               __syncwarp();
               if (lane < nb)
-                tma_load_3d(pg + lane * 4096, map, 0, row, (c0 + lane * kTmBoxCols) / 16,
+                tma_load_3d(pg + lane * kTmBoxBytes, map, 0, row, (c0 + lane * kTmBoxCols) / 64,
                             &ctl->full[pi], pol);
             } else if (W4 && is_w4_task(p.w4, t.type)) {
               // 4-bit: the row tile's packed blocks of these columns are
@@ -1267,82 +1269,55 @@ __device__ __forceinline__ void page_mma_w4(float (&acc)[NN][4], const uint8_t *
 }
 
 // One 16-row weight page staged in tensor memory (slot columns at `slot`)
-// against the staged activation.  The page's 128-column boxes sit at slot
-// columns 8 box .. 8 box + 7, and column block b (16 columns) of the box in
-// lanes 16 b .. 16 b + 15: a 16x256b load there is the block's mma A
-// fragment for the k order (4q, 4q + 1 | 4q + 2, 4q + 3) of lane quarter q,
-// which the activation fragment follows (columns 4q .. 4q + 3 of the block,
-// 8 bytes of the staged hi or lo half).  A warp reads only its lane quarter
-// qq of tensor memory: column blocks 2 qq and 2 qq + 1 of every box, four
-// boxes per load; the two warps of quarters 1 and 2 take alternate runs of
-// four boxes.
+// against the staged activation.  Box bx (512 columns) sits at slot columns
+// 32 bx .. 32 bx + 31: 64-column block cb of the box in lanes 16 cb ..
+// 16 cb + 15, its 16-column slice j in columns 32 bx + 8 j .. + 7.  A
+// 16x256b load there is the slice's mma A fragment for the k order
+// (4q, 4q + 1 | 4q + 2, 4q + 3) of lane quarter q, which the activation
+// fragment follows (columns 4q .. 4q + 3 of the slice, 8 bytes of the staged
+// hi or lo half).  A warp reads only its lane quarter qq of tensor memory:
+// blocks 2 qq and 2 qq + 1 of every box, its four slices per load; the two
+// warps of quarters 1 and 2 take alternate boxes.
 template <int NN>
 __device__ __forceinline__ void page_tm(float (&acc)[NN][4], uint32_t slot, int nc,
                                         const uint8_t *xs, int xpitch, int xcol0, int B, int warp,
                                         int lane) {
   const int g = lane >> 2, q = lane & 3;
   const int qq = (warp + 1) & 3;
-  const bool pair = qq == 1 || qq == 2;   // two warps on this quarter: alternate 4-box runs
-  const int r0 = (pair && warp >= 4) ? 4 : 0;
-  const int rstep = pair ? 8 : 4;
+  const bool pair = qq == 1 || qq == 2;
+  const int b0 = (pair && warp >= 4) ? 1 : 0;
+  const int bstep = pair ? 2 : 1;
   const int nbox = nc / kTmBoxCols;
-  const int xq = (8 * (q >> 1)) * 4 + (q & 1) * 8 + (g >> 2) * 16;   // bytes, within a block
+  const int xq = (8 * (q >> 1)) * 4 + (q & 1) * 8 + (g >> 2) * 16;   // bytes, within a slice
   float c1[NN][4];
 #pragma unroll
   for (int nt = 0; nt < NN; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) c1[nt][e] = 0.f;
-  // the activation fragment of column block cb (16 columns) of box bx
-  auto xfrag = [&](int bx, int cb, int nt) {
-    const int b = nt * 4 + (g & 3);
-    uint2 xv = make_uint2(0u, 0u);
-    if (b < B)
-      xv = *reinterpret_cast<const uint2 *>(xs + b * xpitch + (xcol0 + 16 * (8 * bx + cb)) * 4 + xq);
-    return xv;
-  };
-  for (int bx0 = r0; bx0 < nbox; bx0 += rstep) {
-    const int nb = min(4, nbox - bx0);
-    if (nb == 4) {
-      // four boxes per load: one wait for 8 fragments
-      uint32_t a[2][16];
+  for (int bx = b0; bx < nbox; bx += bstep) {
+    uint32_t a[2][16];
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-        tm_ld16x256_x4(slot + (static_cast<uint32_t>(32 * qq + 16 * h) << 16) + 8u * bx0, a[h]);
-      tm_wait_ld();
+    for (int h = 0; h < 2; ++h)
+      tm_ld16x256_x4(slot + (static_cast<uint32_t>(32 * qq + 16 * h) << 16) + 32u * bx, a[h]);
+    tm_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+      for (int j = 0; j < 4; ++j) {
+        const int col = kTmBoxCols * bx + 64 * (2 * qq + h) + 16 * j;
 #pragma unroll
-          for (int nt = 0; nt < NN; ++nt) {
-            const uint2 xv = xfrag(bx0 + i, 2 * qq + h, nt);
-            if (h == 0)
-              mma_bf16(acc[nt], a[h][4 * i], a[h][4 * i + 2], a[h][4 * i + 1], a[h][4 * i + 3], xv.x,
-                       xv.y);
-            else
-              mma_bf16(c1[nt], a[h][4 * i], a[h][4 * i + 2], a[h][4 * i + 1], a[h][4 * i + 3], xv.x,
-                       xv.y);
-          }
-    } else {
-      for (int bx = bx0; bx < bx0 + nb; ++bx) {
-        uint32_t a[2][4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          tm_ld16x256(slot + (static_cast<uint32_t>(32 * qq + 16 * h) << 16) + 8u * bx, a[h][0],
-                      a[h][1], a[h][2], a[h][3]);
-        tm_wait_ld();
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int nt = 0; nt < NN; ++nt) {
-            const uint2 xv = xfrag(bx, 2 * qq + h, nt);
-            if (h == 0)
-              mma_bf16(acc[nt], a[h][0], a[h][2], a[h][1], a[h][3], xv.x, xv.y);
-            else
-              mma_bf16(c1[nt], a[h][0], a[h][2], a[h][1], a[h][3], xv.x, xv.y);
-          }
+        for (int nt = 0; nt < NN; ++nt) {
+          const int b = nt * 4 + (g & 3);
+          uint2 xv = make_uint2(0u, 0u);
+          if (b < B) xv = *reinterpret_cast<const uint2 *>(xs + b * xpitch + (xcol0 + col) * 4 + xq);
+          if (j & 1)
+            mma_bf16(c1[nt], a[h][4 * j], a[h][4 * j + 2], a[h][4 * j + 1], a[h][4 * j + 3], xv.x,
+                     xv.y);
+          else
+            mma_bf16(acc[nt], a[h][4 * j], a[h][4 * j + 2], a[h][4 * j + 1], a[h][4 * j + 3], xv.x,
+                     xv.y);
+        }
       }
-    }
   }
 #pragma unroll
   for (int nt = 0; nt < NN; ++nt)

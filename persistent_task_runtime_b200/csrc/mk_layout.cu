@@ -396,7 +396,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   // fewer hand-offs per byte.  Failing 3 pages, the most pages.
   std::vector<Geom> cands;
   for (int cand = tm ? colcap / kTmBoxCols * kTmBoxCols : colcap; cand >= (tm ? kTmBoxCols : 32) && !tc && !o.w4;
-       cand -= (cand > 256 ? 256 : (tm ? kTmBoxCols : 32))) {
+       cand -= tm ? kTmBoxCols : (cand > 256 ? 256 : 32)) {
     Geom g{};
     if (geometry(cand, g)) cands.push_back(g);
   }
@@ -879,18 +879,18 @@ int encode_weight_maps(const mk_model_config &c, const mk_weights &w, const Layo
     return MK_OK;
   };
   // tensor-memory staging (mma.sync pages): a 3-D view of each matrix,
-  // x = 16 columns (32 bytes), y = rows, z = 16-column blocks, so that a box
-  // of 16 x 16 x 8 lands as 128 rows of 32 bytes (row 16 b + r = block b of
-  // weight row r), 32-byte swizzled: one tcgen05.cp source
+  // x = 64 columns (128 bytes), y = rows, z = 64-column blocks, so that a box
+  // of 64 x 16 x 8 lands as 128 rows of 128 bytes (row 16 b + r = block b of
+  // weight row r), 128-byte swizzled: four tcgen05.cp sources
   auto one_tm = [&](int idx, const void *ptr, int rows, int K) {
     CUtensorMap m;
-    cuuint64_t dims[3] = {16, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K / 16)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, 32};
-    cuuint32_t box[3] = {16, 16, static_cast<cuuint32_t>(kTmBoxCols / 16)};
+    cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K / 64)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, 128};
+    cuuint32_t box[3] = {64, 16, static_cast<cuuint32_t>(kTmBoxCols / 64)};
     cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
                               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return lfail(err, MK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", r);
     std::memcpy(out.data() + static_cast<size_t>(idx) * sizeof(CUtensorMap), &m, sizeof(m));

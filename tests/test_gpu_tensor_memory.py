@@ -1,8 +1,8 @@
 """GPU parity of the mma.sync GEMV over weight pages staged in tensor memory
 (gemv_path 3) against the CPU oracle.
 
-The weights of every projection arrive by TMA tensor copies in 128-column
-boxes of 16 rows (32-byte swizzle), are copied into tensor memory by the
+The weights of every projection arrive by TMA tensor copies in 512-column
+boxes of 16 rows (128-byte swizzle), are copied into tensor memory by the
 loader (tcgen05.cp) and read back by the compute warps as mma.sync A
 fragments (tcgen05.ld.16x256b).  The shapes put ragged edges where the path
 has them: a 5000-row LM head (a last row tile of 8 rows, which TMA pads with
@@ -22,7 +22,7 @@ from tests.gpu_harness import Pair, StepReport, assert_report
 
 pytestmark = pytest.mark.gpu
 
-TM_CFG = dict(n_layers=2, hidden=1024, n_q_heads=8, n_kv_heads=2, head_dim=128, ffn=2816,
+TM_CFG = dict(n_layers=2, hidden=1024, n_q_heads=8, n_kv_heads=2, head_dim=128, ffn=3072,
               vocab=5000, rms_eps=1e-6, rope_theta=1e6, qk_norm=True)
 
 
@@ -79,7 +79,7 @@ def test_tensor_memory_and_mma_paths_agree(cuda_device):
 
 
 def test_tensor_memory_full_size_8b_batch1(cuda_device):
-    """The 8B shape at batch 1 through tensor memory (64 KB pages: 16 boxes,
+    """The 8B shape at batch 1 through tensor memory (64 KB pages: 4 boxes,
     a whole slot), one step at context 64 against the oracle's first layers
     is covered by the full-size tests; here the step must run clean and give
     the same token and logits (to 5e-3) as the plain mma.sync path."""

@@ -277,23 +277,26 @@ def test_attention_path_option():
         assert e.value.code == mk.MK_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("name", ["8b", "1.5b"])
 @pytest.mark.parametrize("batch", [1, 2, 4])
-def test_tensor_memory_gemv_plan(name, batch):
+def test_tensor_memory_gemv_plan(batch):
     """gemv_path 3 (mma.sync pages staged in tensor memory): the task graph
     of the plain mma.sync path, with every weight page a whole number of
-    128-column boxes (the loader's TMA boxes and tcgen05.cp sources), and a
-    valid graph by the same checks as every other plan."""
-    cfg = SHAPES[name]
+    512-column boxes (the loader's TMA boxes, each four tcgen05.cp sources),
+    and a valid graph by the same checks as every other plan."""
+    cfg = SHAPES["8b"]
     i3, t3 = mk.describe(cfg, max_batch=batch, max_seq_len=1024, gemv_path=3)
     assert i3["gemv_path"] == 3
-    assert all(c % 128 == 0 for c in i3["page_cols"])
-    assert i3["ffn_part_cols"] % 128 == 0
+    assert all(c % 512 == 0 for c in i3["page_cols"])
+    assert i3["ffn_part_cols"] % 512 == 0
     check_plan(cfg, i3, t3, batch)
 
 
 def test_tensor_memory_gemv_rejections():
-    tiny = SHAPES["tiny"]   # ffn 688: not whole 128-column boxes
+    for cfg in (SHAPES["tiny"], SHAPES["1.5b"]):   # ffn 688, 8960: not whole 512-column boxes
+        with pytest.raises(mk.MkError) as e:
+            mk.describe(cfg, gemv_path=3)
+        assert e.value.code == mk.MK_ERR_UNSUPPORTED
+    tiny = SHAPES["tiny"]
     with pytest.raises(mk.MkError) as e:
         mk.describe(tiny, gemv_path=3)
     assert e.value.code == mk.MK_ERR_UNSUPPORTED
