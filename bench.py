@@ -458,8 +458,8 @@ def main():
     ap.add_argument("--prompt-path", choices=["chunks", "decode"], default="chunks",
                     help="how a workload's prompt fills the cache: prompt chunks of 16 tokens "
                          "(mk_prefill_chunk) or one decode step per token")
-    ap.add_argument("--schedule", type=int, default=0, choices=[0, 1],
-                    help="0 dynamic ticket queue, 1 solidified per-CTA task lists")
+    ap.add_argument("--schedule", type=int, default=0, choices=[0, 1, 2],
+                    help="0 automatic (solidified), 1 solidified per-CTA task lists, 2 dynamic queue")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-threads", type=int, default=0,
                     help="threads for the CPU oracle (0: the process's BLAS thread pool as set up)")

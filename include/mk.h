@@ -192,14 +192,15 @@ typedef struct {
                              stay in flight per SM.  3 needs hidden, ffn and
                              n_q_heads*head_dim multiples of 512, no 4-bit
                              weights and no o_split                         */
-  int schedule;           /* 0 = dynamic: every CTA takes the next task from
-                             one in-GPU ticket queue; 1 = solidified: the
+  int schedule;           /* 0 = automatic: solidified; 1 = solidified: the
                              plan assigns each CTA its task list offline (list
                              scheduling in queue order under a cost model of
                              weight bytes per task; the Ada-MK summary's
                              offline path solidification) and each CTA runs
-                             its list in order.  Per-operator modes always
-                             use the queue                                  */
+                             its list in order; 2 = dynamic: every CTA takes
+                             the next task from one in-GPU ticket queue.
+                             Per-operator modes and mk_decode_step_noalloc
+                             always use the queue                           */
   int weight_bits;        /* 0: as the weights are given (mk_plan_describe:
                              bf16); 16: bf16 projections; 4: 4-bit (the
                              weights must carry w4_layers).  4-bit plans run

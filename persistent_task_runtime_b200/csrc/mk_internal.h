@@ -268,7 +268,7 @@ struct LayoutOptions {
   int max_page_cols = 0;        // 0: kMaxPageCols
   bool o_split = false;         // O projection in two K parts of whole KV groups
   int gemv_path = 0;            // 0 automatic, 1 mma.sync pages, 2 tcgen05 tiles, 3 mma.sync pages through tensor memory
-  int schedule = 0;             // 0 dynamic ticket queue, 1 solidified per-CTA task lists
+  int schedule = 0;             // 0 automatic (solidified), 1 solidified per-CTA task lists, 2 dynamic ticket queue
   bool prefill = false;         // K/V appended by their own tasks (prompt chunks of one sequence)
   bool w4 = false;              // 4-bit projections (packed, MK_W4_BLOCK_BYTES blocks)
   int attn_path = 0;            // 0 automatic / 1 CUDA-core FMA, 2 mma.sync tiles (d 64, 128)

@@ -163,6 +163,7 @@ extern "C" MK_API int mk_decode_step_noalloc(const mk_model_config *cfg, const m
     lo.max_batch = B;
     lo.page_size = P;
     lo.w4 = w->w4_layers != nullptr;
+    lo.schedule = 2;   // the dynamic queue: the scratch array holds no per-CTA lists
     std::string err;
     const int rc = mk::build_layout(c, lo, nsm, smem_optin, up.lay, err);
     if (rc) return nfail(rc, err.c_str());

@@ -68,13 +68,16 @@ def test_odd_shapes(cuda_device, name):
     assert_report(rep)
 
 
-def test_batch_ragged_history(cuda_device):
+@pytest.mark.parametrize("schedule", [0, 2])
+def test_batch_ragged_history(cuda_device, schedule):
     """B = 5 sequences at ragged positions over a synthetic KV history whose
-    lengths sit on and around page and chunk boundaries."""
+    lengths sit on and around page and chunk boundaries; under the default
+    (solidified) schedule and the dynamic ticket queue."""
     cfg = synth.CONFIGS["tiny"]
     lengths = [0, 15, 16, 17, 300]
     steps = 6
-    pair = Pair(cfg, _weights(cfg, seed=5), 5, [n + steps for n in lengths])
+    pair = Pair(cfg, _weights(cfg, seed=5), 5, [n + steps for n in lengths], schedule=schedule)
+    assert pair.plan.info()["schedule"] == (0 if schedule == 2 else 1)
     hist = synth.make_kv_history(cfg, lengths, seed=6)
     pair.load_history(hist, lengths)
     ids = synth.make_ids(cfg["vocab"], (steps, 5), seed=7)
@@ -101,8 +104,8 @@ def test_long_context_many_attention_chunks(cuda_device):
     assert_report(rep)
 
 
-@pytest.mark.parametrize("path", [1, 2])
-def test_large_batch_chunked_activations(cuda_device, path):
+@pytest.mark.parametrize("path,schedule", [(1, 0), (2, 0), (2, 2)])
+def test_large_batch_chunked_activations(cuda_device, path, schedule):
     """B = 16 with activations too wide for one staging buffer: on the
     mma.sync path (four mma n-tiles) every projection stages its input in
     column chunks; on the tensor-core path chunks stream through two
@@ -112,7 +115,7 @@ def test_large_batch_chunked_activations(cuda_device, path):
     B = 16
     lengths = [int(x) for x in np.linspace(1, 200, B)]
     pair = Pair(cfg, _weights(cfg, seed=8, gain="random"), B, [n + 8 for n in lengths],
-                gemv_path=path)
+                gemv_path=path, schedule=schedule)
     pair.load_history(synth.make_kv_history(cfg, lengths, seed=9), lengths)
     ids = synth.make_ids(cfg["vocab"], (3, B), seed=10)
     rep = StepReport()

@@ -206,7 +206,7 @@ def test_solidified_schedule_no_deadlock(name, batch, workers, path):
             assert ctr[wait] == need
     # the dynamic plan describes no schedule
     assert (mk.describe_schedule(cfg, info["n_tasks"], max_batch=batch, max_seq_len=600,
-                                 gemv_path=path, num_sms=workers, schedule=0) == -1).all()
+                                 gemv_path=path, num_sms=workers, schedule=2) == -1).all()
 
 
 @pytest.mark.parametrize("name,batch,workers,path", [("tiny", 16, 9, 0), ("3groups", 16, 148, 2),
