@@ -294,8 +294,8 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     // (epilogue, split-K sum and hand-offs, about 4 us: the time one SM's
     // share of HBM streams 640 columns of a 128-row tile).  Ties go to fewer
     // parts.
+    constexpr long long kTaskCostCols = 640;
     auto parts_for = [&](int tiles, int nm, int K, int i) {
-      constexpr long long kTaskCostCols = 640;
       const int nmax = std::max(1, K / tc_kc);
       long long best = -1;
       int bn = 1, bw = K;
@@ -316,10 +316,23 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
     parts_for(NQKV / kTcRows, 1, H, 0);
     parts_for(cdiv(F, kTcRows), 2, H, 2);
     parts_for(cdiv(H, kTcRows), 1, F, 3);
-    o_groups = 1;
-    n_o_parts = Hkv;
+    // the O projection in parts of whole KV groups (each part waits only for
+    // its groups' attention), as many groups per part as the same model says
+    {
+      long long best = -1;
+      for (int og = 1; og <= Hkv; ++og) {
+        if (Hkv % og != 0) continue;
+        const long long rounds = cdiv(cdiv(H, kTcRows) * (Hkv / og), grid);
+        const long long cost = rounds * (static_cast<long long>(og) * G * d + kTaskCostCols);
+        if (best < 0 || cost < best) {
+          best = cost;
+          o_groups = og;
+        }
+      }
+    }
+    n_o_parts = Hkv / o_groups;
     split[1] = n_o_parts;
-    kt[1] = n_o_parts > 1 ? G * d : 0;
+    kt[1] = n_o_parts > 1 ? o_groups * G * d : 0;
     n_ksplit = split[3];
     kchunk_ffn = kt[3] > 0 ? kt[3] : F;
     if (n_ksplit > 255 || split[0] > 255 || split[2] > 255)
