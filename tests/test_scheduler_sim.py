@@ -204,8 +204,11 @@ def test_solidified_schedule_no_deadlock(name, batch, workers, path):
     for ty, wait, need, *_ in tasks:
         if wait >= 0:
             assert ctr[wait] == need
-    # the dynamic plan describes no schedule
-    assert (mk.describe_schedule(cfg, info["n_tasks"], max_batch=batch, max_seq_len=600,
+    # the dynamic plan (its own task count: gate/up tasks of one row tile)
+    # describes no schedule
+    info2, _ = mk.describe(cfg, max_batch=batch, max_seq_len=600, gemv_path=path, schedule=2,
+                           num_sms=workers)
+    assert (mk.describe_schedule(cfg, info2["n_tasks"], max_batch=batch, max_seq_len=600,
                                  gemv_path=path, num_sms=workers, schedule=2) == -1).all()
 
 
