@@ -311,6 +311,25 @@ def test_tensor_memory_gemv_rejections():
     assert e.value.code == mk.MK_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("name", ["8b", "1.5b", "tiny"])
+def test_schedule_default_and_task_sizes(name):
+    """The solidified lists are the default (schedule 0 and 1), the dynamic
+    queue on request (2); under the lists the mma.sync path's gate/up tasks
+    take two row tiles, under the queue one (many small tasks for the queue's
+    run-time balance).  Both graphs are valid."""
+    cfg = SHAPES[name]
+    i0, t0 = mk.describe(cfg, max_batch=1, max_seq_len=600)
+    i1, _ = mk.describe(cfg, max_batch=1, max_seq_len=600, schedule=1)
+    i2, t2 = mk.describe(cfg, max_batch=1, max_seq_len=600, schedule=2)
+    assert i0["schedule"] == 1 and i1["schedule"] == 1 and i2["schedule"] == 0
+    assert i0["rows_per_task"][2] == 32 and i2["rows_per_task"][2] == 16
+    check_plan(cfg, i0, t0, 1)
+    check_plan(cfg, i2, t2, 1)
+    with pytest.raises(mk.MkError) as e:
+        mk.describe(cfg, schedule=3)
+    assert e.value.code == mk.MK_ERR_INVALID_ARG
+
+
 def test_describe_rejects_what_create_rejects():
     cfg = dict(SHAPES["tiny"], head_dim=96)
     with pytest.raises(mk.MkError):
