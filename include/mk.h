@@ -173,7 +173,7 @@ typedef struct {
                              and >= 1024 columns per part); 0 = one part.
                              mma.sync path only                             */
   int gemv_path;          /* how the projections run: 0 = automatic (tensor
-                             cores when max_batch >= 5 and the shape allows),
+                             cores when max_batch >= 4 and the shape allows),
                              1 = CUDA-core mma.sync over 16-row weight pages,
                              2 = tcgen05 tensor cores over 128-row tiles: the
                              weights arrive by TMA tensor copies in the

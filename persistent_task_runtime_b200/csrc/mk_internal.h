@@ -43,7 +43,7 @@ constexpr int kTcAtomCols = 64;                   // columns of one 128-byte swi
 constexpr int kTcAtomBytes = kTcRows * 128;       // one weight atom: 128 rows x 128 B
 constexpr int kTcXBytes = 32 * 1024;              // one staged activation chunk buffer
 constexpr int kTcTmemCols = 128;                  // tensor-memory columns allocated per CTA
-constexpr int kTcAutoBatch = 5;                   // smallest max_batch that takes it by default
+constexpr int kTcAutoBatch = 4;                   // smallest max_batch that takes it by default
 constexpr int kAttnMmaAutoBatch = 2;              // smallest max_batch that takes the mma.sync attention
 
 // ---- mma.sync GEMV over weights staged in tensor memory -------------------------

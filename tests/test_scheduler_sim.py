@@ -145,7 +145,7 @@ CASES = [("tiny", 1, 1, 0), ("tiny", 1, 5, 0), ("tiny", 3, 148, 0), ("tiny", 16,
 def test_no_deadlock_every_task_once(name, batch, workers, path):
     cfg = SHAPES[name]
     info, t = mk.describe(cfg, max_batch=batch, max_seq_len=600, gemv_path=path)
-    if path == 2 or (batch >= 5 and cfg["head_dim"] == 128):
+    if path == 2 or (batch >= 4 and cfg["head_dim"] == 128):
         assert info["gemv_path"] == 2
     tasks = compile_tasks(cfg, info, t)
     seeds = (1,) if name in ("1.5b", "8b") else (1, 2, 3)
