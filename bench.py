@@ -34,6 +34,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -84,16 +85,36 @@ def model_config(wl: dict) -> dict:
     return cfg
 
 
+# C/C++ tokens that matter to the digest: string and character literals are
+# kept whole, comments are dropped (so that a comment inside a literal, or a
+# quote inside a comment, is read the way the compiler reads it).
+_C_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|//[^\n]*|/\*.*?\*/', re.S)
+
+
+def code_text(src: str) -> str:
+    """C/C++ source without its comments, whitespace runs outside literals
+    collapsed to one space."""
+    parts, at = [], 0
+    for m in _C_TOKENS.finditer(src):
+        parts.append(" ".join(src[at:m.start()].split()))
+        tok = m.group(0)
+        parts.append(tok if tok[0] in "\"'" else "")
+        at = m.end()
+    parts.append(" ".join(src[at:].split()))
+    return " ".join(p for p in parts if p)
+
+
 def source_digest() -> str:
-    """sha256 over the kernel and plan sources (the code a DRAM capture covers)."""
+    """sha256 over the code of the kernel and plan sources (the code a DRAM
+    capture covers); comments and layout do not enter it."""
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "persistent_task_runtime_b200", "csrc")
     for name in sorted(os.listdir(cdir)):
         if name.endswith((".cu", ".h")):
-            with open(os.path.join(cdir, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
-    with open(os.path.join(ROOT, "include", "mk.h"), "rb") as f:
-        h.update(f.read())
+            with open(os.path.join(cdir, name), encoding="utf-8") as f:
+                h.update(name.encode() + b"\0" + code_text(f.read()).encode())
+    with open(os.path.join(ROOT, "include", "mk.h"), encoding="utf-8") as f:
+        h.update(code_text(f.read()).encode())
     return h.hexdigest()
 
 

@@ -174,7 +174,8 @@ typedef struct {
                              mma.sync path only                             */
   int gemv_path;          /* how the projections run: 0 = automatic (tensor
                              cores when max_batch >= 4 and the shape allows),
-                             1 = CUDA-core mma.sync over 16-row weight pages,
+                             1 = warp-level mma.sync (the pre-tcgen05 tensor
+                             core instruction) over 16-row weight pages,
                              2 = tcgen05 tensor cores over 128-row tiles: the
                              weights arrive by TMA tensor copies in the
                              swizzled layout the MMA reads, the activation is
@@ -388,7 +389,7 @@ MK_API int mk_plan_describe(const mk_model_config *cfg, const mk_plan_options *o
                             void *tasks, int64_t max_tasks);
 
 /* The CTA each task of that plan runs on under a solidified schedule
- * (opts->schedule == 1), without any GPU: cta_of_task[i] for i < n_tasks,
+ * (opts->schedule 0 or 1), without any GPU: cta_of_task[i] for i < n_tasks,
  * or -1 for every task when the plan uses the dynamic queue.  Each CTA runs
  * its tasks in ascending index order.  MK_ERR_INVALID_ARG if max_tasks is
  * below the plan's task count. */

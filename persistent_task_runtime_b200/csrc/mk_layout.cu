@@ -162,7 +162,7 @@ int build_layout(const mk_model_config &c, const LayoutOptions &o, int nsm, int 
   const int smem_max = std::min(smem_optin, kMaxSmem);
   const int mt_cap = max_mtiles_for(maxB);
 
-  // ---- GEMV path: CUDA-core mma.sync pages, or tcgen05 tiles of 128 rows -------------
+  // ---- GEMV path: warp-level mma.sync pages, or tcgen05 tiles of 128 rows -------------
   // The tensor-core path needs one 128-row tile per head (head_dim 128) and
   // inputs whose width is a whole number of 64-column swizzle atoms.
   const bool tc_ok = d == kTcRows && H % 64 == 0 && F % 64 == 0 && (Hq * d) % 64 == 0;

@@ -58,3 +58,22 @@ def test_workload_names(name, batch, model):
     wl = bench.parse_workload(name)
     assert wl["batch"] == batch and wl["model"] == model
     assert len(wl["lengths"]) == batch
+
+
+def test_source_digest_ignores_comments_but_not_code():
+    """The digest that gates the committed DRAM figures follows the code only:
+    comments and whitespace leave it alone, a literal or a token does not."""
+    a = 'int f(int x) {  // scale\n  return x * 2; /* two */ }\nconst char *s = "a // b";\n'
+    b = 'int f(int x) {\n\n  return x * 2; }\nconst char *s = "a // b"; // the literal\n'
+    assert bench.code_text(a) == bench.code_text(b)
+    assert bench.code_text(a) != bench.code_text(a.replace("x * 2", "x * 3"))
+    assert bench.code_text(a) != bench.code_text(a.replace('"a // b"', '"a //  b"'))
+    assert bench.code_text("char c = '/'; int y; /* '\"' */") == bench.code_text("char c = '/'; int y;")
+    assert "/*" not in bench.code_text("int y; /* '\"' */")
+
+
+def test_profiled_traffic_matches_current_sources():
+    """The batch-1 summary's digest is that of the current sources, so the
+    bench line carries its measured DRAM bytes."""
+    t = bench.profiled_traffic("8b_b1_ctx512")
+    assert t is not None and t > 15e9
