@@ -244,13 +244,17 @@ def describe(cfg: Dict, max_batch: int = 1, page_size: int = 16, max_seq_len: in
 
 def describe_schedule(cfg: Dict, n_tasks: int, max_batch: int = 1, page_size: int = 16,
                       max_seq_len: int = 4096, num_sms: int = 148, smem_optin: int = 232448,
-                      gemv_path: int = 0, schedule: int = 1):
-    """CTA of every task under the plan's solidified schedule (-1: dynamic queue)."""
+                      gemv_path: int = 0, schedule: int = 1, rows_per_task=(0, 0, 0, 0, 0),
+                      max_page_cols: int = 0, o_split: bool = False, prefill: bool = False,
+                      weight_bits: int = 0, attn_path: int = 0):
+    """CTA of every task under the plan's solidified schedule (-1: dynamic
+    queue); the options are those of describe()."""
     import numpy as np
     lib = load_library()
     c = _config(cfg, max_seq_len)
-    opts = mk_plan_options(max_batch, page_size, 0, 0, (C.c_int * 5)(0, 0, 0, 0, 0), 0, 0, 0,
-                           gemv_path, schedule)
+    opts = mk_plan_options(max_batch, page_size, 0, 0, (C.c_int * 5)(*rows_per_task), 0,
+                           max_page_cols, 1 if o_split else 0, gemv_path, schedule, weight_bits,
+                           1 if prefill else 0, attn_path)
     out = np.zeros(n_tasks, dtype=np.int32)
     _check(lib.mk_plan_describe_schedule(C.byref(c), C.byref(opts), num_sms, smem_optin,
                                          out.ctypes.data, n_tasks))

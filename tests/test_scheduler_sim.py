@@ -223,3 +223,32 @@ def test_prefill_plan_no_deadlock(name, batch, workers, path):
         for ty, wait, need, *_ in tasks:
             if wait >= 0:
                 assert ctr[wait] == need
+
+
+# (shape, max_batch, workers, describe options): the solidified lists of the
+# plans the default options build at batch >= 4 (tensor-core tiles), with
+# prompt chunks, 4-bit weights and tensor-memory staging
+LIST_CASES = [("tiny", 16, 9, dict(prefill=True)),
+              ("3groups", 16, 148, dict(prefill=True, gemv_path=2)),
+              ("3groups", 4, 148, dict()),
+              ("8b", 4, 148, dict()),
+              ("8b", 1, 148, dict(weight_bits=4)),
+              ("8b", 2, 148, dict(gemv_path=3))]
+
+
+@pytest.mark.parametrize("name,batch,workers,opts", LIST_CASES)
+def test_solidified_lists_of_other_plans(name, batch, workers, opts):
+    cfg = SHAPES[name]
+    info, t = mk.describe(cfg, max_batch=batch, max_seq_len=600, num_sms=workers, **opts)
+    assert info["schedule"] == 1
+    if batch >= 4 and cfg["head_dim"] == 128:
+        assert info["gemv_path"] == 2
+    owner = mk.describe_schedule(cfg, info["n_tasks"], max_batch=batch, max_seq_len=600,
+                                 num_sms=workers, schedule=0, **opts)
+    assert owner.min() >= 0 and owner.max() < workers
+    lists = [[int(i) for i in np.flatnonzero(owner == w)] for w in range(workers)]
+    tasks = compile_tasks(cfg, info, t)
+    ctr = simulate(tasks, info["n_events"], workers, seed=2, lists=lists)
+    for ty, wait, need, *_ in tasks:
+        if wait >= 0:
+            assert ctr[wait] == need
